@@ -1,0 +1,241 @@
+/*
+ * lkv.h -- C ABI of liblkv: low-bit quantized KV cache and single-token
+ * decode attention over the packed cache, for NVIDIA B200 (sm_100a).
+ *
+ * The method comes from two web pages:
+ *   [SKV] "Super KV Compression: 突破LLM推理内存瓶颈的三层压缩架构解析"
+ *         §第一层：自适应非对称量化      -- K at 6 bits, V at 4 bits, asymmetric
+ *         §第二层：注意力感知的Token淘汰机制 -- V at 6 / 4 bits or evicted by attention
+ *         §第三层：稀疏V跳过加速          -- do not dequantize low-attention V
+ *   [TQ]  "TurboQuant：将LLM KV缓存压缩5-7倍的突破性技术"
+ *         §TurboQuant的核心创新           -- asymmetric, group-wise quantization
+ *
+ * Conventions for every entry point
+ * ---------------------------------
+ * - All tensor arguments are DEVICE pointers to caller-owned memory; the
+ *   library allocates nothing and keeps no state between calls.
+ * - `stream` is a cudaStream_t passed as void* (NULL = legacy default
+ *   stream).  Every call only enqueues work on it and returns at once; no
+ *   call synchronizes, except lkv_workspace_status().
+ * - Arguments are validated on the host before anything is launched; a
+ *   failed check returns a nonzero lkv_status and enqueues nothing.
+ *   Launch failures return LKV_ERR_CUDA.
+ * - Sequence lengths live on the device, so the host cannot see them:
+ *   kernels clamp each length into [0, T_cap]; the decode entry points also
+ *   record an out-of-range length in the workspace status word.
+ * - bf16 inputs must be finite.  NaN or infinity gives unspecified values
+ *   but never an out-of-bounds access.
+ * - Index arithmetic is 64-bit: any tensor that fits in device memory works.
+ *
+ * Shapes and layouts (row-major, innermost last)
+ *   B batch, Hq query heads, Hkv KV heads (Hq % Hkv == 0), r = Hq / Hkv;
+ *   query head h reads KV head h / r.  D head_dim (64 or 128).  G group:
+ *   G contiguous head_dim channels of one token share one (scale, zero);
+ *   G in {32, 64, 128}, G divides D, ng = D / G.  T_cap cache capacity
+ *   in tokens; T_b = seq_lens[b] valid tokens of sequence b.  bits in
+ *   {2, 4, 6, 8}.
+ *
+ *   K, V (bf16)  [B][Hkv][T_cap][D]
+ *   codes (u8)   [B][Hkv][T_cap][D*bits/8]   one packed row per token:
+ *                code j of the row occupies bits [j*bits, (j+1)*bits) of the
+ *                row read as one little-endian bit string.
+ *   sz (f32)     [B][Hkv][T_cap][ng][2]      (scale, zero) per group.
+ *   q (bf16)     [B][Hq][D];  out (f32) [B][Hq][D].
+ *
+ * Every device pointer must be 16-byte aligned, and T_cap * ng must be even
+ * (the per-token (scale, zero) rows are then 16-byte aligned in bulk).
+ */
+#ifndef LKV_H
+#define LKV_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#if defined(__GNUC__)
+#define LKV_API __attribute__((visibility("default")))
+#else
+#define LKV_API
+#endif
+
+/* Status codes returned by every entry point and kept in the workspace. */
+enum lkv_status {
+    LKV_OK = 0,
+    LKV_ERR_INVALID_ARG = 1, /* null pointer, bad shape, misalignment, bad seq_len */
+    LKV_ERR_UNSUPPORTED = 2, /* a shape or bit width this build does not handle */
+    LKV_ERR_WORKSPACE = 3,   /* workspace smaller than the *_workspace_bytes query */
+    LKV_ERR_CUDA = 4,        /* a CUDA runtime call or launch failed */
+    LKV_ERR_TIMEOUT = 5      /* a bounded cross-block wait gave up (device side) */
+};
+
+/* Quantizer settings: bit widths of K and V codes and the group size. */
+typedef struct {
+    int32_t k_bits; /* 2, 4, 6 or 8 */
+    int32_t v_bits; /* 2, 4, 6 or 8 */
+    int32_t group;  /* 32, 64 or 128; divides D */
+} lkv_qspec;
+
+/* One packed cache segment: codes and (scale, zero) for K and V. */
+typedef struct {
+    void *k_codes;
+    float *k_sz;
+    void *v_codes;
+    float *v_sz;
+} lkv_segment;
+
+/* Human-readable name of a status code (static string, never NULL). */
+LKV_API const char *lkv_status_string(int status);
+
+/* ABI version of this header (major * 100 + minor). */
+LKV_API int lkv_version(void);
+
+/* Bytes of one packed token row: D * bits / 8.  0 for unsupported input. */
+LKV_API size_t lkv_row_bytes(int bits, int D);
+
+/* Bytes of one token's (scale, zero) row: 8 * D / group.  0 if unsupported. */
+LKV_API size_t lkv_sz_row_bytes(int D, int group);
+
+/*
+ * lkv_quantize_kv -- [SKV] §第一层 (K and V at their own widths, asymmetric),
+ * [TQ] §核心创新 (group-wise).  For every valid token t < T_b of every
+ * (b, kv head) and every group of G channels x_0..x_{G-1}, in fp32 with each
+ * operation rounded on its own (no fused multiply-add):
+ *   mn = min x_i, mx = max x_i, d = mx - mn, qmax = 2^bits - 1
+ *   scale = d / qmax, inv = qmax / d      (both 0 when d == 0)
+ *   code_i = clamp(round_half_even((x_i - mn) * inv), 0, qmax)
+ *   stored (scale, zero) = (scale, mn + 0.0f)
+ * and reconstruction is code * scale + zero.  K uses spec.k_bits, V uses
+ * spec.v_bits.  Rows t >= T_b are not written.
+ *
+ *   k, v       in   bf16 [B][Hkv][T_cap][D]
+ *   seq_lens   in   int32 [B] (device)
+ *   k_codes    out  u8  [B][Hkv][T_cap][D*k_bits/8]
+ *   k_sz       out  f32 [B][Hkv][T_cap][D/group][2]
+ *   v_codes    out  u8  [B][Hkv][T_cap][D*v_bits/8]
+ *   v_sz       out  f32 [B][Hkv][T_cap][D/group][2]
+ */
+LKV_API int lkv_quantize_kv(lkv_qspec spec, int B, int Hkv, int T_cap, int D,
+                    const int32_t *seq_lens, const void *k, const void *v,
+                    void *k_codes, float *k_sz, void *v_codes, float *v_sz,
+                    void *stream);
+
+/*
+ * Workspace bytes that lkv_decode_attention needs for these sizes.  The
+ * workspace is caller-owned device memory (256-byte aligned).  It must be
+ * zero-filled before its first use (lkv_workspace_reset); every call leaves
+ * it ready for the next one.  Its first word is a device status word that
+ * calls set on a device-side error and that stays set until a reset.
+ */
+LKV_API size_t lkv_decode_workspace_bytes(lkv_qspec spec, int B, int Hq, int Hkv, int T_cap, int D);
+
+/*
+ * lkv_decode_attention -- one decode step of grouped-query attention read
+ * straight from the packed cache, with the sparse-V skip of [SKV] §第三层.
+ * For every (b, h) with g = h / r and T = T_b:
+ *   khat_t, vhat_t = dequantized rows t < T of KV head g
+ *   s_t  = softmax_scale * sum_d q[b,h,d] * khat_t[d]
+ *   p_t  = exp(s_t - max_u s_u) / sum_u exp(s_u - max_u s_u)
+ *   skip_t = p_t < tau        (the V row is never dequantized for this head)
+ *   out[b,h,:] = sum_{t : !skip_t} p_t * vhat_t     (no renormalisation)
+ * A V row is read from memory only if some head of its group keeps it.
+ * T == 0 gives out = 0.  Arithmetic is fp32; the sequence is split into
+ * chunks whose partial softmax statistics and outputs are merged exactly.
+ *
+ *   q            in   bf16 [B][Hq][D]
+ *   k_codes...   in   the packed cache written by lkv_quantize_kv
+ *   out          out  f32 [B][Hq][D]
+ *   skip_mask    out  u8  [B][Hq][T_cap], nullable; 1 = skipped; only t < T_b written
+ *   skip_counts  out  int64 [2], nullable; {skipped (b, h, t), V rows skipped
+ *                     by every head of their group}
+ *   workspace    in/out  lkv_decode_workspace_bytes() bytes, see above
+ */
+LKV_API int lkv_decode_attention(lkv_qspec spec, int B, int Hq, int Hkv, int T_cap, int D,
+                         const int32_t *seq_lens, const void *q, const void *k_codes,
+                         const float *k_sz, const void *v_codes, const float *v_sz,
+                         float softmax_scale, float tau, float *out, uint8_t *skip_mask,
+                         int64_t *skip_counts, void *workspace, size_t ws_bytes,
+                         void *stream);
+
+/* Zero-fill a workspace (enqueued on stream). */
+LKV_API int lkv_workspace_reset(void *workspace, size_t ws_bytes, void *stream);
+
+/*
+ * Copy the workspace status word to *status (an lkv_status), synchronizing
+ * `stream` first.  The only synchronizing call of the library.
+ */
+LKV_API int lkv_workspace_status(const void *workspace, void *stream, int32_t *status);
+
+/*
+ * lkv_tier_classify -- [SKV] §第二层 (attention-aware tiers).  From the
+ * previous step's attention mass a of each token:
+ *   tier 2 (keep, V at 6 bits) if a > tau_high
+ *   tier 1 (keep, V at 4 bits) if tau_low <= a <= tau_high
+ *   tier 0 (evict K and V)     otherwise (including NaN), and for t >= T_b
+ * Then, per (b, kv head), the positions of tier-2 and of tier-1 tokens are
+ * listed in ascending order (a stable compaction).
+ *
+ *   mass    in   f32 [B][Hkv][T_cap]
+ *   tier    out  i8  [B][Hkv][T_cap]   all T_cap entries written
+ *   counts  out  i32 [B][Hkv][2]       {n2, n1}
+ *   pos_a   out  i32 [B][Hkv][T_cap]   first n2 entries: tier-2 positions
+ *   pos_b   out  i32 [B][Hkv][T_cap]   first n1 entries: tier-1 positions
+ */
+LKV_API int lkv_tier_classify(int B, int Hkv, int T_cap, const int32_t *seq_lens, const float *mass,
+                      float tau_low, float tau_high, int8_t *tier, int32_t *counts,
+                      int32_t *pos_a, int32_t *pos_b, void *stream);
+
+/*
+ * lkv_tier_repack -- [SKV] §第二层 items 1 and 2: every kept token is
+ * quantized again from its bf16 K and V with the lkv_quantize_kv formula --
+ * K at 6 bits in both segments, V at 6 bits in segment A (tier 2) and at 4
+ * bits in segment B (tier 1).  Row i of segment A / B of (b, kv head) holds
+ * position pos_a / pos_b [b][g][i]; rows i >= the count are not written.
+ *
+ *   k, v      in   bf16 [B][Hkv][T_cap][D]
+ *   counts, pos_a, pos_b   in  as written by lkv_tier_classify
+ *   seg_a     out  k_codes u8 [B][Hkv][T_cap][D*6/8], k_sz, v_codes [..][D*6/8], v_sz
+ *   seg_b     out  k_codes u8 [B][Hkv][T_cap][D*6/8], k_sz, v_codes [..][D*4/8], v_sz
+ */
+LKV_API int lkv_tier_repack(int B, int Hkv, int T_cap, int D, int group, const void *k, const void *v,
+                    const int32_t *counts, const int32_t *pos_a, const int32_t *pos_b,
+                    lkv_segment seg_a, lkv_segment seg_b, void *stream);
+
+/* Workspace bytes for lkv_tiered_attention / lkv_tiered_decode (same rules). */
+LKV_API size_t lkv_tiered_workspace_bytes(int B, int Hq, int Hkv, int T_cap, int D, int group);
+
+/*
+ * lkv_tiered_attention -- decode attention over the kept tokens only
+ * ([SKV] §第二层: evicted tokens are gone): one softmax over segment A
+ * (K6, V6) followed by segment B (K6, V4), with the sparse-V skip at tau as
+ * in lkv_decode_attention.  n2 + n1 == 0 gives out = 0.
+ *
+ *   counts   in  i32 [B][Hkv][2]  {rows of segment A, rows of segment B}
+ *   q        in  bf16 [B][Hq][D];  out  f32 [B][Hq][D]
+ *   skip_counts  nullable int64 [2] as in lkv_decode_attention
+ */
+LKV_API int lkv_tiered_attention(int B, int Hq, int Hkv, int T_cap, int D, int group,
+                         const int32_t *counts, const void *q, lkv_segment seg_a,
+                         lkv_segment seg_b, float softmax_scale, float tau, float *out,
+                         int64_t *skip_counts, void *workspace, size_t ws_bytes, void *stream);
+
+/*
+ * lkv_tiered_decode -- the whole attention-tiered step of [SKV] §第二层 in one
+ * call: lkv_tier_classify, then lkv_tier_repack, then lkv_tiered_attention,
+ * enqueued in that order on `stream`.  Arguments as in those three calls.
+ */
+LKV_API int lkv_tiered_decode(int B, int Hq, int Hkv, int T_cap, int D, int group,
+                      const int32_t *seq_lens, const float *mass, float tau_low,
+                      float tau_high, const void *k, const void *v, const void *q,
+                      int8_t *tier, int32_t *counts, int32_t *pos_a, int32_t *pos_b,
+                      lkv_segment seg_a, lkv_segment seg_b, float softmax_scale, float tau,
+                      float *out, int64_t *skip_counts, void *workspace, size_t ws_bytes,
+                      void *stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* LKV_H */

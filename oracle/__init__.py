@@ -49,7 +49,7 @@ def lib():
         L.lkv_oracle_quantize_kv.argtypes = [_I, _I, _I, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P, _P]
         L.lkv_oracle_decode_attention.restype = _I
         L.lkv_oracle_decode_attention.argtypes = [_I, _I, _I, _I, _I, _I, _I, _I, _P, _P, _P, _P,
-                                                  _P, _P, _F, _F, _P, _P, _P]
+                                                  _P, _P, _F, _F, _P, _P, _P, _P]
         L.lkv_oracle_tier_classify.restype = _I
         L.lkv_oracle_tier_classify.argtypes = [_I, _I, _I, _P, _P, _F, _F, _P, _P, _P, _P]
         L.lkv_oracle_tier_repack.restype = _I
@@ -58,7 +58,7 @@ def lib():
         L.lkv_oracle_tiered_attention.restype = _I
         L.lkv_oracle_tiered_attention.argtypes = [_I, _I, _I, _I, _I, _I, _P, _P,
                                                   _P, _P, _P, _P, _P, _P, _P, _P,
-                                                  _F, _F, _P, _P]
+                                                  _F, _F, _P, _P, _P]
         _lib = L
     return _lib
 
@@ -141,8 +141,10 @@ def quantize_kv(kb, vb, G, k_bf16, v_bf16, seq_lens):
     return out
 
 
-def decode_attention(kb, vb, G, seq_lens, q_bf16, cache, softmax_scale, tau, want_mask=True):
-    """Decode attention over a packed cache; returns (out f32 [B,Hq,D], mask, counts).
+def decode_attention(kb, vb, G, seq_lens, q_bf16, cache, softmax_scale, tau, want_mask=True,
+                     want_p=False):
+    """Decode attention over a packed cache; returns (out f32 [B,Hq,D], mask, counts)
+    and, with want_p, also p f64 [B, Hq, T_cap].
 
     mask is u8 [B, Hq, T_cap] (entries t >= T_b stay 0), counts is
     int64 [2] = {skipped (b, h, t) triples, V rows skipped by all heads}.
@@ -155,11 +157,14 @@ def decode_attention(kb, vb, G, seq_lens, q_bf16, cache, softmax_scale, tau, wan
     out = np.zeros((B, Hq, D), np.float32)
     mask = np.zeros((B, Hq, T_cap), np.uint8) if want_mask else None
     counts = np.zeros(2, np.int64)
+    p = np.zeros((B, Hq, T_cap), np.float64) if want_p else None
     _check(lib().lkv_oracle_decode_attention(
         kb, vb, G, B, Hq, Hkv, T_cap, D, _ptr(sl), _ptr(q), _ptr(kc),
         _ptr(_c(cache["k_sz"], np.float32)), _ptr(_c(cache["v_codes"], np.uint8)),
         _ptr(_c(cache["v_sz"], np.float32)), float(softmax_scale), float(tau), _ptr(out),
-        _ptr(mask), _ptr(counts)), "decode_attention")
+        _ptr(mask), _ptr(counts), _ptr(p)), "decode_attention")
+    if want_p:
+        return out, mask, counts, p
     return out, mask, counts
 
 
@@ -205,20 +210,24 @@ def tier_repack(G, k_bf16, v_bf16, counts, pos2, pos1):
     return A, Bs
 
 
-def tiered_attention(G, counts, q_bf16, seg_a, seg_b, softmax_scale, tau):
-    """One softmax over the kept tokens of both segments; returns (out, counts)."""
+def tiered_attention(G, counts, q_bf16, seg_a, seg_b, softmax_scale, tau, want_p=False):
+    """One softmax over the kept tokens of both segments; returns (out, counts)
+    and, with want_p, p f64 [B, Hq, T_cap] over segment-A-then-B rows."""
     q = _c(q_bf16, np.uint16)
     B, Hq, D = q.shape
     Hkv, T_cap = seg_a["k_codes"].shape[1], seg_a["k_codes"].shape[2]
     out = np.zeros((B, Hq, D), np.float32)
     sc = np.zeros(2, np.int64)
+    p = np.zeros((B, Hq, T_cap), np.float64) if want_p else None
     _check(lib().lkv_oracle_tiered_attention(
         B, Hq, Hkv, T_cap, D, G, _ptr(_c(counts, np.int32)), _ptr(q),
         _ptr(_c(seg_a["k_codes"], np.uint8)), _ptr(_c(seg_a["k_sz"], np.float32)),
         _ptr(_c(seg_a["v_codes"], np.uint8)), _ptr(_c(seg_a["v_sz"], np.float32)),
         _ptr(_c(seg_b["k_codes"], np.uint8)), _ptr(_c(seg_b["k_sz"], np.float32)),
         _ptr(_c(seg_b["v_codes"], np.uint8)), _ptr(_c(seg_b["v_sz"], np.float32)),
-        float(softmax_scale), float(tau), _ptr(out), _ptr(sc)), "tiered_attention")
+        float(softmax_scale), float(tau), _ptr(out), _ptr(sc), _ptr(p)), "tiered_attention")
+    if want_p:
+        return out, sc, p
     return out, sc
 
 

@@ -87,7 +87,8 @@ void lkv_oracle_quantize_group(const float *x, int n, int bits,
         float diff = x[i] - mn;
         float y = diff * inv;
         float r = nearbyintf(y); /* default rounding mode: half to even */
-        if (r < 0.0f) r = 0.0f;
+        if (!(r >= 0.0f)) r = 0.0f; /* also NaN: 0 * inf when d is tiny enough
+                                       that qmax / d overflows */
         if (r > qmax) r = qmax;
         codes[i] = (uint32_t)r;
     }
@@ -216,12 +217,12 @@ int lkv_oracle_quantize_kv(int kb, int vb, int G, int B, int Hkv, int T_cap, int
  *   p_t = exp(s_t - max s) / sum_u exp(s_u - max s)
  *   out = sum_{t : p_t >= tau} p_t * vhat_t
  *
- * skip[t] receives 1 for a skipped row and 0 otherwise.  With n == 0 the
- * output is all zeros.
+ * skip[t] receives 1 for a skipped row and 0 otherwise; p_out (nullable)
+ * receives p_t.  With n == 0 the output is all zeros.
  */
 static void attend_one_head(const float *qf, int D, int n, const float *const *khat,
                             const float *const *vhat, float softmax_scale, float tau,
-                            double *s_buf, float *out, uint8_t *skip)
+                            double *s_buf, float *out, uint8_t *skip, double *p_out)
 {
     double acc[256];
     for (int d = 0; d < D; ++d) acc[d] = 0.0;
@@ -239,6 +240,7 @@ static void attend_one_head(const float *qf, int D, int n, const float *const *k
             double p = exp(s_buf[t] - m) / l;
             int skipped = p < (double)tau;
             if (skip) skip[t] = (uint8_t)skipped;
+            if (p_out) p_out[t] = p;
             if (!skipped)
                 for (int d = 0; d < D; ++d) acc[d] += p * (double)vhat[t][d];
         }
@@ -251,14 +253,15 @@ static void attend_one_head(const float *qf, int D, int n, const float *const *k
  * KV head h / (Hq / Hkv).  q is bf16 [B][Hq][D]; out is f32 [B][Hq][D];
  * skip_mask (nullable) is u8 [B][Hq][T_cap] and only entries t < T_b are
  * written; skip_counts (nullable) receives {skipped (b, h, t) triples,
- * V rows skipped by every head of their group}.
+ * V rows skipped by every head of their group}; p_out (nullable) is f64
+ * [B][Hq][T_cap] and receives the probabilities p_t for t < T_b.
  */
 int lkv_oracle_decode_attention(int kb, int vb, int G, int B, int Hq, int Hkv, int T_cap,
                                 int D, const int32_t *seq_lens, const uint16_t *q,
                                 const uint8_t *k_codes, const float *k_sz,
                                 const uint8_t *v_codes, const float *v_sz,
                                 float softmax_scale, float tau, float *out,
-                                uint8_t *skip_mask, int64_t *skip_counts)
+                                uint8_t *skip_mask, int64_t *skip_counts, double *p_out)
 {
     if (!shape_ok(kb, G, D) || !shape_ok(vb, G, D) || Hkv <= 0 || Hq % Hkv != 0 || B < 0)
         return ORACLE_BAD_ARG;
@@ -289,7 +292,8 @@ int lkv_oracle_decode_attention(int kb, int vb, int G, int B, int Hq, int Hkv, i
             float qf[256];
             for (int d = 0; d < D; ++d) qf[d] = bf16_to_float(q[((long long)b * Hq + h) * D + d]);
             attend_one_head(qf, D, T, kp, vp, softmax_scale, tau, s,
-                            out + ((long long)b * Hq + h) * D, sk + (long long)j * (T > 0 ? T : 1));
+                            out + ((long long)b * Hq + h) * D, sk + (long long)j * (T > 0 ? T : 1),
+                            p_out ? p_out + ((long long)b * Hq + h) * T_cap : NULL);
             if (skip_mask)
                 for (int t = 0; t < T; ++t)
                     skip_mask[((long long)b * Hq + h) * T_cap + t] = sk[(long long)j * (T > 0 ? T : 1) + t];
@@ -389,7 +393,7 @@ int lkv_oracle_tiered_attention(int B, int Hq, int Hkv, int T_cap, int D, int G,
                                 const uint8_t *a_kc, const float *a_ksz, const uint8_t *a_vc,
                                 const float *a_vsz, const uint8_t *b_kc, const float *b_ksz,
                                 const uint8_t *b_vc, const float *b_vsz, float softmax_scale,
-                                float tau, float *out, int64_t *skip_counts)
+                                float tau, float *out, int64_t *skip_counts, double *p_out)
 {
     if (!shape_ok(6, G, D) || !shape_ok(4, G, D) || Hkv <= 0 || Hq % Hkv != 0 || B < 0)
         return ORACLE_BAD_ARG;
@@ -424,7 +428,8 @@ int lkv_oracle_tiered_attention(int B, int Hq, int Hkv, int T_cap, int D, int G,
             float qf[256];
             for (int d = 0; d < D; ++d) qf[d] = bf16_to_float(q[((long long)b * Hq + h) * D + d]);
             attend_one_head(qf, D, n, kp, vp, softmax_scale, tau, s,
-                            out + ((long long)b * Hq + h) * D, sk + (size_t)j * cap);
+                            out + ((long long)b * Hq + h) * D, sk + (size_t)j * cap,
+                            p_out ? p_out + ((long long)b * Hq + h) * T_cap : NULL);
         }
         for (int i = 0; i < n; ++i) {
             int all = 1;

@@ -1,0 +1,308 @@
+// api.cu -- the extern "C" entry points of liblkv (declared in include/lkv.h):
+// host-side validation, workspace carving and kernel launches.  Nothing here
+// allocates device memory or synchronizes (except lkv_workspace_status).
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+
+#include "../../include/lkv.h"
+#include "lkv_kernels.cuh"
+
+namespace lkv {
+
+int num_sms() {
+  static int cached[64] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+  if (cached[dev] == 0) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
+    cached[dev] = n;
+  }
+  return cached[dev];
+}
+
+namespace {
+
+constexpr int kChunk = 256;       // decode rows per chunk
+constexpr size_t kAlign = 256;
+
+size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
+
+bool bits_ok(int b) { return b == 2 || b == 4 || b == 6 || b == 8; }
+bool dim_ok(int D) { return D == 64 || D == 128; }
+bool group_ok(int G, int D) { return (G == 32 || G == 64 || G == 128) && G <= D && D % G == 0; }
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+// A pointer that must be valid when its tensor is non-empty.
+bool ptr_ok(const void* p, bool nonempty) { return !nonempty || (p != nullptr && aligned16(p)); }
+
+int from_cuda(cudaError_t e) { return e == cudaSuccess ? LKV_OK : LKV_ERR_CUDA; }
+
+struct WsLayout {
+  size_t status, logits, stats, partial, total;
+  int n_chunks;
+};
+
+WsLayout ws_layout(int B, int Hq, int Hkv, int T_cap, int D) {
+  WsLayout w{};
+  const int r = Hq / Hkv;
+  w.n_chunks = T_cap > 0 ? (T_cap + kChunk - 1) / kChunk : 1;
+  const size_t units = (size_t)B * (size_t)Hkv;
+  w.status = 0;
+  w.logits = align_up(4);
+  w.stats = w.logits + align_up(units * (size_t)T_cap * r * sizeof(float));
+  w.partial = w.stats + align_up(units * (size_t)w.n_chunks * r * 2 * sizeof(float));
+  w.total = w.partial + align_up(units * (size_t)w.n_chunks * r * D * sizeof(float));
+  return w;
+}
+
+// Shapes shared by every attention call.
+int check_attention_shape(int B, int Hq, int Hkv, int T_cap, int D, int G) {
+  if (B < 0 || Hq <= 0 || Hkv <= 0 || T_cap < 0) return LKV_ERR_INVALID_ARG;
+  if (Hq % Hkv != 0) return LKV_ERR_INVALID_ARG;
+  if (!dim_ok(D) || !group_ok(G, D)) return LKV_ERR_UNSUPPORTED;
+  const int r = Hq / Hkv;
+  if (r > 64 || !(r == 1 || r == 2 || r % 4 == 0)) return LKV_ERR_UNSUPPORTED;
+  if (((long long)T_cap * (D / G)) % 2 != 0) return LKV_ERR_UNSUPPORTED;
+  return LKV_OK;
+}
+
+int check_cache_shape(int B, int Hkv, int T_cap, int D, int G) {
+  if (B < 0 || Hkv <= 0 || T_cap < 0) return LKV_ERR_INVALID_ARG;
+  if (!dim_ok(D) || !group_ok(G, D)) return LKV_ERR_UNSUPPORTED;
+  if (((long long)T_cap * (D / G)) % 2 != 0) return LKV_ERR_UNSUPPORTED;
+  return LKV_OK;
+}
+
+bool segment_ok(const lkv_segment& s, bool nonempty) {
+  return ptr_ok(s.k_codes, nonempty) && ptr_ok(s.k_sz, nonempty) && ptr_ok(s.v_codes, nonempty) &&
+         ptr_ok(s.v_sz, nonempty);
+}
+
+int fill_workspace(DecodeArgs& a, int B, int Hq, int Hkv, int T_cap, int D, void* ws, size_t ws_bytes) {
+  const WsLayout w = ws_layout(B, Hq, Hkv, T_cap, D);
+  if (ws == nullptr || (reinterpret_cast<uintptr_t>(ws) % kAlign) != 0) return LKV_ERR_INVALID_ARG;
+  if (ws_bytes < w.total) return LKV_ERR_WORKSPACE;
+  char* base = static_cast<char*>(ws);
+  a.status = reinterpret_cast<int*>(base + w.status);
+  a.logits = reinterpret_cast<float*>(base + w.logits);
+  a.stats = reinterpret_cast<float*>(base + w.stats);
+  a.partial = reinterpret_cast<float*>(base + w.partial);
+  a.chunk = kChunk;
+  a.n_chunks = w.n_chunks;
+  return LKV_OK;
+}
+
+}  // namespace
+}  // namespace lkv
+
+using namespace lkv;
+
+extern "C" {
+
+const char* lkv_status_string(int status) {
+  switch (status) {
+    case LKV_OK: return "LKV_OK";
+    case LKV_ERR_INVALID_ARG: return "LKV_ERR_INVALID_ARG";
+    case LKV_ERR_UNSUPPORTED: return "LKV_ERR_UNSUPPORTED";
+    case LKV_ERR_WORKSPACE: return "LKV_ERR_WORKSPACE";
+    case LKV_ERR_CUDA: return "LKV_ERR_CUDA";
+    case LKV_ERR_TIMEOUT: return "LKV_ERR_TIMEOUT";
+  }
+  return "LKV_ERR_UNKNOWN";
+}
+
+int lkv_version(void) { return 100; }
+
+size_t lkv_row_bytes(int bits, int D) {
+  if (!bits_ok(bits) || D <= 0 || (D * bits) % 8 != 0) return 0;
+  return (size_t)D * bits / 8;
+}
+
+size_t lkv_sz_row_bytes(int D, int group) {
+  if (!group_ok(group, D)) return 0;
+  return (size_t)8 * (D / group);
+}
+
+int lkv_quantize_kv(lkv_qspec spec, int B, int Hkv, int T_cap, int D, const int32_t* seq_lens, const void* k,
+                    const void* v, void* k_codes, float* k_sz, void* v_codes, float* v_sz, void* stream) {
+  if (!bits_ok(spec.k_bits) || !bits_ok(spec.v_bits)) return LKV_ERR_UNSUPPORTED;
+  int rc = check_cache_shape(B, Hkv, T_cap, D, spec.group);
+  if (rc) return rc;
+  const bool ne = (long long)B * Hkv * T_cap > 0;
+  if (!ptr_ok(seq_lens, B > 0) || !ptr_ok(k, ne) || !ptr_ok(v, ne) || !ptr_ok(k_codes, ne) || !ptr_ok(k_sz, ne) ||
+      !ptr_ok(v_codes, ne) || !ptr_ok(v_sz, ne))
+    return LKV_ERR_INVALID_ARG;
+  if (!ne) return LKV_OK;
+  QuantizeArgs a{};
+  a.B = B; a.Hkv = Hkv; a.T_cap = T_cap; a.G = spec.group;
+  a.seq_lens = seq_lens;
+  a.k = static_cast<const uint16_t*>(k);
+  a.v = static_cast<const uint16_t*>(v);
+  a.k_codes = static_cast<uint8_t*>(k_codes);
+  a.k_sz = k_sz;
+  a.v_codes = static_cast<uint8_t*>(v_codes);
+  a.v_sz = v_sz;
+  return from_cuda(launch_quantize_kv(a, spec.k_bits, spec.v_bits, D, static_cast<cudaStream_t>(stream)));
+}
+
+size_t lkv_decode_workspace_bytes(lkv_qspec spec, int B, int Hq, int Hkv, int T_cap, int D) {
+  if (!bits_ok(spec.k_bits) || !bits_ok(spec.v_bits)) return 0;
+  if (check_attention_shape(B, Hq, Hkv, T_cap, D, spec.group)) return 0;
+  return ws_layout(B, Hq, Hkv, T_cap, D).total;
+}
+
+int lkv_decode_attention(lkv_qspec spec, int B, int Hq, int Hkv, int T_cap, int D, const int32_t* seq_lens,
+                         const void* q, const void* k_codes, const float* k_sz, const void* v_codes,
+                         const float* v_sz, float softmax_scale, float tau, float* out, uint8_t* skip_mask,
+                         int64_t* skip_counts, void* workspace, size_t ws_bytes, void* stream) {
+  if (!bits_ok(spec.k_bits) || !bits_ok(spec.v_bits)) return LKV_ERR_UNSUPPORTED;
+  int rc = check_attention_shape(B, Hq, Hkv, T_cap, D, spec.group);
+  if (rc) return rc;
+  if (!std::isfinite(softmax_scale) || std::isnan(tau)) return LKV_ERR_INVALID_ARG;
+  const bool ne = (long long)B * Hkv * T_cap > 0;
+  if (!ptr_ok(seq_lens, B > 0) || !ptr_ok(q, B > 0) || !ptr_ok(out, B > 0) || !ptr_ok(k_codes, ne) ||
+      !ptr_ok(k_sz, ne) || !ptr_ok(v_codes, ne) || !ptr_ok(v_sz, ne))
+    return LKV_ERR_INVALID_ARG;
+  if (skip_counts && !aligned16(skip_counts)) return LKV_ERR_INVALID_ARG;
+  DecodeArgs a{};
+  rc = fill_workspace(a, B, Hq, Hkv, T_cap, D, workspace, ws_bytes);
+  if (rc) return rc;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (B == 0) {
+    if (skip_counts) return from_cuda(cudaMemsetAsync(skip_counts, 0, 2 * sizeof(int64_t), s));
+    return LKV_OK;
+  }
+  a.B = B; a.Hq = Hq; a.Hkv = Hkv; a.T_cap = T_cap; a.G = spec.group; a.r = Hq / Hkv;
+  a.lens = seq_lens; a.len_mode = 0;
+  a.q = static_cast<const uint16_t*>(q);
+  a.kc[0] = a.kc[1] = static_cast<const uint8_t*>(k_codes);
+  a.ksz[0] = a.ksz[1] = k_sz;
+  a.vc[0] = a.vc[1] = static_cast<const uint8_t*>(v_codes);
+  a.vsz[0] = a.vsz[1] = v_sz;
+  a.q_scale = softmax_scale * 1.4426950408889634f;
+  a.tau = tau;
+  a.out = out;
+  a.skip_mask = skip_mask;
+  a.skip_counts = reinterpret_cast<unsigned long long*>(skip_counts);
+  return from_cuda(launch_decode(a, D, spec.k_bits, spec.v_bits, spec.v_bits, s));
+}
+
+int lkv_workspace_reset(void* workspace, size_t ws_bytes, void* stream) {
+  if (workspace == nullptr && ws_bytes > 0) return LKV_ERR_INVALID_ARG;
+  if (ws_bytes == 0) return LKV_OK;
+  return from_cuda(cudaMemsetAsync(workspace, 0, ws_bytes, static_cast<cudaStream_t>(stream)));
+}
+
+int lkv_workspace_status(const void* workspace, void* stream, int32_t* status) {
+  if (workspace == nullptr || status == nullptr) return LKV_ERR_INVALID_ARG;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  int32_t v = 0;
+  cudaError_t e = cudaMemcpyAsync(&v, workspace, sizeof(int32_t), cudaMemcpyDeviceToHost, s);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+  if (e != cudaSuccess) return LKV_ERR_CUDA;
+  *status = v;
+  return LKV_OK;
+}
+
+int lkv_tier_classify(int B, int Hkv, int T_cap, const int32_t* seq_lens, const float* mass, float tau_low,
+                      float tau_high, int8_t* tier, int32_t* counts, int32_t* pos_a, int32_t* pos_b, void* stream) {
+  if (B < 0 || Hkv <= 0 || T_cap < 0) return LKV_ERR_INVALID_ARG;
+  const bool ne = (long long)B * Hkv * T_cap > 0;
+  if (!ptr_ok(seq_lens, B > 0) || !ptr_ok(counts, B > 0) || !ptr_ok(mass, ne) || !ptr_ok(tier, ne) ||
+      !ptr_ok(pos_a, ne) || !ptr_ok(pos_b, ne))
+    return LKV_ERR_INVALID_ARG;
+  if (B == 0) return LKV_OK;
+  ClassifyArgs a{};
+  a.B = B; a.Hkv = Hkv; a.T_cap = T_cap;
+  a.seq_lens = seq_lens; a.mass = mass; a.tau_low = tau_low; a.tau_high = tau_high;
+  a.tier = tier; a.counts = counts; a.pos_a = pos_a; a.pos_b = pos_b;
+  return from_cuda(launch_tier_classify(a, static_cast<cudaStream_t>(stream)));
+}
+
+int lkv_tier_repack(int B, int Hkv, int T_cap, int D, int group, const void* k, const void* v, const int32_t* counts,
+                    const int32_t* pos_a, const int32_t* pos_b, lkv_segment seg_a, lkv_segment seg_b, void* stream) {
+  int rc = check_cache_shape(B, Hkv, T_cap, D, group);
+  if (rc) return rc;
+  const bool ne = (long long)B * Hkv * T_cap > 0;
+  if (!ptr_ok(counts, B > 0) || !ptr_ok(k, ne) || !ptr_ok(v, ne) || !ptr_ok(pos_a, ne) || !ptr_ok(pos_b, ne) ||
+      !segment_ok(seg_a, ne) || !segment_ok(seg_b, ne))
+    return LKV_ERR_INVALID_ARG;
+  if (!ne) return LKV_OK;
+  RepackArgs a{};
+  a.B = B; a.Hkv = Hkv; a.T_cap = T_cap; a.G = group;
+  a.k = static_cast<const uint16_t*>(k);
+  a.v = static_cast<const uint16_t*>(v);
+  a.counts = counts; a.pos_a = pos_a; a.pos_b = pos_b;
+  a.a_kc = static_cast<uint8_t*>(seg_a.k_codes); a.a_ksz = seg_a.k_sz;
+  a.a_vc = static_cast<uint8_t*>(seg_a.v_codes); a.a_vsz = seg_a.v_sz;
+  a.b_kc = static_cast<uint8_t*>(seg_b.k_codes); a.b_ksz = seg_b.k_sz;
+  a.b_vc = static_cast<uint8_t*>(seg_b.v_codes); a.b_vsz = seg_b.v_sz;
+  return from_cuda(launch_tier_repack(a, D, static_cast<cudaStream_t>(stream)));
+}
+
+size_t lkv_tiered_workspace_bytes(int B, int Hq, int Hkv, int T_cap, int D, int group) {
+  if (check_attention_shape(B, Hq, Hkv, T_cap, D, group)) return 0;
+  return ws_layout(B, Hq, Hkv, T_cap, D).total;
+}
+
+int lkv_tiered_attention(int B, int Hq, int Hkv, int T_cap, int D, int group, const int32_t* counts, const void* q,
+                         lkv_segment seg_a, lkv_segment seg_b, float softmax_scale, float tau, float* out,
+                         int64_t* skip_counts, void* workspace, size_t ws_bytes, void* stream) {
+  int rc = check_attention_shape(B, Hq, Hkv, T_cap, D, group);
+  if (rc) return rc;
+  if (!std::isfinite(softmax_scale) || std::isnan(tau)) return LKV_ERR_INVALID_ARG;
+  const bool ne = (long long)B * Hkv * T_cap > 0;
+  if (!ptr_ok(counts, B > 0) || !ptr_ok(q, B > 0) || !ptr_ok(out, B > 0) || !segment_ok(seg_a, ne) ||
+      !segment_ok(seg_b, ne))
+    return LKV_ERR_INVALID_ARG;
+  if (skip_counts && !aligned16(skip_counts)) return LKV_ERR_INVALID_ARG;
+  DecodeArgs a{};
+  rc = fill_workspace(a, B, Hq, Hkv, T_cap, D, workspace, ws_bytes);
+  if (rc) return rc;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (B == 0) {
+    if (skip_counts) return from_cuda(cudaMemsetAsync(skip_counts, 0, 2 * sizeof(int64_t), s));
+    return LKV_OK;
+  }
+  a.B = B; a.Hq = Hq; a.Hkv = Hkv; a.T_cap = T_cap; a.G = group; a.r = Hq / Hkv;
+  a.lens = counts; a.len_mode = 1;
+  a.q = static_cast<const uint16_t*>(q);
+  a.kc[0] = static_cast<const uint8_t*>(seg_a.k_codes); a.kc[1] = static_cast<const uint8_t*>(seg_b.k_codes);
+  a.ksz[0] = seg_a.k_sz; a.ksz[1] = seg_b.k_sz;
+  a.vc[0] = static_cast<const uint8_t*>(seg_a.v_codes); a.vc[1] = static_cast<const uint8_t*>(seg_b.v_codes);
+  a.vsz[0] = seg_a.v_sz; a.vsz[1] = seg_b.v_sz;
+  a.q_scale = softmax_scale * 1.4426950408889634f;
+  a.tau = tau;
+  a.out = out;
+  a.skip_mask = nullptr;
+  a.skip_counts = reinterpret_cast<unsigned long long*>(skip_counts);
+  return from_cuda(launch_decode(a, D, 6, 6, 4, s));
+}
+
+int lkv_tiered_decode(int B, int Hq, int Hkv, int T_cap, int D, int group, const int32_t* seq_lens, const float* mass,
+                      float tau_low, float tau_high, const void* k, const void* v, const void* q, int8_t* tier,
+                      int32_t* counts, int32_t* pos_a, int32_t* pos_b, lkv_segment seg_a, lkv_segment seg_b,
+                      float softmax_scale, float tau, float* out, int64_t* skip_counts, void* workspace,
+                      size_t ws_bytes, void* stream) {
+  // Validate all three stages before enqueueing any of them.
+  int rc = check_attention_shape(B, Hq, Hkv, T_cap, D, group);
+  if (rc) return rc;
+  if (!std::isfinite(softmax_scale) || std::isnan(tau)) return LKV_ERR_INVALID_ARG;
+  const bool ne = (long long)B * Hkv * T_cap > 0;
+  if (!ptr_ok(seq_lens, B > 0) || !ptr_ok(counts, B > 0) || !ptr_ok(q, B > 0) || !ptr_ok(out, B > 0) ||
+      !ptr_ok(mass, ne) || !ptr_ok(tier, ne) || !ptr_ok(pos_a, ne) || !ptr_ok(pos_b, ne) || !ptr_ok(k, ne) ||
+      !ptr_ok(v, ne) || !segment_ok(seg_a, ne) || !segment_ok(seg_b, ne))
+    return LKV_ERR_INVALID_ARG;
+  if (skip_counts && !aligned16(skip_counts)) return LKV_ERR_INVALID_ARG;
+  if (workspace == nullptr || (reinterpret_cast<uintptr_t>(workspace) % 256) != 0) return LKV_ERR_INVALID_ARG;
+  if (ws_bytes < lkv_tiered_workspace_bytes(B, Hq, Hkv, T_cap, D, group)) return LKV_ERR_WORKSPACE;
+  rc = lkv_tier_classify(B, Hkv, T_cap, seq_lens, mass, tau_low, tau_high, tier, counts, pos_a, pos_b, stream);
+  if (rc) return rc;
+  rc = lkv_tier_repack(B, Hkv, T_cap, D, group, k, v, counts, pos_a, pos_b, seg_a, seg_b, stream);
+  if (rc) return rc;
+  return lkv_tiered_attention(B, Hq, Hkv, T_cap, D, group, counts, q, seg_a, seg_b, softmax_scale, tau, out,
+                              skip_counts, workspace, ws_bytes, stream);
+}
+
+}  // extern "C"

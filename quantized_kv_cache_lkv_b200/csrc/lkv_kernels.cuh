@@ -1,0 +1,76 @@
+// lkv_kernels.cuh -- kernel argument blocks and launchers (internal to liblkv).
+#pragma once
+#include "lkv_device.cuh"
+
+namespace lkv {
+
+struct QuantizeArgs {
+  int B, Hkv, T_cap, G;
+  const int32_t* seq_lens;
+  const uint16_t* k;
+  const uint16_t* v;
+  uint8_t* k_codes;
+  float* k_sz;
+  uint8_t* v_codes;
+  float* v_sz;
+};
+
+struct RepackArgs {
+  int B, Hkv, T_cap, G;
+  const uint16_t* k;
+  const uint16_t* v;
+  const int32_t* counts;
+  const int32_t* pos_a;
+  const int32_t* pos_b;
+  uint8_t *a_kc, *a_vc, *b_kc, *b_vc;
+  float *a_ksz, *a_vsz, *b_ksz, *b_vsz;
+};
+
+struct ClassifyArgs {
+  int B, Hkv, T_cap;
+  const int32_t* seq_lens;
+  const float* mass;
+  float tau_low, tau_high;
+  int8_t* tier;
+  int32_t* counts;
+  int32_t* pos_a;
+  int32_t* pos_b;
+};
+
+// A decode problem: per (b, kv head) up to two packed segments that together
+// form one sequence (segment 0 rows first).  Plain decode has one segment of
+// seq_lens[b] rows; the tiered cache has segment A (V6) then segment B (V4)
+// with counts[b][g][0..1] rows.
+struct DecodeArgs {
+  int B, Hq, Hkv, T_cap, G;
+  int r;                 // Hq / Hkv
+  const int32_t* lens;   // seq_lens [B] (len_mode 0) or counts [B][Hkv][2] (len_mode 1)
+  int len_mode;
+  const uint16_t* q;
+  const uint8_t* kc[2];
+  const float* ksz[2];
+  const uint8_t* vc[2];
+  const float* vsz[2];
+  float q_scale;         // softmax_scale * log2(e): logits are kept in base 2
+  float tau;
+  float* out;
+  uint8_t* skip_mask;    // nullable, [B][Hq][T_cap] (plain decode only)
+  unsigned long long* skip_counts;  // nullable, [2]
+  // workspace
+  int* status;
+  int chunk;             // rows per chunk
+  int n_chunks;          // chunks per (b, g) = ceil(2 * T_cap / chunk) for two segments
+  float* logits;         // [B][Hkv][n_chunks * chunk][r]
+  float* stats;          // [B][Hkv][n_chunks][r][2]  (max, sum of exp2)
+  float* partial;        // [B][Hkv][n_chunks][r][D]
+};
+
+int num_sms();
+
+cudaError_t launch_quantize_kv(const QuantizeArgs& a, int kb, int vb, int D, cudaStream_t s);
+cudaError_t launch_tier_repack(const RepackArgs& a, int D, cudaStream_t s);
+cudaError_t launch_tier_classify(const ClassifyArgs& a, cudaStream_t s);
+// vb0 / vb1: V bit widths of segment 0 / 1 (equal for plain decode).
+cudaError_t launch_decode(const DecodeArgs& a, int D, int kb, int vb0, int vb1, cudaStream_t s);
+
+}  // namespace lkv

@@ -1,0 +1,149 @@
+"""The C ABI, without a GPU: liblkv.so loads, exports every entry point that
+include/lkv.h declares, and rejects bad arguments on the host before it
+launches anything (fake device addresses are never dereferenced)."""
+import os
+import re
+
+import pytest
+
+from quantized_kv_cache_lkv_b200 import lkv
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "lkv.h")
+
+FAKE = 0x7F0000000000        # 16-byte aligned, never dereferenced
+MISALIGNED = FAKE + 8
+K6V4 = (6, 4, 64)
+
+
+@pytest.fixture(scope="module")
+def L():
+    from quantized_kv_cache_lkv_b200 import build
+    build.build()
+    return lkv.lib()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    return sorted(set(re.findall(r"^LKV_API\s+[\w\s\*]+?\b(lkv_\w+)\s*\(", text, re.M)))
+
+
+def test_header_declarations_are_all_exported(L):
+    names = declared_functions()
+    assert len(names) >= 14
+    for n in names:
+        assert hasattr(L, n), n
+    # the binding wraps exactly the declared set
+    assert sorted(lkv.SIGNATURES) == names
+
+
+def test_status_strings_and_sizes(L):
+    assert lkv.lkv_status_string(0) == "LKV_OK"
+    assert lkv.lkv_status_string(5) == "LKV_ERR_TIMEOUT"
+    assert lkv.lkv_status_string(99) == "LKV_ERR_UNKNOWN"
+    assert lkv.lkv_version() == 100
+    assert lkv.lkv_row_bytes(6, 128) == 96 and lkv.lkv_row_bytes(4, 128) == 64
+    assert lkv.lkv_row_bytes(2, 64) == 16 and lkv.lkv_row_bytes(8, 64) == 64
+    assert lkv.lkv_row_bytes(5, 128) == 0
+    assert lkv.lkv_sz_row_bytes(128, 64) == 16 and lkv.lkv_sz_row_bytes(64, 32) == 16
+    assert lkv.lkv_sz_row_bytes(64, 128) == 0
+
+
+def test_workspace_sizes(L):
+    n = lkv.lkv_decode_workspace_bytes(K6V4, 16, 32, 8, 8192, 128)
+    logits = 16 * 8 * 8192 * 4 * 4
+    assert logits < n < logits * 2
+    assert lkv.lkv_decode_workspace_bytes(K6V4, 16, 30, 8, 8192, 128) == 0   # Hq % Hkv
+    assert lkv.lkv_decode_workspace_bytes((5, 4, 64), 1, 4, 2, 256, 64) == 0
+    assert lkv.lkv_tiered_workspace_bytes(32, 32, 8, 32768, 128, 64) > 0
+
+
+def rc_of(fn, *args, **kwargs):
+    try:
+        fn(*args, **kwargs)
+    except lkv.LkvError as e:
+        return e.status
+    return 0
+
+
+def quant_args(**kw):
+    a = dict(spec=K6V4, B=2, Hkv=2, T_cap=64, D=128, seq_lens=FAKE, k=FAKE, v=FAKE, k_codes=FAKE,
+             k_sz=FAKE, v_codes=FAKE, v_sz=FAKE, stream=0)
+    a.update(kw)
+    return a
+
+
+@pytest.mark.parametrize("kw,want", [
+    (dict(spec=(5, 4, 64)), lkv.LKV_ERR_UNSUPPORTED),
+    (dict(spec=(6, 4, 48)), lkv.LKV_ERR_UNSUPPORTED),
+    (dict(spec=(6, 4, 256)), lkv.LKV_ERR_UNSUPPORTED),
+    (dict(D=96), lkv.LKV_ERR_UNSUPPORTED),
+    (dict(spec=(6, 4, 128), T_cap=63), lkv.LKV_ERR_UNSUPPORTED),   # T_cap * ng odd
+    (dict(B=-1), lkv.LKV_ERR_INVALID_ARG),
+    (dict(Hkv=0), lkv.LKV_ERR_INVALID_ARG),
+    (dict(k=None), lkv.LKV_ERR_INVALID_ARG),
+    (dict(v_sz=MISALIGNED), lkv.LKV_ERR_INVALID_ARG),
+    (dict(seq_lens=None), lkv.LKV_ERR_INVALID_ARG),
+])
+def test_quantize_rejects(L, kw, want):
+    assert rc_of(lambda **a: lkv.lkv_quantize_kv(**a), **quant_args(**kw)) == want
+
+
+def test_empty_inputs_are_no_ops(L):
+    # nothing to do: succeeds without touching any pointer or the GPU
+    assert rc_of(lambda **a: lkv.lkv_quantize_kv(**a), **quant_args(B=0, k=None, v=None)) == 0
+    assert rc_of(lambda **a: lkv.lkv_quantize_kv(**a), **quant_args(T_cap=0)) == 0
+    assert rc_of(lkv.lkv_tier_classify, 0, 8, 64, None, None, 0.0, 1.0, None, None, None, None, 0) == 0
+
+
+def decode_args(**kw):
+    a = dict(spec=K6V4, B=2, Hq=8, Hkv=2, T_cap=64, D=128, seq_lens=FAKE, q=FAKE, k_codes=FAKE,
+             k_sz=FAKE, v_codes=FAKE, v_sz=FAKE, softmax_scale=0.088, tau=0.0, out=FAKE,
+             skip_mask=None, skip_counts=None, workspace=FAKE, ws_bytes=1 << 40, stream=0)
+    a.update(kw)
+    return a
+
+
+@pytest.mark.parametrize("kw,want", [
+    (dict(Hq=7), lkv.LKV_ERR_INVALID_ARG),
+    (dict(Hq=6), lkv.LKV_ERR_UNSUPPORTED),                    # r = 3
+    (dict(Hq=256, Hkv=2), lkv.LKV_ERR_UNSUPPORTED),           # r > 64
+    (dict(D=256), lkv.LKV_ERR_UNSUPPORTED),
+    (dict(spec=(6, 3, 64)), lkv.LKV_ERR_UNSUPPORTED),
+    (dict(softmax_scale=float("inf")), lkv.LKV_ERR_INVALID_ARG),
+    (dict(tau=float("nan")), lkv.LKV_ERR_INVALID_ARG),
+    (dict(q=None), lkv.LKV_ERR_INVALID_ARG),
+    (dict(out=MISALIGNED), lkv.LKV_ERR_INVALID_ARG),
+    (dict(skip_counts=MISALIGNED), lkv.LKV_ERR_INVALID_ARG),
+    (dict(workspace=None), lkv.LKV_ERR_INVALID_ARG),
+    (dict(workspace=FAKE + 16), lkv.LKV_ERR_INVALID_ARG),     # not 256-byte aligned
+    (dict(ws_bytes=1024), lkv.LKV_ERR_WORKSPACE),
+])
+def test_decode_rejects(L, kw, want):
+    assert rc_of(lambda **a: lkv.lkv_decode_attention(**a), **decode_args(**kw)) == want
+
+
+def test_tiered_rejects(L):
+    seg = lkv.lkv_segment(FAKE, FAKE, FAKE, FAKE)
+    bad = lkv.lkv_segment(FAKE, None, FAKE, FAKE)
+    base = [2, 8, 2, 64, 128, 64, FAKE, FAKE]
+    assert rc_of(lkv.lkv_tiered_attention, *base, seg, bad, 0.088, 0.0, FAKE, None, FAKE, 1 << 40, 0) \
+        == lkv.LKV_ERR_INVALID_ARG
+    assert rc_of(lkv.lkv_tiered_attention, *base, seg, seg, 0.088, 0.0, FAKE, None, FAKE, 64, 0) \
+        == lkv.LKV_ERR_WORKSPACE
+    assert rc_of(lkv.lkv_tier_repack, 2, 2, 64, 128, 48, FAKE, FAKE, FAKE, FAKE, FAKE, seg, seg, 0) \
+        == lkv.LKV_ERR_UNSUPPORTED
+    assert rc_of(lkv.lkv_tier_classify, 2, 0, 64, FAKE, FAKE, 0.0, 1.0, FAKE, FAKE, FAKE, FAKE, 0) \
+        == lkv.LKV_ERR_INVALID_ARG
+    # the composite call validates all three stages before enqueueing any
+    assert rc_of(lkv.lkv_tiered_decode, 2, 8, 2, 64, 128, 64, FAKE, FAKE, 1e-4, 1e-2, FAKE, FAKE, FAKE,
+                 FAKE, FAKE, FAKE, None, seg, seg, 0.088, 0.0, FAKE, None, FAKE, 1 << 40, 0) \
+        == lkv.LKV_ERR_INVALID_ARG
+
+
+def test_binding_raises_without_library(monkeypatch, tmp_path):
+    """No fallback: with the shared library absent every call raises."""
+    monkeypatch.setattr(lkv, "_lib", None)
+    monkeypatch.setattr(lkv, "LIB_PATH", str(tmp_path / "missing.so"))
+    with pytest.raises(RuntimeError):
+        lkv.lkv_version()

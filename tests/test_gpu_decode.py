@@ -1,0 +1,141 @@
+"""lkv_decode_attention on the GPU vs the CPU oracle: attention outputs within
+rel-L2 1e-5 and max-abs 5e-5 * max|V|, skip masks equal outside the 1e-7 tie
+band around tau, skip counts consistent ("Super KV Compression" §第三层)."""
+import numpy as np
+import pytest
+import torch
+
+from gpu_helpers import (assert_attention_close, assert_masks_match, dev, gpu_decode, gpu_quantize,
+                         oracle_inputs, vmax)
+from quantized_kv_cache_lkv_b200 import buffers, lkv
+from quantized_kv_cache_lkv_b200 import workloads as W
+
+pytestmark = pytest.mark.gpu
+
+
+def run_case(orc, cfg, kb, vb, tau, seq_lens=None, batches=None, inp=None):
+    """Quantize + decode the whole batch on the GPU; check the batches listed
+    (all by default) against the oracle, which quantizes from bf16 itself."""
+    if inp is None:
+        inp = W.make_inputs(cfg, seq_lens=seq_lens)
+    cache = gpu_quantize(kb, vb, cfg.G, inp)
+    out, mask, counts = gpu_decode(kb, vb, cfg.G, inp, cache, cfg.softmax_scale, tau)
+    bsel = list(range(cfg.B)) if batches is None else list(batches)
+    sub = {key: inp[key][bsel].contiguous() for key in ("q", "k", "v", "seq_lens")}
+    k, v, q, sl = oracle_inputs(sub)
+    ocache = orc.quantize_kv(kb, vb, cfg.G, k, v, sl)
+    o_out, o_mask, o_counts, p = orc.decode_attention(kb, vb, cfg.G, sl, q, ocache, cfg.softmax_scale, tau,
+                                                      want_p=True)
+    what = f"{cfg.name} K{kb}V{vb} tau={tau}"
+    assert_attention_close(out[bsel], o_out, vmax(sub), what)
+    n_band = assert_masks_match(mask[bsel], o_mask, p, np.float32(tau), sl, what)
+    valid = np.arange(mask.shape[2])[None, None, :] < inp["seq_lens"].numpy()[:, None, None]
+    assert counts[0] == int((mask * valid).sum())        # counts agree with the mask written
+    if batches is None:
+        assert abs(int(counts[0]) - int(o_counts[0])) <= n_band
+        if n_band == 0:
+            assert counts.tolist() == o_counts.tolist()
+    return out, mask, counts
+
+
+def test_decode_config1_tiny(orc):
+    run_case(orc, W.CONFIGS[1], 6, 4, 0.0)
+
+
+@pytest.mark.parametrize("r", [1, 2, 4, 8])
+@pytest.mark.parametrize("D", [64, 128])
+def test_decode_gqa_ratios_ragged(orc, r, D):
+    """Several chunks plus a ragged tail, lengths 0 and 1, every GQA ratio."""
+    G = 32 if D == 64 else 64
+    cfg = W.Config("ragged", B=4, Hq=2 * r, Hkv=2, D=D, T_cap=600, G=G, bits=[(6, 4)], hh_frac=0.01,
+                   seed=10 * r + D)
+    sl = torch.tensor([600, 1, 0, 333], dtype=torch.int32)
+    for tau in (0.0, 1e-3):
+        out, _, _ = run_case(orc, cfg, 6, 4, tau, seq_lens=sl)
+        assert np.all(out[2] == 0.0)
+
+
+@pytest.mark.parametrize("kb,vb", [(8, 8), (6, 4), (4, 4), (4, 2), (2, 2), (2, 8), (8, 6)])
+def test_decode_bit_widths(orc, kb, vb):
+    cfg = W.scaled(W.CONFIGS[4], B=3, T_cap=520, seq_lo=100, seq_hi=520, seed=40 + kb + vb)
+    run_case(orc, cfg, kb, vb, 0.0)
+    run_case(orc, cfg, kb, vb, 2e-3)
+
+
+@pytest.mark.parametrize("tau", [1e-4, 1e-2, 0.5])
+def test_decode_skip_thresholds(orc, tau):
+    cfg = W.scaled(W.CONFIGS[2], B=2, T_cap=1024, seed=77)
+    run_case(orc, cfg, 6, 4, tau)
+
+
+def test_decode_tau_above_every_probability_gives_zero(orc):
+    cfg = W.scaled(W.CONFIGS[2], B=2, T_cap=300, seed=5)
+    out, mask, counts = run_case(orc, cfg, 6, 4, 1.5)
+    assert np.all(out == 0.0) and counts.tolist() == [2 * 32 * 300, 2 * 8 * 300]
+
+
+def test_decode_capacity_invariance(orc):
+    """The same tokens in a larger cache (more chunks launched, most of them
+    empty) give the same skip set and outputs within tolerance."""
+    cfg = W.scaled(W.CONFIGS[2], B=2, T_cap=700, seed=12)
+    inp = W.make_inputs(cfg)
+    big = dict(inp)
+    for key in ("k", "v"):
+        t = torch.zeros(2, 8, 1300, 128, dtype=torch.bfloat16)
+        t[:, :, :700] = inp[key]
+        big[key] = t
+    o1, m1, c1 = run_case(orc, cfg, 6, 4, 1e-4, inp=inp)
+    cfg2 = W.scaled(cfg, T_cap=1300)
+    o2, m2, c2 = run_case(orc, cfg2, 6, 4, 1e-4, inp=big)
+    np.testing.assert_array_equal(m1, m2[:, :, :700])
+    assert c1.tolist() == c2.tolist()
+    assert_attention_close(o2, o1, vmax(inp), "invariance")
+
+
+def test_decode_workspace_reuse_is_deterministic(orc):
+    cfg = W.scaled(W.CONFIGS[2], B=2, T_cap=900, seed=8)
+    inp = W.make_inputs(cfg)
+    cache = gpu_quantize(6, 4, cfg.G, inp)
+    ws = buffers.alloc_workspace(lkv.lkv_decode_workspace_bytes((6, 4, 64), 2, 32, 8, 900, 128))
+    a = gpu_decode(6, 4, 64, inp, cache, cfg.softmax_scale, 1e-4, ws=ws)
+    b = gpu_decode(6, 4, 64, inp, cache, cfg.softmax_scale, 1e-4, ws=ws)
+    for x, y in zip(a, b):
+        np.testing.assert_array_equal(x, y)
+
+
+def test_decode_bad_length_sets_device_status(orc):
+    cfg = W.Config("bad", B=2, Hq=4, Hkv=2, D=64, T_cap=64, G=32, bits=[(6, 4)], seed=1)
+    inp = W.make_inputs(cfg)
+    cache = gpu_quantize(6, 4, 32, inp)
+    inp["seq_lens"] = torch.tensor([64, 65], dtype=torch.int32)
+    nb = lkv.lkv_decode_workspace_bytes((6, 4, 32), 2, 4, 2, 64, 64)
+    ws = buffers.alloc_workspace(nb)
+    out = torch.empty(2, 4, 64, device="cuda")
+    lkv.lkv_decode_attention((6, 4, 32), 2, 4, 2, 64, 64, dev(inp["seq_lens"]), dev(inp["q"]),
+                             cache["k_codes"], cache["k_sz"], cache["v_codes"], cache["v_sz"],
+                             cfg.softmax_scale, 0.0, out, None, None, ws, ws.numel())
+    assert lkv.lkv_workspace_status(ws) == lkv.LKV_ERR_INVALID_ARG
+    assert torch.isfinite(out).all()          # clamped to T_cap, no fault
+    lkv.lkv_workspace_reset(ws, ws.numel())
+    assert lkv.lkv_workspace_status(ws) == lkv.LKV_OK
+
+
+@pytest.mark.slow
+def test_decode_llama8b_full_size_sampled(orc):
+    """The Llama-3.1-8B-shaped workload at full size (B16, 32q/8kv, D128,
+    T8192, 1% heavy hitters, tau 1e-4) in the bench's launch; the oracle
+    checks sequences 0 and 11 in full."""
+    out, mask, counts = run_case(orc, W.CONFIGS[2], 6, 4, 1e-4, batches=[0, 11])
+    assert 0 < counts[1] < 16 * 8 * 8192
+
+
+@pytest.mark.slow
+def test_decode_long_context_full_size(orc):
+    run_case(orc, W.CONFIGS[3], 6, 4, 1e-5)
+
+
+@pytest.mark.slow
+@pytest.mark.parametrize("kb,vb", [(8, 8), (6, 4), (4, 4), (4, 2)])
+def test_decode_sweep_full_size_sampled(orc, kb, vb):
+    cfg = W.CONFIGS[4]
+    run_case(orc, cfg, kb, vb, 0.0, batches=[0, 33, 63])

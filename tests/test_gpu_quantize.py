@@ -1,0 +1,92 @@
+"""lkv_quantize_kv on the GPU vs the CPU oracle: packed codes and (scale,
+zero) must be bit-exact ("Super KV Compression" §第一层, "TurboQuant"
+§TurboQuant的核心创新)."""
+import numpy as np
+import pytest
+import torch
+
+from gpu_helpers import gpu_quantize, oracle_inputs
+from quantized_kv_cache_lkv_b200 import workloads as W
+
+pytestmark = pytest.mark.gpu
+
+
+def compare_cache(gpu, want, seq_lens, what):
+    sl = np.asarray(seq_lens)
+    for key in ("k_codes", "k_sz", "v_codes", "v_sz"):
+        g = gpu[key].cpu().numpy()
+        w = want[key]
+        for b in range(g.shape[0]):
+            T = int(sl[b])
+            gb, wb = g[b, :, :T], w[b, :, :T]
+            if key.endswith("sz"):
+                gb, wb = gb.view(np.uint32), wb.view(np.uint32)
+            if not np.array_equal(gb, wb):
+                n = int((gb != wb).sum())
+                raise AssertionError(f"{what} {key} b={b}: {n} entries differ")
+
+
+def special_rows(inp):
+    """Overwrite a few rows with degenerate groups: constants, zeros of both
+    signs, a single outlier, huge and tiny magnitudes."""
+    k, v = inp["k"], inp["v"]
+    D = k.shape[-1]
+    k[0, 0, 0] = 0.0
+    v[0, 0, 0] = -0.0
+    k[0, 0, 1] = 3.5
+    v[0, 0, 1, : D // 2] = -0.0
+    v[0, 0, 1, D // 2:] = 0.0
+    k[0, 0, 2] = torch.linspace(-1e30, 1e30, D).to(torch.bfloat16)
+    v[0, 0, 2] = torch.linspace(-1e-30, 1e-30, D).to(torch.bfloat16)
+    k[0, 0, 3] = 1.0
+    k[0, 0, 3, 5] = 1000.0
+    v[0, 0, 3] = torch.arange(D, dtype=torch.float32).remainder(16).to(torch.bfloat16)
+    return inp
+
+
+@pytest.mark.parametrize("D,G", [(64, 32), (64, 64), (128, 32), (128, 64), (128, 128)])
+@pytest.mark.parametrize("kb,vb", [(6, 4), (8, 8), (4, 4), (4, 2), (2, 8), (8, 6), (2, 2), (6, 6)])
+def test_quantize_bit_exact_small(orc, D, G, kb, vb):
+    cfg = W.Config("q", B=3, Hq=4, Hkv=2, D=D, T_cap=80, G=G, bits=[(kb, vb)], seed=D + G + kb * 7 + vb)
+    inp = special_rows(W.make_inputs(cfg, seq_lens=torch.tensor([80, 37, 0], dtype=torch.int32)))
+    gpu = gpu_quantize(kb, vb, G, inp)
+    k, v, _, sl = oracle_inputs(inp)
+    want = orc.quantize_kv(kb, vb, G, k, v, sl)
+    compare_cache(gpu, want, sl, f"K{kb}V{vb} D{D} G{G}")
+    # rows beyond the sequence length stay untouched (zero-filled here)
+    assert int(gpu["k_codes"][1, :, 37:].abs().sum()) == 0 and int(gpu["v_sz"][2].abs().sum()) == 0
+
+
+def test_quantize_config1_tiny(orc):
+    cfg = W.CONFIGS[1]
+    inp = W.make_inputs(cfg)
+    gpu = gpu_quantize(6, 4, cfg.G, inp)
+    k, v, _, sl = oracle_inputs(inp)
+    compare_cache(gpu, orc.quantize_kv(6, 4, cfg.G, k, v, sl), sl, "config 1")
+
+
+def test_quantize_long_context_full_size_sampled(orc):
+    """The 131072-token K/V of the long-context workload quantized in one
+    launch; the oracle checks the first, a middle and the last 2048 rows of
+    every KV head."""
+    cfg = W.CONFIGS[3]
+    inp = W.make_inputs(cfg)
+    gpu = gpu_quantize(6, 4, cfg.G, inp)
+    T = cfg.T_cap
+    for t0 in (0, T // 2 - 1000, T - 2048):
+        sub = {"k": inp["k"][:, :, t0:t0 + 2048].contiguous(), "v": inp["v"][:, :, t0:t0 + 2048].contiguous()}
+        sl = np.array([2048], np.int32)
+        want = orc.quantize_kv(6, 4, cfg.G, W.bf16_bits(sub["k"]), W.bf16_bits(sub["v"]), sl)
+        got = {k: v[:, :, t0:t0 + 2048] for k, v in gpu.items()}
+        compare_cache(got, want, sl, f"config 3 rows {t0}..")
+
+
+def test_quantize_out_of_range_lengths_are_clamped(orc):
+    cfg = W.Config("q", B=2, Hq=4, Hkv=2, D=64, T_cap=32, G=32, bits=[(6, 4)], seed=3)
+    inp = W.make_inputs(cfg)
+    inp["seq_lens"] = torch.tensor([999, -5], dtype=torch.int32)
+    gpu = gpu_quantize(6, 4, 32, inp)
+    k, v, _, _ = oracle_inputs(inp)
+    want = orc.quantize_kv(6, 4, 32, k, v, np.array([32, 0], np.int32))
+    compare_cache(gpu, want, [32, 0], "clamped")
+    assert int(gpu["k_codes"][1].abs().sum()) == 0
