@@ -5,10 +5,10 @@ Llama-3.1-8B-shaped workload (B16, 32 query / 8 KV heads, head_dim 128,
 context 8192, group 64, K6V4, 1% heavy hitters):
 
   quantize   lkv_quantize_kv     bf16 K, V -> K6 / V4 codes + (scale, zero)
-  decode     lkv_decode_attention  sparse-V skip at tau = 1e-4 (3 launches)
+  decode     lkv_decode_attention  sparse-V skip at tau = 1e-4 (one launch)
   classify   lkv_tier_classify   Zipf(1.1) previous-step mass, tau_low 1e-4, tau_high 1e-2
   repack     lkv_tier_repack     kept tokens -> K6/V6 and K6/V4 segments
-  tiered     lkv_tiered_attention  decode over the kept tokens (3 launches)
+  tiered     lkv_tiered_attention  decode over the kept tokens (one launch)
 
 value = algorithmic HBM bytes of the step / step time (GB/s), timed with CUDA
 events on the launching stream with L2 flushed before every step; each
@@ -217,7 +217,7 @@ class Step:
                                0.0, self.out2, self.cnt2, self.ws2, self.ws2.numel(), s)
         mark(5)
 
-    LAUNCHES_PER_STEP = 1 + 3 + 1 + 1 + 3
+    LAUNCHES_PER_STEP = 5    # quantize, decode, classify, repack, tiered: one kernel each
 
     def algorithmic_bytes(self):
         """Bytes each kernel must move, from the step's device results."""

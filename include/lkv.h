@@ -123,11 +123,19 @@ LKV_API int lkv_quantize_kv(lkv_qspec spec, int B, int Hkv, int T_cap, int D,
                     void *stream);
 
 /*
- * Workspace bytes that lkv_decode_attention needs for these sizes.  The
- * workspace is caller-owned device memory (256-byte aligned).  It must be
- * zero-filled before its first use (lkv_workspace_reset); every call leaves
- * it ready for the next one.  Its first word is a device status word that
- * calls set on a device-side error and that stays set until a reset.
+ * Workspace bytes that lkv_decode_attention needs for these sizes on the
+ * current device (the size depends on its SM count).  The workspace is
+ * caller-owned device memory (256-byte aligned).  It must be zero-filled
+ * before its first use (lkv_workspace_reset); every successful call leaves
+ * it ready for the next one.  Calls that overlap on the GPU must not share a
+ * workspace.  Layout of its first 256 bytes:
+ *   bytes [0, 4)   device status word (an lkv_status); a call sets it on a
+ *                  device-side error and it stays set until a reset;
+ *   bytes [8, 16)  optional limit, in nanoseconds, of every bounded wait of
+ *                  the single-launch decode (0 = 2 s).  A wait that runs out
+ *                  sets LKV_ERR_TIMEOUT, abandons the rest of the call and
+ *                  leaves finite but meaningless outputs; reset the
+ *                  workspace before reusing it.
  */
 LKV_API size_t lkv_decode_workspace_bytes(lkv_qspec spec, int B, int Hq, int Hkv, int T_cap, int D);
 

@@ -6,6 +6,9 @@
 #include <cstring>
 
 #include "../../include/lkv.h"
+#include <algorithm>
+
+#include "fused_impl.cuh"
 #include "lkv_kernels.cuh"
 
 namespace lkv {
@@ -22,10 +25,25 @@ int num_sms() {
   return cached[dev];
 }
 
+// Opt-in dynamic shared memory per block of the current device.
+static int max_smem_optin() {
+  static int cached[64] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 232448;
+  if (cached[dev] == 0) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) != cudaSuccess || n <= 0)
+      n = 232448;
+    cached[dev] = n;
+  }
+  return cached[dev];
+}
+
 namespace {
 
 constexpr int kChunk = 256;       // decode rows per chunk
 constexpr size_t kAlign = 256;
+constexpr size_t kHeaderBytes = 256;  // status, wait limit, done counter, skip-count accumulators
 
 size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
 
@@ -49,11 +67,106 @@ WsLayout ws_layout(int B, int Hq, int Hkv, int T_cap, int D) {
   w.n_chunks = T_cap > 0 ? (T_cap + kChunk - 1) / kChunk : 1;
   const size_t units = (size_t)B * (size_t)Hkv;
   w.status = 0;
-  w.logits = align_up(4);
+  w.logits = kHeaderBytes;
   w.stats = w.logits + align_up(units * (size_t)T_cap * r * sizeof(float));
   w.partial = w.stats + align_up(units * (size_t)w.n_chunks * r * 2 * sizeof(float));
   w.total = w.partial + align_up(units * (size_t)w.n_chunks * r * D * sizeof(float));
   return w;
+}
+
+// The single-launch decode handles GQA groups of 1, 2 or 4 query heads.
+bool fused_ok(int r) { return r == 1 || r == 2 || r == 4; }
+
+struct FusedLayout {
+  int grid, H, cpc_max, ring_bytes;
+  long long chunks_max, smem_logit_floats;
+  size_t smem_bytes;
+  size_t arrive1, arrive2, pstats, ppart, cstats, ulist, glogits, total;
+  bool need_glogits;
+};
+
+FusedLayout fused_layout(int B, int Hq, int Hkv, int T_cap, int D, int KB) {
+  FusedLayout L{};
+  L.grid = num_sms();
+  L.H = Hq / Hkv;
+  const long long units = (long long)B * Hkv;
+  const long long per_unit = T_cap > 0 ? (T_cap + kChunk - 1) / kChunk : 1;
+  L.chunks_max = units * per_unit > 0 ? units * per_unit : 1;
+  L.cpc_max = (int)((L.chunks_max + L.grid - 1) / L.grid);
+  const int rb = D * KB / 8;
+  const int stage = ((fused::kTile * rb + (fused::kTile + 2) * (D / 32) * 8) + 127) / 128 * 128;
+  const int phase2 = fused::kConsumerWarps * fused::kListCap * 4 + fused::kConsumerWarps * L.H * D * 4;
+  L.ring_bytes = std::max(fused::kStages * stage, phase2);
+  const long long need = (long long)L.cpc_max * kChunk * L.H * 4;
+  const long long avail = (long long)max_smem_optin() - fused::kHeader - L.ring_bytes;
+  if (need <= avail) {
+    L.smem_logit_floats = need / 4;
+    L.need_glogits = false;
+  } else {
+    L.smem_logit_floats = std::max(0ll, avail / 16 * 4);
+    L.need_glogits = true;
+  }
+  L.smem_bytes = fused::kHeader + L.ring_bytes + (size_t)L.smem_logit_floats * 4;
+  size_t off = kHeaderBytes;
+  L.arrive1 = off; off = align_up(off + units * 4);
+  L.arrive2 = off; off = align_up(off + units * 4);
+  L.pstats = off; off = align_up(off + (size_t)L.grid * 2 * L.H * 2 * 4);
+  L.ppart = off; off = align_up(off + (size_t)L.grid * 2 * L.H * D * 4);
+  L.cstats = off; off = align_up(off + (size_t)L.chunks_max * L.H * 2 * 4);
+  L.ulist = off; off = align_up(off + (size_t)L.grid * L.cpc_max * fused::kRec * 4);
+  L.glogits = off;
+  if (L.need_glogits) off = align_up(off + (size_t)L.grid * L.cpc_max * kChunk * L.H * 4);
+  L.total = off;
+  return L;
+}
+
+size_t attention_ws_bytes(int B, int Hq, int Hkv, int T_cap, int D, int KB) {
+  if (fused_ok(Hq / Hkv)) return fused_layout(B, Hq, Hkv, T_cap, D, KB).total;
+  return ws_layout(B, Hq, Hkv, T_cap, D).total;
+}
+
+// Launch the decode of `a` on the single-launch kernel when the group fits,
+// else on the three-launch path.
+int run_attention(DecodeArgs& a, int D, int kb, int vb0, int vb1, void* ws, size_t ws_bytes, cudaStream_t s) {
+  if (ws == nullptr || (reinterpret_cast<uintptr_t>(ws) % kAlign) != 0) return LKV_ERR_INVALID_ARG;
+  char* base = static_cast<char*>(ws);
+  a.status = reinterpret_cast<int*>(base);
+  if (!fused_ok(a.r)) {
+    const WsLayout w = ws_layout(a.B, a.Hq, a.Hkv, a.T_cap, D);
+    if (ws_bytes < w.total) return LKV_ERR_WORKSPACE;
+    a.logits = reinterpret_cast<float*>(base + w.logits);
+    a.stats = reinterpret_cast<float*>(base + w.stats);
+    a.partial = reinterpret_cast<float*>(base + w.partial);
+    a.chunk = kChunk;
+    a.n_chunks = w.n_chunks;
+    return from_cuda(launch_decode(a, D, kb, vb0, vb1, s));
+  }
+  const FusedLayout L = fused_layout(a.B, a.Hq, a.Hkv, a.T_cap, D, kb);
+  if (ws_bytes < L.total) return LKV_ERR_WORKSPACE;
+  FusedArgs f{};
+  f.d = a;
+  f.cpc_max = L.cpc_max;
+  f.ring_bytes = L.ring_bytes;
+  f.smem_logit_floats = L.smem_logit_floats;
+  f.timeout_ns = reinterpret_cast<const unsigned long long*>(base + 8);
+  f.done = reinterpret_cast<int*>(base + 16);
+  f.wcounts = reinterpret_cast<unsigned long long*>(base + 32);
+  f.arrive1 = reinterpret_cast<int*>(base + L.arrive1);
+  f.arrive2 = reinterpret_cast<int*>(base + L.arrive2);
+  f.pstats = reinterpret_cast<float*>(base + L.pstats);
+  f.ppart = reinterpret_cast<float*>(base + L.ppart);
+  f.cstats = reinterpret_cast<float*>(base + L.cstats);
+  f.ulist = reinterpret_cast<int*>(base + L.ulist);
+  f.glogits = L.need_glogits ? reinterpret_cast<float*>(base + L.glogits) : nullptr;
+  cudaError_t e;
+  switch (kb) {
+    case 2: e = launch_fused_k2(f, D, L.H, vb0, vb1, L.smem_bytes, L.grid, s); break;
+    case 4: e = launch_fused_k4(f, D, L.H, vb0, vb1, L.smem_bytes, L.grid, s); break;
+    case 6: e = launch_fused_k6(f, D, L.H, vb0, vb1, L.smem_bytes, L.grid, s); break;
+    case 8: e = launch_fused_k8(f, D, L.H, vb0, vb1, L.smem_bytes, L.grid, s); break;
+    default: return LKV_ERR_UNSUPPORTED;
+  }
+  return from_cuda(e);
 }
 
 // Shapes shared by every attention call.
@@ -77,20 +190,6 @@ int check_cache_shape(int B, int Hkv, int T_cap, int D, int G) {
 bool segment_ok(const lkv_segment& s, bool nonempty) {
   return ptr_ok(s.k_codes, nonempty) && ptr_ok(s.k_sz, nonempty) && ptr_ok(s.v_codes, nonempty) &&
          ptr_ok(s.v_sz, nonempty);
-}
-
-int fill_workspace(DecodeArgs& a, int B, int Hq, int Hkv, int T_cap, int D, void* ws, size_t ws_bytes) {
-  const WsLayout w = ws_layout(B, Hq, Hkv, T_cap, D);
-  if (ws == nullptr || (reinterpret_cast<uintptr_t>(ws) % kAlign) != 0) return LKV_ERR_INVALID_ARG;
-  if (ws_bytes < w.total) return LKV_ERR_WORKSPACE;
-  char* base = static_cast<char*>(ws);
-  a.status = reinterpret_cast<int*>(base + w.status);
-  a.logits = reinterpret_cast<float*>(base + w.logits);
-  a.stats = reinterpret_cast<float*>(base + w.stats);
-  a.partial = reinterpret_cast<float*>(base + w.partial);
-  a.chunk = kChunk;
-  a.n_chunks = w.n_chunks;
-  return LKV_OK;
 }
 
 }  // namespace
@@ -149,7 +248,7 @@ int lkv_quantize_kv(lkv_qspec spec, int B, int Hkv, int T_cap, int D, const int3
 size_t lkv_decode_workspace_bytes(lkv_qspec spec, int B, int Hq, int Hkv, int T_cap, int D) {
   if (!bits_ok(spec.k_bits) || !bits_ok(spec.v_bits)) return 0;
   if (check_attention_shape(B, Hq, Hkv, T_cap, D, spec.group)) return 0;
-  return ws_layout(B, Hq, Hkv, T_cap, D).total;
+  return attention_ws_bytes(B, Hq, Hkv, T_cap, D, spec.k_bits);
 }
 
 int lkv_decode_attention(lkv_qspec spec, int B, int Hq, int Hkv, int T_cap, int D, const int32_t* seq_lens,
@@ -165,9 +264,9 @@ int lkv_decode_attention(lkv_qspec spec, int B, int Hq, int Hkv, int T_cap, int 
       !ptr_ok(k_sz, ne) || !ptr_ok(v_codes, ne) || !ptr_ok(v_sz, ne))
     return LKV_ERR_INVALID_ARG;
   if (skip_counts && !aligned16(skip_counts)) return LKV_ERR_INVALID_ARG;
+  if (workspace == nullptr || (reinterpret_cast<uintptr_t>(workspace) % kAlign) != 0) return LKV_ERR_INVALID_ARG;
+  if (ws_bytes < attention_ws_bytes(B, Hq, Hkv, T_cap, D, spec.k_bits)) return LKV_ERR_WORKSPACE;
   DecodeArgs a{};
-  rc = fill_workspace(a, B, Hq, Hkv, T_cap, D, workspace, ws_bytes);
-  if (rc) return rc;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   if (B == 0) {
     if (skip_counts) return from_cuda(cudaMemsetAsync(skip_counts, 0, 2 * sizeof(int64_t), s));
@@ -185,7 +284,7 @@ int lkv_decode_attention(lkv_qspec spec, int B, int Hq, int Hkv, int T_cap, int 
   a.out = out;
   a.skip_mask = skip_mask;
   a.skip_counts = reinterpret_cast<unsigned long long*>(skip_counts);
-  return from_cuda(launch_decode(a, D, spec.k_bits, spec.v_bits, spec.v_bits, s));
+  return run_attention(a, D, spec.k_bits, spec.v_bits, spec.v_bits, workspace, ws_bytes, s);
 }
 
 int lkv_workspace_reset(void* workspace, size_t ws_bytes, void* stream) {
@@ -243,7 +342,7 @@ int lkv_tier_repack(int B, int Hkv, int T_cap, int D, int group, const void* k, 
 
 size_t lkv_tiered_workspace_bytes(int B, int Hq, int Hkv, int T_cap, int D, int group) {
   if (check_attention_shape(B, Hq, Hkv, T_cap, D, group)) return 0;
-  return ws_layout(B, Hq, Hkv, T_cap, D).total;
+  return attention_ws_bytes(B, Hq, Hkv, T_cap, D, 6);
 }
 
 int lkv_tiered_attention(int B, int Hq, int Hkv, int T_cap, int D, int group, const int32_t* counts, const void* q,
@@ -257,9 +356,9 @@ int lkv_tiered_attention(int B, int Hq, int Hkv, int T_cap, int D, int group, co
       !segment_ok(seg_b, ne))
     return LKV_ERR_INVALID_ARG;
   if (skip_counts && !aligned16(skip_counts)) return LKV_ERR_INVALID_ARG;
+  if (workspace == nullptr || (reinterpret_cast<uintptr_t>(workspace) % kAlign) != 0) return LKV_ERR_INVALID_ARG;
+  if (ws_bytes < attention_ws_bytes(B, Hq, Hkv, T_cap, D, 6)) return LKV_ERR_WORKSPACE;
   DecodeArgs a{};
-  rc = fill_workspace(a, B, Hq, Hkv, T_cap, D, workspace, ws_bytes);
-  if (rc) return rc;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   if (B == 0) {
     if (skip_counts) return from_cuda(cudaMemsetAsync(skip_counts, 0, 2 * sizeof(int64_t), s));
@@ -277,7 +376,7 @@ int lkv_tiered_attention(int B, int Hq, int Hkv, int T_cap, int D, int group, co
   a.out = out;
   a.skip_mask = nullptr;
   a.skip_counts = reinterpret_cast<unsigned long long*>(skip_counts);
-  return from_cuda(launch_decode(a, D, 6, 6, 4, s));
+  return run_attention(a, D, 6, 6, 4, workspace, ws_bytes, s);
 }
 
 int lkv_tiered_decode(int B, int Hq, int Hkv, int T_cap, int D, int group, const int32_t* seq_lens, const float* mass,

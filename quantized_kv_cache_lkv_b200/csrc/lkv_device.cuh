@@ -149,3 +149,161 @@ __device__ __forceinline__ unsigned row_lane_mask(int lane) {
 }
 
 }  // namespace lkv
+
+namespace lkv {
+
+// ------------------------------------------------------------------ exact integer unpack
+//
+// A code c sitting at bits [kk, kk+BITS) of a 32-bit word x with kk + BITS <= 23
+// becomes the float 2^(23-kk) + c with one AND-OR: the mantissa holds c * 2^kk
+// and the exponent field is 150 - kk.  Subtracting 2^(23-kk) (two codes per
+// packed fp32 add) leaves c exactly.  Codes further up the word are first
+// brought down with one (funnel) shift shared by the codes that follow it.
+
+// Stream offset of the shifted copy that code i is read from (greedy plan).
+template <int BITS>
+constexpr int copy_shift(int i) {
+  int s = 0;
+  for (int j = 0; j <= i; ++j) {
+    const int p = j * BITS;
+    if (!(p >= s && p - s + BITS <= 23)) s = p;
+  }
+  return s;
+}
+
+template <int BITS>
+__device__ __forceinline__ uint32_t stream_bits(const LaneWords<BITS>& lw, int s) {
+  const int wi = s >> 5, k = s & 31;
+  if (k == 0) return lw.w[wi];
+  const uint32_t hi = (wi + 1 < LaneWords<BITS>::N) ? lw.w[wi + 1] : 0u;
+  return __funnelshift_r(lw.w[wi], hi, k);
+}
+
+template <int BITS, int I>
+__device__ __forceinline__ float code_plus_magic(const LaneWords<BITS>& lw) {
+  constexpr int s = copy_shift<BITS>(I);
+  constexpr int kk = I * BITS - s;
+  constexpr uint32_t mask = ((1u << BITS) - 1u) << kk;
+  constexpr uint32_t magic = (uint32_t)(150 - kk) << 23;
+  return __uint_as_float((stream_bits<BITS>(lw, s) & mask) | magic);
+}
+
+template <int BITS, int I>
+__device__ __forceinline__ float magic_value() {
+  constexpr int kk = I * BITS - copy_shift<BITS>(I);
+  return __uint_as_float((uint32_t)(150 - kk) << 23);
+}
+
+template <int BITS, int P>
+__device__ __forceinline__ float2 code_pair(const LaneWords<BITS>& lw) {
+  const float2 m = make_float2(code_plus_magic<BITS, 2 * P>(lw), code_plus_magic<BITS, 2 * P + 1>(lw));
+  return __fadd2_rn(m, make_float2(-magic_value<BITS, 2 * P>(), -magic_value<BITS, 2 * P + 1>()));
+}
+
+// The lane's 16 codes as exact floats, in channel pairs.
+template <int BITS>
+__device__ __forceinline__ void unpack16_int(const LaneWords<BITS>& lw, float2 (&c)[8]) {
+  c[0] = code_pair<BITS, 0>(lw);
+  c[1] = code_pair<BITS, 1>(lw);
+  c[2] = code_pair<BITS, 2>(lw);
+  c[3] = code_pair<BITS, 3>(lw);
+  c[4] = code_pair<BITS, 4>(lw);
+  c[5] = code_pair<BITS, 5>(lw);
+  c[6] = code_pair<BITS, 6>(lw);
+  c[7] = code_pair<BITS, 7>(lw);
+}
+
+// Lane words from shared memory (4-byte aligned; wider when the width allows).
+template <int BITS>
+__device__ __forceinline__ void lds_lane_words(const uint8_t* p, LaneWords<BITS>& lw) {
+  if constexpr (BITS == 8) {
+    const uint4 v = *reinterpret_cast<const uint4*>(p);
+    lw.w[0] = v.x; lw.w[1] = v.y; lw.w[2] = v.z; lw.w[3] = v.w;
+  } else if constexpr (BITS == 4) {
+    const uint2 v = *reinterpret_cast<const uint2*>(p);
+    lw.w[0] = v.x; lw.w[1] = v.y;
+  } else {
+#pragma unroll
+    for (int i = 0; i < LaneWords<BITS>::N; ++i) lw.w[i] = reinterpret_cast<const uint32_t*>(p)[i];
+  }
+}
+
+// ------------------------------------------------------------------ mbarrier / bulk copy
+
+__device__ __forceinline__ uint32_t smem_addr(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_addr(bar)), "r"(count) : "memory");
+}
+
+__device__ __forceinline__ void fence_mbar_init() {
+  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_addr(bar)), "r"(bytes)
+               : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_addr(bar)) : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_addr(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+__device__ __forceinline__ uint64_t global_ns() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+
+// Wait for a phase of an mbarrier, giving up after `limit_ns`.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, uint64_t limit_ns) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = global_ns();
+  while (true) {
+    for (int i = 0; i < 64; ++i)
+      if (mbar_try_wait(bar, parity)) return true;
+    if (global_ns() - t0 > limit_ns) return false;
+  }
+}
+
+// 1-D bulk copy global -> shared, completing `bytes` on the mbarrier.  Both
+// addresses and the size are multiples of 16 bytes.
+__device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t bytes, uint64_t* bar,
+                                         uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint [%0], [%1], %2, [%3], %4;"
+      ::"r"(smem_addr(dst)), "l"(src), "r"(bytes), "r"(smem_addr(bar)), "l"(policy)
+      : "memory");
+}
+
+__device__ __forceinline__ uint64_t policy_evict_first() {
+  uint64_t p;
+  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
+  return p;
+}
+
+__device__ __forceinline__ void named_barrier(int id, int threads) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
+}
+
+__device__ __forceinline__ int ld_acquire(const int* p) {
+  int v;
+  asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+
+}  // namespace lkv

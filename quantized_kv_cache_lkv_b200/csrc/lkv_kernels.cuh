@@ -65,6 +65,30 @@ struct DecodeArgs {
   float* partial;        // [B][Hkv][n_chunks][r][D]
 };
 
+// Single-launch decode (fused_impl.cuh): DecodeArgs plus its workspace.
+struct FusedArgs {
+  DecodeArgs d;
+  int cpc_max;                   // upper bound of chunks per CTA
+  int ring_bytes;                // shared-memory ring size
+  long long smem_logit_floats;   // logits that fit in shared memory per CTA
+  const unsigned long long* timeout_ns;  // workspace word: wait limit override (0 = default)
+  int* arrive1;                  // [units] piece statistics published
+  int* arrive2;                  // [units] partial outputs published
+  float* pstats;                 // [grid][2][H][2]
+  float* ppart;                  // [grid][2][H][D]
+  float* cstats;                 // [chunks][H][2]
+  int* ulist;                    // [grid][cpc_max][16]
+  float* glogits;                // [grid][cpc_max * chunk][H] (when shared memory is short)
+  unsigned long long* wcounts;   // [2] skip-count accumulators
+  int* done;                     // CTAs finished
+};
+
+// Dispatch on (D, H, V widths) for one K width; smem = dynamic shared bytes.
+cudaError_t launch_fused_k2(const FusedArgs& a, int D, int H, int vb0, int vb1, size_t smem, int grid, cudaStream_t s);
+cudaError_t launch_fused_k4(const FusedArgs& a, int D, int H, int vb0, int vb1, size_t smem, int grid, cudaStream_t s);
+cudaError_t launch_fused_k6(const FusedArgs& a, int D, int H, int vb0, int vb1, size_t smem, int grid, cudaStream_t s);
+cudaError_t launch_fused_k8(const FusedArgs& a, int D, int H, int vb0, int vb1, size_t smem, int grid, cudaStream_t s);
+
 int num_sms();
 
 cudaError_t launch_quantize_kv(const QuantizeArgs& a, int kb, int vb, int D, cudaStream_t s);

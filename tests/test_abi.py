@@ -50,9 +50,13 @@ def test_status_strings_and_sizes(L):
 
 
 def test_workspace_sizes(L):
+    # groups of up to 4 query heads: single-launch decode, logits stay on chip
     n = lkv.lkv_decode_workspace_bytes(K6V4, 16, 32, 8, 8192, 128)
-    logits = 16 * 8 * 8192 * 4 * 4
-    assert logits < n < logits * 2
+    assert 256 + 16 * 8 * 8 <= n < 16 << 20 and n % 256 == 0
+    # larger groups: three-launch decode, logits in the workspace
+    n8 = lkv.lkv_decode_workspace_bytes(K6V4, 16, 64, 8, 8192, 128)
+    logits = 16 * 8 * 8192 * 8 * 4
+    assert logits < n8 < logits * 2
     assert lkv.lkv_decode_workspace_bytes(K6V4, 16, 30, 8, 8192, 128) == 0   # Hq % Hkv
     assert lkv.lkv_decode_workspace_bytes((5, 4, 64), 1, 4, 2, 256, 64) == 0
     assert lkv.lkv_tiered_workspace_bytes(32, 32, 8, 32768, 128, 64) > 0

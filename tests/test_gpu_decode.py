@@ -120,6 +120,33 @@ def test_decode_bad_length_sets_device_status(orc):
     assert lkv.lkv_workspace_status(ws) == lkv.LKV_OK
 
 
+def test_decode_bounded_wait_times_out(orc):
+    """A unit split over several CTAs waits for its neighbours' statistics.
+    Plant a missing arrival on the host (the unit's arrival counter starts
+    far below its target) with a 1 ms limit: the call must end with
+    LKV_ERR_TIMEOUT and finite outputs, and after a reset the same workspace
+    gives correct results."""
+    cfg = W.Config("wait", B=1, Hq=4, Hkv=1, D=128, T_cap=8192, G=64, bits=[(6, 4)], seed=6)
+    inp = W.make_inputs(cfg)
+    cache = gpu_quantize(6, 4, 64, inp)
+    nb = lkv.lkv_decode_workspace_bytes((6, 4, 64), 1, 4, 1, 8192, 128)
+    ws = buffers.alloc_workspace(nb)
+    ws[8:16].view(torch.int64).fill_(1_000_000)          # wait limit: 1 ms
+    ws[256:260].view(torch.int32).fill_(-(1 << 30))      # arrival counter of unit 0 (first after the header)
+    out = torch.empty(1, 4, 128, device="cuda")
+    lkv.lkv_decode_attention((6, 4, 64), 1, 4, 1, 8192, 128, dev(inp["seq_lens"]), dev(inp["q"]),
+                             cache["k_codes"], cache["k_sz"], cache["v_codes"], cache["v_sz"],
+                             cfg.softmax_scale, 1e-4, out, None, None, ws, ws.numel())
+    assert lkv.lkv_workspace_status(ws) == lkv.LKV_ERR_TIMEOUT
+    assert torch.isfinite(out).all()
+    lkv.lkv_workspace_reset(ws, ws.numel())
+    got, _, _ = gpu_decode(6, 4, 64, inp, cache, cfg.softmax_scale, 1e-4, ws=ws)
+    k, v, q, sl = oracle_inputs(inp)
+    want, _, _ = orc.decode_attention(6, 4, 64, sl, q, orc.quantize_kv(6, 4, 64, k, v, sl),
+                                      cfg.softmax_scale, 1e-4)
+    assert_attention_close(got, want, vmax(inp), "after reset")
+
+
 @pytest.mark.slow
 def test_decode_llama8b_full_size_sampled(orc):
     """The Llama-3.1-8B-shaped workload at full size (B16, 32q/8kv, D128,
