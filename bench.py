@@ -317,7 +317,7 @@ def run_lkv(args):
                 "frac": kern[name]["frac"], "traffic": t_bytes, "kernel": name,
                 "peak_source": f"{peak_kind} hbm_gbs"}
 
-    e2e = run_e2e(step, inp, device, stream, args) if not dist or rank == 0 else None
+    e2e = run_e2e(step, inp, device, stream, args) if (not dist or rank == 0) and not args.no_e2e else None
     if dist:
         e2e_t = torch.tensor([e2e["seconds"] if e2e else 0.0], device=device)
         torch.distributed.all_reduce(e2e_t, op=torch.distributed.ReduceOp.MAX)
@@ -465,6 +465,7 @@ def main():
     ap.add_argument("--e2e-steps", type=int, default=3)
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--no-cpu", action="store_true", help="skip the CPU-oracle baseline leg")
+    ap.add_argument("--no-e2e", action="store_true", help="skip the end-to-end (host buffers) leg")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)   # at least 3 untimed warm-up steps
     if args.impl == "reference":

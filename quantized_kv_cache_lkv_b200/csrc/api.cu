@@ -78,11 +78,11 @@ WsLayout ws_layout(int B, int Hq, int Hkv, int T_cap, int D) {
 bool fused_ok(int r) { return r == 1 || r == 2 || r == 4; }
 
 struct FusedLayout {
-  int grid, H, cpc_max, ring_bytes;
+  int grid, H, cpc_max, ring_bytes, stages;
   long long chunks_max, smem_logit_floats;
   size_t smem_bytes;
-  size_t arrive1, arrive2, pstats, ppart, cstats, ulist, glogits, total;
-  bool need_glogits;
+  size_t arrive1, arrive2, pstats, ppart, cstats, ulist, glogits, gstats, total;
+  bool need_glogits, need_gstats;
 };
 
 FusedLayout fused_layout(int B, int Hq, int Hkv, int T_cap, int D, int KB) {
@@ -90,32 +90,44 @@ FusedLayout fused_layout(int B, int Hq, int Hkv, int T_cap, int D, int KB) {
   L.grid = num_sms();
   L.H = Hq / Hkv;
   const long long units = (long long)B * Hkv;
-  const long long per_unit = T_cap > 0 ? (T_cap + kChunk - 1) / kChunk : 1;
+  // each segment rounds up to whole chunks: at most one more chunk per unit
+  const long long per_unit = T_cap > 0 ? (T_cap + kChunk - 1) / kChunk + 1 : 1;
   L.chunks_max = units * per_unit > 0 ? units * per_unit : 1;
   L.cpc_max = (int)((L.chunks_max + L.grid - 1) / L.grid);
   const int rb = D * KB / 8;
   const int stage = ((fused::kTile * rb + (fused::kTile + 2) * (D / 32) * 8) + 127) / 128 * 128;
   const int phase2 = fused::kConsumerWarps * fused::kListCap * 4 + fused::kConsumerWarps * L.H * D * 4;
-  L.ring_bytes = std::max(fused::kStages * stage, phase2);
   const long long need = (long long)L.cpc_max * kChunk * L.H * 4;
-  const long long avail = (long long)max_smem_optin() - fused::kHeader - L.ring_bytes;
-  if (need <= avail) {
+  const long long smax = max_smem_optin();
+  // deepest ring (a multiple of the consumer groups) that leaves room for the logits
+  L.stages = 0;
+  for (int s = fused::kMaxStages; s >= 6; s -= fused::kGroups) {
+    const int ring = std::max(s * stage, phase2);
+    if (fused::kHeader + ring + need <= smax) { L.stages = s; break; }
+  }
+  if (L.stages > 0) {
+    L.ring_bytes = std::max(L.stages * stage, phase2);
     L.smem_logit_floats = need / 4;
     L.need_glogits = false;
   } else {
-    L.smem_logit_floats = std::max(0ll, avail / 16 * 4);
+    L.stages = 12;
+    L.ring_bytes = std::max(L.stages * stage, phase2);
+    L.smem_logit_floats = std::max(0ll, (smax - fused::kHeader - L.ring_bytes) / 16 * 4);
     L.need_glogits = true;
   }
+  L.need_gstats = L.cpc_max > fused::kCsCap;
   L.smem_bytes = fused::kHeader + L.ring_bytes + (size_t)L.smem_logit_floats * 4;
   size_t off = kHeaderBytes;
   L.arrive1 = off; off = align_up(off + units * 4);
   L.arrive2 = off; off = align_up(off + units * 4);
   L.pstats = off; off = align_up(off + (size_t)L.grid * 2 * L.H * 2 * 4);
   L.ppart = off; off = align_up(off + (size_t)L.grid * 2 * L.H * D * 4);
-  L.cstats = off; off = align_up(off + (size_t)L.chunks_max * L.H * 2 * 4);
+  L.cstats = off;
   L.ulist = off; off = align_up(off + (size_t)L.grid * L.cpc_max * fused::kRec * 4);
   L.glogits = off;
   if (L.need_glogits) off = align_up(off + (size_t)L.grid * L.cpc_max * kChunk * L.H * 4);
+  L.gstats = off;
+  if (L.need_gstats) off = align_up(off + (size_t)L.grid * L.cpc_max * 12 * 4);
   L.total = off;
   return L;
 }
@@ -146,6 +158,7 @@ int run_attention(DecodeArgs& a, int D, int kb, int vb0, int vb1, void* ws, size
   FusedArgs f{};
   f.d = a;
   f.cpc_max = L.cpc_max;
+  f.stages = L.stages;
   f.ring_bytes = L.ring_bytes;
   f.smem_logit_floats = L.smem_logit_floats;
   f.timeout_ns = reinterpret_cast<const unsigned long long*>(base + 8);
@@ -155,9 +168,10 @@ int run_attention(DecodeArgs& a, int D, int kb, int vb0, int vb1, void* ws, size
   f.arrive2 = reinterpret_cast<int*>(base + L.arrive2);
   f.pstats = reinterpret_cast<float*>(base + L.pstats);
   f.ppart = reinterpret_cast<float*>(base + L.ppart);
-  f.cstats = reinterpret_cast<float*>(base + L.cstats);
+  f.cstats = nullptr;
   f.ulist = reinterpret_cast<int*>(base + L.ulist);
   f.glogits = L.need_glogits ? reinterpret_cast<float*>(base + L.glogits) : nullptr;
+  f.gstats = L.need_gstats ? reinterpret_cast<float*>(base + L.gstats) : nullptr;
   cudaError_t e;
   switch (kb) {
     case 2: e = launch_fused_k2(f, D, L.H, vb0, vb1, L.smem_bytes, L.grid, s); break;

@@ -4,19 +4,22 @@
 // (§第二层) as two segments per (batch, KV head) with their own V widths.
 //
 // One persistent CTA per SM (cooperative launch, so all CTAs are resident).
-// Work = the list of chunks (kChunk consecutive tokens of one (b, kv head)
-// "unit"); every CTA takes an equal contiguous range of chunks.
+// Work = the list of chunks (kChunk consecutive tokens of one segment of one
+// (b, kv head) "unit"); every CTA takes an equal contiguous range of chunks.
+// A unit's rows are numbered segment 0 first, padded to whole chunks, then
+// segment 1, so a chunk never straddles the two segments.
 //
 //  phase 1  a producer warp streams the K rows of the CTA's chunks through a
 //           ring of shared-memory stages with 1-D bulk copies (TMA, evict-
-//           first in L2) completing on mbarriers; fifteen consumer warps turn
-//           them into base-2 logits for the group's query heads, which stay
-//           in shared memory.
-//  stats    per chunk: max and sum of exp2 (logits are replaced by
-//           e = exp2(s - max_chunk)); per unit piece: the merged statistics.
-//           A unit owned by one CTA needs nothing else; a unit shared by
-//           neighbouring CTAs exchanges piece statistics through the
-//           workspace (bounded wait on a per-unit arrival counter).
+//           first in L2) completing on mbarriers.  Three groups of four
+//           consumer warps take the tiles in turn and turn them into base-2
+//           logits for the group's query heads, kept in shared memory, while
+//           tracking each chunk's maximum.
+//  stats    per chunk: sum of exp2(s - max) (logits become e = exp2(s - max));
+//           per unit piece: the merged statistics.  A unit owned by one CTA
+//           needs nothing else; a unit shared by neighbouring CTAs exchanges
+//           piece statistics through the workspace (bounded wait on a
+//           per-unit arrival counter).
 //  phase 2  p = e * exp2(max_chunk - max) / sum.  A (b, h, t) with p < tau is
 //           skipped; the V rows some head keeps are listed per warp in row
 //           order, gathered from HBM and accumulated as p * vhat.  Shared
@@ -33,29 +36,38 @@
 namespace lkv {
 namespace fused {
 
-constexpr int kConsumerWarps = 15;
+constexpr int kGroupWarps = 4;                 // consumer warps sharing a tile
+constexpr int kGroups = 3;                     // tiles are dealt to groups in turn
+constexpr int kConsumerWarps = kGroupWarps * kGroups;
 constexpr int kConsumers = kConsumerWarps * 32;
-constexpr int kThreads = kConsumers + 32;
+constexpr int kThreads = kConsumers + 32;      // + producer warp
 constexpr int kChunk = 256;    // tokens per chunk (softmax statistics granularity)
-constexpr int kTile = 128;     // tokens per bulk-copy tile
-constexpr int kStages = 6;
+constexpr int kTile = 64;      // tokens per bulk-copy tile
+constexpr int kMaxStages = 15; // multiple of kGroups
 constexpr int kListCap = 512;  // V-row list entries per warp per batch
 constexpr int kBatchBlocks = kListCap / 32;
 constexpr int kRec = 16;       // ints per unit-list record
-constexpr int kGatherUnroll = 4;
+constexpr int kGatherUnroll = 2;
+constexpr int kCsCap = 64;     // chunk statistics kept in shared memory up to this many chunks
 constexpr unsigned kFull = 0xFFFFFFFFu;
 constexpr int kBarCons = 1;    // named barrier of the consumer warps
-constexpr int kHeader = 1024;  // bytes of shared memory before the ring
+constexpr int kHeader = 4096;  // bytes of shared memory before the ring
 
-// Unit-list record (ints): u, first chunk, chunks, n0, n1, owned, -, -,
-// then (max, sum) of the CTA's piece for up to 4 heads as floats.
+// Shared header layout (bytes): barriers [0, 256), tile descriptors
+// [256, 768), misc ints [768, 1024), chunk statistics [1024, 4096).
+constexpr int kDescOff = 256;
+constexpr int kMiscOff = 768;
+constexpr int kCsOff = 1024;
+
+// Unit-list record (ints): u, first chunk, chunks, n0, n1, owned, chunks of
+// segment 0, -, then (max, sum) of the CTA's piece for up to 4 heads as floats.
 struct Unit {
-  int u, cb, nc, n0, n1, owned;
+  int u, cb, nc, n0, n1, owned, nc0;
 };
 
 __device__ __forceinline__ Unit load_unit(const int* rec) {
   Unit x;
-  x.u = rec[0]; x.cb = rec[1]; x.nc = rec[2]; x.n0 = rec[3]; x.n1 = rec[4]; x.owned = rec[5];
+  x.u = rec[0]; x.cb = rec[1]; x.nc = rec[2]; x.n0 = rec[3]; x.n1 = rec[4]; x.owned = rec[5]; x.nc0 = rec[6];
   return x;
 }
 
@@ -69,6 +81,8 @@ __device__ __forceinline__ void unit_lens(const DecodeArgs& d, int u, int& n0, i
   }
 }
 
+__device__ __forceinline__ int chunks_of(int n) { return (n + kChunk - 1) / kChunk; }
+
 __device__ __forceinline__ void merge_ml(float& m, float& l, float m2, float l2) {
   const float M = fmaxf(m, m2);
   if (M == -INFINITY) return;
@@ -76,19 +90,26 @@ __device__ __forceinline__ void merge_ml(float& m, float& l, float m2, float l2)
   m = M;
 }
 
-// Rows [v_lo, v_hi) (unit coordinates) of the unit that lie in chunks [k0, k1).
-__device__ __forceinline__ void piece_rows(const Unit& x, int k0, int k1, int& v_lo, int& v_hi) {
-  const int ga = max(x.cb, k0), gb = min(x.cb + x.nc, k1);
-  v_lo = (ga - x.cb) * kChunk;
-  v_hi = min((gb - x.cb) * kChunk, x.n0 + x.n1);
+// Order-preserving map of floats to ints (for atomicMax on floats).
+__device__ __forceinline__ int f2ord(float f) {
+  const int i = __float_as_int(f);
+  return i >= 0 ? i : i ^ 0x7FFFFFFF;
 }
+__device__ __forceinline__ float ord2f(int i) { return __int_as_float(i >= 0 ? i : i ^ 0x7FFFFFFF); }
 
-// End of the tile that starts at row v: the next tile boundary, the segment
-// boundary n0, or the piece end.
-__device__ __forceinline__ int tile_end(int v, int n0, int v_hi) {
-  int e = min((v / kTile + 1) * kTile, v_hi);
-  if (v < n0) e = min(e, n0);
-  return e;
+// Rows of chunk c (unit coordinates) and where they live.
+struct ChunkRows {
+  int seg, row0, rows;  // segment, first row inside the segment, valid rows
+};
+
+__device__ __forceinline__ ChunkRows chunk_rows(const Unit& x, int c) {
+  ChunkRows r;
+  r.seg = c >= x.nc0 ? 1 : 0;
+  const int cs = r.seg ? c - x.nc0 : c;
+  const int n = r.seg ? x.n1 : x.n0;
+  r.row0 = cs * kChunk;
+  r.rows = min(kChunk, n - r.row0);
+  return r;
 }
 
 template <int D, int KB>
@@ -97,7 +118,7 @@ struct Geo {
   static constexpr int RPW = 32 / LPR;          // rows per warp step
   static constexpr int RB = D * KB / 8;         // packed K row bytes
   static constexpr int kStageCodes = kTile * RB;
-  static constexpr int kStageSz = (kTile + 2) * (D / 32) * 8;  // ng <= D/32, plus one alignment row each side
+  static constexpr int kStageSz = (kTile + 2) * (D / 32) * 8;  // ng <= D/32, plus alignment rows
   static constexpr int kStageBytes = (kStageCodes + kStageSz + 127) / 128 * 128;
 };
 
@@ -106,7 +127,7 @@ __device__ __forceinline__ bool wait_counter(const int* p, int target, uint64_t 
   if (ld_acquire(p) >= target) return true;
   const uint64_t t0 = global_ns();
   while (true) {
-    __nanosleep(256);
+    __nanosleep(128);
     if (ld_acquire(p) >= target) return true;
     if (global_ns() - t0 > limit_ns) return false;
   }
@@ -135,6 +156,16 @@ struct ReduceScatter {
   }
 };
 
+template <int H, int LPR>
+__device__ __forceinline__ int head_of_lane(int lane) {
+  float dummy[H];
+#pragma unroll
+  for (int h = 0; h < H; ++h) dummy[h] = 0.0f;
+  int hidx = 0;
+  ReduceScatter<H, LPR / 2>::run(dummy, lane, hidx);
+  return hidx;
+}
+
 template <int H>
 __device__ __forceinline__ void load_heads(const float* p, float (&x)[H]) {
   if constexpr (H == 4) {
@@ -159,6 +190,43 @@ __device__ __forceinline__ void store_heads(float* p, const float (&x)[H]) {
   }
 }
 
+// Exponent fields of the unpack's magic floats, kept in registers so that
+// each code costs a single AND-OR (an immediate mask plus this register).
+template <int BITS>
+struct Magic {
+  uint32_t m[32];
+  __device__ __forceinline__ void load(const int* src) {
+#pragma unroll
+    for (int k = 0; k < 24 - BITS; ++k) m[k] = (uint32_t)src[k];
+  }
+};
+
+template <int BITS, int I>
+__device__ __forceinline__ float code_plus_magic_r(const LaneWords<BITS>& lw, const Magic<BITS>& mg) {
+  constexpr int s = copy_shift<BITS>(I);
+  constexpr int kk = I * BITS - s;
+  constexpr uint32_t mask = ((1u << BITS) - 1u) << kk;
+  return __uint_as_float((stream_bits<BITS>(lw, s) & mask) | mg.m[kk]);
+}
+
+template <int BITS, int P>
+__device__ __forceinline__ float2 code_pair_r(const LaneWords<BITS>& lw, const Magic<BITS>& mg) {
+  const float2 m = make_float2(code_plus_magic_r<BITS, 2 * P>(lw, mg), code_plus_magic_r<BITS, 2 * P + 1>(lw, mg));
+  return __fadd2_rn(m, make_float2(-magic_value<BITS, 2 * P>(), -magic_value<BITS, 2 * P + 1>()));
+}
+
+template <int BITS>
+__device__ __forceinline__ void unpack16_int_r(const LaneWords<BITS>& lw, const Magic<BITS>& mg, float2 (&c)[8]) {
+  c[0] = code_pair_r<BITS, 0>(lw, mg);
+  c[1] = code_pair_r<BITS, 1>(lw, mg);
+  c[2] = code_pair_r<BITS, 2>(lw, mg);
+  c[3] = code_pair_r<BITS, 3>(lw, mg);
+  c[4] = code_pair_r<BITS, 4>(lw, mg);
+  c[5] = code_pair_r<BITS, 5>(lw, mg);
+  c[6] = code_pair_r<BITS, 6>(lw, mg);
+  c[7] = code_pair_r<BITS, 7>(lw, mg);
+}
+
 // Global V-row load for the gather (lane's codes + its group's (scale, zero)).
 template <int VB>
 __device__ __forceinline__ void ldg_v(const uint8_t* codes_row, const float* sz_row, int j, int gi,
@@ -168,10 +236,10 @@ __device__ __forceinline__ void ldg_v(const uint8_t* codes_row, const float* sz_
 }
 
 template <int H, int VB>
-__device__ __forceinline__ void accumulate_v(const LaneWords<VB>& lw, float2 sz, const float (&w)[H],
-                                             float2 (&acc)[H][8], float (&Z)[H]) {
+__device__ __forceinline__ void accumulate_v(const LaneWords<VB>& lw, const Magic<VB>& mg, float2 sz,
+                                             const float (&w)[H], float2 (&acc)[H][8], float (&Z)[H]) {
   float2 c[8];
-  unpack16_int<VB>(lw, c);
+  unpack16_int_r<VB>(lw, mg, c);
 #pragma unroll
   for (int h = 0; h < H; ++h) {
     const float ws = w[h] * sz.x;
@@ -181,6 +249,10 @@ __device__ __forceinline__ void accumulate_v(const LaneWords<VB>& lw, float2 sz,
     Z[h] = fmaf(w[h], sz.y, Z[h]);
   }
 }
+
+struct TileDesc {
+  int kk, seg, row0, rows, entry, pad0, pad1, pad2;
+};
 
 // ------------------------------------------------------------------ kernel
 
@@ -194,13 +266,15 @@ __global__ void __launch_bounds__(kThreads, 1) fused_decode_kernel(FusedArgs a) 
   const DecodeArgs& d = a.d;
   const int units = d.B * d.Hkv;
   const int ng = D / d.G;
+  const int S = a.stages;
   const uint64_t limit_ns = (a.timeout_ns && *a.timeout_ns) ? *a.timeout_ns : 2000000000ull;
   const int j = lane % LPR;                 // lane's 16-channel slice of a row
   const int gi = (j * kDimsPerLane) / d.G;  // its quantization group
 
   uint64_t* full = reinterpret_cast<uint64_t*>(smem_raw);
-  uint64_t* empty = full + kStages;
-  int* misc = reinterpret_cast<int*>(smem_raw + 128);   // 224 ints
+  uint64_t* empty = full + kMaxStages;
+  TileDesc* desc = reinterpret_cast<TileDesc*>(smem_raw + kDescOff);
+  int* misc = reinterpret_cast<int*>(smem_raw + kMiscOff);   // 64 ints
   uint8_t* ring = smem_raw + kHeader;
   float* s_logits = reinterpret_cast<float*>(ring + a.ring_bytes);
 
@@ -211,17 +285,19 @@ __global__ void __launch_bounds__(kThreads, 1) fused_decode_kernel(FusedArgs a) 
   int& s_carry_c = misc[4];
   int& s_carry_n = misc[5];
   int& s_last = misc[6];
-  float* s_glob = reinterpret_cast<float*>(misc + 8);  // (max, 1/sum) x 4 heads
-  int* s_wsum = misc + 32;                            // 2 x 16 warp partials
+  float* s_glob = reinterpret_cast<float*>(misc + 8);   // (max, 1/sum) x 4 heads
+  int* s_wsum = misc + 16;                             // 2 x 12 warp partials
+  int* s_magic = misc + 40;                            // 24 magic exponent fields
 
   if (tid == 0) {
-    for (int s = 0; s < kStages; ++s) {
+    for (int s = 0; s < S; ++s) {
       mbar_init(&full[s], 1);
-      mbar_init(&empty[s], kConsumerWarps);
+      mbar_init(&empty[s], kGroupWarps);
     }
     fence_mbar_init();
     s_total = 0; s_e0 = 0; s_nent = 0; s_abort = 0; s_carry_c = 0; s_carry_n = 0; s_last = 0;
   }
+  if (tid < 24) s_magic[tid] = (150 - tid) << 23;
   __syncthreads();
 
   // ------------------------------------------------------------ unit list
@@ -231,7 +307,7 @@ __global__ void __launch_bounds__(kThreads, 1) fused_decode_kernel(FusedArgs a) 
     for (int u = tid; u < units; u += kConsumers) {
       int n0, n1;
       unit_lens(d, u, n0, n1);
-      part += (n0 + n1 + kChunk - 1) / kChunk;
+      part += chunks_of(n0) + chunks_of(n1);
       if (n0 + n1 == 0 && (u % grid) == cta) {  // empty unit: its outputs are zero
         const int b = u / d.Hkv, g = u % d.Hkv;
         for (int e = 0; e < H * D; ++e) d.out[((long long)b * d.Hq + g * H + e / D) * D + e % D] = 0.0f;
@@ -257,13 +333,15 @@ __global__ void __launch_bounds__(kThreads, 1) fused_decode_kernel(FusedArgs a) 
   const int total = s_total;
   const int cpc = (total + grid - 1) / grid;
   const int k0 = min(cta * cpc, total), k1 = min(k0 + cpc, total);
+  const int nck = k1 - k0;
   int* ulist = a.ulist + (long long)cta * a.cpc_max * kRec;
   if (consumer) {
     for (int base = 0; base < units; base += kConsumers) {
       const int u = base + tid;
       int n0 = 0, n1 = 0;
       if (u < units) unit_lens(d, u, n0, n1);
-      const int nc = (n0 + n1 + kChunk - 1) / kChunk;
+      const int nc0 = chunks_of(n0);
+      const int nc = nc0 + chunks_of(n1);
       const int ne = nc > 0 ? 1 : 0;
       int sc = nc, sn = ne;  // warp inclusive scans
 #pragma unroll
@@ -271,12 +349,12 @@ __global__ void __launch_bounds__(kThreads, 1) fused_decode_kernel(FusedArgs a) 
         const int y = __shfl_up_sync(kFull, sc, off), z = __shfl_up_sync(kFull, sn, off);
         if (lane >= off) { sc += y; sn += z; }
       }
-      if (lane == 31) { s_wsum[warp] = sc; s_wsum[16 + warp] = sn; }
+      if (lane == 31) { s_wsum[warp] = sc; s_wsum[12 + warp] = sn; }
       named_barrier(kBarCons, kConsumers);
       int wc = 0, wn = 0, tc = 0, tn = 0;
       for (int w = 0; w < kConsumerWarps; ++w) {
-        if (w < warp) { wc += s_wsum[w]; wn += s_wsum[16 + w]; }
-        tc += s_wsum[w]; tn += s_wsum[16 + w];
+        if (w < warp) { wc += s_wsum[w]; wn += s_wsum[12 + w]; }
+        tc += s_wsum[w]; tn += s_wsum[12 + w];
       }
       const int cb = s_carry_c + wc + sc - nc;
       const int ne_idx = s_carry_n + wn + sn - ne;
@@ -287,6 +365,7 @@ __global__ void __launch_bounds__(kThreads, 1) fused_decode_kernel(FusedArgs a) 
         int* rec = ulist + (long long)idx * kRec;
         rec[0] = u; rec[1] = cb; rec[2] = nc; rec[3] = n0; rec[4] = n1;
         rec[5] = (cb >= k0 && cb + nc <= k1) ? 1 : 0;
+        rec[6] = nc0;
         atomicMax(&s_nent, idx + 1);
       }
       named_barrier(kBarCons, kConsumers);
@@ -294,10 +373,23 @@ __global__ void __launch_bounds__(kThreads, 1) fused_decode_kernel(FusedArgs a) 
       named_barrier(kBarCons, kConsumers);
     }
   }
-  __syncthreads();  // the producer joins: list complete
+  // chunk statistics: in shared memory unless the CTA has many chunks
+  int* cmx;
+  float *csm, *cfc;
+  if (nck <= kCsCap) {
+    cmx = reinterpret_cast<int*>(smem_raw + kCsOff);
+    csm = reinterpret_cast<float*>(cmx + kCsCap * 4);
+    cfc = csm + kCsCap * 4;
+  } else {
+    cmx = reinterpret_cast<int*>(a.gstats + (long long)cta * a.cpc_max * 12);
+    csm = reinterpret_cast<float*>(cmx + a.cpc_max * 4);
+    cfc = csm + a.cpc_max * 4;
+  }
+  for (int i = tid; i < nck * H; i += kThreads) cmx[i] = f2ord(-INFINITY);
+  __syncthreads();  // list complete, maxima reset
   const int nent = s_nent;
 
-  float* lg = ((long long)(k1 - k0) * kChunk * H <= a.smem_logit_floats)
+  float* lg = ((long long)nck * kChunk * H <= a.smem_logit_floats)
                   ? s_logits
                   : a.glogits + (long long)cta * a.cpc_max * kChunk * H;
 
@@ -307,113 +399,131 @@ __global__ void __launch_bounds__(kThreads, 1) fused_decode_kernel(FusedArgs a) 
       const uint64_t pol = policy_evict_first();
       int t = 0;
       bool ok = true;
+      auto acquire_stage = [&](int tt) -> bool {
+        if (tt < S) return true;
+        const int st = tt % S;
+        if (mbar_wait(&empty[st], ((tt / S) - 1) & 1, limit_ns)) return true;
+        atomicExch(d.status, kStatusTimeout);
+        atomicExch(&s_abort, 1);
+        return false;
+      };
       for (int e = 0; e < nent && ok; ++e) {
         const Unit x = load_unit(ulist + (long long)e * kRec);
-        int v_lo, v_hi;
-        piece_rows(x, k0, k1, v_lo, v_hi);
         const long long ubase = (long long)x.u * d.T_cap;
-        for (int v = v_lo; v < v_hi && ok;) {
-          const int ve = tile_end(v, x.n0, v_hi);
-          const int seg = v >= x.n0 ? 1 : 0;
-          const int row = seg ? v - x.n0 : v;
-          const int rows = ve - v;
-          const int stage = t % kStages;
-          if (t >= kStages && !mbar_wait(&empty[stage], ((t / kStages) - 1) & 1, limit_ns)) {
-            atomicExch(d.status, kStatusTimeout);
-            atomicExch(&s_abort, 1);
-            ok = false;
-            break;
+        const int ga = max(x.cb, k0), gb = min(x.cb + x.nc, k1);
+        for (int g = ga; g < gb && ok; ++g) {
+          const ChunkRows cr = chunk_rows(x, g - x.cb);
+          for (int r = 0; r < cr.rows && ok; r += kTile) {
+            const int rows = min(kTile, cr.rows - r);
+            const int row = cr.row0 + r;
+            if (!acquire_stage(t)) { ok = false; break; }
+            const int stage = t % S;
+            const int r0 = (ng == 1) ? (row & ~1) : row;
+            const int r1 = (ng == 1) ? ((row + rows + 1) & ~1) : row + rows;
+            const uint32_t cbytes = (uint32_t)rows * Gk::RB;
+            const uint32_t sbytes = (uint32_t)(r1 - r0) * ng * 8;
+            TileDesc td;
+            td.kk = g - k0; td.seg = cr.seg; td.row0 = row; td.rows = rows; td.entry = e;
+            desc[stage] = td;
+            uint8_t* dst = ring + (size_t)stage * Gk::kStageBytes;
+            mbar_arrive_expect_tx(&full[stage], cbytes + sbytes);
+            bulk_g2s(dst, d.kc[cr.seg] + (ubase + row) * Gk::RB, cbytes, &full[stage], pol);
+            bulk_g2s(dst + Gk::kStageCodes, d.ksz[cr.seg] + (ubase + r0) * ng * 2, sbytes, &full[stage], pol);
+            ++t;
           }
-          const int r0 = (ng == 1) ? (row & ~1) : row;
-          const int r1 = (ng == 1) ? ((row + rows + 1) & ~1) : row + rows;
-          const uint32_t cbytes = (uint32_t)rows * Gk::RB;
-          const uint32_t sbytes = (uint32_t)(r1 - r0) * ng * 8;
-          uint8_t* dst = ring + (size_t)stage * Gk::kStageBytes;
-          mbar_arrive_expect_tx(&full[stage], cbytes + sbytes);
-          bulk_g2s(dst, d.kc[seg] + (ubase + row) * Gk::RB, cbytes, &full[stage], pol);
-          bulk_g2s(dst + Gk::kStageCodes, d.ksz[seg] + (ubase + r0) * ng * 2, sbytes, &full[stage], pol);
-          ++t;
-          v = ve;
         }
       }
+      // one end marker per consumer group (a plain arrival completes the phase)
+      for (int k = 0; k < kGroups && ok; ++k) {
+        if (!acquire_stage(t)) { ok = false; break; }
+        const int stage = t % S;
+        desc[stage].rows = -1;
+        mbar_arrive(&full[stage]);
+        ++t;
+      }
       // Never leave copies in flight: wait for the last stages issued.
-      for (int k = max(0, t - kStages); k < t; ++k)
-        mbar_wait(&full[k % kStages], (k / kStages) & 1, limit_ns);
+      for (int k = max(0, t - S); k < t; ++k) mbar_wait(&full[k % S], (k / S) & 1, limit_ns);
     }
     return;  // the producer warp takes no further part
   }
 
   // consumers
   {
-    int t = 0, rs0 = 0;
+    const int grp = warp / kGroupWarps, wig = warp % kGroupWarps;
+    const int hidx_lane = head_of_lane<H, LPR>(lane);
+    const bool leader = (lane % (LPR / H)) == 0;
+    Magic<KB> mg;
+    mg.load(s_magic);
     float2 qf[H][8];
     float Q[H];
-    for (int e = 0; e < nent; ++e) {
-      const Unit x = load_unit(ulist + (long long)e * kRec);
-      int v_lo, v_hi;
-      piece_rows(x, k0, k1, v_lo, v_hi);
-      const int b = x.u / d.Hkv, g = x.u % d.Hkv;
-#pragma unroll
-      for (int h = 0; h < H; ++h) {
-        float xq[16];
-        load16_bf16(d.q + ((long long)b * d.Hq + g * H + h) * D + j * kDimsPerLane, xq);
-        float s = 0.0f;
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          qf[h][i] = make_float2(xq[2 * i] * d.q_scale, xq[2 * i + 1] * d.q_scale);
-          s += qf[h][i].x + qf[h][i].y;
-        }
-        Q[h] = s;
+    int cur_e = -1;
+    volatile int* abort_flag = &s_abort;
+    for (int t = grp;; t += kGroups) {
+      const int stage = t % S;
+      if (*abort_flag) break;
+      if (!mbar_wait(&full[stage], (t / S) & 1, limit_ns)) {
+        atomicExch(d.status, kStatusTimeout);
+        atomicExch(&s_abort, 1);
+        break;
       }
-      float* lgu = lg + (long long)(x.cb - k0) * kChunk * H;
-      for (int v = v_lo; v < v_hi;) {
-        const int ve = tile_end(v, x.n0, v_hi);
-        const int seg = v >= x.n0 ? 1 : 0;
-        const int row = seg ? v - x.n0 : v;
-        const int rows = ve - v;
-        const int stage = t % kStages;
-        volatile int* abort_flag = &s_abort;
-        if (!*abort_flag && !mbar_wait(&full[stage], (t / kStages) & 1, limit_ns)) {
-          atomicExch(d.status, kStatusTimeout);
-          atomicExch(&s_abort, 1);
-        }
-        if (!*abort_flag) {
-          const uint8_t* codes = ring + (size_t)stage * Gk::kStageBytes;
-          const float* szs = reinterpret_cast<const float*>(codes + Gk::kStageCodes) +
-                             ((ng == 1) ? (row & 1) : 0) * ng * 2;
-          const int nrs = (rows + RPW - 1) / RPW;
-          for (int rs = ((warp - rs0) % kConsumerWarps + kConsumerWarps) % kConsumerWarps; rs < nrs;
-               rs += kConsumerWarps) {
-            const int i = rs * RPW + lane / LPR;
-            const bool valid = i < rows;
-            float dot[H];
+      const TileDesc td = desc[stage];
+      if (td.rows < 0) break;
+      if (td.entry != cur_e) {
+        cur_e = td.entry;
+        const Unit x = load_unit(ulist + (long long)cur_e * kRec);
+        const int b = x.u / d.Hkv, g = x.u % d.Hkv;
 #pragma unroll
-            for (int h = 0; h < H; ++h) dot[h] = 0.0f;
-            if (valid) {
-              LaneWords<KB> lw;
-              lds_lane_words<KB>(codes + i * Gk::RB + j * (2 * KB), lw);
-              const float2 sz = *reinterpret_cast<const float2*>(szs + (i * ng + gi) * 2);
-              float2 c[8];
-              unpack16_int<KB>(lw, c);
+        for (int h = 0; h < H; ++h) {
+          float xq[16];
+          load16_bf16(d.q + ((long long)b * d.Hq + g * H + h) * D + j * kDimsPerLane, xq);
+          float s = 0.0f;
 #pragma unroll
-              for (int h = 0; h < H; ++h) {
-                float2 acc = make_float2(0.0f, 0.0f);
-#pragma unroll
-                for (int p = 0; p < 8; ++p) acc = __ffma2_rn(qf[h][p], c[p], acc);
-                dot[h] = fmaf(sz.x, acc.x + acc.y, sz.y * Q[h]);
-              }
-            }
-            int hidx = 0;
-            ReduceScatter<H, LPR / 2>::run(dot, lane, hidx);
-            if (valid && (lane % (LPR / H)) == 0) lgu[(long long)(v + i) * H + hidx] = dot[0];
+          for (int i = 0; i < 8; ++i) {
+            qf[h][i] = make_float2(xq[2 * i] * d.q_scale, xq[2 * i + 1] * d.q_scale);
+            s += qf[h][i].x + qf[h][i].y;
           }
-          rs0 += nrs;
+          Q[h] = s;
         }
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&empty[stage]);
-        ++t;
-        v = ve;
       }
+      const uint8_t* codes = ring + (size_t)stage * Gk::kStageBytes;
+      const float* szs = reinterpret_cast<const float*>(codes + Gk::kStageCodes) +
+                         ((ng == 1) ? (td.row0 & 1) : 0) * ng * 2;
+      float* lgt = lg + (td.kk * kChunk + (td.row0 % kChunk)) * H;
+      const int nrs = (td.rows + RPW - 1) / RPW;
+      float tmax = -INFINITY;
+      for (int rs = wig; rs < nrs; rs += kGroupWarps) {
+        const int i = rs * RPW + lane / LPR;
+        const bool valid = i < td.rows;
+        float dot[H];
+#pragma unroll
+        for (int h = 0; h < H; ++h) dot[h] = 0.0f;
+        if (valid) {
+          LaneWords<KB> lw;
+          lds_lane_words<KB>(codes + i * Gk::RB + j * (2 * KB), lw);
+          const float2 sz = *reinterpret_cast<const float2*>(szs + (i * ng + gi) * 2);
+          float2 c[8];
+          unpack16_int_r<KB>(lw, mg, c);
+#pragma unroll
+          for (int h = 0; h < H; ++h) {
+            float2 acc = make_float2(0.0f, 0.0f);
+#pragma unroll
+            for (int p = 0; p < 8; ++p) acc = __ffma2_rn(qf[h][p], c[p], acc);
+            dot[h] = fmaf(sz.x, acc.x + acc.y, sz.y * Q[h]);
+          }
+        }
+        int hidx = 0;
+        ReduceScatter<H, LPR / 2>::run(dot, lane, hidx);
+        if (valid && leader) {
+          lgt[i * H + hidx] = dot[0];
+          tmax = fmaxf(tmax, dot[0]);
+        }
+      }
+      // tile maximum per head -> the chunk's running maximum
+#pragma unroll
+      for (int off = LPR; off < 32; off <<= 1) tmax = fmaxf(tmax, __shfl_xor_sync(kFull, tmax, off));
+      if (lane < LPR && leader && tmax > -INFINITY) atomicMax(&cmx[td.kk * H + hidx_lane], f2ord(tmax));
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&empty[stage]);
     }
   }
   named_barrier(kBarCons, kConsumers);
@@ -421,9 +531,9 @@ __global__ void __launch_bounds__(kThreads, 1) fused_decode_kernel(FusedArgs a) 
   // phase 2 reuses: skip straight to the end (the status word says why).
   const bool aborted = *static_cast<volatile int*>(&s_abort) != 0;
   const int n_work = aborted ? 0 : nent;
-  const int n_chunks_work = aborted ? 0 : k1 - k0;
+  const int n_chunks_work = aborted ? 0 : nck;
 
-  // ------------------------------------------------------------ chunk statistics
+  // ------------------------------------------------------------ chunk sums
   for (int kk = warp; kk < n_chunks_work; kk += kConsumerWarps) {
     const int g_chunk = k0 + kk;
     int lo = 0, hi = nent - 1;  // entry holding chunk g_chunk
@@ -432,21 +542,11 @@ __global__ void __launch_bounds__(kThreads, 1) fused_decode_kernel(FusedArgs a) 
       if (ulist[(long long)mid * kRec + 1] <= g_chunk) lo = mid; else hi = mid - 1;
     }
     const Unit x = load_unit(ulist + (long long)lo * kRec);
-    const int rows = min(kChunk, x.n0 + x.n1 - (g_chunk - x.cb) * kChunk);
+    const int rows = chunk_rows(x, g_chunk - x.cb).rows;
     float* base = lg + (long long)kk * kChunk * H;
     float m[H], l[H];
 #pragma unroll
-    for (int h = 0; h < H; ++h) { m[h] = -INFINITY; l[h] = 0.0f; }
-    for (int i = lane; i < rows; i += 32) {
-      float s[H];
-      load_heads<H>(base + (long long)i * H, s);
-#pragma unroll
-      for (int h = 0; h < H; ++h) m[h] = fmaxf(m[h], s[h]);
-    }
-#pragma unroll
-    for (int h = 0; h < H; ++h)
-#pragma unroll
-      for (int off = 16; off >= 1; off >>= 1) m[h] = fmaxf(m[h], __shfl_xor_sync(kFull, m[h], off));
+    for (int h = 0; h < H; ++h) { m[h] = ord2f(cmx[kk * H + h]); l[h] = 0.0f; }
     for (int i = lane; i < rows; i += 32) {
       float s[H];
       load_heads<H>(base + (long long)i * H, s);
@@ -461,11 +561,7 @@ __global__ void __launch_bounds__(kThreads, 1) fused_decode_kernel(FusedArgs a) 
     for (int h = 0; h < H; ++h)
 #pragma unroll
       for (int off = 16; off >= 1; off >>= 1) l[h] += __shfl_xor_sync(kFull, l[h], off);
-    if (lane == 0) {
-      float* cs = a.cstats + (long long)g_chunk * H * 2;
-#pragma unroll
-      for (int h = 0; h < H; ++h) { cs[2 * h] = m[h]; cs[2 * h + 1] = l[h]; }
-    }
+    if (lane < H) csm[kk * H + lane] = l[lane];
   }
   named_barrier(kBarCons, kConsumers);
 
@@ -473,38 +569,50 @@ __global__ void __launch_bounds__(kThreads, 1) fused_decode_kernel(FusedArgs a) 
   for (int e = warp; e < n_work; e += kConsumerWarps) {
     int* rec = ulist + (long long)e * kRec;
     const Unit x = load_unit(rec);
-    if (lane < H) {
-      const int h = lane;
+    const int ga = max(x.cb, k0), gb = min(x.cb + x.nc, k1);
+#pragma unroll
+    for (int h = 0; h < H; ++h) {
       float m = -INFINITY, l = 0.0f;
-      const int ga = max(x.cb, k0), gb = min(x.cb + x.nc, k1);
-      for (int g2 = ga; g2 < gb; ++g2) {
-        const float* cs = a.cstats + (long long)g2 * H * 2;
-        merge_ml(m, l, cs[2 * h], cs[2 * h + 1]);
+      for (int g2 = ga + lane; g2 < gb; g2 += 32) merge_ml(m, l, ord2f(cmx[(g2 - k0) * H + h]), csm[(g2 - k0) * H + h]);
+#pragma unroll
+      for (int off = 16; off >= 1; off >>= 1) {
+        const float m2 = __shfl_xor_sync(kFull, m, off), l2 = __shfl_xor_sync(kFull, l, off);
+        merge_ml(m, l, m2, l2);
       }
-      reinterpret_cast<float*>(rec + 8)[2 * h] = m;
-      reinterpret_cast<float*>(rec + 8)[2 * h + 1] = l;
-      if (!x.owned) {
-        if (e == 0) {
-          a.pstats[((long long)cta * 2 + 0) * H * 2 + 2 * h] = m;
-          a.pstats[((long long)cta * 2 + 0) * H * 2 + 2 * h + 1] = l;
-        }
-        if (e == nent - 1) {
-          a.pstats[((long long)cta * 2 + 1) * H * 2 + 2 * h] = m;
-          a.pstats[((long long)cta * 2 + 1) * H * 2 + 2 * h + 1] = l;
+      if (lane == 0) {
+        reinterpret_cast<float*>(rec + 8)[2 * h] = m;
+        reinterpret_cast<float*>(rec + 8)[2 * h + 1] = l;
+        if (!x.owned) {
+          if (e == 0) {
+            a.pstats[((long long)cta * 2 + 0) * H * 2 + 2 * h] = m;
+            a.pstats[((long long)cta * 2 + 0) * H * 2 + 2 * h + 1] = l;
+          }
+          if (e == nent - 1) {
+            a.pstats[((long long)cta * 2 + 1) * H * 2 + 2 * h] = m;
+            a.pstats[((long long)cta * 2 + 1) * H * 2 + 2 * h + 1] = l;
+          }
         }
       }
-    }
-    if (!x.owned) {
-      __threadfence();
-      __syncwarp();
-      if (lane == 0) atomicAdd(a.arrive1 + x.u, 1);
     }
   }
   named_barrier(kBarCons, kConsumers);
+  if (tid == 0 && n_work > 0) {
+    __threadfence();  // orders every consumer's statistics before the arrivals
+    const Unit x0 = load_unit(ulist);
+    if (!x0.owned) atomicAdd(a.arrive1 + x0.u, 1);
+    if (nent > 1) {
+      const Unit x1 = load_unit(ulist + (long long)(nent - 1) * kRec);
+      if (!x1.owned) atomicAdd(a.arrive1 + x1.u, 1);
+    }
+  }
 
   // ------------------------------------------------------------ phase 2
-  int* lists = reinterpret_cast<int*>(ring);                        // [16][kListCap]
-  float* red = reinterpret_cast<float*>(ring + kConsumerWarps * kListCap * 4);  // [16][H][D]
+  int* lists = reinterpret_cast<int*>(ring);                                    // [12][kListCap]
+  float* red = reinterpret_cast<float*>(ring + kConsumerWarps * kListCap * 4);  // [12][H][D]
+  Magic<VB0> mg0;
+  mg0.load(s_magic);
+  Magic<VB1> mg1;
+  mg1.load(s_magic);
   unsigned long long cnt_heads = 0, cnt_rows = 0;
   for (int pass = 0; pass < 2; ++pass) {
     for (int e = 0; e < n_work; ++e) {
@@ -541,23 +649,19 @@ __global__ void __launch_bounds__(kThreads, 1) fused_decode_kernel(FusedArgs a) 
         }
       }
       named_barrier(kBarCons, kConsumers);
-      // per-chunk factors exp2(max_c - max) / sum, written over the chunk sums
-      {
-        const int ga = max(x.cb, k0), gb = min(x.cb + x.nc, k1);
-        for (int g2 = ga + tid / H; g2 < gb; g2 += kConsumers / H) {
-          const int h = tid % H;
-          float* cs = a.cstats + (long long)g2 * H * 2;
-          const float M = s_glob[2 * h], il = s_glob[2 * h + 1];
-          cs[2 * h + 1] = (il > 0.0f) ? exp2f(cs[2 * h] - M) * il : 0.0f;
-        }
+      const int ga = max(x.cb, k0), gb = min(x.cb + x.nc, k1);
+      // per-chunk factors exp2(max_c - max) / sum
+      for (int q = tid; q < (gb - ga) * H; q += kConsumers) {
+        const int kk = ga - k0 + q / H, h = q % H;
+        const float M = s_glob[2 * h], il = s_glob[2 * h + 1];
+        cfc[kk * H + h] = (il > 0.0f) ? exp2f(ord2f(cmx[kk * H + h]) - M) * il : 0.0f;
       }
       named_barrier(kBarCons, kConsumers);
 
-      int v_lo, v_hi;
-      piece_rows(x, k0, k1, v_lo, v_hi);
       const float* lgu = lg + (long long)(x.cb - k0) * kChunk * H;
-      const float* csu = a.cstats + (long long)x.cb * H * 2;
+      const float* cfu = cfc + (x.cb - k0) * H;
       const long long ubase = (long long)x.u * d.T_cap;
+      const int v_lo = (ga - x.cb) * kChunk, v_hi = (gb - x.cb) * kChunk;  // chunk-aligned (padded) rows
       float2 acc[H][8];
       float Z[H];
 #pragma unroll
@@ -571,17 +675,18 @@ __global__ void __launch_bounds__(kThreads, 1) fused_decode_kernel(FusedArgs a) 
         int* list = lists + warp * kListCap;
         int n_w = 0;
         for (int blk = warp; blk < kConsumerWarps * kBatchBlocks; blk += kConsumerWarps) {
-          const int v = vb + blk * 32 + lane;
           if (vb + blk * 32 >= v_hi) break;
+          const int v = vb + blk * 32 + lane;
+          const int c = v / kChunk;
+          const ChunkRows cr = chunk_rows(x, c);
           bool need = false;
-          if (v < v_hi) {
+          if (v % kChunk < cr.rows) {
             float ev[H];
             load_heads<H>(lgu + (long long)v * H, ev);
             int nskip = 0;
 #pragma unroll
             for (int h = 0; h < H; ++h) {
-              const float fac = csu[(long long)(v / kChunk) * H * 2 + 2 * h + 1];
-              const float p = ev[h] * fac;
+              const float p = ev[h] * cfu[c * H + h];
               const bool keep = !(p < d.tau);
               need |= keep;
               nskip += keep ? 0 : 1;
@@ -608,11 +713,11 @@ __global__ void __launch_bounds__(kThreads, 1) fused_decode_kernel(FusedArgs a) 
             vv[s] = idx < n_w ? list[idx] : -1;
             if (vv[s] >= 0) {
               const int v = vv[s];
-              const int seg = v >= x.n0 ? 1 : 0;
-              const long long row = ubase + (seg ? v - x.n0 : v);
+              const ChunkRows cr = chunk_rows(x, v / kChunk);
+              const long long row = ubase + cr.row0 + v % kChunk;
               if constexpr (kOneWidth) {
-                ldg_v<VB0>(d.vc[seg] + row * (D * VB0 / 8), d.vsz[seg] + row * ng * 2, j, gi, w0[s], szv[s]);
-              } else if (seg == 0) {
+                ldg_v<VB0>(d.vc[cr.seg] + row * (D * VB0 / 8), d.vsz[cr.seg] + row * ng * 2, j, gi, w0[s], szv[s]);
+              } else if (cr.seg == 0) {
                 ldg_v<VB0>(d.vc[0] + row * (D * VB0 / 8), d.vsz[0] + row * ng * 2, j, gi, w0[s], szv[s]);
               } else {
                 ldg_v<VB1>(d.vc[1] + row * (D * VB1 / 8), d.vsz[1] + row * ng * 2, j, gi, w1[s], szv[s]);
@@ -623,18 +728,19 @@ __global__ void __launch_bounds__(kThreads, 1) fused_decode_kernel(FusedArgs a) 
           for (int s = 0; s < kGatherUnroll; ++s) {
             const int v = vv[s];
             if (v < 0) continue;
+            const int c = v / kChunk;
             float ev[H], w[H];
             load_heads<H>(lgu + (long long)v * H, ev);
 #pragma unroll
             for (int h = 0; h < H; ++h) {
-              const float p = ev[h] * csu[(long long)(v / kChunk) * H * 2 + 2 * h + 1];
+              const float p = ev[h] * cfu[c * H + h];
               w[h] = (p < d.tau) ? 0.0f : p;
             }
             if constexpr (kOneWidth) {
-              accumulate_v<H, VB0>(w0[s], szv[s], w, acc, Z);
+              accumulate_v<H, VB0>(w0[s], mg0, szv[s], w, acc, Z);
             } else {
-              if (v < x.n0) accumulate_v<H, VB0>(w0[s], szv[s], w, acc, Z);
-              else accumulate_v<H, VB1>(w1[s], szv[s], w, acc, Z);
+              if (c < x.nc0) accumulate_v<H, VB0>(w0[s], mg0, szv[s], w, acc, Z);
+              else accumulate_v<H, VB1>(w1[s], mg1, szv[s], w, acc, Z);
             }
           }
         }
@@ -654,19 +760,18 @@ __global__ void __launch_bounds__(kThreads, 1) fused_decode_kernel(FusedArgs a) 
             acc[h][i].x += __shfl_xor_sync(kFull, acc[h][i].x, off);
             acc[h][i].y += __shfl_xor_sync(kFull, acc[h][i].y, off);
           }
-      named_barrier(kBarCons, kConsumers);  // lists no longer read; red free
       if (lane < LPR) {
 #pragma unroll
         for (int h = 0; h < H; ++h)
 #pragma unroll
           for (int i = 0; i < 8; ++i)
-            *reinterpret_cast<float2*>(red + ((long long)warp * H + h) * D + j * kDimsPerLane + 2 * i) = acc[h][i];
+            *reinterpret_cast<float2*>(red + (warp * H + h) * D + j * kDimsPerLane + 2 * i) = acc[h][i];
       }
       named_barrier(kBarCons, kConsumers);
       for (int o = tid; o < H * D; o += kConsumers) {
         float s = 0.0f;
 #pragma unroll
-        for (int w = 0; w < kConsumerWarps; ++w) s += red[(long long)w * H * D + o];
+        for (int w = 0; w < kConsumerWarps; ++w) s += red[w * H * D + o];
         const int h = o / D, dd = o % D;
         if (x.owned) {
           d.out[((long long)b * d.Hq + g * H + h) * D + dd] = s;
@@ -676,9 +781,9 @@ __global__ void __launch_bounds__(kThreads, 1) fused_decode_kernel(FusedArgs a) 
         }
       }
       if (!x.owned) {
-        __threadfence();
         named_barrier(kBarCons, kConsumers);
         if (tid == 0) {
+          __threadfence();  // every thread's partial before the arrival
           const int old = atomicAdd(a.arrive2 + x.u, 1);
           s_last = (old == i_last - i_first) ? 1 : 0;
         }
@@ -716,9 +821,9 @@ __global__ void __launch_bounds__(kThreads, 1) fused_decode_kernel(FusedArgs a) 
       atomicAdd(a.wcounts + 1, cnt_rows);
     }
   }
-  __threadfence();
   named_barrier(kBarCons, kConsumers);
   if (tid == 0) {
+    __threadfence();
     const int old = atomicAdd(a.done, 1);
     if (old == grid - 1) {
       __threadfence();

@@ -69,6 +69,7 @@ struct DecodeArgs {
 struct FusedArgs {
   DecodeArgs d;
   int cpc_max;                   // upper bound of chunks per CTA
+  int stages;                    // ring stages in use
   int ring_bytes;                // shared-memory ring size
   long long smem_logit_floats;   // logits that fit in shared memory per CTA
   const unsigned long long* timeout_ns;  // workspace word: wait limit override (0 = default)
@@ -79,6 +80,7 @@ struct FusedArgs {
   float* cstats;                 // [chunks][H][2]
   int* ulist;                    // [grid][cpc_max][16]
   float* glogits;                // [grid][cpc_max * chunk][H] (when shared memory is short)
+  float* gstats;                 // [grid][cpc_max][12] chunk statistics (when there are many chunks)
   unsigned long long* wcounts;   // [2] skip-count accumulators
   int* done;                     // CTAs finished
 };
