@@ -79,10 +79,9 @@ bool fused_ok(int r) { return r == 1 || r == 2 || r == 4; }
 
 struct FusedLayout {
   int grid, H, cpc_max, ring_bytes, stages;
-  long long chunks_max, smem_logit_floats;
   size_t smem_bytes;
-  size_t arrive1, arrive2, pstats, ppart, cstats, ulist, glogits, gstats, total;
-  bool need_glogits, need_gstats;
+  size_t arrive1, arrive2, pstats, ppart, ulist, glogits, gstats, qbuf, qgsum, total;
+  bool need_gstats;
 };
 
 FusedLayout fused_layout(int B, int Hq, int Hkv, int T_cap, int D, int KB) {
@@ -92,42 +91,26 @@ FusedLayout fused_layout(int B, int Hq, int Hkv, int T_cap, int D, int KB) {
   const long long units = (long long)B * Hkv;
   // each segment rounds up to whole chunks: at most one more chunk per unit
   const long long per_unit = T_cap > 0 ? (T_cap + kChunk - 1) / kChunk + 1 : 1;
-  L.chunks_max = units * per_unit > 0 ? units * per_unit : 1;
-  L.cpc_max = (int)((L.chunks_max + L.grid - 1) / L.grid);
-  const int rb = D * KB / 8;
-  const int stage = ((fused::kTile * rb + (fused::kTile + 2) * (D / 32) * 8) + 127) / 128 * 128;
-  const int phase2 = fused::kConsumerWarps * fused::kListCap * 4 + fused::kConsumerWarps * L.H * D * 4;
-  const long long need = (long long)L.cpc_max * kChunk * L.H * 4;
-  const long long smax = max_smem_optin();
-  // deepest ring (a multiple of the consumer groups) that leaves room for the logits
-  L.stages = 0;
-  for (int s = fused::kMaxStages; s >= 6; s -= fused::kGroups) {
-    const int ring = std::max(s * stage, phase2);
-    if (fused::kHeader + ring + need <= smax) { L.stages = s; break; }
-  }
-  if (L.stages > 0) {
-    L.ring_bytes = std::max(L.stages * stage, phase2);
-    L.smem_logit_floats = need / 4;
-    L.need_glogits = false;
-  } else {
-    L.stages = 12;
-    L.ring_bytes = std::max(L.stages * stage, phase2);
-    L.smem_logit_floats = std::max(0ll, (smax - fused::kHeader - L.ring_bytes) / 16 * 4);
-    L.need_glogits = true;
-  }
-  L.need_gstats = L.cpc_max > fused::kCsCap;
-  L.smem_bytes = fused::kHeader + L.ring_bytes + (size_t)L.smem_logit_floats * 4;
+  const long long chunks_max = units * per_unit > 0 ? units * per_unit : 1;
+  L.cpc_max = (int)((chunks_max + L.grid - 1) / L.grid);
+  const fused::GeoHost g = fused::geo_host(D, KB);
+  L.stages = g.stages;
+  const int phase2 = fused::kMaxConsumerWarps * fused::kListCap * 4 + g.consumer_warps * L.H * D * 4;
+  L.ring_bytes = std::max(g.stages * g.stage_bytes, phase2);
+  L.smem_bytes = fused::kHeader + L.ring_bytes;
+  const int tpc = fused::kChunk / g.tile_rows;
+  L.need_gstats = (long long)L.cpc_max * tpc > fused::kTsCap;
   size_t off = kHeaderBytes;
   L.arrive1 = off; off = align_up(off + units * 4);
   L.arrive2 = off; off = align_up(off + units * 4);
   L.pstats = off; off = align_up(off + (size_t)L.grid * 2 * L.H * 2 * 4);
   L.ppart = off; off = align_up(off + (size_t)L.grid * 2 * L.H * D * 4);
-  L.cstats = off;
   L.ulist = off; off = align_up(off + (size_t)L.grid * L.cpc_max * fused::kRec * 4);
-  L.glogits = off;
-  if (L.need_glogits) off = align_up(off + (size_t)L.grid * L.cpc_max * kChunk * L.H * 4);
+  L.glogits = off; off = align_up(off + (size_t)L.grid * L.cpc_max * kChunk * L.H * 4);
   L.gstats = off;
-  if (L.need_gstats) off = align_up(off + (size_t)L.grid * L.cpc_max * 12 * 4);
+  if (L.need_gstats) off = align_up(off + (size_t)L.grid * L.cpc_max * 8 * 12 * 4);
+  L.qbuf = off; off = align_up(off + (size_t)units * L.H * D * 4);
+  L.qgsum = off; off = align_up(off + (size_t)units * L.H * 4 * 4);
   L.total = off;
   return L;
 }
@@ -160,7 +143,7 @@ int run_attention(DecodeArgs& a, int D, int kb, int vb0, int vb1, void* ws, size
   f.cpc_max = L.cpc_max;
   f.stages = L.stages;
   f.ring_bytes = L.ring_bytes;
-  f.smem_logit_floats = L.smem_logit_floats;
+  f.smem_logit_floats = 0;
   f.timeout_ns = reinterpret_cast<const unsigned long long*>(base + 8);
   f.done = reinterpret_cast<int*>(base + 16);
   f.wcounts = reinterpret_cast<unsigned long long*>(base + 32);
@@ -170,8 +153,10 @@ int run_attention(DecodeArgs& a, int D, int kb, int vb0, int vb1, void* ws, size
   f.ppart = reinterpret_cast<float*>(base + L.ppart);
   f.cstats = nullptr;
   f.ulist = reinterpret_cast<int*>(base + L.ulist);
-  f.glogits = L.need_glogits ? reinterpret_cast<float*>(base + L.glogits) : nullptr;
+  f.glogits = reinterpret_cast<float*>(base + L.glogits);
   f.gstats = L.need_gstats ? reinterpret_cast<float*>(base + L.gstats) : nullptr;
+  f.qbuf = reinterpret_cast<float*>(base + L.qbuf);
+  f.qgsum = reinterpret_cast<float*>(base + L.qgsum);
   cudaError_t e;
   switch (kb) {
     case 2: e = launch_fused_k2(f, D, L.H, vb0, vb1, L.smem_bytes, L.grid, s); break;

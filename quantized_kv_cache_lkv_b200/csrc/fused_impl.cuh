@@ -9,24 +9,25 @@
 // A unit's rows are numbered segment 0 first, padded to whole chunks, then
 // segment 1, so a chunk never straddles the two segments.
 //
-//  phase 1  a producer warp streams the K rows of the CTA's chunks through a
-//           ring of shared-memory stages with 1-D bulk copies (TMA, evict-
-//           first in L2) completing on mbarriers.  Three groups of four
-//           consumer warps take the tiles in turn and turn them into base-2
-//           logits for the group's query heads, kept in shared memory, while
-//           tracking each chunk's maximum.
-//  stats    per chunk: sum of exp2(s - max) (logits become e = exp2(s - max));
-//           per unit piece: the merged statistics.  A unit owned by one CTA
-//           needs nothing else; a unit shared by neighbouring CTAs exchanges
-//           piece statistics through the workspace (bounded wait on a
-//           per-unit arrival counter).
-//  phase 2  p = e * exp2(max_chunk - max) / sum.  A (b, h, t) with p < tau is
+//  phase 1  a producer warp streams the K rows of the CTA's chunks, tile by
+//           tile, with 1-D bulk copies (TMA, evict-first in L2) into a
+//           two-deep ring of shared-memory stages per consumer warp.  A
+//           consumer lane computes whole rows (two per tile), so the 512
+//           multiply-adds of a row need no cross-lane reduction; q is read
+//           as warp-uniform broadcasts.  Each tile's per-head maximum and sum
+//           of exp2 are reduced in the warp, and e = exp2(s - max_tile) is
+//           written to an L2-resident workspace.
+//  stats    per unit piece: the merged tile statistics.  A unit owned by one
+//           CTA needs nothing else; a unit shared by neighbouring CTAs
+//           exchanges piece statistics through the workspace (bounded wait
+//           on a per-unit arrival counter).
+//  phase 2  p = e * exp2(max_tile - max) / sum.  A (b, h, t) with p < tau is
 //           skipped; the V rows some head keeps are listed per warp in row
 //           order, gathered from HBM and accumulated as p * vhat.  Shared
 //           units publish partial outputs; the last CTA to arrive adds them.
 //
 // Dequantization is folded into the dot products: codes become exact
-// integers (unpack16_int) and, with the group's (scale, zero),
+// integers (unpack) and, with the group's (scale, zero),
 //   sum_d q_d * (scale * c_d + zero) = scale * sum_d q_d c_d + zero * sum_d q_d.
 #pragma once
 #include <cfloat>
@@ -36,28 +37,58 @@
 namespace lkv {
 namespace fused {
 
-constexpr int kGroupWarps = 4;                 // consumer warps sharing a tile
-constexpr int kGroups = 3;                     // tiles are dealt to groups in turn
-constexpr int kConsumerWarps = kGroupWarps * kGroups;
-constexpr int kConsumers = kConsumerWarps * 32;
-constexpr int kThreads = kConsumers + 32;      // + producer warp
-constexpr int kChunk = 256;    // tokens per chunk (softmax statistics granularity)
-constexpr int kTile = 64;      // tokens per bulk-copy tile
-constexpr int kMaxStages = 15; // multiple of kGroups
+constexpr int kChunk = 256;    // tokens per chunk (work-partition granularity)
+constexpr int kSlotsPerWarp = 2;
+constexpr int kMaxConsumerWarps = 12;
 constexpr int kListCap = 512;  // V-row list entries per warp per batch
 constexpr int kBatchBlocks = kListCap / 32;
 constexpr int kRec = 16;       // ints per unit-list record
 constexpr int kGatherUnroll = 2;
-constexpr int kCsCap = 64;     // chunk statistics kept in shared memory up to this many chunks
+constexpr int kTsCap = 128;    // tile statistics kept in shared memory up to this many tiles
+constexpr int kQSlots = 4;     // units whose prescaled q is staged in shared memory
 constexpr unsigned kFull = 0xFFFFFFFFu;
 constexpr int kBarCons = 1;    // named barrier of the consumer warps
-constexpr int kHeader = 4096;  // bytes of shared memory before the ring
+// Shared header (bytes): barriers [0, 512), unused [512, 1536),
+// misc ints [1536, 2048), tile statistics [2048, 8192), q of up to kQSlots
+// units [8192, 16384).
+constexpr int kMiscOff = 1536;
+constexpr int kTsOff = 2048;
+constexpr int kQOff = 8192;
+constexpr int kHeader = 16384;
 
-// Shared header layout (bytes): barriers [0, 256), tile descriptors
-// [256, 768), misc ints [768, 1024), chunk statistics [1024, 4096).
-constexpr int kDescOff = 256;
-constexpr int kMiscOff = 768;
-constexpr int kCsOff = 1024;
+// Compile-time geometry of one instantiation.
+template <int D, int KB>
+struct Geo {
+  static constexpr int RB = D * KB / 8;                       // packed K row bytes
+  static constexpr int RW = RB / 4;                           // ... in 32-bit words
+  static constexpr int RPL = RW <= 24 ? 2 : 1;                // rows per lane in a tile
+  static constexpr int kTileRows = 32 * RPL;
+  static constexpr int kTilesPerChunk = kChunk / kTileRows;
+  static constexpr int kCW = RPL == 2 ? 12 : 8;               // consumer warps
+  static constexpr int kConsumers = kCW * 32;
+  static constexpr int kThreads = kConsumers;                 // every warp streams its own tiles
+  static constexpr int kStages = kCW * kSlotsPerWarp;
+  static constexpr int kStageCodes = kTileRows * RB;
+  static constexpr int kStageSz = (kTileRows + 2) * (D / 32) * 8;  // ng <= D/32, plus alignment rows
+  static constexpr int kStageBytes = (kStageCodes + kStageSz + 127) / 128 * 128;
+  static constexpr int kDimsPerWord = 32 / KB;                // not used for 6-bit
+};
+
+// Host-side view of the geometry (the same formulas as Geo).
+struct GeoHost {
+  int threads, stages, stage_bytes, tile_rows, consumer_warps;
+};
+inline GeoHost geo_host(int D, int KB) {
+  const int rb = D * KB / 8, rw = rb / 4;
+  const int rpl = rw <= 24 ? 2 : 1;
+  GeoHost g;
+  g.tile_rows = 32 * rpl;
+  g.consumer_warps = rpl == 2 ? 12 : 8;
+  g.threads = g.consumer_warps * 32;
+  g.stages = g.consumer_warps * kSlotsPerWarp;
+  g.stage_bytes = (g.tile_rows * rb + (g.tile_rows + 2) * (D / 32) * 8 + 127) / 128 * 128;
+  return g;
+}
 
 // Unit-list record (ints): u, first chunk, chunks, n0, n1, owned, chunks of
 // segment 0, -, then (max, sum) of the CTA's piece for up to 4 heads as floats.
@@ -90,13 +121,6 @@ __device__ __forceinline__ void merge_ml(float& m, float& l, float m2, float l2)
   m = M;
 }
 
-// Order-preserving map of floats to ints (for atomicMax on floats).
-__device__ __forceinline__ int f2ord(float f) {
-  const int i = __float_as_int(f);
-  return i >= 0 ? i : i ^ 0x7FFFFFFF;
-}
-__device__ __forceinline__ float ord2f(int i) { return __int_as_float(i >= 0 ? i : i ^ 0x7FFFFFFF); }
-
 // Rows of chunk c (unit coordinates) and where they live.
 struct ChunkRows {
   int seg, row0, rows;  // segment, first row inside the segment, valid rows
@@ -112,16 +136,6 @@ __device__ __forceinline__ ChunkRows chunk_rows(const Unit& x, int c) {
   return r;
 }
 
-template <int D, int KB>
-struct Geo {
-  static constexpr int LPR = D / kDimsPerLane;  // lanes per row
-  static constexpr int RPW = 32 / LPR;          // rows per warp step
-  static constexpr int RB = D * KB / 8;         // packed K row bytes
-  static constexpr int kStageCodes = kTile * RB;
-  static constexpr int kStageSz = (kTile + 2) * (D / 32) * 8;  // ng <= D/32, plus alignment rows
-  static constexpr int kStageBytes = (kStageCodes + kStageSz + 127) / 128 * 128;
-};
-
 // Bounded spin on a counter written by other CTAs.
 __device__ __forceinline__ bool wait_counter(const int* p, int target, uint64_t limit_ns) {
   if (ld_acquire(p) >= target) return true;
@@ -131,39 +145,6 @@ __device__ __forceinline__ bool wait_counter(const int* p, int target, uint64_t 
     if (ld_acquire(p) >= target) return true;
     if (global_ns() - t0 > limit_ns) return false;
   }
-}
-
-template <int NH, int OFF>
-struct ReduceScatter {
-  static __device__ __forceinline__ void run(float* v, int lane, int& hidx) {
-    if constexpr (OFF >= 1) {
-      if constexpr (NH > 1) {
-        constexpr int half = NH / 2;
-        const bool up = (lane & OFF) != 0;
-#pragma unroll
-        for (int i = 0; i < half; ++i) {
-          const float send = up ? v[i] : v[half + i];
-          const float keep = up ? v[half + i] : v[i];
-          v[i] = keep + __shfl_xor_sync(kFull, send, OFF);
-        }
-        if (up) hidx += half;
-        ReduceScatter<half, OFF / 2>::run(v, lane, hidx);
-      } else {
-        v[0] += __shfl_xor_sync(kFull, v[0], OFF);
-        ReduceScatter<1, OFF / 2>::run(v, lane, hidx);
-      }
-    }
-  }
-};
-
-template <int H, int LPR>
-__device__ __forceinline__ int head_of_lane(int lane) {
-  float dummy[H];
-#pragma unroll
-  for (int h = 0; h < H; ++h) dummy[h] = 0.0f;
-  int hidx = 0;
-  ReduceScatter<H, LPR / 2>::run(dummy, lane, hidx);
-  return hidx;
 }
 
 template <int H>
@@ -180,6 +161,19 @@ __device__ __forceinline__ void load_heads(const float* p, float (&x)[H]) {
 }
 
 template <int H>
+__device__ __forceinline__ void ldcg_heads(const float* p, float (&x)[H]) {
+  if constexpr (H == 4) {
+    const float4 v = __ldcg(reinterpret_cast<const float4*>(p));
+    x[0] = v.x; x[1] = v.y; x[2] = v.z; x[3] = v.w;
+  } else if constexpr (H == 2) {
+    const float2 v = __ldcg(reinterpret_cast<const float2*>(p));
+    x[0] = v.x; x[1] = v.y;
+  } else {
+    x[0] = __ldcg(p);
+  }
+}
+
+template <int H>
 __device__ __forceinline__ void store_heads(float* p, const float (&x)[H]) {
   if constexpr (H == 4) {
     *reinterpret_cast<float4*>(p) = make_float4(x[0], x[1], x[2], x[3]);
@@ -190,17 +184,18 @@ __device__ __forceinline__ void store_heads(float* p, const float (&x)[H]) {
   }
 }
 
-// Exponent fields of the unpack's magic floats, kept in registers so that
-// each code costs a single AND-OR (an immediate mask plus this register).
+// Exponent fields of the unpack's magic floats, kept in registers so that a
+// code costs a single AND-OR (an immediate mask plus this register).
 template <int BITS>
 struct Magic {
-  uint32_t m[32];
+  uint32_t m[24];
   __device__ __forceinline__ void load(const int* src) {
 #pragma unroll
     for (int k = 0; k < 24 - BITS; ++k) m[k] = (uint32_t)src[k];
   }
 };
 
+// Code I of a 16-code lane slice, plus its magic constant 2^(23-kk).
 template <int BITS, int I>
 __device__ __forceinline__ float code_plus_magic_r(const LaneWords<BITS>& lw, const Magic<BITS>& mg) {
   constexpr int s = copy_shift<BITS>(I);
@@ -209,6 +204,7 @@ __device__ __forceinline__ float code_plus_magic_r(const LaneWords<BITS>& lw, co
   return __uint_as_float((stream_bits<BITS>(lw, s) & mask) | mg.m[kk]);
 }
 
+// Codes (2P, 2P+1) of the slice as exact floats.
 template <int BITS, int P>
 __device__ __forceinline__ float2 code_pair_r(const LaneWords<BITS>& lw, const Magic<BITS>& mg) {
   const float2 m = make_float2(code_plus_magic_r<BITS, 2 * P>(lw, mg), code_plus_magic_r<BITS, 2 * P + 1>(lw, mg));
@@ -251,32 +247,46 @@ __device__ __forceinline__ void accumulate_v(const LaneWords<VB>& lw, const Magi
 }
 
 struct TileDesc {
-  int kk, seg, row0, rows, entry, pad0, pad1, pad2;
+  int slot, seg, row0, rows, entry, u;
 };
+
+// Pair P (0..7) of a 16-code slice; P is a constant once loops are unrolled.
+template <int BITS>
+__device__ __forceinline__ float2 code_pair_at(const LaneWords<BITS>& lw, const Magic<BITS>& mg, int P) {
+  switch (P) {
+    case 0: return code_pair_r<BITS, 0>(lw, mg);
+    case 1: return code_pair_r<BITS, 1>(lw, mg);
+    case 2: return code_pair_r<BITS, 2>(lw, mg);
+    case 3: return code_pair_r<BITS, 3>(lw, mg);
+    case 4: return code_pair_r<BITS, 4>(lw, mg);
+    case 5: return code_pair_r<BITS, 5>(lw, mg);
+    case 6: return code_pair_r<BITS, 6>(lw, mg);
+    default: return code_pair_r<BITS, 7>(lw, mg);
+  }
+}
 
 // ------------------------------------------------------------------ kernel
 
 template <int D, int H, int KB, int VB0, int VB1>
-__global__ void __launch_bounds__(kThreads, 1) fused_decode_kernel(FusedArgs a) {
+__global__ void __launch_bounds__(Geo<D, KB>::kThreads, 1) fused_decode_kernel(FusedArgs a) {
   using Gk = Geo<D, KB>;
-  constexpr int LPR = Gk::LPR, RPW = Gk::RPW;
+  constexpr int CW = Gk::kCW, NCONS = Gk::kConsumers, NTHR = Gk::kThreads;
+  constexpr int RPL = Gk::RPL, TR = Gk::kTileRows, TPC = Gk::kTilesPerChunk;
+  constexpr int LPR = D / kDimsPerLane, RPW = 32 / LPR;  // phase-2 lane mapping (16 channels per lane)
+  constexpr int CH = D / 16, NW = KB / 2;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int cta = blockIdx.x, grid = gridDim.x;
   const DecodeArgs& d = a.d;
   const int units = d.B * d.Hkv;
   const int ng = D / d.G;
-  const int S = a.stages;
   const uint64_t limit_ns = (a.timeout_ns && *a.timeout_ns) ? *a.timeout_ns : 2000000000ull;
-  const int j = lane % LPR;                 // lane's 16-channel slice of a row
+  const int j = lane % LPR;                 // phase 2: lane's 16-channel slice of a row
   const int gi = (j * kDimsPerLane) / d.G;  // its quantization group
 
   uint64_t* full = reinterpret_cast<uint64_t*>(smem_raw);
-  uint64_t* empty = full + kMaxStages;
-  TileDesc* desc = reinterpret_cast<TileDesc*>(smem_raw + kDescOff);
-  int* misc = reinterpret_cast<int*>(smem_raw + kMiscOff);   // 64 ints
+  int* misc = reinterpret_cast<int*>(smem_raw + kMiscOff);  // 128 ints
   uint8_t* ring = smem_raw + kHeader;
-  float* s_logits = reinterpret_cast<float*>(ring + a.ring_bytes);
 
   int& s_total = misc[0];
   int& s_e0 = misc[1];
@@ -285,15 +295,12 @@ __global__ void __launch_bounds__(kThreads, 1) fused_decode_kernel(FusedArgs a) 
   int& s_carry_c = misc[4];
   int& s_carry_n = misc[5];
   int& s_last = misc[6];
-  float* s_glob = reinterpret_cast<float*>(misc + 8);   // (max, 1/sum) x 4 heads
-  int* s_wsum = misc + 16;                             // 2 x 12 warp partials
-  int* s_magic = misc + 40;                            // 24 magic exponent fields
+  float* s_glob = reinterpret_cast<float*>(misc + 8);  // (max, 1/sum) x 4 heads
+  int* s_wsum = misc + 16;                            // 2 x 12 warp partials
+  int* s_magic = misc + 48;                           // 24 magic exponent fields
 
   if (tid == 0) {
-    for (int s = 0; s < S; ++s) {
-      mbar_init(&full[s], 1);
-      mbar_init(&empty[s], kGroupWarps);
-    }
+    for (int s = 0; s < Gk::kStages; ++s) mbar_init(&full[s], 1);
     fence_mbar_init();
     s_total = 0; s_e0 = 0; s_nent = 0; s_abort = 0; s_carry_c = 0; s_carry_n = 0; s_last = 0;
   }
@@ -301,10 +308,10 @@ __global__ void __launch_bounds__(kThreads, 1) fused_decode_kernel(FusedArgs a) 
   __syncthreads();
 
   // ------------------------------------------------------------ unit list
-  const bool consumer = warp < kConsumerWarps;
+  const bool consumer = warp < CW;
   if (consumer) {
     int part = 0;
-    for (int u = tid; u < units; u += kConsumers) {
+    for (int u = tid; u < units; u += NCONS) {
       int n0, n1;
       unit_lens(d, u, n0, n1);
       part += chunks_of(n0) + chunks_of(n1);
@@ -334,9 +341,10 @@ __global__ void __launch_bounds__(kThreads, 1) fused_decode_kernel(FusedArgs a) 
   const int cpc = (total + grid - 1) / grid;
   const int k0 = min(cta * cpc, total), k1 = min(k0 + cpc, total);
   const int nck = k1 - k0;
+  const int ntile = nck * TPC;
   int* ulist = a.ulist + (long long)cta * a.cpc_max * kRec;
   if (consumer) {
-    for (int base = 0; base < units; base += kConsumers) {
+    for (int base = 0; base < units; base += NCONS) {
       const int u = base + tid;
       int n0 = 0, n1 = 0;
       if (u < units) unit_lens(d, u, n0, n1);
@@ -349,17 +357,17 @@ __global__ void __launch_bounds__(kThreads, 1) fused_decode_kernel(FusedArgs a) 
         const int y = __shfl_up_sync(kFull, sc, off), z = __shfl_up_sync(kFull, sn, off);
         if (lane >= off) { sc += y; sn += z; }
       }
-      if (lane == 31) { s_wsum[warp] = sc; s_wsum[12 + warp] = sn; }
-      named_barrier(kBarCons, kConsumers);
+      if (lane == 31) { s_wsum[warp] = sc; s_wsum[16 + warp] = sn; }
+      named_barrier(kBarCons, NCONS);
       int wc = 0, wn = 0, tc = 0, tn = 0;
-      for (int w = 0; w < kConsumerWarps; ++w) {
-        if (w < warp) { wc += s_wsum[w]; wn += s_wsum[12 + w]; }
-        tc += s_wsum[w]; tn += s_wsum[12 + w];
+      for (int w = 0; w < CW; ++w) {
+        if (w < warp) { wc += s_wsum[w]; wn += s_wsum[16 + w]; }
+        tc += s_wsum[w]; tn += s_wsum[16 + w];
       }
       const int cb = s_carry_c + wc + sc - nc;
       const int ne_idx = s_carry_n + wn + sn - ne;
       if (ne && cb <= k0 && k0 < cb + nc) s_e0 = ne_idx;
-      named_barrier(kBarCons, kConsumers);
+      named_barrier(kBarCons, NCONS);
       if (ne && cb < k1 && cb + nc > k0) {
         const int idx = ne_idx - s_e0;
         int* rec = ulist + (long long)idx * kRec;
@@ -368,212 +376,263 @@ __global__ void __launch_bounds__(kThreads, 1) fused_decode_kernel(FusedArgs a) 
         rec[6] = nc0;
         atomicMax(&s_nent, idx + 1);
       }
-      named_barrier(kBarCons, kConsumers);
+      named_barrier(kBarCons, NCONS);
       if (tid == 0) { s_carry_c += tc; s_carry_n += tn; }
-      named_barrier(kBarCons, kConsumers);
+      named_barrier(kBarCons, NCONS);
     }
   }
-  // chunk statistics: in shared memory unless the CTA has many chunks
-  int* cmx;
-  float *csm, *cfc;
-  if (nck <= kCsCap) {
-    cmx = reinterpret_cast<int*>(smem_raw + kCsOff);
-    csm = reinterpret_cast<float*>(cmx + kCsCap * 4);
-    cfc = csm + kCsCap * 4;
+  // tile statistics (max, sum, factor per head): shared memory unless many tiles
+  float* tsm;
+  float* tsl;
+  float* tsf;
+  if (ntile <= kTsCap) {
+    tsm = reinterpret_cast<float*>(smem_raw + kTsOff);
+    tsl = tsm + kTsCap * 4;
+    tsf = tsl + kTsCap * 4;
   } else {
-    cmx = reinterpret_cast<int*>(a.gstats + (long long)cta * a.cpc_max * 12);
-    csm = reinterpret_cast<float*>(cmx + a.cpc_max * 4);
-    cfc = csm + a.cpc_max * 4;
+    tsm = a.gstats + (long long)cta * a.cpc_max * 8 * 12;
+    tsl = tsm + a.cpc_max * 8 * 4;
+    tsf = tsl + a.cpc_max * 8 * 4;
   }
-  for (int i = tid; i < nck * H; i += kThreads) cmx[i] = f2ord(-INFINITY);
-  __syncthreads();  // list complete, maxima reset
+  for (int i = tid; i < ntile * H; i += NTHR) { tsm[i] = -INFINITY; tsl[i] = 0.0f; }
+  __syncthreads();  // list complete
   const int nent = s_nent;
+  // prescaled q of the CTA's units and its per-group sums (one warp per (unit, head))
+  if (consumer) {
+    constexpr int DPL = D / 32;  // channels per lane
+    for (int task = warp; task < nent * H; task += CW) {
+      const int e = task / H, h = task % H;
+      const Unit x = load_unit(ulist + (long long)e * kRec);
+      const int b = x.u / d.Hkv, g = x.u % d.Hkv;
+      const uint16_t* qs = d.q + ((long long)b * d.Hq + g * H + h) * D + lane * DPL;
+      float* qd = (e < kQSlots ? reinterpret_cast<float*>(smem_raw + kQOff) + e * H * D
+                               : a.qbuf + (long long)x.u * H * D) + h * D + lane * DPL;
+      float s = 0.0f;
+#pragma unroll
+      for (int i = 0; i < DPL; ++i) {
+        const float v = __uint_as_float(((uint32_t)qs[i]) << 16) * d.q_scale;
+        qd[i] = v;
+        s += v;
+      }
+      const int lpg = d.G / DPL;  // lanes per quantization group
+      for (int off = 1; off < lpg; off <<= 1) s += __shfl_xor_sync(kFull, s, off);
+      if (lane % lpg == 0) a.qgsum[((long long)x.u * H + h) * 4 + lane / lpg] = s;
+    }
+  }
+  __syncthreads();  // q ready; phase 1 starts
 
-  float* lg = ((long long)nck * kChunk * H <= a.smem_logit_floats)
-                  ? s_logits
-                  : a.glogits + (long long)cta * a.cpc_max * kChunk * H;
+  float* lg = a.glogits + (long long)cta * a.cpc_max * kChunk * H;  // [slot][H], slot = kk * kChunk + row
 
   // ------------------------------------------------------------ phase 1
-  if (!consumer) {
-    if (lane == 0) {
-      const uint64_t pol = policy_evict_first();
-      int t = 0;
-      bool ok = true;
-      auto acquire_stage = [&](int tt) -> bool {
-        if (tt < S) return true;
-        const int st = tt % S;
-        if (mbar_wait(&empty[st], ((tt / S) - 1) & 1, limit_ns)) return true;
-        atomicExch(d.status, kStatusTimeout);
-        atomicExch(&s_abort, 1);
-        return false;
-      };
-      for (int e = 0; e < nent && ok; ++e) {
-        const Unit x = load_unit(ulist + (long long)e * kRec);
-        const long long ubase = (long long)x.u * d.T_cap;
-        const int ga = max(x.cb, k0), gb = min(x.cb + x.nc, k1);
-        for (int g = ga; g < gb && ok; ++g) {
-          const ChunkRows cr = chunk_rows(x, g - x.cb);
-          for (int r = 0; r < cr.rows && ok; r += kTile) {
-            const int rows = min(kTile, cr.rows - r);
-            const int row = cr.row0 + r;
-            if (!acquire_stage(t)) { ok = false; break; }
-            const int stage = t % S;
-            const int r0 = (ng == 1) ? (row & ~1) : row;
-            const int r1 = (ng == 1) ? ((row + rows + 1) & ~1) : row + rows;
-            const uint32_t cbytes = (uint32_t)rows * Gk::RB;
-            const uint32_t sbytes = (uint32_t)(r1 - r0) * ng * 8;
-            TileDesc td;
-            td.kk = g - k0; td.seg = cr.seg; td.row0 = row; td.rows = rows; td.entry = e;
-            desc[stage] = td;
-            uint8_t* dst = ring + (size_t)stage * Gk::kStageBytes;
-            mbar_arrive_expect_tx(&full[stage], cbytes + sbytes);
-            bulk_g2s(dst, d.kc[cr.seg] + (ubase + row) * Gk::RB, cbytes, &full[stage], pol);
-            bulk_g2s(dst + Gk::kStageCodes, d.ksz[cr.seg] + (ubase + r0) * ng * 2, sbytes, &full[stage], pol);
-            ++t;
-          }
-        }
-      }
-      // one end marker per consumer group (a plain arrival completes the phase)
-      for (int k = 0; k < kGroups && ok; ++k) {
-        if (!acquire_stage(t)) { ok = false; break; }
-        const int stage = t % S;
-        desc[stage].rows = -1;
-        mbar_arrive(&full[stage]);
-        ++t;
-      }
-      // Never leave copies in flight: wait for the last stages issued.
-      for (int k = max(0, t - S); k < t; ++k) mbar_wait(&full[k % S], (k / S) & 1, limit_ns);
-    }
-    return;  // the producer warp takes no further part
-  }
-
-  // consumers
+  // Warp w takes tiles w, w + CW, ... of the CTA (tile t = chunk t / TPC,
+  // rows (t % TPC) * TR ...) and keeps two of them in flight in its own two
+  // ring stages, issuing each bulk copy itself.
   {
-    const int grp = warp / kGroupWarps, wig = warp % kGroupWarps;
-    const int hidx_lane = head_of_lane<H, LPR>(lane);
-    const bool leader = (lane % (LPR / H)) == 0;
     Magic<KB> mg;
     mg.load(s_magic);
-    float2 qf[H][8];
-    float Q[H];
-    int cur_e = -1;
+    const uint64_t pol = policy_evict_first();
     volatile int* abort_flag = &s_abort;
-    for (int t = grp;; t += kGroups) {
-      const int stage = t % S;
+    int nt = warp, ent = 0;
+    // next non-empty tile of this warp, or false
+    auto next_tile = [&](TileDesc& td) -> bool {
+      while (nt < ntile) {
+        const int t = nt;
+        nt += CW;
+        const int g = k0 + t / TPC, sub = t % TPC;
+        while (ent + 1 < nent && ulist[(long long)(ent + 1) * kRec + 1] <= g) ++ent;
+        const Unit x = load_unit(ulist + (long long)ent * kRec);
+        const ChunkRows cr = chunk_rows(x, g - x.cb);
+        const int rows = min(TR, cr.rows - sub * TR);
+        if (rows > 0) {
+          td.slot = t; td.seg = cr.seg; td.row0 = cr.row0 + sub * TR; td.rows = rows; td.entry = ent;
+          td.u = x.u;
+          return true;
+        }
+      }
+      return false;
+    };
+    auto issue = [&](const TileDesc& td, int stage) {
+      if (lane == 0) {
+        const long long ubase = (long long)td.u * d.T_cap;
+        const int row = td.row0, rows = td.rows;
+        const int r0 = (ng == 1) ? (row & ~1) : row;
+        const int r1 = (ng == 1) ? ((row + rows + 1) & ~1) : row + rows;
+        const uint32_t cbytes = (uint32_t)rows * Gk::RB;
+        const uint32_t sbytes = (uint32_t)(r1 - r0) * ng * 8;
+        uint8_t* dst = ring + (size_t)stage * Gk::kStageBytes;
+        mbar_arrive_expect_tx(&full[stage], cbytes + sbytes);
+        bulk_g2s(dst, d.kc[td.seg] + (ubase + row) * Gk::RB, cbytes, &full[stage], pol);
+        bulk_g2s(dst + Gk::kStageCodes, d.ksz[td.seg] + (ubase + r0) * ng * 2, sbytes, &full[stage], pol);
+      }
+    };
+    TileDesc p0, p1;
+    int issued = 0, consumed = 0;
+    if (next_tile(p0)) { issue(p0, warp * kSlotsPerWarp + 0); ++issued; }
+    if (issued == 1 && next_tile(p1)) { issue(p1, warp * kSlotsPerWarp + 1); ++issued; }
+    int cur_e = -1;
+    const float* qv = nullptr;
+    const float* qg = nullptr;
+    while (consumed < issued) {
+      const int slotw = consumed % kSlotsPerWarp;
+      const int stage = warp * kSlotsPerWarp + slotw;
       if (*abort_flag) break;
-      if (!mbar_wait(&full[stage], (t / S) & 1, limit_ns)) {
+      if (!mbar_wait(&full[stage], (consumed / kSlotsPerWarp) & 1, limit_ns)) {
         atomicExch(d.status, kStatusTimeout);
         atomicExch(&s_abort, 1);
         break;
       }
-      const TileDesc td = desc[stage];
-      if (td.rows < 0) break;
+      const TileDesc td = slotw ? p1 : p0;
       if (td.entry != cur_e) {
         cur_e = td.entry;
-        const Unit x = load_unit(ulist + (long long)cur_e * kRec);
-        const int b = x.u / d.Hkv, g = x.u % d.Hkv;
-#pragma unroll
-        for (int h = 0; h < H; ++h) {
-          float xq[16];
-          load16_bf16(d.q + ((long long)b * d.Hq + g * H + h) * D + j * kDimsPerLane, xq);
-          float s = 0.0f;
-#pragma unroll
-          for (int i = 0; i < 8; ++i) {
-            qf[h][i] = make_float2(xq[2 * i] * d.q_scale, xq[2 * i + 1] * d.q_scale);
-            s += qf[h][i].x + qf[h][i].y;
-          }
-          Q[h] = s;
-        }
+        const int u = td.u;
+        qv = cur_e < kQSlots ? reinterpret_cast<const float*>(smem_raw + kQOff) + cur_e * H * D
+                             : a.qbuf + (long long)u * H * D;
+        qg = a.qgsum + (long long)u * H * 4;
       }
       const uint8_t* codes = ring + (size_t)stage * Gk::kStageBytes;
       const float* szs = reinterpret_cast<const float*>(codes + Gk::kStageCodes) +
                          ((ng == 1) ? (td.row0 & 1) : 0) * ng * 2;
-      float* lgt = lg + (td.kk * kChunk + (td.row0 % kChunk)) * H;
-      const int nrs = (td.rows + RPW - 1) / RPW;
-      float tmax = -INFINITY;
-      for (int rs = wig; rs < nrs; rs += kGroupWarps) {
-        const int i = rs * RPW + lane / LPR;
-        const bool valid = i < td.rows;
-        float dot[H];
+      bool valid[RPL];
+      const uint4* src[RPL];
 #pragma unroll
-        for (int h = 0; h < H; ++h) dot[h] = 0.0f;
-        if (valid) {
-          LaneWords<KB> lw;
-          lds_lane_words<KB>(codes + i * Gk::RB + j * (2 * KB), lw);
-          const float2 sz = *reinterpret_cast<const float2*>(szs + (i * ng + gi) * 2);
-          float2 c[8];
-          unpack16_int_r<KB>(lw, mg, c);
+      for (int r = 0; r < RPL; ++r) {
+        const int i = lane + 32 * r;
+        valid[r] = i < td.rows;
+        src[r] = reinterpret_cast<const uint4*>(codes + (valid[r] ? i : 0) * Gk::RB);
+      }
+      float dot[RPL][H];
+      float2 acc[RPL][H];
 #pragma unroll
-          for (int h = 0; h < H; ++h) {
-            float2 acc = make_float2(0.0f, 0.0f);
+      for (int r = 0; r < RPL; ++r)
 #pragma unroll
-            for (int p = 0; p < 8; ++p) acc = __ffma2_rn(qf[h][p], c[p], acc);
-            dot[h] = fmaf(sz.x, acc.x + acc.y, sz.y * Q[h]);
+        for (int h = 0; h < H; ++h) { dot[r][h] = 0.0f; acc[r][h] = make_float2(0.0f, 0.0f); }
+      // q of the next 4-channel block, fetched one block ahead
+      float4 qn[H];
+#pragma unroll
+      for (int h = 0; h < H; ++h) qn[h] = *reinterpret_cast<const float4*>(qv + h * D);
+      constexpr int SW = 2 * KB;  // words of 64 channels of a row
+#pragma unroll
+      for (int sgm = 0; sgm < D / 64; ++sgm) {
+        uint32_t w[RPL][SW];
+#pragma unroll
+        for (int r = 0; r < RPL; ++r)
+#pragma unroll
+          for (int q4 = 0; q4 < SW / 4; ++q4) {
+            const uint4 v = src[r][sgm * (SW / 4) + q4];
+            w[r][4 * q4] = v.x; w[r][4 * q4 + 1] = v.y; w[r][4 * q4 + 2] = v.z; w[r][4 * q4 + 3] = v.w;
+          }
+#pragma unroll
+        for (int cc = 0; cc < 4; ++cc) {
+          const int c = sgm * 4 + cc;
+          LaneWords<KB> lw[RPL];
+#pragma unroll
+          for (int r = 0; r < RPL; ++r)
+#pragma unroll
+            for (int k2 = 0; k2 < NW; ++k2) lw[r].w[k2] = w[r][cc * NW + k2];
+#pragma unroll
+          for (int b4 = 0; b4 < 4; ++b4) {
+            const int blk = c * 4 + b4;
+            float4 qc[H];
+#pragma unroll
+            for (int h = 0; h < H; ++h) qc[h] = qn[h];
+            if (blk + 1 < D / 4) {
+#pragma unroll
+              for (int h = 0; h < H; ++h) qn[h] = *reinterpret_cast<const float4*>(qv + h * D + (blk + 1) * 4);
+            }
+            float2 cp[RPL][2];
+#pragma unroll
+            for (int r = 0; r < RPL; ++r) {
+              cp[r][0] = code_pair_at<KB>(lw[r], mg, 2 * b4);
+              cp[r][1] = code_pair_at<KB>(lw[r], mg, 2 * b4 + 1);
+            }
+#pragma unroll
+            for (int h = 0; h < H; ++h)
+#pragma unroll
+              for (int r = 0; r < RPL; ++r) {
+                acc[r][h] = __ffma2_rn(make_float2(qc[h].x, qc[h].y), cp[r][0], acc[r][h]);
+                acc[r][h] = __ffma2_rn(make_float2(qc[h].z, qc[h].w), cp[r][1], acc[r][h]);
+              }
+          }
+          if (((c + 1) * 16) % d.G == 0) {  // end of a quantization group: fold (scale, zero)
+            const int gidx = (c * 16) / d.G;
+            float qsum[H];
+#pragma unroll
+            for (int h = 0; h < H; ++h) qsum[h] = qg[h * 4 + gidx];
+#pragma unroll
+            for (int r = 0; r < RPL; ++r) {
+              const int i = valid[r] ? lane + 32 * r : 0;
+              const float2 sz = *reinterpret_cast<const float2*>(szs + (i * ng + gidx) * 2);
+#pragma unroll
+              for (int h = 0; h < H; ++h) {
+                dot[r][h] = fmaf(sz.x, acc[r][h].x + acc[r][h].y, fmaf(sz.y, qsum[h], dot[r][h]));
+                acc[r][h] = make_float2(0.0f, 0.0f);
+              }
+            }
           }
         }
-        int hidx = 0;
-        ReduceScatter<H, LPR / 2>::run(dot, lane, hidx);
-        if (valid && leader) {
-          lgt[i * H + hidx] = dot[0];
-          tmax = fmaxf(tmax, dot[0]);
+      }
+      // The stage's data is in registers now: refill it with this warp's next tile.
+      ++consumed;
+      fence_proxy_async_smem();
+      __syncwarp();
+      {
+        TileDesc tn;
+        if (next_tile(tn)) {
+          if (slotw) p1 = tn; else p0 = tn;
+          issue(tn, stage);
+          ++issued;
         }
       }
-      // tile maximum per head -> the chunk's running maximum
+      // tile statistics: per-head maximum and sum of exp2 over the tile's rows
+      float tm[H], tl[H];
 #pragma unroll
-      for (int off = LPR; off < 32; off <<= 1) tmax = fmaxf(tmax, __shfl_xor_sync(kFull, tmax, off));
-      if (lane < LPR && leader && tmax > -INFINITY) atomicMax(&cmx[td.kk * H + hidx_lane], f2ord(tmax));
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&empty[stage]);
+      for (int h = 0; h < H; ++h) {
+        float m = -INFINITY;
+#pragma unroll
+        for (int r = 0; r < RPL; ++r) m = valid[r] ? fmaxf(m, dot[r][h]) : m;
+#pragma unroll
+        for (int off = 16; off >= 1; off >>= 1) m = fmaxf(m, __shfl_xor_sync(kFull, m, off));
+        tm[h] = m;
+        float l = 0.0f;
+#pragma unroll
+        for (int r = 0; r < RPL; ++r) {
+          dot[r][h] = exp2f(dot[r][h] - m);
+          l += valid[r] ? dot[r][h] : 0.0f;
+        }
+#pragma unroll
+        for (int off = 16; off >= 1; off >>= 1) l += __shfl_xor_sync(kFull, l, off);
+        tl[h] = l;
+      }
+#pragma unroll
+      for (int r = 0; r < RPL; ++r)
+        if (valid[r]) store_heads<H>(lg + ((long long)td.slot * TR + lane + 32 * r) * H, dot[r]);
+      if (lane < H) {
+        float mv = tm[0], lv = tl[0];
+#pragma unroll
+        for (int h = 1; h < H; ++h) if (lane == h) { mv = tm[h]; lv = tl[h]; }
+        tsm[td.slot * H + lane] = mv;
+        tsl[td.slot * H + lane] = lv;
+      }
     }
+    // Never leave copies in flight (only after an abort can any be pending).
+    for (; consumed < issued; ++consumed)
+      mbar_wait(&full[warp * kSlotsPerWarp + consumed % kSlotsPerWarp], (consumed / kSlotsPerWarp) & 1, limit_ns);
   }
-  named_barrier(kBarCons, kConsumers);
+  named_barrier(kBarCons, NCONS);
   // After a timed-out wait a bulk copy may still land in the ring, which
   // phase 2 reuses: skip straight to the end (the status word says why).
   const bool aborted = *static_cast<volatile int*>(&s_abort) != 0;
   const int n_work = aborted ? 0 : nent;
-  const int n_chunks_work = aborted ? 0 : nck;
-
-  // ------------------------------------------------------------ chunk sums
-  for (int kk = warp; kk < n_chunks_work; kk += kConsumerWarps) {
-    const int g_chunk = k0 + kk;
-    int lo = 0, hi = nent - 1;  // entry holding chunk g_chunk
-    while (lo < hi) {
-      const int mid = (lo + hi + 1) / 2;
-      if (ulist[(long long)mid * kRec + 1] <= g_chunk) lo = mid; else hi = mid - 1;
-    }
-    const Unit x = load_unit(ulist + (long long)lo * kRec);
-    const int rows = chunk_rows(x, g_chunk - x.cb).rows;
-    float* base = lg + (long long)kk * kChunk * H;
-    float m[H], l[H];
-#pragma unroll
-    for (int h = 0; h < H; ++h) { m[h] = ord2f(cmx[kk * H + h]); l[h] = 0.0f; }
-    for (int i = lane; i < rows; i += 32) {
-      float s[H];
-      load_heads<H>(base + (long long)i * H, s);
-#pragma unroll
-      for (int h = 0; h < H; ++h) {
-        s[h] = exp2f(s[h] - m[h]);
-        l[h] += s[h];
-      }
-      store_heads<H>(base + (long long)i * H, s);
-    }
-#pragma unroll
-    for (int h = 0; h < H; ++h)
-#pragma unroll
-      for (int off = 16; off >= 1; off >>= 1) l[h] += __shfl_xor_sync(kFull, l[h], off);
-    if (lane < H) csm[kk * H + lane] = l[lane];
-  }
-  named_barrier(kBarCons, kConsumers);
 
   // ------------------------------------------------------------ piece statistics
-  for (int e = warp; e < n_work; e += kConsumerWarps) {
+  for (int e = warp; e < n_work; e += CW) {
     int* rec = ulist + (long long)e * kRec;
     const Unit x = load_unit(rec);
-    const int ga = max(x.cb, k0), gb = min(x.cb + x.nc, k1);
+    const int ta = (max(x.cb, k0) - k0) * TPC, tb = (min(x.cb + x.nc, k1) - k0) * TPC;
 #pragma unroll
     for (int h = 0; h < H; ++h) {
       float m = -INFINITY, l = 0.0f;
-      for (int g2 = ga + lane; g2 < gb; g2 += 32) merge_ml(m, l, ord2f(cmx[(g2 - k0) * H + h]), csm[(g2 - k0) * H + h]);
+      for (int t2 = ta + lane; t2 < tb; t2 += 32) merge_ml(m, l, tsm[t2 * H + h], tsl[t2 * H + h]);
 #pragma unroll
       for (int off = 16; off >= 1; off >>= 1) {
         const float m2 = __shfl_xor_sync(kFull, m, off), l2 = __shfl_xor_sync(kFull, l, off);
@@ -595,7 +654,7 @@ __global__ void __launch_bounds__(kThreads, 1) fused_decode_kernel(FusedArgs a) 
       }
     }
   }
-  named_barrier(kBarCons, kConsumers);
+  named_barrier(kBarCons, NCONS);
   if (tid == 0 && n_work > 0) {
     __threadfence();  // orders every consumer's statistics before the arrivals
     const Unit x0 = load_unit(ulist);
@@ -607,8 +666,8 @@ __global__ void __launch_bounds__(kThreads, 1) fused_decode_kernel(FusedArgs a) 
   }
 
   // ------------------------------------------------------------ phase 2
-  int* lists = reinterpret_cast<int*>(ring);                                    // [12][kListCap]
-  float* red = reinterpret_cast<float*>(ring + kConsumerWarps * kListCap * 4);  // [12][H][D]
+  int* lists = reinterpret_cast<int*>(ring);                                         // [CW][kListCap]
+  float* red = reinterpret_cast<float*>(ring + kMaxConsumerWarps * kListCap * 4);    // [CW][H][D]
   Magic<VB0> mg0;
   mg0.load(s_magic);
   Magic<VB1> mg1;
@@ -648,18 +707,19 @@ __global__ void __launch_bounds__(kThreads, 1) fused_decode_kernel(FusedArgs a) 
           s_glob[2 * lane + 1] = l > 0.0f ? 1.0f / l : 0.0f;
         }
       }
-      named_barrier(kBarCons, kConsumers);
+      named_barrier(kBarCons, NCONS);
       const int ga = max(x.cb, k0), gb = min(x.cb + x.nc, k1);
-      // per-chunk factors exp2(max_c - max) / sum
-      for (int q = tid; q < (gb - ga) * H; q += kConsumers) {
-        const int kk = ga - k0 + q / H, h = q % H;
+      // per-tile factors exp2(max_tile - max) / sum
+      for (int q = tid; q < (gb - ga) * TPC * H; q += NCONS) {
+        const int t2 = (ga - k0) * TPC + q / H, h = q % H;
         const float M = s_glob[2 * h], il = s_glob[2 * h + 1];
-        cfc[kk * H + h] = (il > 0.0f) ? exp2f(ord2f(cmx[kk * H + h]) - M) * il : 0.0f;
+        const float mt = tsm[t2 * H + h];
+        tsf[t2 * H + h] = (il > 0.0f && mt > -INFINITY) ? exp2f(mt - M) * il : 0.0f;
       }
-      named_barrier(kBarCons, kConsumers);
+      named_barrier(kBarCons, NCONS);
 
-      const float* lgu = lg + (long long)(x.cb - k0) * kChunk * H;
-      const float* cfu = cfc + (x.cb - k0) * H;
+      const float* lgu = lg + (long long)(x.cb - k0) * kChunk * H;   // row v of the unit at lgu[v * H]
+      const float* tfu = tsf + (x.cb - k0) * TPC * H;                 // tile v / TR at tfu[(v / TR) * H]
       const long long ubase = (long long)x.u * d.T_cap;
       const int v_lo = (ga - x.cb) * kChunk, v_hi = (gb - x.cb) * kChunk;  // chunk-aligned (padded) rows
       float2 acc[H][8];
@@ -670,23 +730,22 @@ __global__ void __launch_bounds__(kThreads, 1) fused_decode_kernel(FusedArgs a) 
 #pragma unroll
         for (int i = 0; i < 8; ++i) acc[h][i] = make_float2(0.0f, 0.0f);
       }
-      for (int vb = v_lo; vb < v_hi; vb += kConsumers * kBatchBlocks) {
+      for (int vb = v_lo; vb < v_hi; vb += NCONS * kBatchBlocks) {
         // scan: 32-row blocks round robin over warps, row order kept per warp
         int* list = lists + warp * kListCap;
         int n_w = 0;
-        for (int blk = warp; blk < kConsumerWarps * kBatchBlocks; blk += kConsumerWarps) {
+        for (int blk = warp; blk < CW * kBatchBlocks; blk += CW) {
           if (vb + blk * 32 >= v_hi) break;
           const int v = vb + blk * 32 + lane;
-          const int c = v / kChunk;
-          const ChunkRows cr = chunk_rows(x, c);
+          const ChunkRows cr = chunk_rows(x, v / kChunk);
           bool need = false;
           if (v % kChunk < cr.rows) {
             float ev[H];
-            load_heads<H>(lgu + (long long)v * H, ev);
+            ldcg_heads<H>(lgu + (long long)v * H, ev);
             int nskip = 0;
 #pragma unroll
             for (int h = 0; h < H; ++h) {
-              const float p = ev[h] * cfu[c * H + h];
+              const float p = ev[h] * tfu[(v / TR) * H + h];
               const bool keep = !(p < d.tau);
               need |= keep;
               nskip += keep ? 0 : 1;
@@ -708,39 +767,38 @@ __global__ void __launch_bounds__(kThreads, 1) fused_decode_kernel(FusedArgs a) 
           float2 szv[kGatherUnroll];
           int vv[kGatherUnroll];
 #pragma unroll
-          for (int s = 0; s < kGatherUnroll; ++s) {
-            const int idx = i0 + s * RPW + lane / LPR;
-            vv[s] = idx < n_w ? list[idx] : -1;
-            if (vv[s] >= 0) {
-              const int v = vv[s];
+          for (int s2 = 0; s2 < kGatherUnroll; ++s2) {
+            const int idx = i0 + s2 * RPW + lane / LPR;
+            vv[s2] = idx < n_w ? list[idx] : -1;
+            if (vv[s2] >= 0) {
+              const int v = vv[s2];
               const ChunkRows cr = chunk_rows(x, v / kChunk);
               const long long row = ubase + cr.row0 + v % kChunk;
               if constexpr (kOneWidth) {
-                ldg_v<VB0>(d.vc[cr.seg] + row * (D * VB0 / 8), d.vsz[cr.seg] + row * ng * 2, j, gi, w0[s], szv[s]);
+                ldg_v<VB0>(d.vc[cr.seg] + row * (D * VB0 / 8), d.vsz[cr.seg] + row * ng * 2, j, gi, w0[s2], szv[s2]);
               } else if (cr.seg == 0) {
-                ldg_v<VB0>(d.vc[0] + row * (D * VB0 / 8), d.vsz[0] + row * ng * 2, j, gi, w0[s], szv[s]);
+                ldg_v<VB0>(d.vc[0] + row * (D * VB0 / 8), d.vsz[0] + row * ng * 2, j, gi, w0[s2], szv[s2]);
               } else {
-                ldg_v<VB1>(d.vc[1] + row * (D * VB1 / 8), d.vsz[1] + row * ng * 2, j, gi, w1[s], szv[s]);
+                ldg_v<VB1>(d.vc[1] + row * (D * VB1 / 8), d.vsz[1] + row * ng * 2, j, gi, w1[s2], szv[s2]);
               }
             }
           }
 #pragma unroll
-          for (int s = 0; s < kGatherUnroll; ++s) {
-            const int v = vv[s];
+          for (int s2 = 0; s2 < kGatherUnroll; ++s2) {
+            const int v = vv[s2];
             if (v < 0) continue;
-            const int c = v / kChunk;
-            float ev[H], w[H];
-            load_heads<H>(lgu + (long long)v * H, ev);
+            float ev[H], wgt[H];
+            ldcg_heads<H>(lgu + (long long)v * H, ev);
 #pragma unroll
             for (int h = 0; h < H; ++h) {
-              const float p = ev[h] * cfu[c * H + h];
-              w[h] = (p < d.tau) ? 0.0f : p;
+              const float p = ev[h] * tfu[(v / TR) * H + h];
+              wgt[h] = (p < d.tau) ? 0.0f : p;
             }
             if constexpr (kOneWidth) {
-              accumulate_v<H, VB0>(w0[s], mg0, szv[s], w, acc, Z);
+              accumulate_v<H, VB0>(w0[s2], mg0, szv[s2], wgt, acc, Z);
             } else {
-              if (c < x.nc0) accumulate_v<H, VB0>(w0[s], mg0, szv[s], w, acc, Z);
-              else accumulate_v<H, VB1>(w1[s], mg1, szv[s], w, acc, Z);
+              if (v / kChunk < x.nc0) accumulate_v<H, VB0>(w0[s2], mg0, szv[s2], wgt, acc, Z);
+              else accumulate_v<H, VB1>(w1[s2], mg1, szv[s2], wgt, acc, Z);
             }
           }
         }
@@ -767,37 +825,37 @@ __global__ void __launch_bounds__(kThreads, 1) fused_decode_kernel(FusedArgs a) 
           for (int i = 0; i < 8; ++i)
             *reinterpret_cast<float2*>(red + (warp * H + h) * D + j * kDimsPerLane + 2 * i) = acc[h][i];
       }
-      named_barrier(kBarCons, kConsumers);
-      for (int o = tid; o < H * D; o += kConsumers) {
-        float s = 0.0f;
+      named_barrier(kBarCons, NCONS);
+      for (int o = tid; o < H * D; o += NCONS) {
+        float s2 = 0.0f;
 #pragma unroll
-        for (int w = 0; w < kConsumerWarps; ++w) s += red[w * H * D + o];
+        for (int w2 = 0; w2 < CW; ++w2) s2 += red[w2 * H * D + o];
         const int h = o / D, dd = o % D;
         if (x.owned) {
-          d.out[((long long)b * d.Hq + g * H + h) * D + dd] = s;
+          d.out[((long long)b * d.Hq + g * H + h) * D + dd] = s2;
         } else {
-          if (e == 0) a.ppart[(((long long)cta * 2 + 0) * H + h) * D + dd] = s;
-          if (e == nent - 1) a.ppart[(((long long)cta * 2 + 1) * H + h) * D + dd] = s;
+          if (e == 0) a.ppart[(((long long)cta * 2 + 0) * H + h) * D + dd] = s2;
+          if (e == nent - 1) a.ppart[(((long long)cta * 2 + 1) * H + h) * D + dd] = s2;
         }
       }
       if (!x.owned) {
-        named_barrier(kBarCons, kConsumers);
+        named_barrier(kBarCons, NCONS);
         if (tid == 0) {
           __threadfence();  // every thread's partial before the arrival
           const int old = atomicAdd(a.arrive2 + x.u, 1);
           s_last = (old == i_last - i_first) ? 1 : 0;
         }
-        named_barrier(kBarCons, kConsumers);
+        named_barrier(kBarCons, NCONS);
         if (s_last) {
           __threadfence();
-          for (int o = tid; o < H * D; o += kConsumers) {
-            float s = 0.0f;
+          for (int o = tid; o < H * D; o += NCONS) {
+            float s2 = 0.0f;
             for (int i = i_first; i <= i_last; ++i) {
               const int slot = (i == i_first) ? 1 : 0;
-              s += __ldcg(a.ppart + (((long long)i * 2 + slot) * H) * D + o);
+              s2 += __ldcg(a.ppart + (((long long)i * 2 + slot) * H) * D + o);
             }
             const int h = o / D, dd = o % D;
-            d.out[((long long)b * d.Hq + g * H + h) * D + dd] = s;
+            d.out[((long long)b * d.Hq + g * H + h) * D + dd] = s2;
           }
           if (tid == 0) {
             a.arrive1[x.u] = 0;
@@ -805,7 +863,7 @@ __global__ void __launch_bounds__(kThreads, 1) fused_decode_kernel(FusedArgs a) 
           }
         }
       }
-      named_barrier(kBarCons, kConsumers);
+      named_barrier(kBarCons, NCONS);
     }
   }
 
@@ -821,7 +879,7 @@ __global__ void __launch_bounds__(kThreads, 1) fused_decode_kernel(FusedArgs a) 
       atomicAdd(a.wcounts + 1, cnt_rows);
     }
   }
-  named_barrier(kBarCons, kConsumers);
+  named_barrier(kBarCons, NCONS);
   if (tid == 0) {
     __threadfence();
     const int old = atomicAdd(a.done, 1);

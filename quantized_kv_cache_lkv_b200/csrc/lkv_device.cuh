@@ -296,6 +296,12 @@ __device__ __forceinline__ uint64_t policy_evict_first() {
   return p;
 }
 
+// Orders this thread's earlier shared-memory accesses before later
+// async-proxy (bulk copy) writes to shared memory.
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
 __device__ __forceinline__ void named_barrier(int id, int threads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
 }

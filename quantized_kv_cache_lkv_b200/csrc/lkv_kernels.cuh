@@ -80,7 +80,9 @@ struct FusedArgs {
   float* cstats;                 // [chunks][H][2]
   int* ulist;                    // [grid][cpc_max][16]
   float* glogits;                // [grid][cpc_max * chunk][H] (when shared memory is short)
-  float* gstats;                 // [grid][cpc_max][12] chunk statistics (when there are many chunks)
+  float* gstats;                 // [grid][cpc_max * 8][12] tile statistics (when there are many tiles)
+  float* qbuf;                   // [units][H][D] q * softmax_scale * log2(e)
+  float* qgsum;                  // [units][H][4] sums of qbuf per quantization group
   unsigned long long* wcounts;   // [2] skip-count accumulators
   int* done;                     // CTAs finished
 };
