@@ -167,6 +167,44 @@ LKV_API int lkv_decode_attention(lkv_qspec spec, int B, int Hq, int Hkv, int T_c
                          int64_t *skip_counts, void *workspace, size_t ws_bytes,
                          void *stream);
 
+/*
+ * Size of the fixed device scratch that lkv_decode_attention_static uses:
+ * 32 MiB per device, enough for e.g. B = 16, Hkv = 8, T_cap = 8192, D = 128
+ * with groups of 4 query heads (about 18 MiB on 148 SMs).
+ */
+#define LKV_STATIC_WORKSPACE_BYTES (32u << 20)
+
+/*
+ * lkv_decode_attention_static -- lkv_decode_attention without a caller
+ * workspace and without allocating: its scratch is a fixed array of
+ * LKV_STATIC_WORKSPACE_BYTES bytes of device memory inside the library, one
+ * per device.  The paper has no counterpart; it exists for callers that
+ * cannot hand out device memory (a plain-C host with no device allocator,
+ * or a process whose memory another allocator has reserved in full).
+ * Arguments, outputs and numerics are those of lkv_decode_attention.
+ *
+ *   status  out  nullable device int32: the call's device-side status (an
+ *                lkv_status: LKV_OK, LKV_ERR_INVALID_ARG for a length outside
+ *                [0, T_cap], LKV_ERR_TIMEOUT), written on `stream` after the
+ *                decode.  Bounded waits use the default 2 s limit.
+ *
+ * Returns LKV_ERR_WORKSPACE, before enqueueing anything, when the decode
+ * needs more than LKV_STATIC_WORKSPACE_BYTES (lkv_decode_workspace_bytes
+ * gives the need).  Nothing is allocated or freed.  Each call first clears,
+ * on `stream`, the part of the scratch that must start at zero, so an
+ * earlier failed call leaves nothing behind.  The first call on a device
+ * looks up the scratch's address (which may load the library's device
+ * code); make it before any stream capture.  All calls on one device share
+ * the one scratch: calls that overlap on the GPU (other streams, other host
+ * threads) race and give wrong results, so order them (one stream, or
+ * events).
+ */
+LKV_API int lkv_decode_attention_static(lkv_qspec spec, int B, int Hq, int Hkv, int T_cap, int D,
+                         const int32_t *seq_lens, const void *q, const void *k_codes,
+                         const float *k_sz, const void *v_codes, const float *v_sz,
+                         float softmax_scale, float tau, float *out, uint8_t *skip_mask,
+                         int64_t *skip_counts, int32_t *status, void *stream);
+
 /* Zero-fill a workspace (enqueued on stream). */
 LKV_API int lkv_workspace_reset(void *workspace, size_t ws_bytes, void *stream);
 

@@ -7,6 +7,7 @@
 
 #include "../../include/lkv.h"
 #include <algorithm>
+#include <mutex>
 
 #include "fused_impl.cuh"
 #include "lkv_kernels.cuh"
@@ -196,6 +197,50 @@ bool segment_ok(const lkv_segment& s, bool nonempty) {
 
 using namespace lkv;
 
+// ---------------------------------------------------------------- fixed scratch
+// Scratch of lkv_decode_attention_static: a fixed array of device memory that
+// belongs to this library's module, so that callers which cannot allocate
+// device memory still get a decode.  Examples: a host embedding the library
+// from plain C with no device allocator of its own, or a serving process
+// whose memory is all reserved up front by another allocator, where a new
+// cudaMalloc would fail and a cudaFree would synchronize the whole device.
+// Its size is fixed at LKV_STATIC_WORKSPACE_BYTES; larger decodes are
+// rejected.  Host code never uses the array's name as a device address: the
+// address comes from cudaGetSymbolAddress, looked up once per device.
+static __device__ __align__(256) unsigned char g_static_ws[LKV_STATIC_WORKSPACE_BYTES];
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+std::mutex g_static_mu;
+void* g_static_ptr[kMaxDevices] = {};
+
+// Device address of g_static_ws on the current device; the first call for a
+// device looks it up (with that device current, as it is here).
+int static_scratch(void** ptr) {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess) return LKV_ERR_CUDA;
+  if (dev < 0 || dev >= kMaxDevices) return LKV_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lock(g_static_mu);
+  if (g_static_ptr[dev] == nullptr) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_static_ws) != cudaSuccess || p == nullptr) return LKV_ERR_CUDA;
+    g_static_ptr[dev] = p;
+  }
+  *ptr = g_static_ptr[dev];
+  return LKV_OK;
+}
+
+// Bytes at the start of the scratch that a decode expects to find zero: the
+// status word, the wait limit and the cross-CTA counters.  Everything past
+// them is written before it is read.
+size_t static_zero_prefix(int B, int Hq, int Hkv, int T_cap, int D, int KB) {
+  if (fused_ok(Hq / Hkv)) return fused_layout(B, Hq, Hkv, T_cap, D, KB).pstats;
+  return kHeaderBytes;
+}
+
+}  // namespace
+
 extern "C" {
 
 const char* lkv_status_string(int status) {
@@ -284,6 +329,54 @@ int lkv_decode_attention(lkv_qspec spec, int B, int Hq, int Hkv, int T_cap, int 
   a.skip_mask = skip_mask;
   a.skip_counts = reinterpret_cast<unsigned long long*>(skip_counts);
   return run_attention(a, D, spec.k_bits, spec.v_bits, spec.v_bits, workspace, ws_bytes, s);
+}
+
+int lkv_decode_attention_static(lkv_qspec spec, int B, int Hq, int Hkv, int T_cap, int D, const int32_t* seq_lens,
+                                const void* q, const void* k_codes, const float* k_sz, const void* v_codes,
+                                const float* v_sz, float softmax_scale, float tau, float* out,
+                                uint8_t* skip_mask, int64_t* skip_counts, int32_t* status, void* stream) {
+  if (!bits_ok(spec.k_bits) || !bits_ok(spec.v_bits)) return LKV_ERR_UNSUPPORTED;
+  int rc = check_attention_shape(B, Hq, Hkv, T_cap, D, spec.group);
+  if (rc) return rc;
+  if (!std::isfinite(softmax_scale) || std::isnan(tau)) return LKV_ERR_INVALID_ARG;
+  const bool ne = (long long)B * Hkv * T_cap > 0;
+  if (!ptr_ok(seq_lens, B > 0) || !ptr_ok(q, B > 0) || !ptr_ok(out, B > 0) || !ptr_ok(k_codes, ne) ||
+      !ptr_ok(k_sz, ne) || !ptr_ok(v_codes, ne) || !ptr_ok(v_sz, ne))
+    return LKV_ERR_INVALID_ARG;
+  if (skip_counts && !aligned16(skip_counts)) return LKV_ERR_INVALID_ARG;
+  if (status && (reinterpret_cast<uintptr_t>(status) & 3u) != 0) return LKV_ERR_INVALID_ARG;
+  const size_t need = attention_ws_bytes(B, Hq, Hkv, T_cap, D, spec.k_bits);
+  if (need > (size_t)LKV_STATIC_WORKSPACE_BYTES) return LKV_ERR_WORKSPACE;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (B == 0) {
+    if (skip_counts) rc = from_cuda(cudaMemsetAsync(skip_counts, 0, 2 * sizeof(int64_t), s));
+    if (rc == LKV_OK && status) rc = from_cuda(cudaMemsetAsync(status, 0, sizeof(int32_t), s));
+    return rc;
+  }
+  void* ws = nullptr;
+  rc = static_scratch(&ws);
+  if (rc) return rc;
+  // Clear what must start at zero, so that a failed earlier call (a timeout,
+  // a bad length) leaves nothing behind for this one.
+  rc = from_cuda(cudaMemsetAsync(ws, 0, static_zero_prefix(B, Hq, Hkv, T_cap, D, spec.k_bits), s));
+  if (rc) return rc;
+  DecodeArgs a{};
+  a.B = B; a.Hq = Hq; a.Hkv = Hkv; a.T_cap = T_cap; a.G = spec.group; a.r = Hq / Hkv;
+  a.lens = seq_lens; a.len_mode = 0;
+  a.q = static_cast<const uint16_t*>(q);
+  a.kc[0] = a.kc[1] = static_cast<const uint8_t*>(k_codes);
+  a.ksz[0] = a.ksz[1] = k_sz;
+  a.vc[0] = a.vc[1] = static_cast<const uint8_t*>(v_codes);
+  a.vsz[0] = a.vsz[1] = v_sz;
+  a.q_scale = softmax_scale * 1.4426950408889634f;
+  a.tau = tau;
+  a.out = out;
+  a.skip_mask = skip_mask;
+  a.skip_counts = reinterpret_cast<unsigned long long*>(skip_counts);
+  rc = run_attention(a, D, spec.k_bits, spec.v_bits, spec.v_bits, ws, LKV_STATIC_WORKSPACE_BYTES, s);
+  if (rc == LKV_OK && status)
+    rc = from_cuda(cudaMemcpyAsync(status, ws, sizeof(int32_t), cudaMemcpyDeviceToDevice, s));
+  return rc;
 }
 
 int lkv_workspace_reset(void* workspace, size_t ws_bytes, void* stream) {

@@ -51,6 +51,8 @@ SIGNATURES = {
     "lkv_decode_workspace_bytes": (_Z, [lkv_qspec, _I, _I, _I, _I, _I]),
     "lkv_decode_attention": (_I, [lkv_qspec, _I, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P, _F, _F,
                                   _P, _P, _P, _P, _Z, _P]),
+    "lkv_decode_attention_static": (_I, [lkv_qspec, _I, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P, _F,
+                                         _F, _P, _P, _P, _P, _P]),
     "lkv_workspace_reset": (_I, [_P, _Z, _P]),
     "lkv_workspace_status": (_I, [_P, _P, _P]),
     "lkv_tier_classify": (_I, [_I, _I, _I, _P, _P, _F, _F, _P, _P, _P, _P, _P]),
@@ -150,6 +152,18 @@ def lkv_decode_attention(spec, B, Hq, Hkv, T_cap, D, seq_lens, q, k_codes, k_sz,
                                       float(softmax_scale), float(tau), _ptr(out), _ptr(skip_mask),
                                       _ptr(skip_counts), _ptr(workspace), int(ws_bytes),
                                       _stream(stream)), "lkv_decode_attention")
+
+
+LKV_STATIC_WORKSPACE_BYTES = 32 << 20
+
+
+def lkv_decode_attention_static(spec, B, Hq, Hkv, T_cap, D, seq_lens, q, k_codes, k_sz, v_codes, v_sz,
+                                softmax_scale, tau, out, skip_mask, skip_counts, status, stream=None):
+    _check(lib().lkv_decode_attention_static(_spec(spec), B, Hq, Hkv, T_cap, D, _ptr(seq_lens), _ptr(q),
+                                             _ptr(k_codes), _ptr(k_sz), _ptr(v_codes), _ptr(v_sz),
+                                             float(softmax_scale), float(tau), _ptr(out),
+                                             _ptr(skip_mask), _ptr(skip_counts), _ptr(status),
+                                             _stream(stream)), "lkv_decode_attention_static")
 
 
 def lkv_workspace_reset(workspace, ws_bytes, stream=None):

@@ -127,6 +127,22 @@ def test_decode_rejects(L, kw, want):
     assert rc_of(lambda **a: lkv.lkv_decode_attention(**a), **decode_args(**kw)) == want
 
 
+def test_static_decode_rejects_before_any_device_call(L):
+    """The fixed-scratch decode refuses sizes beyond its scratch on the host."""
+    def static_args(**kw):
+        a = decode_args(status=None)
+        del a["workspace"], a["ws_bytes"]
+        a.update(kw)
+        return a
+    call = lambda **a: lkv.lkv_decode_attention_static(**a)
+    # B64 x 8 kv heads x T4096 needs about 40 MiB of scratch
+    assert lkv.lkv_decode_workspace_bytes(K6V4, 64, 32, 8, 4096, 128) > lkv.LKV_STATIC_WORKSPACE_BYTES
+    assert rc_of(call, **static_args(B=64, Hq=32, Hkv=8, T_cap=4096)) == lkv.LKV_ERR_WORKSPACE
+    assert rc_of(call, **static_args(status=FAKE + 2)) == lkv.LKV_ERR_INVALID_ARG
+    assert rc_of(call, **static_args(Hq=6)) == lkv.LKV_ERR_UNSUPPORTED
+    assert rc_of(call, **static_args(q=None)) == lkv.LKV_ERR_INVALID_ARG
+
+
 def test_tiered_rejects(L):
     seg = lkv.lkv_segment(FAKE, FAKE, FAKE, FAKE)
     bad = lkv.lkv_segment(FAKE, None, FAKE, FAKE)
