@@ -97,21 +97,58 @@ __device__ __forceinline__ void store_lane_words(uint8_t* p, const LaneWords<BIT
   }
 }
 
-// Quantize the 16 values a lane holds, sharing min/max with the other lanes
-// of its group (LPG = G / 16 consecutive lanes).  The formula is the fixed
-// fp32 one of lkv_quantize_kv, every operation rounded separately.
-// `mask` names the lanes of the calling row (all of them take this call).
+// Packed fp32 add and multiply, each rounded to nearest even, written as PTX
+// so that the compiler front end cannot reassociate them.  A multiply whose
+// result feeds an add directly may still be contracted by the code generator;
+// callers that need the product rounded separately put another operation
+// between the two.
+__device__ __forceinline__ uint64_t pack_f2(float2 a) {
+  return ((uint64_t)__float_as_uint(a.y) << 32) | __float_as_uint(a.x);
+}
+__device__ __forceinline__ float2 unpack_f2(uint64_t r) {
+  return make_float2(__uint_as_float((uint32_t)r), __uint_as_float((uint32_t)(r >> 32)));
+}
+__device__ __forceinline__ float2 exact_add2(float2 a, float2 b) {
+  uint64_t r;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(pack_f2(a)), "l"(pack_f2(b)));
+  return unpack_f2(r);
+}
+__device__ __forceinline__ float2 exact_mul2(float2 a, float2 b) {
+  uint64_t r;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(pack_f2(a)), "l"(pack_f2(b)));
+  return unpack_f2(r);
+}
+
+// Quantize the 16 bf16 values a lane holds (raw words w, value 2i in the low
+// half of w[i]), sharing min/max with the other lanes of its group (LPG =
+// G / 16 consecutive lanes), and pack the codes into lw.  The formula is the
+// fixed fp32 one of lkv_quantize_kv, every operation rounded separately:
+//   d = mx - mn;  scale = d / qmax;  inv = qmax / d  (both 0 when d == 0);
+//   code = clamp(rint((x - mn) * inv), 0, qmax);  zero = mn + 0.
+// While d and inv are finite, x - mn <= d, so (x - mn) * inv < qmax + 1/2 and
+// the clamp never bites: the code is rounded half-even by adding 1.5 * 2^23
+// (two values per packed fp32 add) and read from the low mantissa bits.
+// Otherwise (inv overflowing for a tiny d, or d overflowing) every value takes
+// the clamped scalar path.  `mask` names the lanes of the calling row.
 template <int BITS>
-__device__ __forceinline__ void quantize16(const float (&x)[16], int lpg, unsigned mask, uint32_t (&c)[16],
+__device__ __forceinline__ void quantize16(const uint32_t (&w)[8], int lpg, unsigned mask, LaneWords<BITS>& lw,
                                            float& scale, float& zero) {
-  float mn = x[0], mx = x[0];
+  // min and max are exact in bf16, two values per instruction
+  __nv_bfloat162 lo = *reinterpret_cast<const __nv_bfloat162*>(&w[0]), hi = lo;
 #pragma unroll
-  for (int i = 1; i < 16; ++i) { mn = fminf(mn, x[i]); mx = fmaxf(mx, x[i]); }
+  for (int i = 1; i < 8; ++i) {
+    const __nv_bfloat162 p = *reinterpret_cast<const __nv_bfloat162*>(&w[i]);
+    lo = __hmin2(lo, p);
+    hi = __hmax2(hi, p);
+  }
+  float mn = fminf(__low2float(lo), __high2float(lo));
+  float mx = fmaxf(__low2float(hi), __high2float(hi));
   for (int off = 1; off < lpg; off <<= 1) {
     mn = fminf(mn, __shfl_xor_sync(mask, mn, off));
     mx = fmaxf(mx, __shfl_xor_sync(mask, mx, off));
   }
-  const float qmax = static_cast<float>((1u << BITS) - 1u);
+  constexpr uint32_t cmask = (1u << BITS) - 1u;
+  const float qmax = static_cast<float>(cmask);
   const float d = __fsub_rn(mx, mn);
   float inv = 0.0f;
   scale = 0.0f;
@@ -119,15 +156,35 @@ __device__ __forceinline__ void quantize16(const float (&x)[16], int lpg, unsign
     scale = __fdiv_rn(d, qmax);
     inv = __fdiv_rn(qmax, d);
   }
-#pragma unroll
-  for (int i = 0; i < 16; ++i) {
-    const float y = __fmul_rn(__fsub_rn(x[i], mn), inv);
-    int ci = __float2int_rn(y);
-    ci = ci < 0 ? 0 : ci;
-    ci = ci > (int)((1u << BITS) - 1u) ? (int)((1u << BITS) - 1u) : ci;
-    c[i] = static_cast<uint32_t>(ci);
-  }
   zero = __fadd_rn(mn, 0.0f);
+  uint32_t c[16];
+  if (d <= 3.4028234663852886e38f && inv <= 3.4028234663852886e38f) {
+    const float2 nmn = make_float2(-mn, -mn), inv2 = make_float2(inv, inv);
+    const float2 rnd = make_float2(12582912.0f, 12582912.0f);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const float2 x = make_float2(bf16_lo(w[i]), bf16_hi(w[i]));
+      float2 y = exact_mul2(exact_add2(x, nmn), inv2);
+      // The max sits between the packed multiply and the packed rounding add
+      // on purpose: with the two adjacent, the code generator contracts them
+      // into one fused multiply-add even when both are written with explicit
+      // round-to-nearest, and the product would no longer be rounded on its
+      // own.  It also sends a NaN input to code 0.
+      y = make_float2(fmaxf(y.x, 0.0f), fmaxf(y.y, 0.0f));
+      const float2 r = exact_add2(y, rnd);
+      c[2 * i] = __float_as_uint(r.x) & cmask;
+      c[2 * i + 1] = __float_as_uint(r.y) & cmask;
+    }
+  } else {
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      const float x = (i & 1) ? bf16_hi(w[i / 2]) : bf16_lo(w[i / 2]);
+      int ci = __float2int_rn(__fmul_rn(__fsub_rn(x, mn), inv));  // NaN gives 0
+      ci = ci < 0 ? 0 : ci;
+      c[i] = static_cast<uint32_t>(ci > (int)cmask ? (int)cmask : ci);
+    }
+  }
+  pack16<BITS>(c, lw);
 }
 
 // Load 16 bf16 values (32 bytes, 32-byte aligned) as floats.

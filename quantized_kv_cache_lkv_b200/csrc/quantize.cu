@@ -8,114 +8,172 @@
 // registers: one lane quantizes 16 channels, the G/16 lanes of a group share
 // their min/max by warp shuffles, and the lane packs its 16 codes into
 // 2*BITS bytes that it stores itself.
+#include <algorithm>
+
 #include "lkv_kernels.cuh"
 
 namespace lkv {
 
-// One row (token) of one tensor: lane j of the row's D/16 lanes.
-template <int D, int BITS>
-__device__ __forceinline__ void quantize_row_lane(const uint16_t* __restrict__ src, uint8_t* __restrict__ codes,
-                                                  float* __restrict__ sz, int j, int G) {
-  constexpr int LPR = D / kDimsPerLane;
-  const unsigned mask = row_lane_mask<LPR>(threadIdx.x & 31);
-  float x[16];
-  load16_bf16(src + j * kDimsPerLane, x);
-  uint32_t c[16];
-  float scale, zero;
-  const int lpg = G / kDimsPerLane;
-  quantize16<BITS>(x, lpg, mask, c, scale, zero);
+// Streaming 16-byte load that does not keep the line in L1 (each bf16 row is
+// read exactly once).
+__device__ __forceinline__ uint4 ld_stream(const void* p) {
+  uint4 v;
+  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "l"(p));
+  return v;
+}
+
+// The 16 bf16 channels [16j, 16j + 16) of one row of K and of V, in flight.
+struct LaneRows {
+  uint4 k0, k1, v0, v1;
+};
+
+__device__ __forceinline__ void fetch_lane_rows(const uint16_t* k, const uint16_t* v, LaneRows& r) {
+  r.k0 = ld_stream(k); r.k1 = ld_stream(k + 8);
+  r.v0 = ld_stream(v); r.v1 = ld_stream(v + 8);
+}
+
+// Quantize one lane's 16 channels of a row (raw bf16 words w0, w1) and store
+// its codes and, for the group's first lane, the (scale, zero) pair.
+template <int BITS>
+__device__ __forceinline__ void quantize_lane(const uint4& w0, const uint4& w1, uint8_t* __restrict__ codes,
+                                              float* __restrict__ sz, int j, int lpg, unsigned mask) {
+  const uint32_t w[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
   LaneWords<BITS> lw;
-  pack16<BITS>(c, lw);
+  float scale, zero;
+  quantize16<BITS>(w, lpg, mask, lw, scale, zero);
   store_lane_words<BITS>(codes + j * (2 * BITS), lw);
   if (j % lpg == 0) *reinterpret_cast<float2*>(sz + 2 * (j / lpg)) = make_float2(scale, zero);
 }
 
-// Grid-stride over row slots of [B][Hkv][T_cap]; a warp covers 32/(D/16) rows.
+// Row batches: batch i of unit bg = i / nbu covers tokens (i % nbu) * RPW ...
+// of that unit, one row per D/16 lanes.  Each warp walks its batches with the
+// next batch's loads issued before the current one is quantized, so two
+// batches of K and V per warp are in flight.
 template <int D, int KB, int VB>
-__global__ void __launch_bounds__(256) quantize_kv_kernel(QuantizeArgs a) {
+__global__ void __launch_bounds__(256, 4) quantize_kv_kernel(QuantizeArgs a) {
   constexpr int LPR = D / kDimsPerLane;
   constexpr int RPW = 32 / LPR;
   const int lane = threadIdx.x & 31;
-  const int j = lane % LPR;
-  const int ng = D / a.G;
-  const long long n_rows = (long long)a.B * a.Hkv * a.T_cap;
-  const long long warp0 = ((long long)blockIdx.x * blockDim.x + threadIdx.x) / 32;
-  const long long n_warps = (long long)gridDim.x * blockDim.x / 32;
-  for (long long base = warp0 * RPW; base < n_rows; base += n_warps * RPW) {
-    const long long row = base + lane / LPR;
-    if (row >= n_rows) continue;
-    const long long bg = row / a.T_cap;
-    const int t = (int)(row - bg * a.T_cap);
-    const int b = (int)(bg / a.Hkv);
-    if (t >= clamp_len(a.seq_lens[b], a.T_cap)) continue;
-    // The lanes of one row take this path together, so the group shuffles
-    // inside quantize16 only ever pair lanes that are both active.
-    quantize_row_lane<D, KB>(a.k + row * D, a.k_codes + row * (D * KB / 8), a.k_sz + row * ng * 2, j, a.G);
-    quantize_row_lane<D, VB>(a.v + row * D, a.v_codes + row * (D * VB / 8), a.v_sz + row * ng * 2, j, a.G);
+  const int j = lane % LPR, sub = lane / LPR;
+  const unsigned mask = row_lane_mask<LPR>(lane);
+  const int ng = D / a.G, lpg = a.G / kDimsPerLane;
+  const uint32_t nbu = (uint32_t)(a.T_cap + RPW - 1) / RPW;
+  const uint32_t n_batches = (uint32_t)(a.B * a.Hkv) * nbu;
+  const uint32_t stride = gridDim.x * (blockDim.x / 32);
+  auto fetch = [&](uint32_t i, LaneRows& r, long long& row) -> bool {
+    if (i >= n_batches) return false;
+    const uint32_t bg = i / nbu;
+    const int t = (int)(i - bg * nbu) * RPW + sub;
+    if (t >= clamp_len(__ldg(a.seq_lens + bg / a.Hkv), a.T_cap)) return false;
+    row = (long long)bg * a.T_cap + t;
+    fetch_lane_rows(a.k + row * D + j * kDimsPerLane, a.v + row * D + j * kDimsPerLane, r);
+    return true;
+  };
+  uint32_t i = blockIdx.x * (blockDim.x / 32) + threadIdx.x / 32;
+  LaneRows cur, nxt;
+  long long row = 0, row_n = 0;
+  bool ok = fetch(i, cur, row);
+  for (; i < n_batches; i += stride) {
+    const bool ok_n = fetch(i + stride, nxt, row_n);
+    // The lanes of one row share `ok`, so the group shuffles inside
+    // quantize16 only ever pair lanes that are both active.
+    if (ok) {
+      quantize_lane<KB>(cur.k0, cur.k1, a.k_codes + row * (D * KB / 8), a.k_sz + row * ng * 2, j, lpg, mask);
+      quantize_lane<VB>(cur.v0, cur.v1, a.v_codes + row * (D * VB / 8), a.v_sz + row * ng * 2, j, lpg, mask);
+    }
+    cur = nxt; row = row_n; ok = ok_n;
   }
 }
 
 // Tier repack: row i of segment A (tier 2) or B (tier 1) of (b, g) is the
 // token at pos[b][g][i], quantized from bf16 with K at 6 bits and V at 6 (A)
-// or 4 (B) bits ("Super KV Compression", §第二层 items 1-2).
+// or 4 (B) bits ("Super KV Compression", §第二层 items 1-2).  Block
+// (bg * S + s, seg) walks only the n rows that segment seg of unit bg holds,
+// S blocks per unit and segment, with the same one-ahead loads as above.
 template <int D>
-__global__ void __launch_bounds__(256) tier_repack_kernel(RepackArgs a) {
+__global__ void __launch_bounds__(256, 4) tier_repack_kernel(RepackArgs a, int S) {
   constexpr int LPR = D / kDimsPerLane;
   constexpr int RPW = 32 / LPR;
   const int lane = threadIdx.x & 31;
-  const int j = lane % LPR;
-  const int ng = D / a.G;
-  const long long n_slots = (long long)a.B * a.Hkv * a.T_cap;
-  const long long warp0 = ((long long)blockIdx.x * blockDim.x + threadIdx.x) / 32;
-  const long long n_warps = (long long)gridDim.x * blockDim.x / 32;
+  const int j = lane % LPR, sub = lane / LPR;
+  const unsigned mask = row_lane_mask<LPR>(lane);
+  const int ng = D / a.G, lpg = a.G / kDimsPerLane;
   const int seg = blockIdx.y;  // 0: segment A, 1: segment B
-  const int32_t* pos = seg == 0 ? a.pos_a : a.pos_b;
-  for (long long base = warp0 * RPW; base < n_slots; base += n_warps * RPW) {
-    const long long slot = base + lane / LPR;
-    if (slot >= n_slots) continue;
-    const long long bg = slot / a.T_cap;
-    const int i = (int)(slot - bg * a.T_cap);
-    const int n = clamp_len(a.counts[2 * bg + seg], a.T_cap);
-    if (i >= n) continue;
-    int t = pos[slot];
+  const long long bg = blockIdx.x / S;
+  const int s = blockIdx.x % S;
+  const int n = clamp_len(a.counts[2 * bg + seg], a.T_cap);
+  const int32_t* pos = (seg == 0 ? a.pos_a : a.pos_b) + bg * a.T_cap;
+  const int nw = blockDim.x / 32;
+  const int stride = S * nw * RPW;
+  auto fetch = [&](int i, LaneRows& r) -> bool {
+    if (i >= n) return false;
+    int t = __ldg(pos + i);
     t = t < 0 ? 0 : (t >= a.T_cap ? a.T_cap - 1 : t);
     const long long src = bg * a.T_cap + t;
-    if (seg == 0) {
-      quantize_row_lane<D, 6>(a.k + src * D, a.a_kc + slot * (D * 6 / 8), a.a_ksz + slot * ng * 2, j, a.G);
-      quantize_row_lane<D, 6>(a.v + src * D, a.a_vc + slot * (D * 6 / 8), a.a_vsz + slot * ng * 2, j, a.G);
-    } else {
-      quantize_row_lane<D, 6>(a.k + src * D, a.b_kc + slot * (D * 6 / 8), a.b_ksz + slot * ng * 2, j, a.G);
-      quantize_row_lane<D, 4>(a.v + src * D, a.b_vc + slot * (D * 4 / 8), a.b_vsz + slot * ng * 2, j, a.G);
+    fetch_lane_rows(a.k + src * D + j * kDimsPerLane, a.v + src * D + j * kDimsPerLane, r);
+    return true;
+  };
+  int i = (s * nw + (int)threadIdx.x / 32) * RPW + sub;
+  LaneRows cur, nxt;
+  bool ok = fetch(i, cur);
+  for (; i - sub < n; i += stride) {
+    const bool ok_n = fetch(i + stride, nxt);
+    if (ok) {
+      const long long slot = bg * a.T_cap + i;
+      if (seg == 0) {
+        quantize_lane<6>(cur.k0, cur.k1, a.a_kc + slot * (D * 6 / 8), a.a_ksz + slot * ng * 2, j, lpg, mask);
+        quantize_lane<6>(cur.v0, cur.v1, a.a_vc + slot * (D * 6 / 8), a.a_vsz + slot * ng * 2, j, lpg, mask);
+      } else {
+        quantize_lane<6>(cur.k0, cur.k1, a.b_kc + slot * (D * 6 / 8), a.b_ksz + slot * ng * 2, j, lpg, mask);
+        quantize_lane<4>(cur.v0, cur.v1, a.b_vc + slot * (D * 4 / 8), a.b_vsz + slot * ng * 2, j, lpg, mask);
+      }
     }
+    cur = nxt; ok = ok_n;
   }
 }
 
-static int grid_for_rows(long long n_rows, int rows_per_block, int sms) {
-  long long blocks = (n_rows + rows_per_block - 1) / rows_per_block;
-  const long long cap = (long long)sms * 8;
-  if (blocks > cap) blocks = cap;
-  return (int)(blocks < 1 ? 1 : blocks);
+// Resident blocks of 256 threads per SM for a kernel (cached per kernel and
+// device by the caller's static).
+static int resident_blocks(const void* kern) {
+  int n = 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kern, 256, 0) != cudaSuccess || n < 1) n = 1;
+  return n;
 }
 
-template <int D, int KB>
-static cudaError_t launch_quantize_vb(const QuantizeArgs& a, int vb, int grid, cudaStream_t s) {
-  switch (vb) {
-    case 2: quantize_kv_kernel<D, KB, 2><<<grid, 256, 0, s>>>(a); break;
-    case 4: quantize_kv_kernel<D, KB, 4><<<grid, 256, 0, s>>>(a); break;
-    case 6: quantize_kv_kernel<D, KB, 6><<<grid, 256, 0, s>>>(a); break;
-    case 8: quantize_kv_kernel<D, KB, 8><<<grid, 256, 0, s>>>(a); break;
-    default: return cudaErrorInvalidValue;
-  }
+template <int D, int KB, int VB>
+static cudaError_t launch_quantize_t(const QuantizeArgs& a, cudaStream_t s) {
+  constexpr int RPW = 32 / (D / kDimsPerLane);
+  static int per_sm[64] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) dev = 0;
+  if (per_sm[dev] == 0) per_sm[dev] = resident_blocks((const void*)quantize_kv_kernel<D, KB, VB>);
+  const long long n_batches = (long long)a.B * a.Hkv * ((a.T_cap + RPW - 1) / RPW);
+  if (n_batches >= (1ll << 31)) return cudaErrorInvalidValue;
+  long long blocks = std::min<long long>((long long)num_sms() * per_sm[dev], (n_batches + 7) / 8);
+  quantize_kv_kernel<D, KB, VB><<<(int)std::max<long long>(blocks, 1), 256, 0, s>>>(a);
   return cudaGetLastError();
 }
 
+template <int D, int KB>
+static cudaError_t launch_quantize_vb(const QuantizeArgs& a, int vb, cudaStream_t s) {
+  switch (vb) {
+    case 2: return launch_quantize_t<D, KB, 2>(a, s);
+    case 4: return launch_quantize_t<D, KB, 4>(a, s);
+    case 6: return launch_quantize_t<D, KB, 6>(a, s);
+    case 8: return launch_quantize_t<D, KB, 8>(a, s);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
 template <int D>
-static cudaError_t launch_quantize_d(const QuantizeArgs& a, int kb, int vb, int grid, cudaStream_t s) {
+static cudaError_t launch_quantize_d(const QuantizeArgs& a, int kb, int vb, cudaStream_t s) {
   switch (kb) {
-    case 2: return launch_quantize_vb<D, 2>(a, vb, grid, s);
-    case 4: return launch_quantize_vb<D, 4>(a, vb, grid, s);
-    case 6: return launch_quantize_vb<D, 6>(a, vb, grid, s);
-    case 8: return launch_quantize_vb<D, 8>(a, vb, grid, s);
+    case 2: return launch_quantize_vb<D, 2>(a, vb, s);
+    case 4: return launch_quantize_vb<D, 4>(a, vb, s);
+    case 6: return launch_quantize_vb<D, 6>(a, vb, s);
+    case 8: return launch_quantize_vb<D, 8>(a, vb, s);
     default: return cudaErrorInvalidValue;
   }
 }
@@ -123,20 +181,21 @@ static cudaError_t launch_quantize_d(const QuantizeArgs& a, int kb, int vb, int 
 cudaError_t launch_quantize_kv(const QuantizeArgs& a, int kb, int vb, int D, cudaStream_t s) {
   const long long n_rows = (long long)a.B * a.Hkv * a.T_cap;
   if (n_rows == 0) return cudaSuccess;
-  const int rows_per_block = 8 * (32 / (D / kDimsPerLane));
-  const int grid = grid_for_rows(n_rows, rows_per_block, num_sms());
-  if (D == 64) return launch_quantize_d<64>(a, kb, vb, grid, s);
-  if (D == 128) return launch_quantize_d<128>(a, kb, vb, grid, s);
+  if (D == 64) return launch_quantize_d<64>(a, kb, vb, s);
+  if (D == 128) return launch_quantize_d<128>(a, kb, vb, s);
   return cudaErrorInvalidValue;
 }
 
 cudaError_t launch_tier_repack(const RepackArgs& a, int D, cudaStream_t s) {
-  const long long n_slots = (long long)a.B * a.Hkv * a.T_cap;
-  if (n_slots == 0) return cudaSuccess;
-  const int rows_per_block = 8 * (32 / (D / kDimsPerLane));
-  dim3 grid(grid_for_rows(n_slots, rows_per_block, num_sms()), 2);
-  if (D == 64) tier_repack_kernel<64><<<grid, 256, 0, s>>>(a);
-  else if (D == 128) tier_repack_kernel<128><<<grid, 256, 0, s>>>(a);
+  const long long units = (long long)a.B * a.Hkv;
+  if (units == 0 || a.T_cap == 0) return cudaSuccess;
+  // about eight blocks per SM over both segments, at least one per unit
+  const long long want = (long long)num_sms() * 8;
+  const int S = (int)std::max<long long>(1, std::min<long long>(64, want / (2 * units)));
+  if (units * S >= (1ll << 31)) return cudaErrorInvalidValue;
+  dim3 grid((unsigned)(units * S), 2);
+  if (D == 64) tier_repack_kernel<64><<<grid, 256, 0, s>>>(a, S);
+  else if (D == 128) tier_repack_kernel<128><<<grid, 256, 0, s>>>(a, S);
   else return cudaErrorInvalidValue;
   return cudaGetLastError();
 }

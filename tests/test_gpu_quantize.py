@@ -41,6 +41,10 @@ def special_rows(inp):
     k[0, 0, 3] = 1.0
     k[0, 0, 3, 5] = 1000.0
     v[0, 0, 3] = torch.arange(D, dtype=torch.float32).remainder(16).to(torch.bfloat16)
+    # range so small that qmax / d overflows (subnormal steps), and so large
+    # that d = mx - mn overflows: both take the clamped path of the formula
+    v[0, 0, 4] = torch.linspace(0.0, 1e-38, 16, dtype=torch.float64).repeat(D // 16).to(torch.bfloat16)
+    k[0, 0, 4] = torch.linspace(-3e38, 3e38, 16, dtype=torch.float64).repeat(D // 16).to(torch.bfloat16)
     return inp
 
 
