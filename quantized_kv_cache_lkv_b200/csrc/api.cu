@@ -278,7 +278,7 @@ int lkv_quantize_kv(lkv_qspec spec, int B, int Hkv, int T_cap, int D, const int3
     return LKV_ERR_INVALID_ARG;
   if (!ne) return LKV_OK;
   QuantizeArgs a{};
-  a.B = B; a.Hkv = Hkv; a.T_cap = T_cap; a.G = spec.group;
+  a.B = B; a.Hkv = Hkv; a.T_cap = T_cap; a.G = spec.group; a.one = 1.0f;
   a.seq_lens = seq_lens;
   a.k = static_cast<const uint16_t*>(k);
   a.v = static_cast<const uint16_t*>(v);
@@ -421,7 +421,7 @@ int lkv_tier_repack(int B, int Hkv, int T_cap, int D, int group, const void* k, 
     return LKV_ERR_INVALID_ARG;
   if (!ne) return LKV_OK;
   RepackArgs a{};
-  a.B = B; a.Hkv = Hkv; a.T_cap = T_cap; a.G = group;
+  a.B = B; a.Hkv = Hkv; a.T_cap = T_cap; a.G = group; a.one = 1.0f;
   a.k = static_cast<const uint16_t*>(k);
   a.v = static_cast<const uint16_t*>(v);
   a.counts = counts; a.pos_a = pos_a; a.pos_b = pos_b;

@@ -119,6 +119,42 @@ __device__ __forceinline__ float2 exact_mul2(float2 a, float2 b) {
   return unpack_f2(r);
 }
 
+__device__ __forceinline__ float2 exact_fma2(float2 a, float2 b, float2 c) {
+  uint64_t r;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(pack_f2(a)), "l"(pack_f2(b)), "l"(pack_f2(c)));
+  return unpack_f2(r);
+}
+
+// Magic-rounded codes: rb[i] = 0x4B400000 + code_i (the bits of 1.5 * 2^23 +
+// code).  Packs them LSB first without masking: adding rb << pos for every
+// code of a word and one constant that cancels the 0x4B400000 << pos terms
+// (mod 2^32) leaves exactly the OR of code << pos.
+template <int BITS>
+constexpr uint32_t magic_pack_const(int wi) {
+  uint32_t c = 0u;
+  for (int i = 0; i < 16; ++i) {
+    const int bit = i * BITS;
+    if ((bit >> 5) == wi) c -= 0x4B400000u << (bit & 31);
+  }
+  return c;
+}
+
+template <int BITS>
+__device__ __forceinline__ void pack16_magic(const uint32_t (&rb)[16], LaneWords<BITS>& lw) {
+  constexpr uint32_t mask = (1u << BITS) - 1u;
+#pragma unroll
+  for (int wi = 0; wi < LaneWords<BITS>::N; ++wi) {
+    uint32_t acc = magic_pack_const<BITS>(wi);
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      const int bit = i * BITS, w0 = bit >> 5, pos = bit & 31;
+      if (w0 == wi) acc += rb[i] << pos;
+      else if (w0 + 1 == wi && pos + BITS > 32) acc += (rb[i] & mask) >> (32 - pos);
+    }
+    lw.w[wi] = acc;
+  }
+}
+
 // Quantize the 16 bf16 values a lane holds (raw words w, value 2i in the low
 // half of w[i]), sharing min/max with the other lanes of its group (LPG =
 // G / 16 consecutive lanes), and pack the codes into lw.  The formula is the
@@ -127,12 +163,13 @@ __device__ __forceinline__ float2 exact_mul2(float2 a, float2 b) {
 //   code = clamp(rint((x - mn) * inv), 0, qmax);  zero = mn + 0.
 // While d and inv are finite, x - mn <= d, so (x - mn) * inv < qmax + 1/2 and
 // the clamp never bites: the code is rounded half-even by adding 1.5 * 2^23
-// (two values per packed fp32 add) and read from the low mantissa bits.
+// (two values per packed fp32 operation) and read from the low mantissa bits.
+// `one` must be 1.0f, passed in at run time (see the rounding step).
 // Otherwise (inv overflowing for a tiny d, or d overflowing) every value takes
 // the clamped scalar path.  `mask` names the lanes of the calling row.
 template <int BITS>
-__device__ __forceinline__ void quantize16(const uint32_t (&w)[8], int lpg, unsigned mask, LaneWords<BITS>& lw,
-                                           float& scale, float& zero) {
+__device__ __forceinline__ void quantize16(const uint32_t (&w)[8], int lpg, unsigned mask, float one,
+                                           LaneWords<BITS>& lw, float& scale, float& zero) {
   // min and max are exact in bf16, two values per instruction
   __nv_bfloat162 lo = *reinterpret_cast<const __nv_bfloat162*>(&w[0]), hi = lo;
 #pragma unroll
@@ -143,9 +180,12 @@ __device__ __forceinline__ void quantize16(const uint32_t (&w)[8], int lpg, unsi
   }
   float mn = fminf(__low2float(lo), __high2float(lo));
   float mx = fmaxf(__low2float(hi), __high2float(hi));
-  for (int off = 1; off < lpg; off <<= 1) {
-    mn = fminf(mn, __shfl_xor_sync(mask, mn, off));
-    mx = fmaxf(mx, __shfl_xor_sync(mask, mx, off));
+#pragma unroll
+  for (int off = 1; off < 8; off <<= 1) {
+    if (off < lpg) {
+      mn = fminf(mn, __shfl_xor_sync(mask, mn, off));
+      mx = fmaxf(mx, __shfl_xor_sync(mask, mx, off));
+    }
   }
   constexpr uint32_t cmask = (1u << BITS) - 1u;
   const float qmax = static_cast<float>(cmask);
@@ -157,25 +197,30 @@ __device__ __forceinline__ void quantize16(const uint32_t (&w)[8], int lpg, unsi
     inv = __fdiv_rn(qmax, d);
   }
   zero = __fadd_rn(mn, 0.0f);
-  uint32_t c[16];
   if (d <= 3.4028234663852886e38f && inv <= 3.4028234663852886e38f) {
-    const float2 nmn = make_float2(-mn, -mn), inv2 = make_float2(inv, inv);
+    // a NaN input becomes mn (code 0), every other value is unchanged
+    const __nv_bfloat162 mn_b = __floats2bfloat162_rn(mn, mn);
+    const float2 nmn = make_float2(-mn, -mn), inv2 = make_float2(inv, inv), one2 = make_float2(one, one);
     const float2 rnd = make_float2(12582912.0f, 12582912.0f);
+    uint32_t rb[16];
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
-      const float2 x = make_float2(bf16_lo(w[i]), bf16_hi(w[i]));
-      float2 y = exact_mul2(exact_add2(x, nmn), inv2);
-      // The max sits between the packed multiply and the packed rounding add
-      // on purpose: with the two adjacent, the code generator contracts them
-      // into one fused multiply-add even when both are written with explicit
-      // round-to-nearest, and the product would no longer be rounded on its
-      // own.  It also sends a NaN input to code 0.
-      y = make_float2(fmaxf(y.x, 0.0f), fmaxf(y.y, 0.0f));
-      const float2 r = exact_add2(y, rnd);
-      c[2 * i] = __float_as_uint(r.x) & cmask;
-      c[2 * i + 1] = __float_as_uint(r.y) & cmask;
+      const __nv_bfloat162 p = __hmax2(*reinterpret_cast<const __nv_bfloat162*>(&w[i]), mn_b);
+      const uint32_t u = *reinterpret_cast<const uint32_t*>(&p);
+      const float2 x = make_float2(bf16_lo(u), bf16_hi(u));
+      const float2 y = exact_mul2(exact_add2(x, nmn), inv2);
+      // y * one + 1.5 * 2^23 with one == 1.0 held in a register: the product
+      // y * 1 is exact, so this is y + 1.5 * 2^23 rounded once, i.e. y rounded
+      // half-even into the low mantissa bits.  (A plain add fed directly by
+      // the multiply above would be contracted into one fused multiply-add,
+      // skipping the rounding of y.)
+      const float2 r = exact_fma2(y, one2, rnd);
+      rb[2 * i] = __float_as_uint(r.x);
+      rb[2 * i + 1] = __float_as_uint(r.y);
     }
+    pack16_magic<BITS>(rb, lw);
   } else {
+    uint32_t c[16];
 #pragma unroll
     for (int i = 0; i < 16; ++i) {
       const float x = (i & 1) ? bf16_hi(w[i / 2]) : bf16_lo(w[i / 2]);
@@ -183,8 +228,8 @@ __device__ __forceinline__ void quantize16(const uint32_t (&w)[8], int lpg, unsi
       ci = ci < 0 ? 0 : ci;
       c[i] = static_cast<uint32_t>(ci > (int)cmask ? (int)cmask : ci);
     }
+    pack16<BITS>(c, lw);
   }
-  pack16<BITS>(c, lw);
 }
 
 // Load 16 bf16 values (32 bytes, 32-byte aligned) as floats.

@@ -6,6 +6,7 @@ namespace lkv {
 
 struct QuantizeArgs {
   int B, Hkv, T_cap, G;
+  float one;  // 1.0f, read at run time by the rounding step of the quantizer
   const int32_t* seq_lens;
   const uint16_t* k;
   const uint16_t* v;
@@ -17,6 +18,7 @@ struct QuantizeArgs {
 
 struct RepackArgs {
   int B, Hkv, T_cap, G;
+  float one;  // 1.0f, as in QuantizeArgs
   const uint16_t* k;
   const uint16_t* v;
   const int32_t* counts;

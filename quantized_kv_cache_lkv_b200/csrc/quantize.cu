@@ -38,19 +38,20 @@ __device__ __forceinline__ void fetch_lane_rows(const uint16_t* k, const uint16_
 // its codes and, for the group's first lane, the (scale, zero) pair.
 template <int BITS>
 __device__ __forceinline__ void quantize_lane(const uint4& w0, const uint4& w1, uint8_t* __restrict__ codes,
-                                              float* __restrict__ sz, int j, int lpg, unsigned mask) {
+                                              float* __restrict__ sz, int j, int lpg, unsigned mask, float one) {
   const uint32_t w[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
   LaneWords<BITS> lw;
   float scale, zero;
-  quantize16<BITS>(w, lpg, mask, lw, scale, zero);
+  quantize16<BITS>(w, lpg, mask, one, lw, scale, zero);
   store_lane_words<BITS>(codes + j * (2 * BITS), lw);
   if (j % lpg == 0) *reinterpret_cast<float2*>(sz + 2 * (j / lpg)) = make_float2(scale, zero);
 }
 
-// Row batches: batch i of unit bg = i / nbu covers tokens (i % nbu) * RPW ...
-// of that unit, one row per D/16 lanes.  Each warp walks its batches with the
-// next batch's loads issued before the current one is quantized, so two
-// batches of K and V per warp are in flight.
+// Row batches: batch (b, g, tb) covers tokens tb * RPW ... of KV head g of
+// sequence b, one row per D/16 lanes.  Warp w of the grid takes batches w,
+// w + W, w + 2W, ... in (b, g, tb) order, stepping its coordinates without
+// divisions, and issues the next batch's loads before quantizing the current
+// one, so two batches of K and V per warp are in flight.
 template <int D, int KB, int VB>
 __global__ void __launch_bounds__(256, 4) quantize_kv_kernel(QuantizeArgs a) {
   constexpr int LPR = D / kDimsPerLane;
@@ -59,31 +60,44 @@ __global__ void __launch_bounds__(256, 4) quantize_kv_kernel(QuantizeArgs a) {
   const int j = lane % LPR, sub = lane / LPR;
   const unsigned mask = row_lane_mask<LPR>(lane);
   const int ng = D / a.G, lpg = a.G / kDimsPerLane;
-  const uint32_t nbu = (uint32_t)(a.T_cap + RPW - 1) / RPW;
-  const uint32_t n_batches = (uint32_t)(a.B * a.Hkv) * nbu;
-  const uint32_t stride = gridDim.x * (blockDim.x / 32);
-  auto fetch = [&](uint32_t i, LaneRows& r, long long& row) -> bool {
-    if (i >= n_batches) return false;
-    const uint32_t bg = i / nbu;
-    const int t = (int)(i - bg * nbu) * RPW + sub;
-    if (t >= clamp_len(__ldg(a.seq_lens + bg / a.Hkv), a.T_cap)) return false;
-    row = (long long)bg * a.T_cap + t;
+  const uint32_t nbu = (uint32_t)(a.T_cap + RPW - 1) / RPW;  // batches per (b, g)
+  const uint32_t W = gridDim.x * (blockDim.x / 32);
+  const uint32_t w0 = blockIdx.x * (blockDim.x / 32) + threadIdx.x / 32;
+  // position (b, g, tb) of batch w0 and the step W in the same coordinates
+  uint32_t tb = w0 % nbu, g = (w0 / nbu) % (uint32_t)a.Hkv, b = (w0 / nbu) / (uint32_t)a.Hkv;
+  const uint32_t s_tb = W % nbu, s_g = (W / nbu) % (uint32_t)a.Hkv, s_b = (W / nbu) / (uint32_t)a.Hkv;
+  auto step = [&](uint32_t& b_, uint32_t& g_, uint32_t& tb_) {
+    tb_ += s_tb;
+    uint32_t c = tb_ >= nbu ? 1u : 0u;
+    tb_ -= c * nbu;
+    g_ += s_g + c;
+    c = g_ >= (uint32_t)a.Hkv ? 1u : 0u;
+    g_ -= c * (uint32_t)a.Hkv;
+    b_ += s_b + c;
+  };
+  auto fetch = [&](uint32_t b_, uint32_t g_, uint32_t tb_, LaneRows& r, long long& row) -> bool {
+    if (b_ >= (uint32_t)a.B) return false;
+    const int t = (int)tb_ * RPW + sub;
+    if (t >= clamp_len(__ldg(a.seq_lens + b_), a.T_cap)) return false;
+    row = ((long long)b_ * a.Hkv + g_) * a.T_cap + t;
     fetch_lane_rows(a.k + row * D + j * kDimsPerLane, a.v + row * D + j * kDimsPerLane, r);
     return true;
   };
-  uint32_t i = blockIdx.x * (blockDim.x / 32) + threadIdx.x / 32;
   LaneRows cur, nxt;
   long long row = 0, row_n = 0;
-  bool ok = fetch(i, cur, row);
-  for (; i < n_batches; i += stride) {
-    const bool ok_n = fetch(i + stride, nxt, row_n);
+  bool ok = fetch(b, g, tb, cur, row);
+  while (b < (uint32_t)a.B) {
+    uint32_t bn = b, gn = g, tbn = tb;
+    step(bn, gn, tbn);
+    const bool ok_n = fetch(bn, gn, tbn, nxt, row_n);
     // The lanes of one row share `ok`, so the group shuffles inside
     // quantize16 only ever pair lanes that are both active.
     if (ok) {
-      quantize_lane<KB>(cur.k0, cur.k1, a.k_codes + row * (D * KB / 8), a.k_sz + row * ng * 2, j, lpg, mask);
-      quantize_lane<VB>(cur.v0, cur.v1, a.v_codes + row * (D * VB / 8), a.v_sz + row * ng * 2, j, lpg, mask);
+      quantize_lane<KB>(cur.k0, cur.k1, a.k_codes + row * (D * KB / 8), a.k_sz + row * ng * 2, j, lpg, mask, a.one);
+      quantize_lane<VB>(cur.v0, cur.v1, a.v_codes + row * (D * VB / 8), a.v_sz + row * ng * 2, j, lpg, mask, a.one);
     }
     cur = nxt; row = row_n; ok = ok_n;
+    b = bn; g = gn; tb = tbn;
   }
 }
 
@@ -123,11 +137,11 @@ __global__ void __launch_bounds__(256, 4) tier_repack_kernel(RepackArgs a, int S
     if (ok) {
       const long long slot = bg * a.T_cap + i;
       if (seg == 0) {
-        quantize_lane<6>(cur.k0, cur.k1, a.a_kc + slot * (D * 6 / 8), a.a_ksz + slot * ng * 2, j, lpg, mask);
-        quantize_lane<6>(cur.v0, cur.v1, a.a_vc + slot * (D * 6 / 8), a.a_vsz + slot * ng * 2, j, lpg, mask);
+        quantize_lane<6>(cur.k0, cur.k1, a.a_kc + slot * (D * 6 / 8), a.a_ksz + slot * ng * 2, j, lpg, mask, a.one);
+        quantize_lane<6>(cur.v0, cur.v1, a.a_vc + slot * (D * 6 / 8), a.a_vsz + slot * ng * 2, j, lpg, mask, a.one);
       } else {
-        quantize_lane<6>(cur.k0, cur.k1, a.b_kc + slot * (D * 6 / 8), a.b_ksz + slot * ng * 2, j, lpg, mask);
-        quantize_lane<4>(cur.v0, cur.v1, a.b_vc + slot * (D * 4 / 8), a.b_vsz + slot * ng * 2, j, lpg, mask);
+        quantize_lane<6>(cur.k0, cur.k1, a.b_kc + slot * (D * 6 / 8), a.b_ksz + slot * ng * 2, j, lpg, mask, a.one);
+        quantize_lane<4>(cur.v0, cur.v1, a.b_vc + slot * (D * 4 / 8), a.b_vsz + slot * ng * 2, j, lpg, mask, a.one);
       }
     }
     cur = nxt; ok = ok_n;
