@@ -43,7 +43,8 @@ constexpr int kMaxConsumerWarps = 12;
 constexpr int kListCap = 512;  // V-row list entries per warp per batch
 constexpr int kBatchBlocks = kListCap / 32;
 constexpr int kRec = 16;       // ints per unit-list record
-constexpr int kGatherUnroll = 2;
+constexpr int kGatherUnroll = 4;
+constexpr int kScanBlocks = 4;  // 32-row blocks whose logits one warp loads at once
 constexpr int kTsCap = 128;    // tile statistics kept in shared memory up to this many tiles
 constexpr int kQSlots = 4;     // units whose prescaled q is staged in shared memory
 constexpr unsigned kFull = 0xFFFFFFFFu;
@@ -170,6 +171,19 @@ __device__ __forceinline__ void ldcg_heads(const float* p, float (&x)[H]) {
     x[0] = v.x; x[1] = v.y;
   } else {
     x[0] = __ldcg(p);
+  }
+}
+
+template <int H>
+__device__ __forceinline__ void lds_heads(const float* p, float (&x)[H]) {
+  if constexpr (H == 4) {
+    const float4 v = *reinterpret_cast<const float4*>(p);
+    x[0] = v.x; x[1] = v.y; x[2] = v.z; x[3] = v.w;
+  } else if constexpr (H == 2) {
+    const float2 v = *reinterpret_cast<const float2*>(p);
+    x[0] = v.x; x[1] = v.y;
+  } else {
+    x[0] = p[0];
   }
 }
 
@@ -666,8 +680,11 @@ __global__ void __launch_bounds__(Geo<D, KB>::kThreads, 1) fused_decode_kernel(F
   }
 
   // ------------------------------------------------------------ phase 2
-  int* lists = reinterpret_cast<int*>(ring);                                         // [CW][kListCap]
-  float* red = reinterpret_cast<float*>(ring + kMaxConsumerWarps * kListCap * 4);    // [CW][H][D]
+  // phase-2 shared memory (in the ring): kept-row lists [CW][kListCap], their
+  // per-head weights [CW][kListCap][H] and the warps' partial outputs [CW][H][D]
+  int* lists = reinterpret_cast<int*>(ring);
+  float* wts = reinterpret_cast<float*>(ring + kMaxConsumerWarps * kListCap * 4);
+  float* red = wts + kMaxConsumerWarps * kListCap * H;
   Magic<VB0> mg0;
   mg0.load(s_magic);
   Magic<VB1> mg1;
@@ -731,32 +748,54 @@ __global__ void __launch_bounds__(Geo<D, KB>::kThreads, 1) fused_decode_kernel(F
         for (int i = 0; i < 8; ++i) acc[h][i] = make_float2(0.0f, 0.0f);
       }
       for (int vb = v_lo; vb < v_hi; vb += NCONS * kBatchBlocks) {
-        // scan: 32-row blocks round robin over warps, row order kept per warp
+        // scan: 32-row blocks round robin over warps, row order kept per warp;
+        // the logits of kScanBlocks blocks are loaded before any is used
         int* list = lists + warp * kListCap;
+        float* lwt = wts + warp * kListCap * H;
         int n_w = 0;
-        for (int blk = warp; blk < CW * kBatchBlocks; blk += CW) {
-          if (vb + blk * 32 >= v_hi) break;
-          const int v = vb + blk * 32 + lane;
-          const ChunkRows cr = chunk_rows(x, v / kChunk);
-          bool need = false;
-          if (v % kChunk < cr.rows) {
-            float ev[H];
-            ldcg_heads<H>(lgu + (long long)v * H, ev);
-            int nskip = 0;
+        for (int blk0 = warp; blk0 < CW * kBatchBlocks; blk0 += kScanBlocks * CW) {
+          if (vb + blk0 * 32 >= v_hi) break;
+          float ev[kScanBlocks][H];
+          bool in[kScanBlocks];
 #pragma unroll
-            for (int h = 0; h < H; ++h) {
-              const float p = ev[h] * tfu[(v / TR) * H + h];
-              const bool keep = !(p < d.tau);
-              need |= keep;
-              nskip += keep ? 0 : 1;
-              if (d.skip_mask) d.skip_mask[((long long)b * d.Hq + g * H + h) * d.T_cap + v] = keep ? 0 : 1;
-            }
-            cnt_heads += nskip;
-            cnt_rows += need ? 0 : 1;
+          for (int u = 0; u < kScanBlocks; ++u) {
+            const int blk = blk0 + u * CW;
+            const int v = vb + blk * 32 + lane;
+            in[u] = false;
+            if (blk < CW * kBatchBlocks && vb + blk * 32 < v_hi) in[u] = v % kChunk < chunk_rows(x, v / kChunk).rows;
+            if (in[u]) ldcg_heads<H>(lgu + (long long)v * H, ev[u]);
           }
-          const unsigned bal = __ballot_sync(kFull, need);
-          if (need) list[n_w + __popc(bal & ((1u << lane) - 1u))] = v;
-          n_w += __popc(bal);
+#pragma unroll
+          for (int u = 0; u < kScanBlocks; ++u) {
+            const int blk = blk0 + u * CW;
+            if (blk >= CW * kBatchBlocks || vb + blk * 32 >= v_hi) break;  // the same for the whole warp
+            const int v = vb + blk * 32 + lane;
+            bool need = false;
+            float wgt[H];
+#pragma unroll
+            for (int h = 0; h < H; ++h) wgt[h] = 0.0f;
+            if (in[u]) {
+              int nskip = 0;
+#pragma unroll
+              for (int h = 0; h < H; ++h) {
+                const float p = ev[u][h] * tfu[(v / TR) * H + h];
+                const bool keep = !(p < d.tau);
+                wgt[h] = keep ? p : 0.0f;
+                need |= keep;
+                nskip += keep ? 0 : 1;
+                if (d.skip_mask) d.skip_mask[((long long)b * d.Hq + g * H + h) * d.T_cap + v] = keep ? 0 : 1;
+              }
+              cnt_heads += nskip;
+              cnt_rows += need ? 0 : 1;
+            }
+            const unsigned bal = __ballot_sync(kFull, need);
+            if (need) {
+              const int idx = n_w + __popc(bal & ((1u << lane) - 1u));
+              list[idx] = v;
+              store_heads<H>(lwt + idx * H, wgt);
+            }
+            n_w += __popc(bal);
+          }
         }
         __syncwarp();
         // gather and accumulate this warp's rows
@@ -787,13 +826,8 @@ __global__ void __launch_bounds__(Geo<D, KB>::kThreads, 1) fused_decode_kernel(F
           for (int s2 = 0; s2 < kGatherUnroll; ++s2) {
             const int v = vv[s2];
             if (v < 0) continue;
-            float ev[H], wgt[H];
-            ldcg_heads<H>(lgu + (long long)v * H, ev);
-#pragma unroll
-            for (int h = 0; h < H; ++h) {
-              const float p = ev[h] * tfu[(v / TR) * H + h];
-              wgt[h] = (p < d.tau) ? 0.0f : p;
-            }
+            float wgt[H];
+            lds_heads<H>(lwt + (i0 + s2 * RPW + lane / LPR) * H, wgt);
             if constexpr (kOneWidth) {
               accumulate_v<H, VB0>(w0[s2], mg0, szv[s2], wgt, acc, Z);
             } else {
