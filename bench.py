@@ -72,9 +72,24 @@ def traffic_table():
     return out
 
 
-def source_hash(rel):
-    with open(os.path.join(ROOT, rel), "rb") as f:
-        return hashlib.sha1(f.read()).hexdigest()[:12]
+# Sources each timed kernel is compiled from (an ncu traffic figure only
+# counts while these files are unchanged).
+CSRC = "quantized_kv_cache_lkv_b200/csrc/"
+KERNEL_SOURCES = {
+    "quantize": [CSRC + "quantize.cu", CSRC + "lkv_device.cuh"],
+    "repack": [CSRC + "quantize.cu", CSRC + "lkv_device.cuh"],
+    "classify": [CSRC + "tier.cu"],
+    "decode": [CSRC + "fused_impl.cuh", CSRC + "fused_k6.cu", CSRC + "lkv_device.cuh"],
+    "tiered": [CSRC + "fused_impl.cuh", CSRC + "fused_k6.cu", CSRC + "lkv_device.cuh"],
+}
+
+
+def source_hash(name):
+    h = hashlib.sha1()
+    for rel in KERNEL_SOURCES[name]:
+        with open(os.path.join(ROOT, rel), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:12]
 
 
 class ClockSampler:
@@ -302,16 +317,11 @@ def run_lkv(args):
                       "frac": round(gbs / peak, 4), "share": round(ms / statistics.mean(step_ms), 4)}
     dominant = max(step.names, key=lambda k: kern[k]["us"])
     traffic = traffic_table()
-    src = {"quantize": "quantized_kv_cache_lkv_b200/csrc/quantize.cu",
-           "decode": "quantized_kv_cache_lkv_b200/csrc/decode.cu",
-           "tiered": "quantized_kv_cache_lkv_b200/csrc/decode.cu",
-           "classify": "quantized_kv_cache_lkv_b200/csrc/tier.cu",
-           "repack": "quantized_kv_cache_lkv_b200/csrc/quantize.cu"}
 
     def roofline(name):
         tr = traffic.get(name)
         t_bytes = None
-        if tr and tr[0] == source_hash(src[name]):
+        if tr and tr[0] == source_hash(name):
             t_bytes = tr[1]
         return {"bound": "hbm", "achieved": kern[name]["gbs"], "peak": peak, "unit": "GB/s",
                 "frac": kern[name]["frac"], "traffic": t_bytes, "kernel": name,
