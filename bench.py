@@ -181,6 +181,31 @@ def path_bytes(cfg, seq_lens, counts, skipped_rows, skipped_rows_tiered):
     return by
 
 
+# ----------------------------------------------------------------- ranks
+
+def rank_workload(rank):
+    """The batch rank `rank` decodes: the bench workload with its own seed, so
+    the ranks process distinct, independent batches (weak scaling)."""
+    base = W.CONFIGS[CFG_ID]
+    return W.scaled(base, seed=base.seed + 1000 * rank)
+
+
+def max_over_ranks(x, device=None):
+    """Maximum of a float over all ranks (the job's time is the slowest
+    rank's); every rank takes part, with or without a process group."""
+    import torch.distributed as tdist
+    if not (tdist.is_available() and tdist.is_initialized()) or tdist.get_world_size() == 1:
+        return float(x)
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    tdist.all_reduce(t, op=tdist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(bytes_per_rank_step, world, steps, max_ms):
+    """Whole-job GB/s: the bytes all ranks moved over the slowest rank's time."""
+    return bytes_per_rank_step * world * steps / (max_ms * 1e-3) / 1e9
+
+
 # ----------------------------------------------------------------- the step
 
 class Step:
@@ -268,7 +293,7 @@ def run_lkv(args):
     from __graft_entry__ import build
     build()
 
-    cfg = W.scaled(W.CONFIGS[CFG_ID], seed=W.CONFIGS[CFG_ID].seed + 1000 * rank)
+    cfg = rank_workload(rank)
     inp = W.make_inputs(cfg, with_mass=True)
     step = Step(cfg, inp, device)
     stream = torch.cuda.current_stream(device)
@@ -297,14 +322,10 @@ def run_lkv(args):
         for j, name in enumerate(step.names):
             per_kernel[name].append(ev[i][j].elapsed_time(ev[i][j + 1]))
         step_ms.append(ev[i][0].elapsed_time(ev[i][n]))
-    total_ms = sum(step_ms)
-    if dist:
-        t = torch.tensor([total_ms], device=device)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        total_ms = float(t.item())
+    total_ms = max_over_ranks(sum(step_ms), device)
     by = step.algorithmic_bytes()
     step_bytes = sum(by.values())
-    value = step_bytes * world * args.steps / (total_ms * 1e-3) / 1e9
+    value = job_throughput(step_bytes, world, args.steps, total_ms)
     kv_tokens = int(inp["seq_lens"].sum()) * world
     peak, peak_kind = peaks()
 
@@ -327,10 +348,11 @@ def run_lkv(args):
                 "frac": kern[name]["frac"], "traffic": t_bytes, "kernel": name,
                 "peak_source": f"{peak_kind} hbm_gbs"}
 
-    e2e = run_e2e(step, inp, device, stream, args) if (not dist or rank == 0) and not args.no_e2e else None
-    if dist:
-        e2e_t = torch.tensor([e2e["seconds"] if e2e else 0.0], device=device)
-        torch.distributed.all_reduce(e2e_t, op=torch.distributed.ReduceOp.MAX)
+    e2e = None
+    if not args.no_e2e:   # every rank runs it; the job's time is the slowest rank's
+        e2e = run_e2e(step, inp, device, stream, args)
+        sec = max_over_ranks(e2e["seconds"], device)
+        e2e["value"] = round(job_throughput(e2e["bytes"], world, e2e["steps"], sec * 1e3), 2)
     cpu = cpu_baseline(cfg, inp, args) if rank == 0 and world == 1 and not args.no_cpu else None
 
     if rank == 0:
@@ -391,7 +413,7 @@ def run_e2e(step, inp, device, stream, args):
     sec = start.elapsed_time(end) * 1e-3
     by = sum(step.algorithmic_bytes().values())
     return {"value": round(by * n / sec / 1e9, 2), "unit": "GB/s", "h2d_bytes_per_step": h2d,
-            "d2h_bytes_per_step": d2h, "seconds": sec}
+            "d2h_bytes_per_step": d2h, "seconds": sec, "bytes": by, "steps": n}
 
 
 # ----------------------------------------------------------------- CPU oracle
