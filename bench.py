@@ -448,9 +448,18 @@ def cpu_baseline(cfg, inp, args):
         t0 = time.perf_counter()
         by = oracle_step(oracle, cfg, oracle_sample(cfg, inp, n_seq))
         dt = time.perf_counter() - t0
-    return {"value": round(by / dt / 1e9, 4), "unit": "GB/s", "cores": oracle.threads(), "kind": "oracle",
-            "sample": f"first {n_seq} of {cfg.B} sequences of {cfg.name}, one oracle pass "
-                      f"(quantize + decode + tiers + repack + tiered), {dt:.1f} s"}
+    # the whole batch may still be quick on a large host: repeat the pass
+    sample = oracle_sample(cfg, inp, n_seq)
+    passes, total_by, total_dt = 1, by, dt
+    while total_dt < target / 2:
+        t0 = time.perf_counter()
+        total_by += oracle_step(oracle, cfg, sample)
+        total_dt += time.perf_counter() - t0
+        passes += 1
+    return {"value": round(total_by / total_dt / 1e9, 4), "unit": "GB/s", "cores": oracle.threads(),
+            "kind": "oracle",
+            "sample": f"first {n_seq} of {cfg.B} sequences of {cfg.name}, {passes} oracle pass(es) "
+                      f"(quantize + decode + tiers + repack + tiered), {total_dt:.1f} s"}
 
 
 def run_reference(args):
