@@ -26,20 +26,6 @@ int num_sms() {
   return cached[dev];
 }
 
-// Opt-in dynamic shared memory per block of the current device.
-static int max_smem_optin() {
-  static int cached[64] = {0};
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 232448;
-  if (cached[dev] == 0) {
-    int n = 0;
-    if (cudaDeviceGetAttribute(&n, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) != cudaSuccess || n <= 0)
-      n = 232448;
-    cached[dev] = n;
-  }
-  return cached[dev];
-}
-
 namespace {
 
 constexpr int kChunk = 256;       // decode rows per chunk

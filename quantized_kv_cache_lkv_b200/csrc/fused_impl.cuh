@@ -30,6 +30,7 @@
 // integers (unpack) and, with the group's (scale, zero),
 //   sum_d q_d * (scale * c_d + zero) = scale * sum_d q_d c_d + zero * sum_d q_d.
 #pragma once
+#include <type_traits>
 #include <cfloat>
 
 #include "lkv_kernels.cuh"
@@ -49,9 +50,10 @@ constexpr int kTsCap = 128;    // tile statistics kept in shared memory up to th
 constexpr int kQSlots = 4;     // units whose prescaled q is staged in shared memory
 constexpr unsigned kFull = 0xFFFFFFFFu;
 constexpr int kBarCons = 1;    // named barrier of the consumer warps
-// Shared header (bytes): barriers [0, 512), unused [512, 1536),
-// misc ints [1536, 2048), tile statistics [2048, 8192), q of up to kQSlots
+// Shared header (bytes): barriers [0, 512), per-group q sums of up to
+// kQSlots units [512, 1536), misc ints [1536, 2048), tile statistics [2048, 8192), q of up to kQSlots
 // units [8192, 16384).
+constexpr int kQgOff = 512;
 constexpr int kMiscOff = 1536;
 constexpr int kTsOff = 2048;
 constexpr int kQOff = 8192;
@@ -287,7 +289,7 @@ __global__ void __launch_bounds__(Geo<D, KB>::kThreads, 1) fused_decode_kernel(F
   constexpr int CW = Gk::kCW, NCONS = Gk::kConsumers, NTHR = Gk::kThreads;
   constexpr int RPL = Gk::RPL, TR = Gk::kTileRows, TPC = Gk::kTilesPerChunk;
   constexpr int LPR = D / kDimsPerLane, RPW = 32 / LPR;  // phase-2 lane mapping (16 channels per lane)
-  constexpr int CH = D / 16, NW = KB / 2;
+  constexpr int NW = KB / 2;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int cta = blockIdx.x, grid = gridDim.x;
@@ -430,7 +432,10 @@ __global__ void __launch_bounds__(Geo<D, KB>::kThreads, 1) fused_decode_kernel(F
       }
       const int lpg = d.G / DPL;  // lanes per quantization group
       for (int off = 1; off < lpg; off <<= 1) s += __shfl_xor_sync(kFull, s, off);
-      if (lane % lpg == 0) a.qgsum[((long long)x.u * H + h) * 4 + lane / lpg] = s;
+      if (lane % lpg == 0) {
+        a.qgsum[((long long)x.u * H + h) * 4 + lane / lpg] = s;
+        if (e < kQSlots) reinterpret_cast<float*>(smem_raw + kQgOff)[(e * H + h) * 4 + lane / lpg] = s;
+      }
     }
   }
   __syncthreads();  // q ready; phase 1 starts
@@ -483,9 +488,6 @@ __global__ void __launch_bounds__(Geo<D, KB>::kThreads, 1) fused_decode_kernel(F
     int issued = 0, consumed = 0;
     if (next_tile(p0)) { issue(p0, warp * kSlotsPerWarp + 0); ++issued; }
     if (issued == 1 && next_tile(p1)) { issue(p1, warp * kSlotsPerWarp + 1); ++issued; }
-    int cur_e = -1;
-    const float* qv = nullptr;
-    const float* qg = nullptr;
     while (consumed < issued) {
       const int slotw = consumed % kSlotsPerWarp;
       const int stage = warp * kSlotsPerWarp + slotw;
@@ -496,13 +498,6 @@ __global__ void __launch_bounds__(Geo<D, KB>::kThreads, 1) fused_decode_kernel(F
         break;
       }
       const TileDesc td = slotw ? p1 : p0;
-      if (td.entry != cur_e) {
-        cur_e = td.entry;
-        const int u = td.u;
-        qv = cur_e < kQSlots ? reinterpret_cast<const float*>(smem_raw + kQOff) + cur_e * H * D
-                             : a.qbuf + (long long)u * H * D;
-        qg = a.qgsum + (long long)u * H * 4;
-      }
       const uint8_t* codes = ring + (size_t)stage * Gk::kStageBytes;
       const float* szs = reinterpret_cast<const float*>(codes + Gk::kStageCodes) +
                          ((ng == 1) ? (td.row0 & 1) : 0) * ng * 2;
@@ -515,6 +510,15 @@ __global__ void __launch_bounds__(Geo<D, KB>::kThreads, 1) fused_decode_kernel(F
         src[r] = reinterpret_cast<const uint4*>(codes + (valid[r] ? i : 0) * Gk::RB);
       }
       float dot[RPL][H];
+      // The dot products of the tile's rows with the unit's prescaled q (qv)
+      // and its per-group sums (qg).  Called with shared-memory pointers for
+      // the CTA's first kQSlots units (shared loads) and with global ones
+      // otherwise.
+      // SPG (16-channel slices per quantization group) is G / 16 when known at
+      // compile time, so the group folds sit at fixed places in the unrolled
+      // loop, or 0 to read G at run time.
+      auto k_rows = [&](auto spg, const float* __restrict__ qv, const float* __restrict__ qg) {
+      constexpr int SPG = decltype(spg)::value;
       float2 acc[RPL][H];
 #pragma unroll
       for (int r = 0; r < RPL; ++r)
@@ -567,8 +571,8 @@ __global__ void __launch_bounds__(Geo<D, KB>::kThreads, 1) fused_decode_kernel(F
                 acc[r][h] = __ffma2_rn(make_float2(qc[h].z, qc[h].w), cp[r][1], acc[r][h]);
               }
           }
-          if (((c + 1) * 16) % d.G == 0) {  // end of a quantization group: fold (scale, zero)
-            const int gidx = (c * 16) / d.G;
+          if (SPG ? ((c + 1) % SPG == 0) : (((c + 1) * 16) % d.G == 0)) {  // end of a group: fold (scale, zero)
+            const int gidx = SPG ? c / SPG : (c * 16) / d.G;
             float qsum[H];
 #pragma unroll
             for (int h = 0; h < H; ++h) qsum[h] = qg[h * 4 + gidx];
@@ -584,6 +588,16 @@ __global__ void __launch_bounds__(Geo<D, KB>::kThreads, 1) fused_decode_kernel(F
             }
           }
         }
+      }
+      };
+      if (td.entry < kQSlots) {
+        const float* qv_s = reinterpret_cast<const float*>(smem_raw + kQOff) + td.entry * H * D;
+        const float* qg_s = reinterpret_cast<const float*>(smem_raw + kQgOff) + td.entry * H * 4;
+        if (d.G == 32) k_rows(std::integral_constant<int, 2>{}, qv_s, qg_s);
+        else if (d.G == 64) k_rows(std::integral_constant<int, 4>{}, qv_s, qg_s);
+        else k_rows(std::integral_constant<int, 8>{}, qv_s, qg_s);
+      } else {
+        k_rows(std::integral_constant<int, 0>{}, a.qbuf + (long long)td.u * H * D, a.qgsum + (long long)td.u * H * 4);
       }
       // The stage's data is in registers now: refill it with this warp's next tile.
       ++consumed;
