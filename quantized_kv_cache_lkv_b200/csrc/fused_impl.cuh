@@ -314,6 +314,7 @@ __global__ void __launch_bounds__(Geo<D, KB>::kThreads, 1) fused_decode_kernel(F
   float* s_glob = reinterpret_cast<float*>(misc + 8);  // (max, 1/sum) x 4 heads
   int* s_wsum = misc + 16;                            // 2 x 12 warp partials
   int* s_magic = misc + 48;                           // 24 magic exponent fields
+  int* s_nw = misc + 96;                              // kept rows per warp in a phase-2 batch
 
   if (tid == 0) {
     for (int s = 0; s < Gk::kStages; ++s) mbar_init(&full[s], 1);
@@ -704,6 +705,7 @@ __global__ void __launch_bounds__(Geo<D, KB>::kThreads, 1) fused_decode_kernel(F
   Magic<VB1> mg1;
   mg1.load(s_magic);
   unsigned long long cnt_heads = 0, cnt_rows = 0;
+  uint8_t* const smask = d.skip_mask;
   for (int pass = 0; pass < 2; ++pass) {
     for (int e = 0; e < n_work; ++e) {
       int* rec = ulist + (long long)e * kRec;
@@ -763,66 +765,87 @@ __global__ void __launch_bounds__(Geo<D, KB>::kThreads, 1) fused_decode_kernel(F
       }
       for (int vb = v_lo; vb < v_hi; vb += NCONS * kBatchBlocks) {
         // scan: 32-row blocks round robin over warps, row order kept per warp;
-        // the logits of kScanBlocks blocks are loaded before any is used
+        // the logits of kScanBlocks blocks are loaded before any is used.  A
+        // block lies in one chunk and one tile, so its valid-row count and
+        // its tile factors are the same for the whole warp.
         int* list = lists + warp * kListCap;
         float* lwt = wts + warp * kListCap * H;
         int n_w = 0;
+        uint32_t my_skip = 0, my_rows = 0;
         for (int blk0 = warp; blk0 < CW * kBatchBlocks; blk0 += kScanBlocks * CW) {
           if (vb + blk0 * 32 >= v_hi) break;
           float ev[kScanBlocks][H];
-          bool in[kScanBlocks];
+          int nvalid[kScanBlocks];
 #pragma unroll
           for (int u = 0; u < kScanBlocks; ++u) {
             const int blk = blk0 + u * CW;
-            const int v = vb + blk * 32 + lane;
-            in[u] = false;
-            if (blk < CW * kBatchBlocks && vb + blk * 32 < v_hi) in[u] = v % kChunk < chunk_rows(x, v / kChunk).rows;
-            if (in[u]) ldcg_heads<H>(lgu + (long long)v * H, ev[u]);
+            const int v0 = vb + blk * 32;
+            nvalid[u] = 0;
+            if (blk < CW * kBatchBlocks && v0 < v_hi) nvalid[u] = chunk_rows(x, v0 / kChunk).rows - v0 % kChunk;
+            if (lane < nvalid[u]) ldcg_heads<H>(lgu + (long long)(v0 + lane) * H, ev[u]);
           }
 #pragma unroll
           for (int u = 0; u < kScanBlocks; ++u) {
             const int blk = blk0 + u * CW;
-            if (blk >= CW * kBatchBlocks || vb + blk * 32 >= v_hi) break;  // the same for the whole warp
-            const int v = vb + blk * 32 + lane;
+            const int v0 = vb + blk * 32;
+            if (blk >= CW * kBatchBlocks || v0 >= v_hi) break;  // the same for the whole warp
+            float f[H], wgt[H];
+            lds_heads<H>(tfu + (v0 / TR) * H, f);
             bool need = false;
-            float wgt[H];
-#pragma unroll
-            for (int h = 0; h < H; ++h) wgt[h] = 0.0f;
-            if (in[u]) {
-              int nskip = 0;
+            if (lane < nvalid[u]) {
 #pragma unroll
               for (int h = 0; h < H; ++h) {
-                const float p = ev[u][h] * tfu[(v / TR) * H + h];
+                const float p = ev[u][h] * f[h];
                 const bool keep = !(p < d.tau);
                 wgt[h] = keep ? p : 0.0f;
                 need |= keep;
-                nskip += keep ? 0 : 1;
-                if (d.skip_mask) d.skip_mask[((long long)b * d.Hq + g * H + h) * d.T_cap + v] = keep ? 0 : 1;
+                my_skip += keep ? 0u : 1u;
               }
-              cnt_heads += nskip;
-              cnt_rows += need ? 0 : 1;
+              my_rows += need ? 0u : 1u;
+              if (smask) {
+#pragma unroll
+                for (int h = 0; h < H; ++h)
+                  smask[((long long)b * d.Hq + g * H + h) * d.T_cap + v0 + lane] = (ev[u][h] * f[h] < d.tau) ? 1 : 0;
+              }
             }
             const unsigned bal = __ballot_sync(kFull, need);
             if (need) {
               const int idx = n_w + __popc(bal & ((1u << lane) - 1u));
-              list[idx] = v;
+              list[idx] = v0 + lane;
               store_heads<H>(lwt + idx * H, wgt);
             }
             n_w += __popc(bal);
           }
         }
+        cnt_heads += my_skip;
+        cnt_rows += my_rows;
         __syncwarp();
-        // gather and accumulate this warp's rows
-        for (int i0 = 0; i0 < n_w; i0 += kGatherUnroll * RPW) {
+        // gather: the CTA's kept rows (warp 0's list, then warp 1's, ...) are
+        // split evenly over the warps, in order, so every warp waits for about
+        // the same number of HBM round trips
+        if (lane == 0) s_nw[warp] = n_w;
+        named_barrier(kBarCons, NCONS);
+        int n_all = 0;
+#pragma unroll
+        for (int w2 = 0; w2 < CW; ++w2) n_all += s_nw[w2];
+        const int per = ((n_all + CW - 1) / CW + RPW - 1) / RPW * RPW;
+        const int g_lo = min(n_all, warp * per), g_hi = min(n_all, g_lo + per);
+        int sw = 0, sbase = 0;  // list holding the lane's next entry, entries before it
+        for (int i0 = g_lo; i0 < g_hi; i0 += kGatherUnroll * RPW) {
           constexpr bool kOneWidth = (VB0 == VB1);
           LaneWords<VB0> w0[kGatherUnroll];
           LaneWords<kOneWidth ? 2 : VB1> w1[kOneWidth ? 1 : kGatherUnroll];
           float2 szv[kGatherUnroll];
-          int vv[kGatherUnroll];
+          int vv[kGatherUnroll], li[kGatherUnroll];
 #pragma unroll
           for (int s2 = 0; s2 < kGatherUnroll; ++s2) {
-            const int idx = i0 + s2 * RPW + lane / LPR;
-            vv[s2] = idx < n_w ? list[idx] : -1;
+            const int gidx = i0 + s2 * RPW + lane / LPR;
+            li[s2] = -1;
+            if (gidx < g_hi) {
+              while (gidx >= sbase + s_nw[sw]) { sbase += s_nw[sw]; ++sw; }
+              li[s2] = sw * kListCap + gidx - sbase;
+            }
+            vv[s2] = li[s2] >= 0 ? lists[li[s2]] : -1;
             if (vv[s2] >= 0) {
               const int v = vv[s2];
               const ChunkRows cr = chunk_rows(x, v / kChunk);
@@ -841,7 +864,7 @@ __global__ void __launch_bounds__(Geo<D, KB>::kThreads, 1) fused_decode_kernel(F
             const int v = vv[s2];
             if (v < 0) continue;
             float wgt[H];
-            lds_heads<H>(lwt + (i0 + s2 * RPW + lane / LPR) * H, wgt);
+            lds_heads<H>(wts + li[s2] * H, wgt);
             if constexpr (kOneWidth) {
               accumulate_v<H, VB0>(w0[s2], mg0, szv[s2], wgt, acc, Z);
             } else {
@@ -850,7 +873,7 @@ __global__ void __launch_bounds__(Geo<D, KB>::kThreads, 1) fused_decode_kernel(F
             }
           }
         }
-        __syncwarp();
+        named_barrier(kBarCons, NCONS);  // other warps read this batch's lists
       }
       // fold the per-group constant, reduce the row slots of the warp
 #pragma unroll
