@@ -123,6 +123,23 @@ LKV_API int lkv_quantize_kv(lkv_qspec spec, int B, int Hkv, int T_cap, int D,
                     void *stream);
 
 /*
+ * lkv_append_kv -- quantize the newest token of every (b, g) into the packed
+ * cache in place: the step before decode in a decode loop ([LKV]
+ * §实现细节与工程考量: quantization must keep pace with generation).  Row
+ * pos[b] of every KV head of sequence b receives the codes and (scale, zero)
+ * that lkv_quantize_kv would write for that token; no other row changes.
+ *
+ *   pos          in   int32 [B], device: the slot to write (normally the
+ *                     length before this token); a value outside [0, T_cap)
+ *                     writes nothing for that sequence
+ *   k_new, v_new in   bf16 [B][Hkv][D]
+ *   k_codes...   in/out  the packed cache of lkv_quantize_kv
+ */
+LKV_API int lkv_append_kv(lkv_qspec spec, int B, int Hkv, int T_cap, int D, const int32_t *pos,
+                  const void *k_new, const void *v_new, void *k_codes, float *k_sz, void *v_codes,
+                  float *v_sz, void *stream);
+
+/*
  * Workspace bytes that lkv_decode_attention needs for these sizes on the
  * current device (the size depends on its SM count).  The workspace is
  * caller-owned device memory (256-byte aligned).  It must be zero-filled
@@ -165,6 +182,27 @@ LKV_API int lkv_decode_attention(lkv_qspec spec, int B, int Hq, int Hkv, int T_c
                          const float *k_sz, const void *v_codes, const float *v_sz,
                          float softmax_scale, float tau, float *out, uint8_t *skip_mask,
                          int64_t *skip_counts, void *workspace, size_t ws_bytes,
+                         void *stream);
+
+/*
+ * lkv_decode_attention_mass -- lkv_decode_attention that also emits, for
+ * every token, the attention its KV group paid to it in this step: the
+ * input of the next step's lkv_tier_classify ([SKV] §第二层: the attention
+ * weights are the signal that ranks tokens into tiers).
+ *
+ *   mass  out  f32 [B][Hkv][T_cap], not NULL (4-byte aligned):
+ *              mass[b][g][t] = (1/r) * sum over the r query heads h of group
+ *              g of p[b][h][t], the softmax probability before the sparse-V
+ *              skip, for t < T_b; slots t >= T_b are not written.  Over t it
+ *              sums to 1 for every (b, g) with T_b > 0.
+ * Every other argument and the return value are those of
+ * lkv_decode_attention.  Arithmetic is fp32.
+ */
+LKV_API int lkv_decode_attention_mass(lkv_qspec spec, int B, int Hq, int Hkv, int T_cap, int D,
+                         const int32_t *seq_lens, const void *q, const void *k_codes,
+                         const float *k_sz, const void *v_codes, const float *v_sz,
+                         float softmax_scale, float tau, float *out, uint8_t *skip_mask,
+                         int64_t *skip_counts, float *mass, void *workspace, size_t ws_bytes,
                          void *stream);
 
 /*

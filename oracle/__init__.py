@@ -168,6 +168,25 @@ def decode_attention(kb, vb, G, seq_lens, q_bf16, cache, softmax_scale, tau, wan
     return out, mask, counts
 
 
+def attention_mass(p, Hkv, seq_lens):
+    """Per-token attention mass of each KV group for the next step's tiers
+    ("Super KV Compression" §第二层: the attention weights rank the tokens):
+    mass[b, g, t] = mean over the r query heads of group g of p[b, h, t]
+    (the softmax probability before the sparse-V skip), for t < T_b; 0 for
+    the slots beyond.  p is the f64 [B, Hq, T_cap] of decode_attention."""
+    p = np.asarray(p, np.float64)
+    B, Hq, T_cap = p.shape
+    r = Hq // Hkv
+    mass = np.zeros((B, Hkv, T_cap), np.float64)
+    for b in range(B):
+        T = int(seq_lens[b])
+        for g in range(Hkv):
+            for h in range(g * r, (g + 1) * r):
+                mass[b, g, :T] += p[b, h, :T]
+            mass[b, g, :T] /= r
+    return mass
+
+
 def tier_classify(seq_lens, mass, tau_low, tau_high):
     """mass f32 [B, Hkv, T_cap] -> (tier i8, counts i32 [B,Hkv,2], pos2, pos1 i32 [B,Hkv,T_cap]).
 

@@ -227,6 +227,13 @@ size_t static_zero_prefix(int B, int Hq, int Hkv, int T_cap, int D, int KB) {
 
 }  // namespace
 
+namespace {
+int decode_impl(lkv_qspec spec, int B, int Hq, int Hkv, int T_cap, int D, const int32_t* seq_lens, const void* q,
+                const void* k_codes, const float* k_sz, const void* v_codes, const float* v_sz, float softmax_scale,
+                float tau, float* out, uint8_t* skip_mask, int64_t* skip_counts, float* mass, void* workspace,
+                size_t ws_bytes, void* stream);
+}  // namespace
+
 extern "C" {
 
 const char* lkv_status_string(int status) {
@@ -275,6 +282,28 @@ int lkv_quantize_kv(lkv_qspec spec, int B, int Hkv, int T_cap, int D, const int3
   return from_cuda(launch_quantize_kv(a, spec.k_bits, spec.v_bits, D, static_cast<cudaStream_t>(stream)));
 }
 
+int lkv_append_kv(lkv_qspec spec, int B, int Hkv, int T_cap, int D, const int32_t* pos, const void* k_new,
+                  const void* v_new, void* k_codes, float* k_sz, void* v_codes, float* v_sz, void* stream) {
+  if (!bits_ok(spec.k_bits) || !bits_ok(spec.v_bits)) return LKV_ERR_UNSUPPORTED;
+  int rc = check_cache_shape(B, Hkv, T_cap, D, spec.group);
+  if (rc) return rc;
+  const bool ne = (long long)B * Hkv * T_cap > 0;
+  if (!ptr_ok(pos, ne) || !ptr_ok(k_new, ne) || !ptr_ok(v_new, ne) || !ptr_ok(k_codes, ne) || !ptr_ok(k_sz, ne) ||
+      !ptr_ok(v_codes, ne) || !ptr_ok(v_sz, ne))
+    return LKV_ERR_INVALID_ARG;
+  if (!ne) return LKV_OK;
+  QuantizeArgs a{};
+  a.B = B; a.Hkv = Hkv; a.T_cap = T_cap; a.G = spec.group; a.one = 1.0f;
+  a.seq_lens = pos;
+  a.k = static_cast<const uint16_t*>(k_new);
+  a.v = static_cast<const uint16_t*>(v_new);
+  a.k_codes = static_cast<uint8_t*>(k_codes);
+  a.k_sz = k_sz;
+  a.v_codes = static_cast<uint8_t*>(v_codes);
+  a.v_sz = v_sz;
+  return from_cuda(launch_append_kv(a, spec.k_bits, spec.v_bits, D, static_cast<cudaStream_t>(stream)));
+}
+
 size_t lkv_decode_workspace_bytes(lkv_qspec spec, int B, int Hq, int Hkv, int T_cap, int D) {
   if (!bits_ok(spec.k_bits) || !bits_ok(spec.v_bits)) return 0;
   if (check_attention_shape(B, Hq, Hkv, T_cap, D, spec.group)) return 0;
@@ -285,6 +314,27 @@ int lkv_decode_attention(lkv_qspec spec, int B, int Hq, int Hkv, int T_cap, int 
                          const void* q, const void* k_codes, const float* k_sz, const void* v_codes,
                          const float* v_sz, float softmax_scale, float tau, float* out, uint8_t* skip_mask,
                          int64_t* skip_counts, void* workspace, size_t ws_bytes, void* stream) {
+  return decode_impl(spec, B, Hq, Hkv, T_cap, D, seq_lens, q, k_codes, k_sz, v_codes, v_sz, softmax_scale, tau,
+                     out, skip_mask, skip_counts, nullptr, workspace, ws_bytes, stream);
+}
+
+int lkv_decode_attention_mass(lkv_qspec spec, int B, int Hq, int Hkv, int T_cap, int D, const int32_t* seq_lens,
+                              const void* q, const void* k_codes, const float* k_sz, const void* v_codes,
+                              const float* v_sz, float softmax_scale, float tau, float* out, uint8_t* skip_mask,
+                              int64_t* skip_counts, float* mass, void* workspace, size_t ws_bytes, void* stream) {
+  if (mass == nullptr && (long long)B * Hkv * T_cap > 0) return LKV_ERR_INVALID_ARG;
+  return decode_impl(spec, B, Hq, Hkv, T_cap, D, seq_lens, q, k_codes, k_sz, v_codes, v_sz, softmax_scale, tau,
+                     out, skip_mask, skip_counts, mass, workspace, ws_bytes, stream);
+}
+
+}  // extern "C"
+
+namespace {
+
+int decode_impl(lkv_qspec spec, int B, int Hq, int Hkv, int T_cap, int D, const int32_t* seq_lens, const void* q,
+                const void* k_codes, const float* k_sz, const void* v_codes, const float* v_sz, float softmax_scale,
+                float tau, float* out, uint8_t* skip_mask, int64_t* skip_counts, float* mass, void* workspace,
+                size_t ws_bytes, void* stream) {
   if (!bits_ok(spec.k_bits) || !bits_ok(spec.v_bits)) return LKV_ERR_UNSUPPORTED;
   int rc = check_attention_shape(B, Hq, Hkv, T_cap, D, spec.group);
   if (rc) return rc;
@@ -294,6 +344,7 @@ int lkv_decode_attention(lkv_qspec spec, int B, int Hq, int Hkv, int T_cap, int 
       !ptr_ok(k_sz, ne) || !ptr_ok(v_codes, ne) || !ptr_ok(v_sz, ne))
     return LKV_ERR_INVALID_ARG;
   if (skip_counts && !aligned16(skip_counts)) return LKV_ERR_INVALID_ARG;
+  if (mass && (reinterpret_cast<uintptr_t>(mass) & 3u) != 0) return LKV_ERR_INVALID_ARG;
   if (workspace == nullptr || (reinterpret_cast<uintptr_t>(workspace) % kAlign) != 0) return LKV_ERR_INVALID_ARG;
   if (ws_bytes < attention_ws_bytes(B, Hq, Hkv, T_cap, D, spec.k_bits)) return LKV_ERR_WORKSPACE;
   DecodeArgs a{};
@@ -313,9 +364,14 @@ int lkv_decode_attention(lkv_qspec spec, int B, int Hq, int Hkv, int T_cap, int 
   a.tau = tau;
   a.out = out;
   a.skip_mask = skip_mask;
+  a.mass = mass;
   a.skip_counts = reinterpret_cast<unsigned long long*>(skip_counts);
   return run_attention(a, D, spec.k_bits, spec.v_bits, spec.v_bits, workspace, ws_bytes, s);
 }
+
+}  // namespace
+
+extern "C" {
 
 int lkv_decode_attention_static(lkv_qspec spec, int B, int Hq, int Hkv, int T_cap, int D, const int32_t* seq_lens,
                                 const void* q, const void* k_codes, const float* k_sz, const void* v_codes,

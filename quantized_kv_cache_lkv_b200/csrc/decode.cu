@@ -278,6 +278,11 @@ __global__ void __launch_bounds__(kThreads) v_phase_kernel(DecodeArgs a) {
       need |= keep[h];
     }
     if (j == 0) {
+      if (a.mass && z == 0) {  // the group's mean attention to the row, over all r heads
+        float ms = 0.0f;
+        for (int hh = 0; hh < a.r; ++hh) ms += exp2f(a.logits[lrow * a.r + hh] - sm_m[hh]) * sm_il[hh];
+        a.mass[lrow] = ms * (1.0f / a.r);
+      }
       if (a.skip_mask) {
 #pragma unroll
         for (int h = 0; h < H; ++h)

@@ -706,6 +706,7 @@ __global__ void __launch_bounds__(Geo<D, KB>::kThreads, 1) fused_decode_kernel(F
   mg1.load(s_magic);
   unsigned long long cnt_heads = 0, cnt_rows = 0;
   uint8_t* const smask = d.skip_mask;
+  float* const mass_out = d.mass;
   for (int pass = 0; pass < 2; ++pass) {
     for (int e = 0; e < n_work; ++e) {
       int* rec = ulist + (long long)e * kRec;
@@ -802,6 +803,12 @@ __global__ void __launch_bounds__(Geo<D, KB>::kThreads, 1) fused_decode_kernel(F
                 my_skip += keep ? 0u : 1u;
               }
               my_rows += need ? 0u : 1u;
+              if (mass_out) {  // the group's mean attention to the row
+                float ms = 0.0f;
+#pragma unroll
+                for (int h = 0; h < H; ++h) ms += ev[u][h] * f[h];
+                mass_out[((long long)b * d.Hkv + g) * d.T_cap + v0 + lane] = ms * (1.0f / H);
+              }
               if (smask) {
 #pragma unroll
                 for (int h = 0; h < H; ++h)

@@ -57,6 +57,7 @@ struct DecodeArgs {
   float tau;
   float* out;
   uint8_t* skip_mask;    // nullable, [B][Hq][T_cap] (plain decode only)
+  float* mass;           // nullable, [B][Hkv][T_cap]: mean over the group's heads of p (plain decode only)
   unsigned long long* skip_counts;  // nullable, [2]
   // workspace
   int* status;
@@ -98,6 +99,8 @@ cudaError_t launch_fused_k8(const FusedArgs& a, int D, int H, int vb0, int vb1, 
 int num_sms();
 
 cudaError_t launch_quantize_kv(const QuantizeArgs& a, int kb, int vb, int D, cudaStream_t s);
+// seq_lens holds the slot to write per sequence; k, v hold [B][Hkv][D].
+cudaError_t launch_append_kv(const QuantizeArgs& a, int kb, int vb, int D, cudaStream_t s);
 cudaError_t launch_tier_repack(const RepackArgs& a, int D, cudaStream_t s);
 cudaError_t launch_tier_classify(const ClassifyArgs& a, cudaStream_t s);
 // vb0 / vb1: V bit widths of segment 0 / 1 (equal for plain decode).

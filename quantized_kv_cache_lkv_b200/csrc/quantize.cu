@@ -101,6 +101,29 @@ __global__ void __launch_bounds__(256, 4) quantize_kv_kernel(QuantizeArgs a) {
   }
 }
 
+// Append: the new token of every (b, g) -- bf16 K and V rows [B][Hkv][D] --
+// quantized into slot pos[b] of the packed cache, with the formula of
+// quantize_kv_kernel (the step just before decode in a decode loop).  A
+// position outside [0, T_cap) writes nothing.
+template <int D, int KB, int VB>
+__global__ void __launch_bounds__(256) append_kv_kernel(QuantizeArgs a) {
+  constexpr int LPR = D / kDimsPerLane;
+  constexpr int RPW = 32 / LPR;
+  const int lane = threadIdx.x & 31;
+  const int j = lane % LPR, sub = lane / LPR;
+  const unsigned mask = row_lane_mask<LPR>(lane);
+  const int ng = D / a.G, lpg = a.G / kDimsPerLane;
+  const long long unit = ((long long)blockIdx.x * (blockDim.x / 32) + threadIdx.x / 32) * RPW + sub;
+  if (unit >= (long long)a.B * a.Hkv) return;  // the lanes of a row agree
+  const int t = __ldg(a.seq_lens + unit / a.Hkv);
+  if (t < 0 || t >= a.T_cap) return;
+  const long long row = unit * a.T_cap + t;
+  LaneRows r;
+  fetch_lane_rows(a.k + unit * D + j * kDimsPerLane, a.v + unit * D + j * kDimsPerLane, r);
+  quantize_lane<KB>(r.k0, r.k1, a.k_codes + row * (D * KB / 8), a.k_sz + row * ng * 2, j, lpg, mask, a.one);
+  quantize_lane<VB>(r.v0, r.v1, a.v_codes + row * (D * VB / 8), a.v_sz + row * ng * 2, j, lpg, mask, a.one);
+}
+
 // Tier repack: row i of segment A (tier 2) or B (tier 1) of (b, g) is the
 // token at pos[b][g][i], quantized from bf16 with K at 6 bits and V at 6 (A)
 // or 4 (B) bits ("Super KV Compression", §第二层 items 1-2).  Block
@@ -170,24 +193,34 @@ static cudaError_t launch_quantize_t(const QuantizeArgs& a, cudaStream_t s) {
   return cudaGetLastError();
 }
 
+template <int D, int KB, int VB>
+static cudaError_t launch_append_t(const QuantizeArgs& a, cudaStream_t s) {
+  constexpr int RPW = 32 / (D / kDimsPerLane);
+  const long long units = (long long)a.B * a.Hkv;
+  const long long blocks = (units + 8 * RPW - 1) / (8 * RPW);
+  if (blocks >= (1ll << 31)) return cudaErrorInvalidValue;
+  append_kv_kernel<D, KB, VB><<<(unsigned)blocks, 256, 0, s>>>(a);
+  return cudaGetLastError();
+}
+
 template <int D, int KB>
-static cudaError_t launch_quantize_vb(const QuantizeArgs& a, int vb, cudaStream_t s) {
+static cudaError_t launch_quantize_vb(const QuantizeArgs& a, int vb, bool append, cudaStream_t s) {
   switch (vb) {
-    case 2: return launch_quantize_t<D, KB, 2>(a, s);
-    case 4: return launch_quantize_t<D, KB, 4>(a, s);
-    case 6: return launch_quantize_t<D, KB, 6>(a, s);
-    case 8: return launch_quantize_t<D, KB, 8>(a, s);
+    case 2: return append ? launch_append_t<D, KB, 2>(a, s) : launch_quantize_t<D, KB, 2>(a, s);
+    case 4: return append ? launch_append_t<D, KB, 4>(a, s) : launch_quantize_t<D, KB, 4>(a, s);
+    case 6: return append ? launch_append_t<D, KB, 6>(a, s) : launch_quantize_t<D, KB, 6>(a, s);
+    case 8: return append ? launch_append_t<D, KB, 8>(a, s) : launch_quantize_t<D, KB, 8>(a, s);
     default: return cudaErrorInvalidValue;
   }
 }
 
 template <int D>
-static cudaError_t launch_quantize_d(const QuantizeArgs& a, int kb, int vb, cudaStream_t s) {
+static cudaError_t launch_quantize_d(const QuantizeArgs& a, int kb, int vb, bool append, cudaStream_t s) {
   switch (kb) {
-    case 2: return launch_quantize_vb<D, 2>(a, vb, s);
-    case 4: return launch_quantize_vb<D, 4>(a, vb, s);
-    case 6: return launch_quantize_vb<D, 6>(a, vb, s);
-    case 8: return launch_quantize_vb<D, 8>(a, vb, s);
+    case 2: return launch_quantize_vb<D, 2>(a, vb, append, s);
+    case 4: return launch_quantize_vb<D, 4>(a, vb, append, s);
+    case 6: return launch_quantize_vb<D, 6>(a, vb, append, s);
+    case 8: return launch_quantize_vb<D, 8>(a, vb, append, s);
     default: return cudaErrorInvalidValue;
   }
 }
@@ -195,8 +228,15 @@ static cudaError_t launch_quantize_d(const QuantizeArgs& a, int kb, int vb, cuda
 cudaError_t launch_quantize_kv(const QuantizeArgs& a, int kb, int vb, int D, cudaStream_t s) {
   const long long n_rows = (long long)a.B * a.Hkv * a.T_cap;
   if (n_rows == 0) return cudaSuccess;
-  if (D == 64) return launch_quantize_d<64>(a, kb, vb, s);
-  if (D == 128) return launch_quantize_d<128>(a, kb, vb, s);
+  if (D == 64) return launch_quantize_d<64>(a, kb, vb, false, s);
+  if (D == 128) return launch_quantize_d<128>(a, kb, vb, false, s);
+  return cudaErrorInvalidValue;
+}
+
+cudaError_t launch_append_kv(const QuantizeArgs& a, int kb, int vb, int D, cudaStream_t s) {
+  if ((long long)a.B * a.Hkv * a.T_cap == 0) return cudaSuccess;
+  if (D == 64) return launch_quantize_d<64>(a, kb, vb, true, s);
+  if (D == 128) return launch_quantize_d<128>(a, kb, vb, true, s);
   return cudaErrorInvalidValue;
 }
 

@@ -48,9 +48,12 @@ SIGNATURES = {
     "lkv_row_bytes": (_Z, [_I, _I]),
     "lkv_sz_row_bytes": (_Z, [_I, _I]),
     "lkv_quantize_kv": (_I, [lkv_qspec, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P, _P, _P]),
+    "lkv_append_kv": (_I, [lkv_qspec, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P, _P, _P]),
     "lkv_decode_workspace_bytes": (_Z, [lkv_qspec, _I, _I, _I, _I, _I]),
     "lkv_decode_attention": (_I, [lkv_qspec, _I, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P, _F, _F,
                                   _P, _P, _P, _P, _Z, _P]),
+    "lkv_decode_attention_mass": (_I, [lkv_qspec, _I, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P, _F, _F,
+                                       _P, _P, _P, _P, _P, _Z, _P]),
     "lkv_decode_attention_static": (_I, [lkv_qspec, _I, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P, _F,
                                          _F, _P, _P, _P, _P, _P]),
     "lkv_workspace_reset": (_I, [_P, _Z, _P]),
@@ -140,6 +143,12 @@ def lkv_quantize_kv(spec, B, Hkv, T_cap, D, seq_lens, k, v, k_codes, k_sz, v_cod
                                  _stream(stream)), "lkv_quantize_kv")
 
 
+def lkv_append_kv(spec, B, Hkv, T_cap, D, pos, k_new, v_new, k_codes, k_sz, v_codes, v_sz, stream=None):
+    _check(lib().lkv_append_kv(_spec(spec), B, Hkv, T_cap, D, _ptr(pos), _ptr(k_new), _ptr(v_new),
+                               _ptr(k_codes), _ptr(k_sz), _ptr(v_codes), _ptr(v_sz), _stream(stream)),
+           "lkv_append_kv")
+
+
 def lkv_decode_workspace_bytes(spec, B, Hq, Hkv, T_cap, D):
     return lib().lkv_decode_workspace_bytes(_spec(spec), B, Hq, Hkv, T_cap, D)
 
@@ -152,6 +161,16 @@ def lkv_decode_attention(spec, B, Hq, Hkv, T_cap, D, seq_lens, q, k_codes, k_sz,
                                       float(softmax_scale), float(tau), _ptr(out), _ptr(skip_mask),
                                       _ptr(skip_counts), _ptr(workspace), int(ws_bytes),
                                       _stream(stream)), "lkv_decode_attention")
+
+
+def lkv_decode_attention_mass(spec, B, Hq, Hkv, T_cap, D, seq_lens, q, k_codes, k_sz, v_codes, v_sz,
+                              softmax_scale, tau, out, skip_mask, skip_counts, mass, workspace, ws_bytes,
+                              stream=None):
+    _check(lib().lkv_decode_attention_mass(_spec(spec), B, Hq, Hkv, T_cap, D, _ptr(seq_lens), _ptr(q),
+                                           _ptr(k_codes), _ptr(k_sz), _ptr(v_codes), _ptr(v_sz),
+                                           float(softmax_scale), float(tau), _ptr(out), _ptr(skip_mask),
+                                           _ptr(skip_counts), _ptr(mass), _ptr(workspace), int(ws_bytes),
+                                           _stream(stream)), "lkv_decode_attention_mass")
 
 
 LKV_STATIC_WORKSPACE_BYTES = 32 << 20

@@ -143,6 +143,21 @@ def test_static_decode_rejects_before_any_device_call(L):
     assert rc_of(call, **static_args(q=None)) == lkv.LKV_ERR_INVALID_ARG
 
 
+def test_append_and_mass_reject(L):
+    call = lambda *a: lkv.lkv_append_kv(*a)
+    base = [K6V4, 2, 2, 64, 128, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 0]
+    assert rc_of(call, (5, 4, 64), *base[1:]) == lkv.LKV_ERR_UNSUPPORTED
+    assert rc_of(call, *base[:5], None, *base[6:]) == lkv.LKV_ERR_INVALID_ARG      # pos
+    assert rc_of(call, *base[:6], MISALIGNED, *base[7:]) == lkv.LKV_ERR_INVALID_ARG
+    assert rc_of(call, K6V4, 0, 2, 64, 128, None, None, None, None, None, None, None, 0) == 0   # nothing to do
+    m = decode_args()
+    del m["workspace"], m["ws_bytes"]
+    mass = lambda **kw: lkv.lkv_decode_attention_mass(**dict(m, **kw))
+    assert rc_of(mass, mass=None, workspace=FAKE, ws_bytes=1 << 40) == lkv.LKV_ERR_INVALID_ARG
+    assert rc_of(mass, mass=FAKE + 2, workspace=FAKE, ws_bytes=1 << 40) == lkv.LKV_ERR_INVALID_ARG
+    assert rc_of(mass, mass=FAKE, workspace=FAKE, ws_bytes=64) == lkv.LKV_ERR_WORKSPACE
+
+
 def test_tiered_rejects(L):
     seg = lkv.lkv_segment(FAKE, FAKE, FAKE, FAKE)
     bad = lkv.lkv_segment(FAKE, None, FAKE, FAKE)

@@ -166,3 +166,74 @@ def test_decode_long_context_full_size(orc):
 def test_decode_sweep_full_size_sampled(orc, kb, vb):
     cfg = W.CONFIGS[4]
     run_case(orc, cfg, kb, vb, 0.0, batches=[0, 33, 63])
+
+
+@pytest.mark.parametrize("r", [1, 2, 4, 8])
+def test_decode_attention_mass(orc, r):
+    """lkv_decode_attention_mass: the group's mean softmax probability per
+    token ("Super KV Compression" §第二层 ranks tokens by it) matches the
+    oracle's within 1e-4 relative (an fp32 logit carries an absolute error of
+    order 1e-5 in base 2, which moves exp2 by about 7e-6 relative per unit
+    of error, plus the error of the shared sum); every other output is
+    bit-identical to
+    lkv_decode_attention; slots beyond T_b are left untouched."""
+    cfg = W.Config("mass", B=3, Hq=2 * r, Hkv=2, D=128, T_cap=700, G=64, bits=[(6, 4)], hh_frac=0.01,
+                   seed=50 + r)
+    sl = torch.tensor([700, 1, 333], dtype=torch.int32)
+    inp = W.make_inputs(cfg, seq_lens=sl)
+    cache = gpu_quantize(6, 4, 64, inp)
+    tau = 1e-3
+    want_out, want_mask, want_counts = gpu_decode(6, 4, 64, inp, cache, cfg.softmax_scale, tau)
+    out = torch.empty(3, 2 * r, 128, device="cuda")
+    mask = torch.zeros(3, 2 * r, 700, dtype=torch.uint8, device="cuda")
+    counts = torch.zeros(2, dtype=torch.int64, device="cuda")
+    mass = torch.full((3, 2, 700), -1.0, device="cuda")
+    nb = lkv.lkv_decode_workspace_bytes((6, 4, 64), 3, 2 * r, 2, 700, 128)
+    ws = buffers.alloc_workspace(nb)
+    lkv.lkv_decode_attention_mass((6, 4, 64), 3, 2 * r, 2, 700, 128, dev(inp["seq_lens"]), dev(inp["q"]),
+                                  cache["k_codes"], cache["k_sz"], cache["v_codes"], cache["v_sz"],
+                                  cfg.softmax_scale, tau, out, mask, counts, mass, ws, nb)
+    torch.cuda.synchronize()
+    assert lkv.lkv_workspace_status(ws) == lkv.LKV_OK
+    np.testing.assert_array_equal(out.cpu().numpy(), want_out)
+    np.testing.assert_array_equal(mask.cpu().numpy(), want_mask)
+    assert counts.cpu().tolist() == want_counts.tolist()
+    k, v, q, s = oracle_inputs(inp)
+    ocache = orc.quantize_kv(6, 4, 64, k, v, s)
+    _, _, _, p = orc.decode_attention(6, 4, 64, s, q, ocache, cfg.softmax_scale, tau, want_p=True)
+    want = orc.attention_mass(p, 2, s)
+    got = mass.cpu().numpy()
+    for b in range(3):
+        T = int(s[b])
+        np.testing.assert_allclose(got[b, :, :T], want[b, :, :T], rtol=1e-4, atol=1e-12)
+        assert np.all(got[b, :, T:] == -1.0)
+
+
+def test_decode_mass_feeds_the_tiers(orc):
+    """One step of the attention-tiered cache driven by its own decode: the
+    mass from lkv_decode_attention_mass classified on the GPU gives the
+    oracle's tiers, except for masses within 1e-4 relative of a threshold."""
+    cfg = W.scaled(W.CONFIGS[2], B=2, T_cap=1024, seed=61)
+    inp = W.make_inputs(cfg)
+    cache = gpu_quantize(6, 4, 64, inp)
+    nb = lkv.lkv_decode_workspace_bytes((6, 4, 64), 2, 32, 8, 1024, 128)
+    ws = buffers.alloc_workspace(nb)
+    out = torch.empty(2, 32, 128, device="cuda")
+    mass = torch.zeros(2, 8, 1024, device="cuda")
+    sl = dev(inp["seq_lens"])
+    lkv.lkv_decode_attention_mass((6, 4, 64), 2, 32, 8, 1024, 128, sl, dev(inp["q"]), cache["k_codes"],
+                                  cache["k_sz"], cache["v_codes"], cache["v_sz"], cfg.softmax_scale, 1e-4, out,
+                                  None, None, mass, ws, nb)
+    t = buffers.alloc_tiers(2, 8, 1024, "cuda", zero=True)
+    lo, hi = 1e-4, 1e-2
+    lkv.lkv_tier_classify(2, 8, 1024, sl, mass, lo, hi, t["tier"], t["counts"], t["pos_a"], t["pos_b"])
+    torch.cuda.synchronize()
+    k, v, q, s = oracle_inputs(inp)
+    ocache = orc.quantize_kv(6, 4, 64, k, v, s)
+    _, _, _, p = orc.decode_attention(6, 4, 64, s, q, ocache, cfg.softmax_scale, 1e-4, want_p=True)
+    m_or = orc.attention_mass(p, 8, s)
+    tier_or, _, _, _ = orc.tier_classify(s, m_or.astype(np.float32), lo, hi)
+    near = (np.abs(m_or - lo) <= 1e-4 * lo) | (np.abs(m_or - hi) <= 1e-4 * hi)
+    got = t["tier"].cpu().numpy()
+    assert np.all((got == tier_or) | near)
+    assert (got == 2).sum() > 0 and (got == 1).sum() > 0 and (got == 0).sum() > 0

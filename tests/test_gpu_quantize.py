@@ -94,3 +94,33 @@ def test_quantize_out_of_range_lengths_are_clamped(orc):
     want = orc.quantize_kv(6, 4, 32, k, v, np.array([32, 0], np.int32))
     compare_cache(gpu, want, [32, 0], "clamped")
     assert int(gpu["k_codes"][1].abs().sum()) == 0
+
+
+@pytest.mark.parametrize("D,G,kb,vb", [(128, 64, 6, 4), (64, 32, 8, 8), (128, 128, 4, 2), (128, 32, 2, 6)])
+def test_append_equals_quantize_of_the_longer_sequence(orc, D, G, kb, vb):
+    """lkv_append_kv writes the new token's row exactly as lkv_quantize_kv
+    would (bit-exact vs the oracle), and touches no other row; positions
+    outside [0, T_cap) write nothing."""
+    from quantized_kv_cache_lkv_b200 import lkv
+    T_cap = 96
+    cfg = W.Config("append", B=4, Hq=4, Hkv=2, D=D, T_cap=T_cap, G=G, bits=[(kb, vb)], seed=90 + D + G + kb)
+    full = torch.tensor([50, 96, 1, 20], dtype=torch.int32)
+    inp = W.make_inputs(cfg, seq_lens=full)
+    before = torch.tensor([49, 95, 0, 20], dtype=torch.int32)   # sequence 3 appends at an invalid slot below
+    cache = gpu_quantize(kb, vb, G, dict(inp, seq_lens=before))
+    pos = torch.tensor([49, 95, 0, T_cap], dtype=torch.int32)    # T_cap: nothing written
+    k_new = torch.stack([inp["k"][b, :, min(int(pos[b]), T_cap - 1)] for b in range(4)]).contiguous()
+    v_new = torch.stack([inp["v"][b, :, min(int(pos[b]), T_cap - 1)] for b in range(4)]).contiguous()
+    snapshot = {k: v.clone() for k, v in cache.items()}
+    lkv.lkv_append_kv((kb, vb, G), 4, 2, T_cap, D, pos.cuda(), k_new.cuda(), v_new.cuda(), cache["k_codes"],
+                      cache["k_sz"], cache["v_codes"], cache["v_sz"])
+    torch.cuda.synchronize()
+    after = torch.tensor([50, 96, 1, 20], dtype=torch.int32)
+    k, v, _, sl = oracle_inputs(dict(inp, seq_lens=after))
+    want = orc.quantize_kv(kb, vb, G, k, v, sl)
+    compare_cache(cache, want, sl, f"append K{kb}V{vb} D{D} G{G}")
+    for key in cache:   # rows other than the appended ones are untouched
+        g, s0 = cache[key].cpu(), snapshot[key].cpu()
+        for b in range(4):
+            keep = [t for t in range(T_cap) if not (b < 3 and t == int(pos[b]))]
+            assert torch.equal(g[b, :, keep], s0[b, :, keep]), (key, b)

@@ -366,6 +366,30 @@ def test_skip_set_matches_torch_probabilities(orc):
     assert counts.tolist() == [int(mask.sum()), int(rows_all)]
 
 
+def test_attention_mass_is_group_mean_of_torch_softmax(orc):
+    """The per-token mass fed to the next step's tiers is the mean over the
+    group's query heads of torch float64 softmax probabilities; over t it
+    sums to 1 per (b, KV head); slots beyond T_b stay 0; with one query head
+    per group it is that head's probability."""
+    cfg = W.scaled(W.CONFIGS[2], B=2, T_cap=384, seed=23)
+    q, cache, sl = _case(orc, cfg, 6, 4)
+    sl = np.array([384, 200], np.int32)
+    _, _, _, p = orc.decode_attention(6, 4, cfg.G, sl, q, cache, cfg.softmax_scale, 1e-3, want_p=True)
+    mass = orc.attention_mass(p, cfg.Hkv, sl)
+    kh, _ = _dequant_cache(orc, cache, 6, 4, cfg.D, cfg.G)
+    for b in range(2):
+        T = int(sl[b])
+        qd = torch.from_numpy(q.view(np.int16)).view(torch.bfloat16).double()[b]
+        K = torch.from_numpy(kh[b, :, :T]).double().repeat_interleave(cfg.r, dim=0)
+        pt = torch.softmax(torch.einsum("hd,htd->ht", qd, K) * float(np.float32(cfg.softmax_scale)), -1).numpy()
+        want = pt.reshape(cfg.Hkv, cfg.r, T).mean(axis=1)
+        np.testing.assert_allclose(mass[b, :, :T], want, rtol=1e-9, atol=1e-15)
+        np.testing.assert_allclose(mass[b, :, :T].sum(axis=1), 1.0, rtol=1e-12)
+        assert np.all(mass[b, :, T:] == 0.0)
+    one = orc.attention_mass(p[:, ::cfg.r], cfg.Hkv, sl)      # one head per group
+    np.testing.assert_array_equal(one, p[:, ::cfg.r])
+
+
 # ---------------------------------------------------------------- tiers
 
 def test_tier_boundaries(orc):
