@@ -4,10 +4,10 @@
 // ("Super KV Compression", §第一层：自适应非对称量化; "TurboQuant",
 // §TurboQuant的核心创新: asymmetric and group-wise).  The kernel is bound by
 // HBM traffic (2*D bytes in, D*bits/8 + 8*D/G bytes out per row and tensor),
-// so it streams rows with 32-byte vector loads and keeps everything else in
-// registers: one lane quantizes 16 channels, the G/16 lanes of a group share
-// their min/max by warp shuffles, and the lane packs its 16 codes into
-// 2*BITS bytes that it stores itself.
+// so it streams rows with 16-byte vector loads and keeps everything else in
+// registers: one lane quantizes 32 channels (16 in the repack and append
+// kernels), the lanes of a group share their min/max by warp shuffles, and
+// each lane packs its codes and stores them itself.
 #include <algorithm>
 
 #include "lkv_kernels.cuh"
@@ -47,19 +47,161 @@ __device__ __forceinline__ void quantize_lane(const uint4& w0, const uint4& w1, 
   if (j % lpg == 0) *reinterpret_cast<float2*>(sz + 2 * (j / lpg)) = make_float2(scale, zero);
 }
 
+// ------------------------------------------------------------ 32 channels per lane
+// The full-cache quantizer gives each lane 32 channels (two 16-channel
+// slices): the per-lane work of a group -- min/max, the two divisions, the
+// group shuffles -- is shared by twice as many values, and for G = 32 a lane
+// holds a whole group.
+
+constexpr int kLaneDims32 = 32;
+
+struct LaneRows32 {
+  uint4 k[4], v[4];
+};
+
+__device__ __forceinline__ void fetch_lane_rows32(const uint16_t* k, const uint16_t* v, LaneRows32& r) {
+#pragma unroll
+  for (int i = 0; i < 4; ++i) r.k[i] = ld_stream(k + 8 * i);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) r.v[i] = ld_stream(v + 8 * i);
+}
+
+// Magic-rounded codes rb[i] = 0x4B400000 + code_i for 32 codes, packed LSB
+// first into BITS words (see pack16_magic).
+template <int BITS>
+constexpr uint32_t magic_pack_const32(int wi) {
+  uint32_t c = 0u;
+  for (int i = 0; i < 32; ++i) {
+    const int bit = i * BITS;
+    if ((bit >> 5) == wi) c -= 0x4B400000u << (bit & 31);
+  }
+  return c;
+}
+
+template <int BITS>
+__device__ __forceinline__ void pack32_magic(const uint32_t (&rb)[32], uint32_t (&out)[BITS]) {
+  constexpr uint32_t mask = (1u << BITS) - 1u;
+#pragma unroll
+  for (int wi = 0; wi < BITS; ++wi) {
+    uint32_t acc = magic_pack_const32<BITS>(wi);
+#pragma unroll
+    for (int i = 0; i < 32; ++i) {
+      const int bit = i * BITS, w0 = bit >> 5, pos = bit & 31;
+      if (w0 == wi) acc += rb[i] << pos;
+      else if (w0 + 1 == wi && pos + BITS > 32) acc += (rb[i] & mask) >> (32 - pos);
+    }
+    out[wi] = acc;
+  }
+}
+
+template <int BITS>
+__device__ __forceinline__ void pack32(const uint32_t (&c)[32], uint32_t (&out)[BITS]) {
+#pragma unroll
+  for (int i = 0; i < BITS; ++i) out[i] = 0u;
+#pragma unroll
+  for (int i = 0; i < 32; ++i) {
+    const int bit = i * BITS, wi = bit >> 5, pos = bit & 31;
+    out[wi] |= c[i] << pos;
+    if (pos + BITS > 32) out[wi + 1] |= c[i] >> (32 - pos);
+  }
+}
+
+// quantize16 for 32 values (16 raw bf16 words); LPG = G / 32 lanes share a
+// group.  The same fixed fp32 formula, the same two paths.
+template <int BITS, int LPG>
+__device__ __forceinline__ void quantize32(const uint32_t (&w)[16], unsigned mask, float one, uint32_t (&out)[BITS],
+                                           float& scale, float& zero) {
+  __nv_bfloat162 lo = *reinterpret_cast<const __nv_bfloat162*>(&w[0]), hi = lo;
+#pragma unroll
+  for (int i = 1; i < 16; ++i) {
+    const __nv_bfloat162 p = *reinterpret_cast<const __nv_bfloat162*>(&w[i]);
+    lo = __hmin2(lo, p);
+    hi = __hmax2(hi, p);
+  }
+  float mn = fminf(__low2float(lo), __high2float(lo));
+  float mx = fmaxf(__low2float(hi), __high2float(hi));
+#pragma unroll
+  for (int off = 1; off < LPG; off <<= 1) {
+    mn = fminf(mn, __shfl_xor_sync(mask, mn, off));
+    mx = fmaxf(mx, __shfl_xor_sync(mask, mx, off));
+  }
+  constexpr uint32_t cmask = (1u << BITS) - 1u;
+  const float qmax = static_cast<float>(cmask);
+  const float d = __fsub_rn(mx, mn);
+  float inv = 0.0f;
+  scale = 0.0f;
+  if (d != 0.0f) {
+    scale = __fdiv_rn(d, qmax);
+    inv = __fdiv_rn(qmax, d);
+  }
+  zero = __fadd_rn(mn, 0.0f);
+  if (d <= 3.4028234663852886e38f && inv <= 3.4028234663852886e38f) {
+    const __nv_bfloat162 mn_b = __floats2bfloat162_rn(mn, mn);
+    const float2 nmn = make_float2(-mn, -mn), inv2 = make_float2(inv, inv), one2 = make_float2(one, one);
+    const float2 rnd = make_float2(12582912.0f, 12582912.0f);
+    uint32_t rb[32];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      const __nv_bfloat162 p = __hmax2(*reinterpret_cast<const __nv_bfloat162*>(&w[i]), mn_b);
+      const uint32_t u = *reinterpret_cast<const uint32_t*>(&p);
+      const float2 x = make_float2(bf16_lo(u), bf16_hi(u));
+      const float2 y = exact_mul2(exact_add2(x, nmn), inv2);
+      const float2 r = exact_fma2(y, one2, rnd);  // y rounded half-even (see quantize16)
+      rb[2 * i] = __float_as_uint(r.x);
+      rb[2 * i + 1] = __float_as_uint(r.y);
+    }
+    pack32_magic<BITS>(rb, out);
+  } else {
+    uint32_t c[32];
+#pragma unroll
+    for (int i = 0; i < 32; ++i) {
+      const float x = (i & 1) ? bf16_hi(w[i / 2]) : bf16_lo(w[i / 2]);
+      int ci = __float2int_rn(__fmul_rn(__fsub_rn(x, mn), inv));  // NaN gives 0
+      ci = ci < 0 ? 0 : ci;
+      c[i] = static_cast<uint32_t>(ci > (int)cmask ? (int)cmask : ci);
+    }
+    pack32<BITS>(c, out);
+  }
+}
+
+// Store a lane's BITS words (4 * BITS bytes at a multiple of 4 * BITS).
+template <int BITS>
+__device__ __forceinline__ void store_words32(uint8_t* p, const uint32_t (&w)[BITS]) {
+  if constexpr (BITS % 4 == 0) {
+#pragma unroll
+    for (int i = 0; i < BITS; i += 4) *reinterpret_cast<uint4*>(p + 4 * i) = make_uint4(w[i], w[i + 1], w[i + 2], w[i + 3]);
+  } else {
+#pragma unroll
+    for (int i = 0; i < BITS; i += 2) *reinterpret_cast<uint2*>(p + 4 * i) = make_uint2(w[i], w[i + 1]);
+  }
+}
+
+template <int BITS, int LPG>
+__device__ __forceinline__ void quantize_lane32(const uint4 (&w4)[4], uint8_t* __restrict__ codes,
+                                                float* __restrict__ sz, int j, unsigned mask, float one) {
+  uint32_t w[16];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) { w[4 * i] = w4[i].x; w[4 * i + 1] = w4[i].y; w[4 * i + 2] = w4[i].z; w[4 * i + 3] = w4[i].w; }
+  uint32_t out[BITS];
+  float scale, zero;
+  quantize32<BITS, LPG>(w, mask, one, out, scale, zero);
+  store_words32<BITS>(codes + j * (4 * BITS), out);
+  if (j % LPG == 0) *reinterpret_cast<float2*>(sz + 2 * (j / LPG)) = make_float2(scale, zero);
+}
+
 // Row batches: batch (b, g, tb) covers tokens tb * RPW ... of KV head g of
 // sequence b, one row per D/16 lanes.  Warp w of the grid takes batches w,
 // w + W, w + 2W, ... in (b, g, tb) order, stepping its coordinates without
 // divisions, and issues the next batch's loads before quantizing the current
 // one, so two batches of K and V per warp are in flight.
-template <int D, int KB, int VB>
-__global__ void __launch_bounds__(256, 4) quantize_kv_kernel(QuantizeArgs a) {
-  constexpr int LPR = D / kDimsPerLane;
+template <int D, int KB, int VB, int LPG>
+__global__ void __launch_bounds__(256, 2) quantize_kv_kernel(QuantizeArgs a) {
+  constexpr int LPR = D / kLaneDims32;
   constexpr int RPW = 32 / LPR;
   const int lane = threadIdx.x & 31;
   const int j = lane % LPR, sub = lane / LPR;
   const unsigned mask = row_lane_mask<LPR>(lane);
-  const int ng = D / a.G, lpg = a.G / kDimsPerLane;
+  const int ng = D / a.G;
   const uint32_t nbu = (uint32_t)(a.T_cap + RPW - 1) / RPW;  // batches per (b, g)
   const uint32_t W = gridDim.x * (blockDim.x / 32);
   const uint32_t w0 = blockIdx.x * (blockDim.x / 32) + threadIdx.x / 32;
@@ -75,15 +217,15 @@ __global__ void __launch_bounds__(256, 4) quantize_kv_kernel(QuantizeArgs a) {
     g_ -= c * (uint32_t)a.Hkv;
     b_ += s_b + c;
   };
-  auto fetch = [&](uint32_t b_, uint32_t g_, uint32_t tb_, LaneRows& r, long long& row) -> bool {
+  auto fetch = [&](uint32_t b_, uint32_t g_, uint32_t tb_, LaneRows32& r, long long& row) -> bool {
     if (b_ >= (uint32_t)a.B) return false;
     const int t = (int)tb_ * RPW + sub;
     if (t >= clamp_len(__ldg(a.seq_lens + b_), a.T_cap)) return false;
     row = ((long long)b_ * a.Hkv + g_) * a.T_cap + t;
-    fetch_lane_rows(a.k + row * D + j * kDimsPerLane, a.v + row * D + j * kDimsPerLane, r);
+    fetch_lane_rows32(a.k + row * D + j * kLaneDims32, a.v + row * D + j * kLaneDims32, r);
     return true;
   };
-  LaneRows cur, nxt;
+  LaneRows32 cur, nxt;
   long long row = 0, row_n = 0;
   bool ok = fetch(b, g, tb, cur, row);
   while (b < (uint32_t)a.B) {
@@ -91,10 +233,10 @@ __global__ void __launch_bounds__(256, 4) quantize_kv_kernel(QuantizeArgs a) {
     step(bn, gn, tbn);
     const bool ok_n = fetch(bn, gn, tbn, nxt, row_n);
     // The lanes of one row share `ok`, so the group shuffles inside
-    // quantize16 only ever pair lanes that are both active.
+    // quantize32 only ever pair lanes that are both active.
     if (ok) {
-      quantize_lane<KB>(cur.k0, cur.k1, a.k_codes + row * (D * KB / 8), a.k_sz + row * ng * 2, j, lpg, mask, a.one);
-      quantize_lane<VB>(cur.v0, cur.v1, a.v_codes + row * (D * VB / 8), a.v_sz + row * ng * 2, j, lpg, mask, a.one);
+      quantize_lane32<KB, LPG>(cur.k, a.k_codes + row * (D * KB / 8), a.k_sz + row * ng * 2, j, mask, a.one);
+      quantize_lane32<VB, LPG>(cur.v, a.v_codes + row * (D * VB / 8), a.v_sz + row * ng * 2, j, mask, a.one);
     }
     cur = nxt; row = row_n; ok = ok_n;
     b = bn; g = gn; tb = tbn;
@@ -179,18 +321,27 @@ static int resident_blocks(const void* kern) {
   return n;
 }
 
-template <int D, int KB, int VB>
-static cudaError_t launch_quantize_t(const QuantizeArgs& a, cudaStream_t s) {
-  constexpr int RPW = 32 / (D / kDimsPerLane);
+template <int D, int KB, int VB, int LPG>
+static cudaError_t launch_quantize_g(const QuantizeArgs& a, cudaStream_t s) {
+  constexpr int RPW = 32 / (D / kLaneDims32);
   static int per_sm[64] = {0};
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) dev = 0;
-  if (per_sm[dev] == 0) per_sm[dev] = resident_blocks((const void*)quantize_kv_kernel<D, KB, VB>);
+  if (per_sm[dev] == 0) per_sm[dev] = resident_blocks((const void*)quantize_kv_kernel<D, KB, VB, LPG>);
   const long long n_batches = (long long)a.B * a.Hkv * ((a.T_cap + RPW - 1) / RPW);
   if (n_batches >= (1ll << 31)) return cudaErrorInvalidValue;
   long long blocks = std::min<long long>((long long)num_sms() * per_sm[dev], (n_batches + 7) / 8);
-  quantize_kv_kernel<D, KB, VB><<<(int)std::max<long long>(blocks, 1), 256, 0, s>>>(a);
+  quantize_kv_kernel<D, KB, VB, LPG><<<(int)std::max<long long>(blocks, 1), 256, 0, s>>>(a);
   return cudaGetLastError();
+}
+
+template <int D, int KB, int VB>
+static cudaError_t launch_quantize_t(const QuantizeArgs& a, cudaStream_t s) {
+  // lanes per group: G / 32 (groups never exceed D)
+  if (a.G == 32) return launch_quantize_g<D, KB, VB, 1>(a, s);
+  if (a.G == 64) return launch_quantize_g<D, KB, VB, 2>(a, s);
+  if constexpr (D >= 128) return launch_quantize_g<D, KB, VB, 4>(a, s);
+  return cudaErrorInvalidValue;
 }
 
 template <int D, int KB, int VB>
