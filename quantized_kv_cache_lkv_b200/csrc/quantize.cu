@@ -271,14 +271,14 @@ __global__ void __launch_bounds__(256) append_kv_kernel(QuantizeArgs a) {
 // or 4 (B) bits ("Super KV Compression", §第二层 items 1-2).  Block
 // (bg * S + s, seg) walks only the n rows that segment seg of unit bg holds,
 // S blocks per unit and segment, with the same one-ahead loads as above.
-template <int D>
-__global__ void __launch_bounds__(256, 4) tier_repack_kernel(RepackArgs a, int S) {
-  constexpr int LPR = D / kDimsPerLane;
+template <int D, int LPG>
+__global__ void __launch_bounds__(256, 2) tier_repack_kernel(RepackArgs a, int S) {
+  constexpr int LPR = D / kLaneDims32;
   constexpr int RPW = 32 / LPR;
   const int lane = threadIdx.x & 31;
   const int j = lane % LPR, sub = lane / LPR;
   const unsigned mask = row_lane_mask<LPR>(lane);
-  const int ng = D / a.G, lpg = a.G / kDimsPerLane;
+  const int ng = D / a.G;
   const int seg = blockIdx.y;  // 0: segment A, 1: segment B
   const long long bg = blockIdx.x / S;
   const int s = blockIdx.x % S;
@@ -286,27 +286,27 @@ __global__ void __launch_bounds__(256, 4) tier_repack_kernel(RepackArgs a, int S
   const int32_t* pos = (seg == 0 ? a.pos_a : a.pos_b) + bg * a.T_cap;
   const int nw = blockDim.x / 32;
   const int stride = S * nw * RPW;
-  auto fetch = [&](int i, LaneRows& r) -> bool {
+  auto fetch = [&](int i, LaneRows32& r) -> bool {
     if (i >= n) return false;
     int t = __ldg(pos + i);
     t = t < 0 ? 0 : (t >= a.T_cap ? a.T_cap - 1 : t);
     const long long src = bg * a.T_cap + t;
-    fetch_lane_rows(a.k + src * D + j * kDimsPerLane, a.v + src * D + j * kDimsPerLane, r);
+    fetch_lane_rows32(a.k + src * D + j * kLaneDims32, a.v + src * D + j * kLaneDims32, r);
     return true;
   };
   int i = (s * nw + (int)threadIdx.x / 32) * RPW + sub;
-  LaneRows cur, nxt;
+  LaneRows32 cur, nxt;
   bool ok = fetch(i, cur);
   for (; i - sub < n; i += stride) {
     const bool ok_n = fetch(i + stride, nxt);
     if (ok) {
       const long long slot = bg * a.T_cap + i;
       if (seg == 0) {
-        quantize_lane<6>(cur.k0, cur.k1, a.a_kc + slot * (D * 6 / 8), a.a_ksz + slot * ng * 2, j, lpg, mask, a.one);
-        quantize_lane<6>(cur.v0, cur.v1, a.a_vc + slot * (D * 6 / 8), a.a_vsz + slot * ng * 2, j, lpg, mask, a.one);
+        quantize_lane32<6, LPG>(cur.k, a.a_kc + slot * (D * 6 / 8), a.a_ksz + slot * ng * 2, j, mask, a.one);
+        quantize_lane32<6, LPG>(cur.v, a.a_vc + slot * (D * 6 / 8), a.a_vsz + slot * ng * 2, j, mask, a.one);
       } else {
-        quantize_lane<6>(cur.k0, cur.k1, a.b_kc + slot * (D * 6 / 8), a.b_ksz + slot * ng * 2, j, lpg, mask, a.one);
-        quantize_lane<4>(cur.v0, cur.v1, a.b_vc + slot * (D * 4 / 8), a.b_vsz + slot * ng * 2, j, lpg, mask, a.one);
+        quantize_lane32<6, LPG>(cur.k, a.b_kc + slot * (D * 6 / 8), a.b_ksz + slot * ng * 2, j, mask, a.one);
+        quantize_lane32<4, LPG>(cur.v, a.b_vc + slot * (D * 4 / 8), a.b_vsz + slot * ng * 2, j, mask, a.one);
       }
     }
     cur = nxt; ok = ok_n;
@@ -399,8 +399,11 @@ cudaError_t launch_tier_repack(const RepackArgs& a, int D, cudaStream_t s) {
   const int S = (int)std::max<long long>(1, std::min<long long>(64, want / (2 * units)));
   if (units * S >= (1ll << 31)) return cudaErrorInvalidValue;
   dim3 grid((unsigned)(units * S), 2);
-  if (D == 64) tier_repack_kernel<64><<<grid, 256, 0, s>>>(a, S);
-  else if (D == 128) tier_repack_kernel<128><<<grid, 256, 0, s>>>(a, S);
+  if (D == 64 && a.G == 32) tier_repack_kernel<64, 1><<<grid, 256, 0, s>>>(a, S);
+  else if (D == 64 && a.G == 64) tier_repack_kernel<64, 2><<<grid, 256, 0, s>>>(a, S);
+  else if (D == 128 && a.G == 32) tier_repack_kernel<128, 1><<<grid, 256, 0, s>>>(a, S);
+  else if (D == 128 && a.G == 64) tier_repack_kernel<128, 2><<<grid, 256, 0, s>>>(a, S);
+  else if (D == 128 && a.G == 128) tier_repack_kernel<128, 4><<<grid, 256, 0, s>>>(a, S);
   else return cudaErrorInvalidValue;
   return cudaGetLastError();
 }
