@@ -82,7 +82,8 @@ FusedLayout fused_layout(int B, int Hq, int Hkv, int T_cap, int D, int KB) {
   L.cpc_max = (int)((chunks_max + L.grid - 1) / L.grid);
   const fused::GeoHost g = fused::geo_host(D, KB);
   L.stages = g.stages;
-  const int phase2 = fused::kMaxConsumerWarps * fused::kListCap * 4 * (1 + L.H) + g.consumer_warps * L.H * D * 4;
+  const int lists = fused::kMaxConsumerWarps * fused::kListCap * 4 * (1 + L.H);
+  const int phase2 = std::max(lists, fused::kDenseStaging) + fused::kMaxConsumerWarps * L.H * D * 4;
   L.ring_bytes = std::max(g.stages * g.stage_bytes, phase2);
   L.smem_bytes = fused::kHeader + L.ring_bytes;
   const int tpc = fused::kChunk / g.tile_rows;

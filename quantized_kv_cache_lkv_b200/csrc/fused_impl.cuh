@@ -48,6 +48,14 @@ constexpr int kGatherUnroll = 4;
 constexpr int kScanBlocks = 4;  // 32-row blocks whose logits one warp loads at once
 constexpr int kTsCap = 128;    // tile statistics kept in shared memory up to this many tiles
 constexpr int kQSlots = 4;     // units whose prescaled q is staged in shared memory
+// Dense V pass (tau <= 0): per warp two buffers of one 32-row block each:
+// V codes (up to 6 bits), (scale, zero) of 34 rows and the block's logits.
+constexpr int kDenseCodes = 32 * 96;
+constexpr int kDenseSz = 34 * 4 * 8;
+constexpr int kDenseLogits = 32 * 4 * 4;
+constexpr int kDenseBuf = (kDenseCodes + kDenseSz + kDenseLogits + 127) / 128 * 128;
+constexpr int kDenseStaging = kMaxConsumerWarps * 2 * kDenseBuf;
+constexpr int kDenseBar = 32;  // first mbarrier of the dense buffers
 constexpr unsigned kFull = 0xFFFFFFFFu;
 constexpr int kBarCons = 1;    // named barrier of the consumer warps
 // Shared header (bytes): barriers [0, 512), per-group q sums of up to
@@ -318,6 +326,7 @@ __global__ void __launch_bounds__(Geo<D, KB>::kThreads, 1) fused_decode_kernel(F
 
   if (tid == 0) {
     for (int s = 0; s < Gk::kStages; ++s) mbar_init(&full[s], 1);
+    for (int s = 0; s < 2 * kMaxConsumerWarps; ++s) mbar_init(&full[kDenseBar + s], 1);
     fence_mbar_init();
     s_total = 0; s_e0 = 0; s_nent = 0; s_abort = 0; s_carry_c = 0; s_carry_n = 0; s_last = 0;
   }
@@ -699,7 +708,11 @@ __global__ void __launch_bounds__(Geo<D, KB>::kThreads, 1) fused_decode_kernel(F
   // per-head weights [CW][kListCap][H] and the warps' partial outputs [CW][H][D]
   int* lists = reinterpret_cast<int*>(ring);
   float* wts = reinterpret_cast<float*>(ring + kMaxConsumerWarps * kListCap * 4);
-  float* red = wts + kMaxConsumerWarps * kListCap * H;
+  constexpr int kListsBytes = kMaxConsumerWarps * kListCap * 4 * (1 + H);
+  float* red = reinterpret_cast<float*>(ring + (kListsBytes > kDenseStaging ? kListsBytes : kDenseStaging));
+  // the dense V pass applies when every row is kept and the V rows fit its buffers
+  const bool dense = d.tau <= 0.0f && VB0 <= 6 && VB1 <= 6;
+  int dense_uses[2] = {0, 0};
   Magic<VB0> mg0;
   mg0.load(s_magic);
   Magic<VB1> mg1;
@@ -764,6 +777,102 @@ __global__ void __launch_bounds__(Geo<D, KB>::kThreads, 1) fused_decode_kernel(F
 #pragma unroll
         for (int i = 0; i < 8; ++i) acc[h][i] = make_float2(0.0f, 0.0f);
       }
+      if (dense) {
+        // Dense V pass: every valid row is kept, so the warp streams its
+        // 32-row blocks (round robin over warps) into shared memory with bulk
+        // copies, two blocks in flight, and accumulates them from there.
+        uint8_t* stg = ring + (size_t)warp * 2 * kDenseBuf;
+        const int nblk = (v_hi - v_lo) / 32;
+        const uint64_t pol = policy_evict_first();
+        int rows_of[2] = {0, 0};
+        auto issue = [&](int k, int buf) {
+          rows_of[buf] = 0;
+          const int blk = warp + k * CW;
+          if (blk >= nblk) return;
+          const int v0 = v_lo + blk * 32;
+          const ChunkRows cr = chunk_rows(x, v0 / kChunk);
+          const int rows = min(32, cr.rows - v0 % kChunk);
+          if (rows <= 0) return;
+          rows_of[buf] = rows;
+          if (lane == 0) {
+            const int seg = cr.seg, row = cr.row0 + v0 % kChunk;
+            const int rbv = seg ? D * VB1 / 8 : D * VB0 / 8;
+            const int r0 = (ng == 1) ? (row & ~1) : row;
+            const int r1 = (ng == 1) ? ((row + rows + 1) & ~1) : row + rows;
+            const uint32_t cbytes = (uint32_t)rows * rbv, sbytes = (uint32_t)(r1 - r0) * ng * 8;
+            const uint32_t lbytes = 32u * H * 4u;
+            uint8_t* dst = stg + buf * kDenseBuf;
+            uint64_t* bar = &full[kDenseBar + warp * 2 + buf];
+            mbar_arrive_expect_tx(bar, cbytes + sbytes + lbytes);
+            bulk_g2s(dst, d.vc[seg] + (ubase + row) * rbv, cbytes, bar, pol);
+            bulk_g2s(dst + kDenseCodes, d.vsz[seg] + (ubase + r0) * ng * 2, sbytes, bar, pol);
+            bulk_g2s(dst + kDenseCodes + kDenseSz, lgu + (long long)v0 * H, lbytes, bar, pol);
+          }
+        };
+        issue(0, 0);
+        issue(1, 1);
+        bool stalled = false;
+        for (int k = 0; warp + k * CW < nblk && !stalled; ++k) {
+          const int buf = k & 1;
+          const int rows = rows_of[buf];
+          if (rows > 0) {
+            if (!mbar_wait(&full[kDenseBar + warp * 2 + buf], dense_uses[buf] & 1, limit_ns)) {
+              atomicExch(d.status, kStatusTimeout);
+              stalled = true;  // leave the copy pending: it is drained below
+              break;
+            }
+            ++dense_uses[buf];
+            rows_of[buf] = 0;
+            {
+              const int v0 = v_lo + (warp + k * CW) * 32;
+              const ChunkRows cr = chunk_rows(x, v0 / kChunk);
+              const int row = cr.row0 + v0 % kChunk;
+              const int sz_skip = (ng == 1) ? (row & 1) : 0;
+              const uint8_t* src = stg + buf * kDenseBuf;
+              const float* lgs = reinterpret_cast<const float*>(src + kDenseCodes + kDenseSz);
+              const float* szs = reinterpret_cast<const float*>(src + kDenseCodes);
+              float f[H];
+              lds_heads<H>(tfu + (v0 / TR) * H, f);
+              for (int s2 = 0; s2 < 32 / RPW; ++s2) {
+                const int i = s2 * RPW + lane / LPR;
+                if (i >= rows) continue;  // the lanes of a row agree
+                float e[H], wgt[H];
+                lds_heads<H>(lgs + i * H, e);
+                float ms = 0.0f;
+#pragma unroll
+                for (int h = 0; h < H; ++h) { wgt[h] = e[h] * f[h]; ms += wgt[h]; }
+                if (j == 0) {
+                  if (smask) {
+#pragma unroll
+                    for (int h = 0; h < H; ++h) smask[((long long)b * d.Hq + g * H + h) * d.T_cap + v0 + i] = 0;
+                  }
+                  if (mass_out) mass_out[((long long)b * d.Hkv + g) * d.T_cap + v0 + i] = ms * (1.0f / H);
+                }
+                const float2 sz = *reinterpret_cast<const float2*>(szs + ((sz_skip + i) * ng + gi) * 2);
+                if (cr.seg == 0) {
+                  LaneWords<VB0> lw;
+                  lds_lane_words<VB0>(src + i * (D * VB0 / 8) + j * 2 * VB0, lw);
+                  accumulate_v<H, VB0>(lw, mg0, sz, wgt, acc, Z);
+                } else {
+                  LaneWords<VB1> lw;
+                  lds_lane_words<VB1>(src + i * (D * VB1 / 8) + j * 2 * VB1, lw);
+                  accumulate_v<H, VB1>(lw, mg1, sz, wgt, acc, Z);
+                }
+              }
+            }
+          }
+          // the buffer's data is in registers: refill it
+          fence_proxy_async_smem();
+          __syncwarp();
+          issue(k + 2, buf);
+        }
+        // never leave copies in flight (only a timed-out wait leaves one)
+        for (int buf = 0; buf < 2; ++buf)
+          if (rows_of[buf] > 0) {
+            mbar_wait(&full[kDenseBar + warp * 2 + buf], dense_uses[buf] & 1, limit_ns);
+            ++dense_uses[buf];
+          }
+      } else
       for (int vb = v_lo; vb < v_hi; vb += NCONS * kBatchBlocks) {
         // scan: 32-row blocks round robin over warps, row order kept per warp;
         // the logits of kScanBlocks blocks are loaded before any is used.  A
