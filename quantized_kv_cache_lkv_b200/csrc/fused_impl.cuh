@@ -667,7 +667,7 @@ __global__ void __launch_bounds__(Geo<D, KB>::kThreads, 1) fused_decode_kernel(F
     int* rec = ulist + (long long)e * kRec;
     const Unit x = load_unit(rec);
     const int ta = (max(x.cb, k0) - k0) * TPC, tb = (min(x.cb + x.nc, k1) - k0) * TPC;
-#pragma unroll
+#pragma unroll 1
     for (int h = 0; h < H; ++h) {
       float m = -INFINITY, l = 0.0f;
       for (int t2 = ta + lane; t2 < tb; t2 += 32) merge_ml(m, l, tsm[t2 * H + h], tsl[t2 * H + h]);
@@ -992,25 +992,33 @@ __global__ void __launch_bounds__(Geo<D, KB>::kThreads, 1) fused_decode_kernel(F
         named_barrier(kBarCons, NCONS);  // other warps read this batch's lists
       }
       // fold the per-group constant, reduce the row slots of the warp
+      // (code that runs once per piece is kept short: loops stay rolled)
 #pragma unroll
       for (int h = 0; h < H; ++h)
 #pragma unroll
         for (int i = 0; i < 8; ++i) { acc[h][i].x += Z[h]; acc[h][i].y += Z[h]; }
-#pragma unroll
-      for (int off = LPR; off < 32; off <<= 1)
-#pragma unroll
-        for (int h = 0; h < H; ++h)
-#pragma unroll
-          for (int i = 0; i < 8; ++i) {
-            acc[h][i].x += __shfl_xor_sync(kFull, acc[h][i].x, off);
-            acc[h][i].y += __shfl_xor_sync(kFull, acc[h][i].y, off);
-          }
       if (lane < LPR) {
 #pragma unroll
         for (int h = 0; h < H; ++h)
 #pragma unroll
           for (int i = 0; i < 8; ++i)
-            *reinterpret_cast<float2*>(red + (warp * H + h) * D + j * kDimsPerLane + 2 * i) = acc[h][i];
+            *reinterpret_cast<float2*>(red + (warp * H + h) * D + j * kDimsPerLane + 2 * i) = make_float2(0.0f, 0.0f);
+      }
+      __syncwarp();
+      // the RPW row slots of the warp add their partial sums in shared memory
+#pragma unroll 1
+      for (int slot = 0; slot < RPW; ++slot) {
+        if (lane / LPR == slot) {
+#pragma unroll
+          for (int h = 0; h < H; ++h)
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+              float2* o = reinterpret_cast<float2*>(red + (warp * H + h) * D + j * kDimsPerLane + 2 * i);
+              const float2 pv = *o;
+              *o = make_float2(pv.x + acc[h][i].x, pv.y + acc[h][i].y);
+            }
+        }
+        __syncwarp();
       }
       named_barrier(kBarCons, NCONS);
       for (int o = tid; o < H * D; o += NCONS) {
