@@ -140,6 +140,49 @@ LKV_API int lkv_append_kv(lkv_qspec spec, int B, int Hkv, int T_cap, int D, cons
                   float *v_sz, void *stream);
 
 /*
+ * Paged caches ([TQ] §与其他优化技术的对比: the quantized cache is meant to
+ * work with paged KV management).  A page holds LKV_PAGE_TOKENS consecutive
+ * tokens of one KV head; the four pools are
+ *   codes  [num_pages][Hkv][LKV_PAGE_TOKENS][D * bits / 8]
+ *   sz     [num_pages][Hkv][LKV_PAGE_TOKENS][D / group][2]
+ * and block_table (int32 [B][pages_per_seq], device) names the page of
+ * tokens [i * LKV_PAGE_TOKENS, (i + 1) * LKV_PAGE_TOKENS) of sequence b.
+ * The logical capacity is T_cap = pages_per_seq * LKV_PAGE_TOKENS.  Codes,
+ * (scale, zero) and all results are those of the contiguous calls on the
+ * same tokens.  A page id outside [0, num_pages) makes quantize and append
+ * skip that token; the decode reads page 0 instead and sets
+ * LKV_ERR_INVALID_ARG in its workspace status word.
+ * Returns LKV_ERR_INVALID_ARG for pages_per_seq or num_pages < 1 or a
+ * missing block table.
+ */
+#define LKV_PAGE_TOKENS 256
+
+/* lkv_quantize_kv into a paged cache; k, v are bf16 [B][Hkv][T_cap][D]. */
+LKV_API int lkv_quantize_kv_paged(lkv_qspec spec, int B, int Hkv, int pages_per_seq, int num_pages,
+                         int D, const int32_t *seq_lens, const void *k, const void *v,
+                         const int32_t *block_table, void *k_pool, float *k_sz_pool, void *v_pool,
+                         float *v_sz_pool, void *stream);
+
+/* lkv_append_kv into a paged cache (pos[b] is the logical token index). */
+LKV_API int lkv_append_kv_paged(lkv_qspec spec, int B, int Hkv, int pages_per_seq, int num_pages,
+                         int D, const int32_t *pos, const void *k_new, const void *v_new,
+                         const int32_t *block_table, void *k_pool, float *k_sz_pool, void *v_pool,
+                         float *v_sz_pool, void *stream);
+
+/*
+ * lkv_decode_attention over a paged cache.  Groups of 1, 2 or 4 query heads
+ * (LKV_ERR_UNSUPPORTED otherwise).  The workspace is that of
+ * lkv_decode_attention with T_cap = pages_per_seq * LKV_PAGE_TOKENS; the
+ * skip mask is [B][Hq][T_cap] over logical positions.
+ */
+LKV_API int lkv_decode_attention_paged(lkv_qspec spec, int B, int Hq, int Hkv, int pages_per_seq,
+                         int num_pages, int D, const int32_t *seq_lens, const void *q,
+                         const int32_t *block_table, const void *k_pool, const float *k_sz_pool,
+                         const void *v_pool, const float *v_sz_pool, float softmax_scale,
+                         float tau, float *out, uint8_t *skip_mask, int64_t *skip_counts,
+                         void *workspace, size_t ws_bytes, void *stream);
+
+/*
  * Workspace bytes that lkv_decode_attention needs for these sizes on the
  * current device (the size depends on its SM count).  The workspace is
  * caller-owned device memory (256-byte aligned).  It must be zero-filled

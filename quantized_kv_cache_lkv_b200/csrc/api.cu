@@ -110,7 +110,8 @@ size_t attention_ws_bytes(int B, int Hq, int Hkv, int T_cap, int D, int KB) {
 
 // Launch the decode of `a` on the single-launch kernel when the group fits,
 // else on the three-launch path.
-int run_attention(DecodeArgs& a, int D, int kb, int vb0, int vb1, void* ws, size_t ws_bytes, cudaStream_t s) {
+int run_attention(DecodeArgs& a, int D, int kb, int vb0, int vb1, void* ws, size_t ws_bytes, cudaStream_t s,
+                  const int32_t* block_table = nullptr, int pages_per_seq = 0, int num_pages = 0) {
   if (ws == nullptr || (reinterpret_cast<uintptr_t>(ws) % kAlign) != 0) return LKV_ERR_INVALID_ARG;
   char* base = static_cast<char*>(ws);
   a.status = reinterpret_cast<int*>(base);
@@ -145,7 +146,21 @@ int run_attention(DecodeArgs& a, int D, int kb, int vb0, int vb1, void* ws, size
   f.gstats = L.need_gstats ? reinterpret_cast<float*>(base + L.gstats) : nullptr;
   f.qbuf = reinterpret_cast<float*>(base + L.qbuf);
   f.qgsum = reinterpret_cast<float*>(base + L.qgsum);
+  f.block_table = block_table;
+  f.pages_per_seq = pages_per_seq;
+  f.num_pages = num_pages;
   cudaError_t e;
+  if (block_table != nullptr) {
+    if (vb0 != vb1) return LKV_ERR_UNSUPPORTED;
+    switch (kb) {
+      case 2: e = launch_fused_paged_k2(f, D, L.H, vb0, L.smem_bytes, L.grid, s); break;
+      case 4: e = launch_fused_paged_k4(f, D, L.H, vb0, L.smem_bytes, L.grid, s); break;
+      case 6: e = launch_fused_paged_k6(f, D, L.H, vb0, L.smem_bytes, L.grid, s); break;
+      case 8: e = launch_fused_paged_k8(f, D, L.H, vb0, L.smem_bytes, L.grid, s); break;
+      default: return LKV_ERR_UNSUPPORTED;
+    }
+    return from_cuda(e);
+  }
   switch (kb) {
     case 2: e = launch_fused_k2(f, D, L.H, vb0, vb1, L.smem_bytes, L.grid, s); break;
     case 4: e = launch_fused_k4(f, D, L.H, vb0, vb1, L.smem_bytes, L.grid, s); break;
@@ -229,10 +244,77 @@ size_t static_zero_prefix(int B, int Hq, int Hkv, int T_cap, int D, int KB) {
 }  // namespace
 
 namespace {
+
+// A paged cache: block_table [B][pps] of page ids in [0, pages); nullptr
+// table = the contiguous [B][Hkv][T_cap] layout.
+struct Paging {
+  const int32_t* table = nullptr;
+  int pps = 0, pages = 0;
+  int T_cap() const { return pps * kPageTokens; }
+};
+
+int check_paging(const Paging& pg, int B) {
+  if (pg.pps <= 0 || pg.pages <= 0) return LKV_ERR_INVALID_ARG;
+  if ((long long)pg.pps * kPageTokens > (1ll << 30)) return LKV_ERR_UNSUPPORTED;
+  if (B > 0 && (pg.table == nullptr || (reinterpret_cast<uintptr_t>(pg.table) & 3u) != 0)) return LKV_ERR_INVALID_ARG;
+  return LKV_OK;
+}
+
+int quantize_impl(lkv_qspec spec, int B, int Hkv, int T_cap, int D, const int32_t* seq_lens, const void* k,
+                  const void* v, const Paging& pg, void* k_codes, float* k_sz, void* v_codes, float* v_sz,
+                  void* stream) {
+  if (!bits_ok(spec.k_bits) || !bits_ok(spec.v_bits)) return LKV_ERR_UNSUPPORTED;
+  int rc = check_cache_shape(B, Hkv, T_cap, D, spec.group);
+  if (rc) return rc;
+  const bool ne = (long long)B * Hkv * T_cap > 0;
+  if (!ptr_ok(seq_lens, B > 0) || !ptr_ok(k, ne) || !ptr_ok(v, ne) || !ptr_ok(k_codes, ne) || !ptr_ok(k_sz, ne) ||
+      !ptr_ok(v_codes, ne) || !ptr_ok(v_sz, ne))
+    return LKV_ERR_INVALID_ARG;
+  if (!ne) return LKV_OK;
+  QuantizeArgs a{};
+  a.B = B; a.Hkv = Hkv; a.T_cap = T_cap; a.G = spec.group; a.one = 1.0f;
+  a.block_table = pg.table; a.pages_per_seq = pg.pps; a.num_pages = pg.pages;
+  a.seq_lens = seq_lens;
+  a.k = static_cast<const uint16_t*>(k);
+  a.v = static_cast<const uint16_t*>(v);
+  a.k_codes = static_cast<uint8_t*>(k_codes);
+  a.k_sz = k_sz;
+  a.v_codes = static_cast<uint8_t*>(v_codes);
+  a.v_sz = v_sz;
+  return from_cuda(launch_quantize_kv(a, spec.k_bits, spec.v_bits, D, static_cast<cudaStream_t>(stream)));
+}
+
+int append_impl(lkv_qspec spec, int B, int Hkv, int T_cap, int D, const int32_t* pos, const void* k_new,
+                const void* v_new, const Paging& pg, void* k_codes, float* k_sz, void* v_codes, float* v_sz,
+                void* stream) {
+  if (!bits_ok(spec.k_bits) || !bits_ok(spec.v_bits)) return LKV_ERR_UNSUPPORTED;
+  int rc = check_cache_shape(B, Hkv, T_cap, D, spec.group);
+  if (rc) return rc;
+  const bool ne = (long long)B * Hkv * T_cap > 0;
+  if (!ptr_ok(pos, ne) || !ptr_ok(k_new, ne) || !ptr_ok(v_new, ne) || !ptr_ok(k_codes, ne) || !ptr_ok(k_sz, ne) ||
+      !ptr_ok(v_codes, ne) || !ptr_ok(v_sz, ne))
+    return LKV_ERR_INVALID_ARG;
+  if (!ne) return LKV_OK;
+  QuantizeArgs a{};
+  a.B = B; a.Hkv = Hkv; a.T_cap = T_cap; a.G = spec.group; a.one = 1.0f;
+  a.block_table = pg.table; a.pages_per_seq = pg.pps; a.num_pages = pg.pages;
+  a.seq_lens = pos;
+  a.k = static_cast<const uint16_t*>(k_new);
+  a.v = static_cast<const uint16_t*>(v_new);
+  a.k_codes = static_cast<uint8_t*>(k_codes);
+  a.k_sz = k_sz;
+  a.v_codes = static_cast<uint8_t*>(v_codes);
+  a.v_sz = v_sz;
+  return from_cuda(launch_append_kv(a, spec.k_bits, spec.v_bits, D, static_cast<cudaStream_t>(stream)));
+}
+
+}  // namespace
+
+namespace {
 int decode_impl(lkv_qspec spec, int B, int Hq, int Hkv, int T_cap, int D, const int32_t* seq_lens, const void* q,
                 const void* k_codes, const float* k_sz, const void* v_codes, const float* v_sz, float softmax_scale,
                 float tau, float* out, uint8_t* skip_mask, int64_t* skip_counts, float* mass, void* workspace,
-                size_t ws_bytes, void* stream);
+                size_t ws_bytes, void* stream, const Paging& pg);
 }  // namespace
 
 extern "C" {
@@ -263,46 +345,32 @@ size_t lkv_sz_row_bytes(int D, int group) {
 
 int lkv_quantize_kv(lkv_qspec spec, int B, int Hkv, int T_cap, int D, const int32_t* seq_lens, const void* k,
                     const void* v, void* k_codes, float* k_sz, void* v_codes, float* v_sz, void* stream) {
-  if (!bits_ok(spec.k_bits) || !bits_ok(spec.v_bits)) return LKV_ERR_UNSUPPORTED;
-  int rc = check_cache_shape(B, Hkv, T_cap, D, spec.group);
+  return quantize_impl(spec, B, Hkv, T_cap, D, seq_lens, k, v, Paging{}, k_codes, k_sz, v_codes, v_sz, stream);
+}
+
+int lkv_quantize_kv_paged(lkv_qspec spec, int B, int Hkv, int pages_per_seq, int num_pages, int D,
+                          const int32_t* seq_lens, const void* k, const void* v, const int32_t* block_table,
+                          void* k_pool, float* k_sz_pool, void* v_pool, float* v_sz_pool, void* stream) {
+  Paging pg{block_table, pages_per_seq, num_pages};
+  int rc = check_paging(pg, B);
   if (rc) return rc;
-  const bool ne = (long long)B * Hkv * T_cap > 0;
-  if (!ptr_ok(seq_lens, B > 0) || !ptr_ok(k, ne) || !ptr_ok(v, ne) || !ptr_ok(k_codes, ne) || !ptr_ok(k_sz, ne) ||
-      !ptr_ok(v_codes, ne) || !ptr_ok(v_sz, ne))
-    return LKV_ERR_INVALID_ARG;
-  if (!ne) return LKV_OK;
-  QuantizeArgs a{};
-  a.B = B; a.Hkv = Hkv; a.T_cap = T_cap; a.G = spec.group; a.one = 1.0f;
-  a.seq_lens = seq_lens;
-  a.k = static_cast<const uint16_t*>(k);
-  a.v = static_cast<const uint16_t*>(v);
-  a.k_codes = static_cast<uint8_t*>(k_codes);
-  a.k_sz = k_sz;
-  a.v_codes = static_cast<uint8_t*>(v_codes);
-  a.v_sz = v_sz;
-  return from_cuda(launch_quantize_kv(a, spec.k_bits, spec.v_bits, D, static_cast<cudaStream_t>(stream)));
+  return quantize_impl(spec, B, Hkv, pg.T_cap(), D, seq_lens, k, v, pg, k_pool, k_sz_pool, v_pool, v_sz_pool,
+                       stream);
 }
 
 int lkv_append_kv(lkv_qspec spec, int B, int Hkv, int T_cap, int D, const int32_t* pos, const void* k_new,
                   const void* v_new, void* k_codes, float* k_sz, void* v_codes, float* v_sz, void* stream) {
-  if (!bits_ok(spec.k_bits) || !bits_ok(spec.v_bits)) return LKV_ERR_UNSUPPORTED;
-  int rc = check_cache_shape(B, Hkv, T_cap, D, spec.group);
+  return append_impl(spec, B, Hkv, T_cap, D, pos, k_new, v_new, Paging{}, k_codes, k_sz, v_codes, v_sz, stream);
+}
+
+int lkv_append_kv_paged(lkv_qspec spec, int B, int Hkv, int pages_per_seq, int num_pages, int D, const int32_t* pos,
+                        const void* k_new, const void* v_new, const int32_t* block_table, void* k_pool,
+                        float* k_sz_pool, void* v_pool, float* v_sz_pool, void* stream) {
+  Paging pg{block_table, pages_per_seq, num_pages};
+  int rc = check_paging(pg, B);
   if (rc) return rc;
-  const bool ne = (long long)B * Hkv * T_cap > 0;
-  if (!ptr_ok(pos, ne) || !ptr_ok(k_new, ne) || !ptr_ok(v_new, ne) || !ptr_ok(k_codes, ne) || !ptr_ok(k_sz, ne) ||
-      !ptr_ok(v_codes, ne) || !ptr_ok(v_sz, ne))
-    return LKV_ERR_INVALID_ARG;
-  if (!ne) return LKV_OK;
-  QuantizeArgs a{};
-  a.B = B; a.Hkv = Hkv; a.T_cap = T_cap; a.G = spec.group; a.one = 1.0f;
-  a.seq_lens = pos;
-  a.k = static_cast<const uint16_t*>(k_new);
-  a.v = static_cast<const uint16_t*>(v_new);
-  a.k_codes = static_cast<uint8_t*>(k_codes);
-  a.k_sz = k_sz;
-  a.v_codes = static_cast<uint8_t*>(v_codes);
-  a.v_sz = v_sz;
-  return from_cuda(launch_append_kv(a, spec.k_bits, spec.v_bits, D, static_cast<cudaStream_t>(stream)));
+  return append_impl(spec, B, Hkv, pg.T_cap(), D, pos, k_new, v_new, pg, k_pool, k_sz_pool, v_pool, v_sz_pool,
+                     stream);
 }
 
 size_t lkv_decode_workspace_bytes(lkv_qspec spec, int B, int Hq, int Hkv, int T_cap, int D) {
@@ -316,7 +384,21 @@ int lkv_decode_attention(lkv_qspec spec, int B, int Hq, int Hkv, int T_cap, int 
                          const float* v_sz, float softmax_scale, float tau, float* out, uint8_t* skip_mask,
                          int64_t* skip_counts, void* workspace, size_t ws_bytes, void* stream) {
   return decode_impl(spec, B, Hq, Hkv, T_cap, D, seq_lens, q, k_codes, k_sz, v_codes, v_sz, softmax_scale, tau,
-                     out, skip_mask, skip_counts, nullptr, workspace, ws_bytes, stream);
+                     out, skip_mask, skip_counts, nullptr, workspace, ws_bytes, stream, Paging{});
+}
+
+int lkv_decode_attention_paged(lkv_qspec spec, int B, int Hq, int Hkv, int pages_per_seq, int num_pages, int D,
+                               const int32_t* seq_lens, const void* q, const int32_t* block_table,
+                               const void* k_pool, const float* k_sz_pool, const void* v_pool,
+                               const float* v_sz_pool, float softmax_scale, float tau, float* out,
+                               uint8_t* skip_mask, int64_t* skip_counts, void* workspace, size_t ws_bytes,
+                               void* stream) {
+  Paging pg{block_table, pages_per_seq, num_pages};
+  int rc = check_paging(pg, B);
+  if (rc) return rc;
+  if (Hkv > 0 && !fused_ok(Hq / Hkv)) return LKV_ERR_UNSUPPORTED;  // paged: groups of 1, 2 or 4 query heads
+  return decode_impl(spec, B, Hq, Hkv, pg.T_cap(), D, seq_lens, q, k_pool, k_sz_pool, v_pool, v_sz_pool,
+                     softmax_scale, tau, out, skip_mask, skip_counts, nullptr, workspace, ws_bytes, stream, pg);
 }
 
 int lkv_decode_attention_mass(lkv_qspec spec, int B, int Hq, int Hkv, int T_cap, int D, const int32_t* seq_lens,
@@ -325,7 +407,7 @@ int lkv_decode_attention_mass(lkv_qspec spec, int B, int Hq, int Hkv, int T_cap,
                               int64_t* skip_counts, float* mass, void* workspace, size_t ws_bytes, void* stream) {
   if (mass == nullptr && (long long)B * Hkv * T_cap > 0) return LKV_ERR_INVALID_ARG;
   return decode_impl(spec, B, Hq, Hkv, T_cap, D, seq_lens, q, k_codes, k_sz, v_codes, v_sz, softmax_scale, tau,
-                     out, skip_mask, skip_counts, mass, workspace, ws_bytes, stream);
+                     out, skip_mask, skip_counts, mass, workspace, ws_bytes, stream, Paging{});
 }
 
 }  // extern "C"
@@ -335,7 +417,7 @@ namespace {
 int decode_impl(lkv_qspec spec, int B, int Hq, int Hkv, int T_cap, int D, const int32_t* seq_lens, const void* q,
                 const void* k_codes, const float* k_sz, const void* v_codes, const float* v_sz, float softmax_scale,
                 float tau, float* out, uint8_t* skip_mask, int64_t* skip_counts, float* mass, void* workspace,
-                size_t ws_bytes, void* stream) {
+                size_t ws_bytes, void* stream, const Paging& pg) {
   if (!bits_ok(spec.k_bits) || !bits_ok(spec.v_bits)) return LKV_ERR_UNSUPPORTED;
   int rc = check_attention_shape(B, Hq, Hkv, T_cap, D, spec.group);
   if (rc) return rc;
@@ -367,7 +449,8 @@ int decode_impl(lkv_qspec spec, int B, int Hq, int Hkv, int T_cap, int D, const 
   a.skip_mask = skip_mask;
   a.mass = mass;
   a.skip_counts = reinterpret_cast<unsigned long long*>(skip_counts);
-  return run_attention(a, D, spec.k_bits, spec.v_bits, spec.v_bits, workspace, ws_bytes, s);
+  return run_attention(a, D, spec.k_bits, spec.v_bits, spec.v_bits, workspace, ws_bytes, s, pg.table,
+                       pg.pps, pg.pages);
 }
 
 }  // namespace

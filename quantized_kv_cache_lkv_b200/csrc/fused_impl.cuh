@@ -39,6 +39,7 @@ namespace lkv {
 namespace fused {
 
 constexpr int kChunk = 256;    // tokens per chunk (work-partition granularity)
+static_assert(kChunk == kPageTokens, "a chunk of a paged cache is one page");
 constexpr int kSlotsPerWarp = 2;
 constexpr int kMaxConsumerWarps = 12;
 constexpr int kListCap = 512;  // V-row list entries per warp per batch
@@ -145,6 +146,25 @@ __device__ __forceinline__ ChunkRows chunk_rows(const Unit& x, int c) {
   r.row0 = cs * kChunk;
   r.rows = min(kChunk, n - r.row0);
   return r;
+}
+
+// Physical cache row of row `row` of unit u: contiguous, or (PAGED) the
+// unit's slot in the page the block table names; a page id outside the pool
+// is read as page 0 and reported in the status word.
+template <bool PAGED>
+__device__ __forceinline__ long long unit_row(const FusedArgs& a, int u, int row) {
+  const DecodeArgs& d = a.d;
+  if constexpr (!PAGED) {
+    return (long long)u * d.T_cap + row;
+  } else {
+    const int b = u / d.Hkv, g = u - b * d.Hkv;
+    int page = __ldg(a.block_table + (long long)b * a.pages_per_seq + row / kPageTokens);
+    if (page < 0 || page >= a.num_pages) {
+      atomicExch(d.status, kStatusInvalidArg);
+      page = 0;
+    }
+    return ((long long)page * d.Hkv + g) * kPageTokens + row % kPageTokens;
+  }
 }
 
 // Bounded spin on a counter written by other CTAs.
@@ -291,7 +311,7 @@ __device__ __forceinline__ float2 code_pair_at(const LaneWords<BITS>& lw, const 
 
 // ------------------------------------------------------------------ kernel
 
-template <int D, int H, int KB, int VB0, int VB1>
+template <int D, int H, int KB, int VB0, int VB1, bool PAGED>
 __global__ void __launch_bounds__(Geo<D, KB>::kThreads, 1) fused_decode_kernel(FusedArgs a) {
   using Gk = Geo<D, KB>;
   constexpr int CW = Gk::kCW, NCONS = Gk::kConsumers, NTHR = Gk::kThreads;
@@ -490,8 +510,11 @@ __global__ void __launch_bounds__(Geo<D, KB>::kThreads, 1) fused_decode_kernel(F
         const uint32_t sbytes = (uint32_t)(r1 - r0) * ng * 8;
         uint8_t* dst = ring + (size_t)stage * Gk::kStageBytes;
         mbar_arrive_expect_tx(&full[stage], cbytes + sbytes);
-        bulk_g2s(dst, d.kc[td.seg] + (ubase + row) * Gk::RB, cbytes, &full[stage], pol);
-        bulk_g2s(dst + Gk::kStageCodes, d.ksz[td.seg] + (ubase + r0) * ng * 2, sbytes, &full[stage], pol);
+        // a tile lies in one chunk, which is one page of a paged cache
+        const long long pr = PAGED ? unit_row<PAGED>(a, td.u, row) : ubase + row;
+        const long long pr0 = PAGED ? unit_row<PAGED>(a, td.u, r0) : ubase + r0;
+        bulk_g2s(dst, d.kc[td.seg] + pr * Gk::RB, cbytes, &full[stage], pol);
+        bulk_g2s(dst + Gk::kStageCodes, d.ksz[td.seg] + pr0 * ng * 2, sbytes, &full[stage], pol);
       }
     };
     TileDesc p0, p1;
@@ -804,8 +827,10 @@ __global__ void __launch_bounds__(Geo<D, KB>::kThreads, 1) fused_decode_kernel(F
             uint8_t* dst = stg + buf * kDenseBuf;
             uint64_t* bar = &full[kDenseBar + warp * 2 + buf];
             mbar_arrive_expect_tx(bar, cbytes + sbytes + lbytes);
-            bulk_g2s(dst, d.vc[seg] + (ubase + row) * rbv, cbytes, bar, pol);
-            bulk_g2s(dst + kDenseCodes, d.vsz[seg] + (ubase + r0) * ng * 2, sbytes, bar, pol);
+            const long long pr = PAGED ? unit_row<PAGED>(a, x.u, row) : ubase + row;
+            const long long pr0 = PAGED ? unit_row<PAGED>(a, x.u, r0) : ubase + r0;
+            bulk_g2s(dst, d.vc[seg] + pr * rbv, cbytes, bar, pol);
+            bulk_g2s(dst + kDenseCodes, d.vsz[seg] + pr0 * ng * 2, sbytes, bar, pol);
             bulk_g2s(dst + kDenseCodes + kDenseSz, lgu + (long long)v0 * H, lbytes, bar, pol);
           }
         };
@@ -965,7 +990,7 @@ __global__ void __launch_bounds__(Geo<D, KB>::kThreads, 1) fused_decode_kernel(F
             if (vv[s2] >= 0) {
               const int v = vv[s2];
               const ChunkRows cr = chunk_rows(x, v / kChunk);
-              const long long row = ubase + cr.row0 + v % kChunk;
+              const long long row = PAGED ? unit_row<PAGED>(a, x.u, cr.row0 + v % kChunk) : ubase + cr.row0 + v % kChunk;
               if constexpr (kOneWidth) {
                 ldg_v<VB0>(d.vc[cr.seg] + row * (D * VB0 / 8), d.vsz[cr.seg] + row * ng * 2, j, gi, w0[s2], szv[s2]);
               } else if (cr.seg == 0) {

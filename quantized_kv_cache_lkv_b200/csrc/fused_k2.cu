@@ -4,6 +4,6 @@
 namespace lkv {
 cudaError_t launch_fused_k2(const FusedArgs& a, int D, int H, int vb0, int vb1, size_t smem, int grid,
                              cudaStream_t s) {
-  return fused::launch_kb<2>(a, D, H, vb0, vb1, smem, grid, s);
+  return fused::launch_kb<2, false>(a, D, H, vb0, vb1, smem, grid, s);
 }
 }  // namespace lkv

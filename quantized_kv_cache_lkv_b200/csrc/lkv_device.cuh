@@ -28,6 +28,22 @@ __device__ __forceinline__ int clamp_len(int32_t t, int T_cap) {
   return t < 0 ? 0 : (t > T_cap ? T_cap : t);
 }
 
+// Paged caches: a page holds kPageTokens consecutive tokens of one KV head;
+// the pool is [num_pages][Hkv][kPageTokens][row], and block_table[b][i] is the
+// page of tokens [i * kPageTokens, (i + 1) * kPageTokens) of sequence b.
+constexpr int kPageTokens = 256;
+
+// Physical row of token t of KV head g of sequence b: the contiguous cache
+// row (b * Hkv + g) * T_cap + t, or its slot in the page that the block
+// table names.  A page id outside [0, num_pages) gives -1.
+__device__ __forceinline__ long long cache_row(const int32_t* block_table, int pages_per_seq, int num_pages,
+                                               int Hkv, int T_cap, int b, int g, int t) {
+  if (block_table == nullptr) return ((long long)b * Hkv + g) * T_cap + t;
+  const int page = __ldg(block_table + (long long)b * pages_per_seq + t / kPageTokens);
+  if (page < 0 || page >= num_pages) return -1;
+  return ((long long)page * Hkv + g) * kPageTokens + (t % kPageTokens);
+}
+
 // Words of one lane's 16 codes.
 template <int BITS>
 struct LaneWords {

@@ -7,6 +7,8 @@ namespace lkv {
 struct QuantizeArgs {
   int B, Hkv, T_cap, G;
   float one;  // 1.0f, read at run time by the rounding step of the quantizer
+  const int32_t* block_table;  // nullable: contiguous [B][Hkv][T_cap] cache
+  int pages_per_seq, num_pages;
   const int32_t* seq_lens;
   const uint16_t* k;
   const uint16_t* v;
@@ -88,6 +90,9 @@ struct FusedArgs {
   float* qgsum;                  // [units][H][4] sums of qbuf per quantization group
   unsigned long long* wcounts;   // [2] skip-count accumulators
   int* done;                     // CTAs finished
+  // paged cache (plain decode only): block table [B][pages_per_seq], T_cap = pages_per_seq * kPageTokens
+  const int32_t* block_table;
+  int pages_per_seq, num_pages;
 };
 
 // Dispatch on (D, H, V widths) for one K width; smem = dynamic shared bytes.
@@ -95,6 +100,11 @@ cudaError_t launch_fused_k2(const FusedArgs& a, int D, int H, int vb0, int vb1, 
 cudaError_t launch_fused_k4(const FusedArgs& a, int D, int H, int vb0, int vb1, size_t smem, int grid, cudaStream_t s);
 cudaError_t launch_fused_k6(const FusedArgs& a, int D, int H, int vb0, int vb1, size_t smem, int grid, cudaStream_t s);
 cudaError_t launch_fused_k8(const FusedArgs& a, int D, int H, int vb0, int vb1, size_t smem, int grid, cudaStream_t s);
+// The same over a paged cache (plain decode: one V width).
+cudaError_t launch_fused_paged_k2(const FusedArgs& a, int D, int H, int vb, size_t smem, int grid, cudaStream_t s);
+cudaError_t launch_fused_paged_k4(const FusedArgs& a, int D, int H, int vb, size_t smem, int grid, cudaStream_t s);
+cudaError_t launch_fused_paged_k6(const FusedArgs& a, int D, int H, int vb, size_t smem, int grid, cudaStream_t s);
+cudaError_t launch_fused_paged_k8(const FusedArgs& a, int D, int H, int vb, size_t smem, int grid, cudaStream_t s);
 
 int num_sms();
 

@@ -221,8 +221,10 @@ __global__ void __launch_bounds__(256, 2) quantize_kv_kernel(QuantizeArgs a) {
     if (b_ >= (uint32_t)a.B) return false;
     const int t = (int)tb_ * RPW + sub;
     if (t >= clamp_len(__ldg(a.seq_lens + b_), a.T_cap)) return false;
-    row = ((long long)b_ * a.Hkv + g_) * a.T_cap + t;
-    fetch_lane_rows32(a.k + row * D + j * kLaneDims32, a.v + row * D + j * kLaneDims32, r);
+    const long long src = ((long long)b_ * a.Hkv + g_) * a.T_cap + t;
+    row = cache_row(a.block_table, a.pages_per_seq, a.num_pages, a.Hkv, a.T_cap, (int)b_, (int)g_, t);
+    if (row < 0) return false;  // a page outside the pool: nothing is written
+    fetch_lane_rows32(a.k + src * D + j * kLaneDims32, a.v + src * D + j * kLaneDims32, r);
     return true;
   };
   LaneRows32 cur, nxt;
@@ -259,7 +261,9 @@ __global__ void __launch_bounds__(256) append_kv_kernel(QuantizeArgs a) {
   if (unit >= (long long)a.B * a.Hkv) return;  // the lanes of a row agree
   const int t = __ldg(a.seq_lens + unit / a.Hkv);
   if (t < 0 || t >= a.T_cap) return;
-  const long long row = unit * a.T_cap + t;
+  const long long row = cache_row(a.block_table, a.pages_per_seq, a.num_pages, a.Hkv, a.T_cap,
+                                  (int)(unit / a.Hkv), (int)(unit % a.Hkv), t);
+  if (row < 0) return;  // a page outside the pool: nothing is written
   LaneRows r;
   fetch_lane_rows(a.k + unit * D + j * kDimsPerLane, a.v + unit * D + j * kDimsPerLane, r);
   quantize_lane<KB>(r.k0, r.k1, a.k_codes + row * (D * KB / 8), a.k_sz + row * ng * 2, j, lpg, mask, a.one);

@@ -49,6 +49,10 @@ SIGNATURES = {
     "lkv_sz_row_bytes": (_Z, [_I, _I]),
     "lkv_quantize_kv": (_I, [lkv_qspec, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P, _P, _P]),
     "lkv_append_kv": (_I, [lkv_qspec, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P, _P, _P]),
+    "lkv_quantize_kv_paged": (_I, [lkv_qspec, _I, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P, _P, _P, _P]),
+    "lkv_append_kv_paged": (_I, [lkv_qspec, _I, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P, _P, _P, _P]),
+    "lkv_decode_attention_paged": (_I, [lkv_qspec, _I, _I, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P, _P, _F,
+                                        _F, _P, _P, _P, _P, _Z, _P]),
     "lkv_decode_workspace_bytes": (_Z, [lkv_qspec, _I, _I, _I, _I, _I]),
     "lkv_decode_attention": (_I, [lkv_qspec, _I, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P, _F, _F,
                                   _P, _P, _P, _P, _Z, _P]),
@@ -147,6 +151,34 @@ def lkv_append_kv(spec, B, Hkv, T_cap, D, pos, k_new, v_new, k_codes, k_sz, v_co
     _check(lib().lkv_append_kv(_spec(spec), B, Hkv, T_cap, D, _ptr(pos), _ptr(k_new), _ptr(v_new),
                                _ptr(k_codes), _ptr(k_sz), _ptr(v_codes), _ptr(v_sz), _stream(stream)),
            "lkv_append_kv")
+
+
+LKV_PAGE_TOKENS = 256
+
+
+def lkv_quantize_kv_paged(spec, B, Hkv, pages_per_seq, num_pages, D, seq_lens, k, v, block_table, k_pool,
+                          k_sz_pool, v_pool, v_sz_pool, stream=None):
+    _check(lib().lkv_quantize_kv_paged(_spec(spec), B, Hkv, pages_per_seq, num_pages, D, _ptr(seq_lens),
+                                       _ptr(k), _ptr(v), _ptr(block_table), _ptr(k_pool), _ptr(k_sz_pool),
+                                       _ptr(v_pool), _ptr(v_sz_pool), _stream(stream)), "lkv_quantize_kv_paged")
+
+
+def lkv_append_kv_paged(spec, B, Hkv, pages_per_seq, num_pages, D, pos, k_new, v_new, block_table, k_pool,
+                        k_sz_pool, v_pool, v_sz_pool, stream=None):
+    _check(lib().lkv_append_kv_paged(_spec(spec), B, Hkv, pages_per_seq, num_pages, D, _ptr(pos), _ptr(k_new),
+                                     _ptr(v_new), _ptr(block_table), _ptr(k_pool), _ptr(k_sz_pool),
+                                     _ptr(v_pool), _ptr(v_sz_pool), _stream(stream)), "lkv_append_kv_paged")
+
+
+def lkv_decode_attention_paged(spec, B, Hq, Hkv, pages_per_seq, num_pages, D, seq_lens, q, block_table, k_pool,
+                               k_sz_pool, v_pool, v_sz_pool, softmax_scale, tau, out, skip_mask, skip_counts,
+                               workspace, ws_bytes, stream=None):
+    _check(lib().lkv_decode_attention_paged(_spec(spec), B, Hq, Hkv, pages_per_seq, num_pages, D,
+                                            _ptr(seq_lens), _ptr(q), _ptr(block_table), _ptr(k_pool),
+                                            _ptr(k_sz_pool), _ptr(v_pool), _ptr(v_sz_pool), float(softmax_scale),
+                                            float(tau), _ptr(out), _ptr(skip_mask), _ptr(skip_counts),
+                                            _ptr(workspace), int(ws_bytes), _stream(stream)),
+           "lkv_decode_attention_paged")
 
 
 def lkv_decode_workspace_bytes(spec, B, Hq, Hkv, T_cap, D):

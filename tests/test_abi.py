@@ -158,6 +158,20 @@ def test_append_and_mass_reject(L):
     assert rc_of(mass, mass=FAKE, workspace=FAKE, ws_bytes=64) == lkv.LKV_ERR_WORKSPACE
 
 
+def test_paged_rejects(L):
+    pq = [K6V4, 2, 2, 3, 8, 128, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 0]
+    assert rc_of(lkv.lkv_quantize_kv_paged, *pq[:3], 0, *pq[4:]) == lkv.LKV_ERR_INVALID_ARG       # pages_per_seq
+    assert rc_of(lkv.lkv_quantize_kv_paged, *pq[:4], 0, *pq[5:]) == lkv.LKV_ERR_INVALID_ARG       # num_pages
+    assert rc_of(lkv.lkv_quantize_kv_paged, *pq[:9], None, *pq[10:]) == lkv.LKV_ERR_INVALID_ARG   # table
+    assert rc_of(lkv.lkv_append_kv_paged, *pq[:9], None, *pq[10:]) == lkv.LKV_ERR_INVALID_ARG
+    pd = [K6V4, 2, 16, 2, 3, 8, 128, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 0.088, 0.0, FAKE, None, None,
+          FAKE, 1 << 40, 0]
+    assert rc_of(lkv.lkv_decode_attention_paged, *pd) == lkv.LKV_ERR_UNSUPPORTED                # groups of 8
+    pd[2] = 8
+    assert rc_of(lkv.lkv_decode_attention_paged, *pd[:9], None, *pd[10:]) == lkv.LKV_ERR_INVALID_ARG
+    assert rc_of(lkv.lkv_decode_attention_paged, *pd[:20], 64, pd[21]) == lkv.LKV_ERR_WORKSPACE
+
+
 def test_tiered_rejects(L):
     seg = lkv.lkv_segment(FAKE, FAKE, FAKE, FAKE)
     bad = lkv.lkv_segment(FAKE, None, FAKE, FAKE)
