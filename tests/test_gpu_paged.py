@@ -115,3 +115,34 @@ def test_paged_decode_bad_page_is_reported():
     torch.cuda.synchronize()
     assert lkv.lkv_workspace_status(ws) == lkv.LKV_ERR_INVALID_ARG
     assert torch.isfinite(out).all()
+
+
+@pytest.mark.slow
+def test_paged_decode_full_size_equals_contiguous():
+    """The Llama-3.1-8B-shaped decode (B16, 32 q / 8 kv heads, T8192 = 32
+    pages per sequence, tau 1e-4) over a shuffled pool of 520 pages is
+    bit-identical to the contiguous decode."""
+    cfg = W.CONFIGS[2]
+    B, Hq, Hkv, D, T, G = cfg.B, cfg.Hq, cfg.Hkv, cfg.D, cfg.T_cap, cfg.G
+    pps = T // P
+    inp = W.make_inputs(cfg)
+    num_pages = B * pps + 8
+    table = torch.randperm(num_pages, generator=torch.Generator().manual_seed(5))[:B * pps].view(B, pps)
+    table = table.to(torch.int32)
+    pool = make_pool(6, 4, G, Hkv, D, num_pages)
+    sl = dev(inp["seq_lens"])
+    lkv.lkv_quantize_kv_paged((6, 4, G), B, Hkv, pps, num_pages, D, sl, dev(inp["k"]), dev(inp["v"]), dev(table),
+                              pool["k_codes"], pool["k_sz"], pool["v_codes"], pool["v_sz"])
+    cache = gpu_quantize(6, 4, G, inp)
+    want_out, want_mask, want_counts = gpu_decode(6, 4, G, inp, cache, cfg.softmax_scale, cfg.tau, want_mask=False)
+    nb = lkv.lkv_decode_workspace_bytes((6, 4, G), B, Hq, Hkv, T, D)
+    ws = buffers.alloc_workspace(nb)
+    out = torch.empty(B, Hq, D, device="cuda")
+    counts = torch.zeros(2, dtype=torch.int64, device="cuda")
+    lkv.lkv_decode_attention_paged((6, 4, G), B, Hq, Hkv, pps, num_pages, D, sl, dev(inp["q"]), dev(table),
+                                   pool["k_codes"], pool["k_sz"], pool["v_codes"], pool["v_sz"], cfg.softmax_scale,
+                                   cfg.tau, out, None, counts, ws, nb)
+    torch.cuda.synchronize()
+    assert lkv.lkv_workspace_status(ws) == lkv.LKV_OK
+    np.testing.assert_array_equal(out.cpu().numpy(), want_out)
+    assert counts.cpu().tolist() == want_counts.tolist()
