@@ -317,6 +317,83 @@ __global__ void __launch_bounds__(256, 2) tier_repack_kernel(RepackArgs a, int S
   }
 }
 
+// The same repack over a grid of resident blocks, with the rows of every
+// (segment, unit) pair laid end to end (segment A's units, then segment B's)
+// and dealt out evenly, so that a unit's short segment A and long segment B
+// cost the same per row.  Each block rebuilds the pairs' first rows in shared
+// memory from the clamped counts.
+constexpr int kRepackMaxPairs = 8192;
+
+template <int D, int LPG>
+__global__ void __launch_bounds__(256, 2) tier_repack_flat_kernel(RepackArgs a) {
+  constexpr int LPR = D / kLaneDims32;
+  constexpr int RPW = 32 / LPR;
+  extern __shared__ int s_first[];  // [pairs + 1]: first row of pair p = seg * units + unit, then the total
+  __shared__ int s_wsum[32];
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, nw = blockDim.x / 32;
+  const int j = lane % LPR, sub = lane / LPR;
+  const unsigned mask = row_lane_mask<LPR>(lane);
+  const int ng = D / a.G;
+  const int units = a.B * a.Hkv, pairs = 2 * units;
+  auto rows_of = [&](int p) { return clamp_len(a.counts[2 * (p % units) + p / units], a.T_cap); };
+  // exclusive scan of the pairs' row counts: a run of pairs per thread
+  const int per = (pairs + (int)blockDim.x - 1) / (int)blockDim.x;
+  const int p0 = min(pairs, tid * per), p1 = min(pairs, p0 + per);
+  int mine = 0;
+  for (int p = p0; p < p1; ++p) mine += rows_of(p);
+  int incl = mine;
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    const int y = __shfl_up_sync(0xFFFFFFFFu, incl, off);
+    if (lane >= off) incl += y;
+  }
+  if (lane == 31) s_wsum[warp] = incl;
+  __syncthreads();
+  int run = incl - mine;
+  for (int w = 0; w < warp; ++w) run += s_wsum[w];
+  for (int p = p0; p < p1; ++p) { s_first[p] = run; run += rows_of(p); }
+  if (tid == (int)blockDim.x - 1) s_first[pairs] = run;  // the last thread's inclusive prefix: every row
+  __syncthreads();
+  const int total = s_first[pairs];
+  // row r lies in the last pair whose first row is <= r (empty pairs are passed over)
+  auto fetch = [&](int r, LaneRows32& x, int& seg, long long& slot) -> bool {
+    if (r >= total) return false;
+    int lo = 0, hi = pairs - 1;
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (s_first[mid] <= r) lo = mid; else hi = mid - 1;
+    }
+    seg = lo / units;
+    const long long bg = lo % units;
+    const int i = r - s_first[lo];
+    int t = __ldg((seg == 0 ? a.pos_a : a.pos_b) + bg * a.T_cap + i);
+    t = t < 0 ? 0 : (t >= a.T_cap ? a.T_cap - 1 : t);
+    const long long src = bg * a.T_cap + t;
+    fetch_lane_rows32(a.k + src * D + j * kLaneDims32, a.v + src * D + j * kLaneDims32, x);
+    slot = bg * a.T_cap + i;
+    return true;
+  };
+  const int stride = (int)gridDim.x * nw * RPW;
+  int r = ((int)blockIdx.x * nw + warp) * RPW + sub;
+  LaneRows32 cur, nxt;
+  int seg = 0, seg_n = 0;
+  long long slot = 0, slot_n = 0;
+  bool ok = fetch(r, cur, seg, slot);
+  for (; r - sub < total; r += stride) {  // r - sub is the same for the whole warp
+    const bool ok_n = fetch(r + stride, nxt, seg_n, slot_n);
+    if (ok) {
+      if (seg == 0) {
+        quantize_lane32<6, LPG>(cur.k, a.a_kc + slot * (D * 6 / 8), a.a_ksz + slot * ng * 2, j, mask, a.one);
+        quantize_lane32<6, LPG>(cur.v, a.a_vc + slot * (D * 6 / 8), a.a_vsz + slot * ng * 2, j, mask, a.one);
+      } else {
+        quantize_lane32<6, LPG>(cur.k, a.b_kc + slot * (D * 6 / 8), a.b_ksz + slot * ng * 2, j, mask, a.one);
+        quantize_lane32<4, LPG>(cur.v, a.b_vc + slot * (D * 4 / 8), a.b_vsz + slot * ng * 2, j, mask, a.one);
+      }
+    }
+    cur = nxt; ok = ok_n; seg = seg_n; slot = slot_n;
+  }
+}
+
 // Resident blocks of 256 threads per SM for a kernel (cached per kernel and
 // device by the caller's static).
 static int resident_blocks(const void* kern) {
@@ -398,6 +475,17 @@ cudaError_t launch_append_kv(const QuantizeArgs& a, int kb, int vb, int D, cudaS
 cudaError_t launch_tier_repack(const RepackArgs& a, int D, cudaStream_t s) {
   const long long units = (long long)a.B * a.Hkv;
   if (units == 0 || a.T_cap == 0) return cudaSuccess;
+  if (2 * units <= kRepackMaxPairs && 2 * units * a.T_cap < (1ll << 30)) {
+    const dim3 grid((unsigned)(num_sms() * 2));
+    const size_t smem = (size_t)(2 * units + 1) * sizeof(int);
+    if (D == 64 && a.G == 32) tier_repack_flat_kernel<64, 1><<<grid, 256, smem, s>>>(a);
+    else if (D == 64 && a.G == 64) tier_repack_flat_kernel<64, 2><<<grid, 256, smem, s>>>(a);
+    else if (D == 128 && a.G == 32) tier_repack_flat_kernel<128, 1><<<grid, 256, smem, s>>>(a);
+    else if (D == 128 && a.G == 64) tier_repack_flat_kernel<128, 2><<<grid, 256, smem, s>>>(a);
+    else if (D == 128 && a.G == 128) tier_repack_flat_kernel<128, 4><<<grid, 256, smem, s>>>(a);
+    else return cudaErrorInvalidValue;
+    return cudaGetLastError();
+  }
   // about eight blocks per SM over both segments, at least one per unit
   const long long want = (long long)num_sms() * 8;
   const int S = (int)std::max<long long>(1, std::min<long long>(64, want / (2 * units)));
