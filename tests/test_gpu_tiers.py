@@ -157,3 +157,14 @@ def test_tiered_full_size_sampled(orc):
     """The tiered workload at full size (B32, context log-uniform in
     [1024, 32768], Zipf(1.1) mass); sequences 0, 17 and 31 checked."""
     tiered_case(orc, W.CONFIGS[5], W.CONFIGS[5].tau_low, W.CONFIGS[5].tau_high, batches=[0, 17, 31])
+
+
+@pytest.mark.parametrize("B", [512, 1040])
+def test_repack_both_row_layouts(orc, B):
+    """Up to 8192 (segment, unit) pairs the repack deals all kept rows evenly
+    over resident blocks; past that it gives each pair its own blocks.  B512
+    (8192 pairs) and B1040 (16640 pairs) with 8 KV heads and short ragged
+    contexts take one layout each; segments are bit-exact with the oracle
+    on sampled sequences."""
+    cfg = W.scaled(W.CONFIGS[5], B=B, T_cap=24, seq_lo=1, seq_hi=24, seed=71 + B)
+    tiered_case(orc, cfg, 2e-3, 5e-2, batches=[0, B // 2 + 1, B - 1])
