@@ -369,8 +369,8 @@ __global__ void __launch_bounds__(Geo<D, KB>::kThreads, 1) fused_decode_kernel(F
 #pragma unroll
     for (int off = 16; off >= 1; off >>= 1) part += __shfl_xor_sync(kFull, part, off);
     if (lane == 0) atomicAdd(&s_total, part);
-    if (tid == 0 && cta == 0) {
-      for (int u = 0; u < (d.len_mode == 0 ? d.B : units); ++u) {
+    if (cta == 0) {  // length checks, spread over the CTA's threads (a serial loop here delays CTA 0)
+      for (int u = tid; u < (d.len_mode == 0 ? d.B : units); u += NCONS) {
         bool bad;
         if (d.len_mode == 0) {
           bad = d.lens[u] < 0 || d.lens[u] > d.T_cap;
