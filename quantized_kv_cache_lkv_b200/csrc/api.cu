@@ -65,11 +65,13 @@ WsLayout ws_layout(int B, int Hq, int Hkv, int T_cap, int D) {
 bool fused_ok(int r) { return r == 1 || r == 2 || r == 4; }
 
 struct FusedLayout {
-  int grid, H, cpc_max, ring_bytes, stages;
+  int grid, H, cpc_max, ring_bytes, stages, cand_cap;
   size_t smem_bytes;
   size_t arrive1, arrive2, pstats, ppart, ulist, glogits, gstats, qbuf, qgsum, total;
   bool need_gstats;
 };
+
+constexpr int kMaxSmem = 227 * 1024;  // dynamic shared memory of one CTA on sm_100
 
 FusedLayout fused_layout(int B, int Hq, int Hkv, int T_cap, int D, int KB) {
   FusedLayout L{};
@@ -80,13 +82,24 @@ FusedLayout fused_layout(int B, int Hq, int Hkv, int T_cap, int D, int KB) {
   const long long per_unit = T_cap > 0 ? (T_cap + kChunk - 1) / kChunk + 1 : 1;
   const long long chunks_max = units * per_unit > 0 ? units * per_unit : 1;
   L.cpc_max = (int)((chunks_max + L.grid - 1) / L.grid);
-  const fused::GeoHost g = fused::geo_host(D, KB);
-  L.stages = g.stages;
-  const int lists = fused::kMaxConsumerWarps * fused::kListCap * 4 * (1 + L.H);
-  const int phase2 = std::max(lists, fused::kDenseStaging) + fused::kMaxConsumerWarps * L.H * D * 4;
-  L.ring_bytes = std::max(g.stages * g.stage_bytes, phase2);
+  // phase 1: as many ring stages as shared memory holds (at most kMaxStages);
+  // phase 2 reuses the ring: sparse-mode lists of kept rows (256 per warp)
+  // and V staging slots, the fallback scan's lists, or the dense-mode
+  // buffers, each followed by the warps' partial outputs
+  const int sb = fused::stage_bytes_host(D, KB);
+  const int red = fused::kWarps * L.H * D * 4;
+  const int slot = D * 8 / 8 + 8 * std::max(2, D / 32);  // widest V row plus (scale, zero)
+  int lcap = 256;
+  if ((long long)L.cpc_max * kChunk >= (1ll << fused::kCandRowBits) || L.cpc_max >= 2048) lcap = 0;
+  const int sparse = fused::kWarps * lcap * (1 + L.H) * 4 + 128 * slot + red;
+  const int scan_fb = fused::kWarps * fused::kListCap * 4 * (1 + L.H) + red;
+  const int dense = fused::kDenseStaging + red;
+  const int phase2 = std::max(sparse, std::max(scan_fb, dense));
+  L.stages = std::min(fused::kMaxStages, (kMaxSmem - fused::kHeader) / sb);
+  L.ring_bytes = (std::max(L.stages * sb, phase2) + 127) / 128 * 128;
+  L.cand_cap = lcap;
   L.smem_bytes = fused::kHeader + L.ring_bytes;
-  const int tpc = fused::kChunk / g.tile_rows;
+  const int tpc = fused::kTilesPerChunk;
   L.need_gstats = (long long)L.cpc_max * tpc > fused::kTsCap;
   size_t off = kHeaderBytes;
   L.arrive1 = off; off = align_up(off + units * 4);
@@ -97,8 +110,8 @@ FusedLayout fused_layout(int B, int Hq, int Hkv, int T_cap, int D, int KB) {
   L.glogits = off; off = align_up(off + (size_t)L.grid * L.cpc_max * kChunk * L.H * 4);
   L.gstats = off;
   if (L.need_gstats) off = align_up(off + (size_t)L.grid * L.cpc_max * 8 * 12 * 4);
-  L.qbuf = off; off = align_up(off + (size_t)units * L.H * D * 4);
-  L.qgsum = off; off = align_up(off + (size_t)units * L.H * 4 * 4);
+  L.qbuf = off; off = align_up(off + (size_t)units * L.H * D * 2);
+  L.qgsum = off; off = align_up(off + (size_t)units * L.H * 8 * 4);
   L.total = off;
   return L;
 }
@@ -132,6 +145,7 @@ int run_attention(DecodeArgs& a, int D, int kb, int vb0, int vb1, void* ws, size
   f.cpc_max = L.cpc_max;
   f.stages = L.stages;
   f.ring_bytes = L.ring_bytes;
+  f.cand_cap = L.cand_cap;
   f.smem_logit_floats = 0;
   f.timeout_ns = reinterpret_cast<const unsigned long long*>(base + 8);
   f.done = reinterpret_cast<int*>(base + 16);

@@ -3,103 +3,106 @@
 // up to four query heads.  The same kernel reads the attention-tiered cache
 // (§第二层) as two segments per (batch, KV head) with their own V widths.
 //
-// One persistent CTA per SM (cooperative launch, so all CTAs are resident).
-// Work = the list of chunks (kChunk consecutive tokens of one segment of one
-// (b, kv head) "unit"); every CTA takes an equal contiguous range of chunks.
-// A unit's rows are numbered segment 0 first, padded to whole chunks, then
-// segment 1, so a chunk never straddles the two segments.
+// One persistent CTA of sixteen warps per SM (cooperative launch, so all
+// CTAs are resident).  Work = the list of chunks (kChunk consecutive tokens
+// of one segment of one (b, kv head) "unit"); every CTA takes an equal
+// contiguous range of chunks.  A unit's rows are numbered segment 0 first,
+// padded to whole chunks, then segment 1, so a chunk never straddles the
+// two segments.
 //
-//  phase 1  a producer warp streams the K rows of the CTA's chunks, tile by
-//           tile, with 1-D bulk copies (TMA, evict-first in L2) into a
-//           two-deep ring of shared-memory stages per consumer warp.  A
-//           consumer lane computes whole rows (two per tile), so the 512
-//           multiply-adds of a row need no cross-lane reduction; q is read
-//           as warp-uniform broadcasts.  Each tile's per-head maximum and sum
-//           of exp2 are reduced in the warp, and e = exp2(s - max_tile) is
-//           written to an L2-resident workspace.
+//  phase 1  a producer warp streams the CTA's 64-row K tiles in order into a
+//           ring of shared-memory stages with 1-D bulk copies (evict-first
+//           in L2); fifteen consumer warps take the tiles round robin and
+//           compute their logits on the tensor cores (mma_k.cuh): codes
+//           become exact fp16 integers, q the head's exact fp16 value times
+//           a power of two, and the (scale, zero) of each group is folded
+//           after the MMA.  Each tile's per-head maximum and sum of exp2 are
+//           reduced in the warp; e = exp2(s - max_tile) is written to an
+//           L2-resident workspace.
 //  stats    per unit piece: the merged tile statistics.  A unit owned by one
 //           CTA needs nothing else; a unit shared by neighbouring CTAs
 //           exchanges piece statistics through the workspace (bounded wait
-//           on a per-unit arrival counter).
-//  phase 2  p = e * exp2(max_tile - max) / sum.  A (b, h, t) with p < tau is
-//           skipped; the V rows some head keeps are listed per warp in row
-//           order, gathered from HBM and accumulated as p * vhat.  Shared
-//           units publish partial outputs; the last CTA to arrive adds them.
-//
-// Dequantization is folded into the dot products: codes become exact
-// integers (unpack) and, with the group's (scale, zero),
-//   sum_d q_d * (scale * c_d + zero) = scale * sum_d q_d c_d + zero * sum_d q_d.
+//           on a per-unit arrival counter).  Every tile then gets its factor
+//           exp2(max_tile - max) / sum.
+//  phase 2  p = e * factor; (b, h, t) with p < tau is skipped.  Sparse mode
+//           (tau > 0): one pass over the CTA's rows takes every decision,
+//           writes the optional skip mask and attention mass, and lists the
+//           rows some head keeps with their weights; their V rows are
+//           brought into shared memory with 16-byte asynchronous copies and
+//           accumulated piece by piece.  Dense mode (tau <= 0): every V row
+//           is streamed.  (Lists that overflow shared memory fall back to a
+//           per-piece scan and gather.)  Shared units publish partial
+//           outputs; the last CTA to arrive adds them.
 #pragma once
 #include <type_traits>
 #include <cfloat>
 
 #include "lkv_kernels.cuh"
+#include "mma_k.cuh"
 
 namespace lkv {
 namespace fused {
 
 constexpr int kChunk = 256;    // tokens per chunk (work-partition granularity)
 static_assert(kChunk == kPageTokens, "a chunk of a paged cache is one page");
-constexpr int kSlotsPerWarp = 2;
-constexpr int kMaxConsumerWarps = 12;
-constexpr int kListCap = 512;  // V-row list entries per warp per batch
+constexpr int kTileRows = 64;  // rows of a K tile: four 16-row MMA tiles
+constexpr int kTilesPerChunk = kChunk / kTileRows;
+constexpr int kWarps = 16;
+constexpr int kThreads = kWarps * 32;
+constexpr int kConsumers = 15;   // warps 0..14 compute, warp 15 streams
+constexpr int kProducer = 15;
+constexpr int kMaxStages = 24;   // ring stages, one chunk each
+constexpr int kListCap = 256;  // fallback scan: V-row list entries per warp per batch
 constexpr int kBatchBlocks = kListCap / 32;
 constexpr int kRec = 16;       // ints per unit-list record
 constexpr int kGatherUnroll = 4;
 constexpr int kScanBlocks = 4;  // 32-row blocks whose logits one warp loads at once
 constexpr int kTsCap = 128;    // tile statistics kept in shared memory up to this many tiles
-constexpr int kQSlots = 4;     // units whose prescaled q is staged in shared memory
+constexpr int kQSlots = 4;     // units whose q is staged in shared memory
+constexpr int kCandRowBits = 20;  // kept-row entry: CTA-local row | unit entry << 20
+constexpr int kScanTiles = 4;      // tiles whose e-values one warp loads at once in the sparse scan
 // Dense V pass (tau <= 0): per warp two buffers of one 32-row block each:
 // V codes (up to 6 bits), (scale, zero) of 34 rows and the block's logits.
 constexpr int kDenseCodes = 32 * 96;
 constexpr int kDenseSz = 34 * 4 * 8;
 constexpr int kDenseLogits = 32 * 4 * 4;
 constexpr int kDenseBuf = (kDenseCodes + kDenseSz + kDenseLogits + 127) / 128 * 128;
-constexpr int kDenseStaging = kMaxConsumerWarps * 2 * kDenseBuf;
-constexpr int kDenseBar = 32;  // first mbarrier of the dense buffers
+constexpr int kDenseStaging = kWarps * 2 * kDenseBuf;
 constexpr unsigned kFull = 0xFFFFFFFFu;
-constexpr int kBarCons = 1;    // named barrier of the consumer warps
-// Shared header (bytes): barriers [0, 512), per-group q sums of up to
-// kQSlots units [512, 1536), misc ints [1536, 2048), tile statistics [2048, 8192), q of up to kQSlots
-// units [8192, 16384).
-constexpr int kQgOff = 512;
+// Shared header (bytes): mbarriers [0, 1024) (full and empty per stage, two
+// per warp for the dense pass), per q slot and head A and Z[4] [1024, 1536),
+// misc ints [1536, 2560), tile statistics [2560, 8704), fp16 q of up to
+// kQSlots units [8704, 12800), unit list [12800, 16896), stage descriptors
+// [16896, 17664).
+constexpr int kBarOff = 0;
+constexpr int kAzOff = 1024;
 constexpr int kMiscOff = 1536;
-constexpr int kTsOff = 2048;
-constexpr int kQOff = 8192;
-constexpr int kHeader = 16384;
+constexpr int kTsOff = 2560;
+constexpr int kQOff = 8704;
+constexpr int kUlOff = 12800;
+constexpr int kUlCap = 64;
+constexpr int kDescOff = 16896;
+constexpr int kHeader = 17664;
+static_assert(2 * kMaxStages + 2 * kWarps <= 128, "barriers fit their 1024 bytes");
+static_assert(kDescOff + kMaxStages * 32 <= kHeader, "stage descriptors fit");
+static_assert(kHeader % 128 == 0, "the ring starts 128-byte aligned");
 
 // Compile-time geometry of one instantiation.
 template <int D, int KB>
 struct Geo {
-  static constexpr int RB = D * KB / 8;                       // packed K row bytes
-  static constexpr int RW = RB / 4;                           // ... in 32-bit words
-  static constexpr int RPL = RW <= 24 ? 2 : 1;                // rows per lane in a tile
-  static constexpr int kTileRows = 32 * RPL;
-  static constexpr int kTilesPerChunk = kChunk / kTileRows;
-  static constexpr int kCW = RPL == 2 ? 12 : 8;               // consumer warps
-  static constexpr int kConsumers = kCW * 32;
-  static constexpr int kThreads = kConsumers;                 // every warp streams its own tiles
-  static constexpr int kStages = kCW * kSlotsPerWarp;
-  static constexpr int kStageCodes = kTileRows * RB;
-  static constexpr int kStageSz = (kTileRows + 2) * (D / 32) * 8;  // ng <= D/32, plus alignment rows
+  static constexpr int RB = D * KB / 8;            // packed K row bytes
+  static constexpr int SW = D * KB / 128;          // words of a lane's slice (D/4 codes)
+  static constexpr int SWB = SW * 4;
+  static constexpr int KS = D / 16;                // MMA k-steps per row
+  static constexpr int kStageCodes = kChunk * RB;             // a stage holds one chunk
+  static constexpr int kStageSz = (kChunk + 2) * (D / 32) * 8;  // ng <= D/32, plus alignment rows
   static constexpr int kStageBytes = (kStageCodes + kStageSz + 127) / 128 * 128;
-  static constexpr int kDimsPerWord = 32 / KB;                // not used for 6-bit
 };
 
 // Host-side view of the geometry (the same formulas as Geo).
-struct GeoHost {
-  int threads, stages, stage_bytes, tile_rows, consumer_warps;
-};
-inline GeoHost geo_host(int D, int KB) {
-  const int rb = D * KB / 8, rw = rb / 4;
-  const int rpl = rw <= 24 ? 2 : 1;
-  GeoHost g;
-  g.tile_rows = 32 * rpl;
-  g.consumer_warps = rpl == 2 ? 12 : 8;
-  g.threads = g.consumer_warps * 32;
-  g.stages = g.consumer_warps * kSlotsPerWarp;
-  g.stage_bytes = (g.tile_rows * rb + (g.tile_rows + 2) * (D / 32) * 8 + 127) / 128 * 128;
-  return g;
+inline int stage_bytes_host(int D, int KB) {
+  const int rb = D * KB / 8;
+  return (kChunk * rb + (kChunk + 2) * (D / 32) * 8 + 127) / 128 * 128;
 }
 
 // Unit-list record (ints): u, first chunk, chunks, n0, n1, owned, chunks of
@@ -178,16 +181,18 @@ __device__ __forceinline__ bool wait_counter(const int* p, int target, uint64_t 
   }
 }
 
-template <int H>
-__device__ __forceinline__ void load_heads(const float* p, float (&x)[H]) {
-  if constexpr (H == 4) {
-    const float4 v = *reinterpret_cast<const float4*>(p);
-    x[0] = v.x; x[1] = v.y; x[2] = v.z; x[3] = v.w;
-  } else if constexpr (H == 2) {
-    const float2 v = *reinterpret_cast<const float2*>(p);
-    x[0] = v.x; x[1] = v.y;
-  } else {
-    x[0] = p[0];
+// Bounded wait until the producer has issued `target` chunks (or the CTA
+// aborted); false after a timeout.
+__device__ __forceinline__ bool wait_issued(const int* issued, int target, const volatile int* abort_flag,
+                                            uint64_t limit_ns) {
+  const volatile int* p = issued;
+  if (*p >= target) { __threadfence_block(); return true; }
+  const uint64_t t0 = global_ns();
+  while (true) {
+    __nanosleep(32);
+    if (*p >= target) { __threadfence_block(); return true; }
+    if (*abort_flag) return false;
+    if (global_ns() - t0 > limit_ns) return false;
   }
 }
 
@@ -228,43 +233,35 @@ __device__ __forceinline__ void store_heads(float* p, const float (&x)[H]) {
   }
 }
 
-// Exponent fields of the unpack's magic floats, kept in registers so that a
-// code costs a single AND-OR (an immediate mask plus this register).
-template <int BITS>
-struct Magic {
-  uint32_t m[24];
-  __device__ __forceinline__ void load(const int* src) {
-#pragma unroll
-    for (int k = 0; k < 24 - BITS; ++k) m[k] = (uint32_t)src[k];
-  }
-};
-
-// Code I of a 16-code lane slice, plus its magic constant 2^(23-kk).
+// Code I of a 16-code lane slice, plus its magic constant 2^(23-kk): the
+// code sits at bit kk of a (shifted) word and the exponent field 150 - kk
+// makes the float 2^(23-kk) + code exactly.
 template <int BITS, int I>
-__device__ __forceinline__ float code_plus_magic_r(const LaneWords<BITS>& lw, const Magic<BITS>& mg) {
+__device__ __forceinline__ float code_plus_magic_r(const LaneWords<BITS>& lw) {
   constexpr int s = copy_shift<BITS>(I);
   constexpr int kk = I * BITS - s;
   constexpr uint32_t mask = ((1u << BITS) - 1u) << kk;
-  return __uint_as_float((stream_bits<BITS>(lw, s) & mask) | mg.m[kk]);
+  constexpr uint32_t magic = (uint32_t)(150 - kk) << 23;
+  return __uint_as_float((stream_bits<BITS>(lw, s) & mask) | magic);
 }
 
 // Codes (2P, 2P+1) of the slice as exact floats.
 template <int BITS, int P>
-__device__ __forceinline__ float2 code_pair_r(const LaneWords<BITS>& lw, const Magic<BITS>& mg) {
-  const float2 m = make_float2(code_plus_magic_r<BITS, 2 * P>(lw, mg), code_plus_magic_r<BITS, 2 * P + 1>(lw, mg));
+__device__ __forceinline__ float2 code_pair_r(const LaneWords<BITS>& lw) {
+  const float2 m = make_float2(code_plus_magic_r<BITS, 2 * P>(lw), code_plus_magic_r<BITS, 2 * P + 1>(lw));
   return __fadd2_rn(m, make_float2(-magic_value<BITS, 2 * P>(), -magic_value<BITS, 2 * P + 1>()));
 }
 
 template <int BITS>
-__device__ __forceinline__ void unpack16_int_r(const LaneWords<BITS>& lw, const Magic<BITS>& mg, float2 (&c)[8]) {
-  c[0] = code_pair_r<BITS, 0>(lw, mg);
-  c[1] = code_pair_r<BITS, 1>(lw, mg);
-  c[2] = code_pair_r<BITS, 2>(lw, mg);
-  c[3] = code_pair_r<BITS, 3>(lw, mg);
-  c[4] = code_pair_r<BITS, 4>(lw, mg);
-  c[5] = code_pair_r<BITS, 5>(lw, mg);
-  c[6] = code_pair_r<BITS, 6>(lw, mg);
-  c[7] = code_pair_r<BITS, 7>(lw, mg);
+__device__ __forceinline__ void unpack16_int_r(const LaneWords<BITS>& lw, float2 (&c)[8]) {
+  c[0] = code_pair_r<BITS, 0>(lw);
+  c[1] = code_pair_r<BITS, 1>(lw);
+  c[2] = code_pair_r<BITS, 2>(lw);
+  c[3] = code_pair_r<BITS, 3>(lw);
+  c[4] = code_pair_r<BITS, 4>(lw);
+  c[5] = code_pair_r<BITS, 5>(lw);
+  c[6] = code_pair_r<BITS, 6>(lw);
+  c[7] = code_pair_r<BITS, 7>(lw);
 }
 
 // Global V-row load for the gather (lane's codes + its group's (scale, zero)).
@@ -276,10 +273,10 @@ __device__ __forceinline__ void ldg_v(const uint8_t* codes_row, const float* sz_
 }
 
 template <int H, int VB>
-__device__ __forceinline__ void accumulate_v(const LaneWords<VB>& lw, const Magic<VB>& mg, float2 sz,
-                                             const float (&w)[H], float2 (&acc)[H][8], float (&Z)[H]) {
+__device__ __forceinline__ void accumulate_v(const LaneWords<VB>& lw, float2 sz, const float (&w)[H],
+                                             float2 (&acc)[H][8], float (&Z)[H]) {
   float2 c[8];
-  unpack16_int_r<VB>(lw, mg, c);
+  unpack16_int_r<VB>(lw, c);
 #pragma unroll
   for (int h = 0; h < H; ++h) {
     const float ws = w[h] * sz.x;
@@ -294,42 +291,117 @@ struct TileDesc {
   int slot, seg, row0, rows, entry, u;
 };
 
-// Pair P (0..7) of a 16-code slice; P is a constant once loops are unrolled.
-template <int BITS>
-__device__ __forceinline__ float2 code_pair_at(const LaneWords<BITS>& lw, const Magic<BITS>& mg, int P) {
-  switch (P) {
-    case 0: return code_pair_r<BITS, 0>(lw, mg);
-    case 1: return code_pair_r<BITS, 1>(lw, mg);
-    case 2: return code_pair_r<BITS, 2>(lw, mg);
-    case 3: return code_pair_r<BITS, 3>(lw, mg);
-    case 4: return code_pair_r<BITS, 4>(lw, mg);
-    case 5: return code_pair_r<BITS, 5>(lw, mg);
-    case 6: return code_pair_r<BITS, 6>(lw, mg);
-    default: return code_pair_r<BITS, 7>(lw, mg);
+// Lane slice words of row `r` of a staged tile (D/4 codes at tig * SWB).
+template <int D, int KB>
+__device__ __forceinline__ void lds_slice(const uint8_t* codes, int r, int tig, int gid,
+                                          uint32_t (&w)[Geo<D, KB>::SW]) {
+  using G = Geo<D, KB>;
+  const uint8_t* p = codes + r * G::RB + tig * G::SWB;
+  if constexpr (G::SWB % 16 == 0) {
+#pragma unroll
+    for (int q = 0; q < G::SW / 4; ++q) {
+      // stagger the two 16-byte halves of 32-byte slices over odd rows (bank spread)
+      const int qq = (G::SW / 4 == 2) ? (q ^ (gid & 1)) : q;
+      const uint4 v = *reinterpret_cast<const uint4*>(p + 16 * qq);
+      w[4 * qq] = v.x; w[4 * qq + 1] = v.y; w[4 * qq + 2] = v.z; w[4 * qq + 3] = v.w;
+    }
+  } else if constexpr (G::SWB % 8 == 0) {
+#pragma unroll
+    for (int q = 0; q < G::SW / 2; ++q) {
+      const uint2 v = *reinterpret_cast<const uint2*>(p + 8 * q);
+      w[2 * q] = v.x; w[2 * q + 1] = v.y;
+    }
+  } else {
+#pragma unroll
+    for (int q = 0; q < G::SW; ++q) w[q] = reinterpret_cast<const uint32_t*>(p)[q];
+  }
+}
+
+// Two 16-row MMA tiles (rows 16 mt + {gid, gid + 8} for mt = MT0, MT0 + 1)
+// of a staged 64-row K tile: acc[m][nt] = C fragment of tile MT0 + m and
+// n-tile nt.  The k-steps are the outer loop so that consecutive MMAs belong
+// to different row tiles and do not wait on one another.
+template <int D, int KB, int NT, int MT0>
+__device__ __forceinline__ void mma_pair(const uint8_t* codes, int tig, int gid, const uint32_t (&bf)[2][D / 8],
+                                         float (&acc)[2][2][4]) {
+  using G = Geo<D, KB>;
+  uint32_t w[2][2][G::SW];
+#pragma unroll
+  for (int m = 0; m < 2; ++m)
+#pragma unroll
+    for (int hf = 0; hf < 2; ++hf) lds_slice<D, KB>(codes, 16 * (MT0 + m) + gid + 8 * hf, tig, gid, w[m][hf]);
+#pragma unroll
+  for (int m = 0; m < 2; ++m)
+#pragma unroll
+    for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+      for (int i = 0; i < 4; ++i) acc[m][nt][i] = 0.0f;
+  auto step = [&](auto sc) {
+    constexpr int s = decltype(sc)::value;
+#pragma unroll
+    for (int m = 0; m < 2; ++m) {
+      const uint32_t a0 = a_reg<KB, 2 * s>(w[m][0]), a1 = a_reg<KB, 2 * s>(w[m][1]);
+      const uint32_t a2 = a_reg<KB, 2 * s + 1>(w[m][0]), a3 = a_reg<KB, 2 * s + 1>(w[m][1]);
+      hmma16816(acc[m][0], a0, a1, a2, a3, bf[0][2 * s], bf[0][2 * s + 1]);
+      if constexpr (NT == 2) hmma16816(acc[m][1], a0, a1, a2, a3, bf[1][2 * s], bf[1][2 * s + 1]);
+    }
+  };
+  step(std::integral_constant<int, 0>{});
+  step(std::integral_constant<int, 1>{});
+  step(std::integral_constant<int, 2>{});
+  step(std::integral_constant<int, 3>{});
+  if constexpr (D == 128) {
+    step(std::integral_constant<int, 4>{});
+    step(std::integral_constant<int, 5>{});
+    step(std::integral_constant<int, 6>{});
+    step(std::integral_constant<int, 7>{});
+  }
+}
+
+// B fragments of the unit for this lane (see mma_k.cuh): column n = 8 nt +
+// gid is (head n / ng, group n % ng); q16 holds the unit's scaled fp16 q
+// [H][D].
+template <int D, int KB, int H>
+__device__ __forceinline__ void build_bfrags(const __half* q16, int ng, int G, int tig, int gid,
+                                             uint32_t (&bf)[2][D / 8]) {
+  const int lane_group = (tig * (D / 4)) / G;
+#pragma unroll
+  for (int nt = 0; nt < 2; ++nt) {
+    const int n = 8 * nt + gid;
+    const int h = n / ng, g = n - h * ng;
+    const bool on = h < H && g == lane_group;
+    const __half* qh = q16 + (on ? h : 0) * D;
+    bfrag_one<KB, D, 0>(qh, tig * (D / 4), on, bf[nt]);
   }
 }
 
 // ------------------------------------------------------------------ kernel
 
 template <int D, int H, int KB, int VB0, int VB1, bool PAGED>
-__global__ void __launch_bounds__(Geo<D, KB>::kThreads, 1) fused_decode_kernel(FusedArgs a) {
+__global__ void __launch_bounds__(kThreads, 1) fused_decode_kernel(FusedArgs a) {
   using Gk = Geo<D, KB>;
-  constexpr int CW = Gk::kCW, NCONS = Gk::kConsumers, NTHR = Gk::kThreads;
-  constexpr int RPL = Gk::RPL, TR = Gk::kTileRows, TPC = Gk::kTilesPerChunk;
+  constexpr int CW = kWarps, NTHR = kThreads;
+  constexpr int TR = kTileRows, TPC = kTilesPerChunk;
   constexpr int LPR = D / kDimsPerLane, RPW = 32 / LPR;  // phase-2 lane mapping (16 channels per lane)
-  constexpr int NW = KB / 2;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int gid = lane >> 2, tig = lane & 3;
   const int cta = blockIdx.x, grid = gridDim.x;
   const DecodeArgs& d = a.d;
   const int units = d.B * d.Hkv;
   const int ng = D / d.G;
+  const int NT = (H * ng > 8) ? 2 : 1;
+  const int S = a.stages;
   const uint64_t limit_ns = (a.timeout_ns && *a.timeout_ns) ? *a.timeout_ns : 2000000000ull;
   const int j = lane % LPR;                 // phase 2: lane's 16-channel slice of a row
   const int gi = (j * kDimsPerLane) / d.G;  // its quantization group
 
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem_raw);
-  int* misc = reinterpret_cast<int*>(smem_raw + kMiscOff);  // 128 ints
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem_raw + kBarOff);
+  uint64_t* full = bars;                    // [kMaxStages] stage holds its tile
+  uint64_t* empty = bars + kMaxStages;      // [kMaxStages] stage read by its consumer
+  uint64_t* dbar = bars + 2 * kMaxStages;   // [2 * kWarps] dense V buffers
+  int* misc = reinterpret_cast<int*>(smem_raw + kMiscOff);  // 256 ints
+  int* desc = reinterpret_cast<int*>(smem_raw + kDescOff);  // [kMaxStages][8] tile descriptors
   uint8_t* ring = smem_raw + kHeader;
 
   int& s_total = misc[0];
@@ -339,25 +411,26 @@ __global__ void __launch_bounds__(Geo<D, KB>::kThreads, 1) fused_decode_kernel(F
   int& s_carry_c = misc[4];
   int& s_carry_n = misc[5];
   int& s_last = misc[6];
-  float* s_glob = reinterpret_cast<float*>(misc + 8);  // (max, 1/sum) x 4 heads
-  int* s_wsum = misc + 16;                            // 2 x 12 warp partials
-  int* s_magic = misc + 48;                           // 24 magic exponent fields
-  int* s_nw = misc + 96;                              // kept rows per warp in a phase-2 batch
+  int& s_ovf = misc[7];
+  int& s_issued = misc[8];                            // chunks the producer has issued
+  int* s_wsum = misc + 16;                            // 2 x 16 warp partials
+  int* s_coff = misc + 72;                            // sparse mode: staging offset per warp
+  int* s_nw = misc + 88;                              // sparse mode: list length per warp
+  int* s_cs = misc + 104;                             // sparse mode: per warp (start, count) in a piece
 
   if (tid == 0) {
-    for (int s = 0; s < Gk::kStages; ++s) mbar_init(&full[s], 1);
-    for (int s = 0; s < 2 * kMaxConsumerWarps; ++s) mbar_init(&full[kDenseBar + s], 1);
+    for (int s = 0; s < kMaxStages; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], kTilesPerChunk); }
+    for (int s = 0; s < 2 * kWarps; ++s) mbar_init(&dbar[s], 1);
     fence_mbar_init();
-    s_total = 0; s_e0 = 0; s_nent = 0; s_abort = 0; s_carry_c = 0; s_carry_n = 0; s_last = 0;
+    s_total = 0; s_e0 = 0; s_nent = 0; s_abort = 0; s_carry_c = 0; s_carry_n = 0; s_last = 0; s_ovf = 0;
+    s_issued = 0;
   }
-  if (tid < 24) s_magic[tid] = (150 - tid) << 23;
   __syncthreads();
 
   // ------------------------------------------------------------ unit list
-  const bool consumer = warp < CW;
-  if (consumer) {
+  {
     int part = 0;
-    for (int u = tid; u < units; u += NCONS) {
+    for (int u = tid; u < units; u += NTHR) {
       int n0, n1;
       unit_lens(d, u, n0, n1);
       part += chunks_of(n0) + chunks_of(n1);
@@ -370,7 +443,7 @@ __global__ void __launch_bounds__(Geo<D, KB>::kThreads, 1) fused_decode_kernel(F
     for (int off = 16; off >= 1; off >>= 1) part += __shfl_xor_sync(kFull, part, off);
     if (lane == 0) atomicAdd(&s_total, part);
     if (cta == 0) {  // length checks, spread over the CTA's threads (a serial loop here delays CTA 0)
-      for (int u = tid; u < (d.len_mode == 0 ? d.B : units); u += NCONS) {
+      for (int u = tid; u < (d.len_mode == 0 ? d.B : units); u += NTHR) {
         bool bad;
         if (d.len_mode == 0) {
           bad = d.lens[u] < 0 || d.lens[u] > d.T_cap;
@@ -388,44 +461,48 @@ __global__ void __launch_bounds__(Geo<D, KB>::kThreads, 1) fused_decode_kernel(F
   const int k0 = min(cta * cpc, total), k1 = min(k0 + cpc, total);
   const int nck = k1 - k0;
   const int ntile = nck * TPC;
-  int* ulist = a.ulist + (long long)cta * a.cpc_max * kRec;
-  if (consumer) {
-    for (int base = 0; base < units; base += NCONS) {
-      const int u = base + tid;
-      int n0 = 0, n1 = 0;
-      if (u < units) unit_lens(d, u, n0, n1);
-      const int nc0 = chunks_of(n0);
-      const int nc = nc0 + chunks_of(n1);
-      const int ne = nc > 0 ? 1 : 0;
-      int sc = nc, sn = ne;  // warp inclusive scans
+  int* ulist_g = a.ulist + (long long)cta * a.cpc_max * kRec;
+  int* ulist_s = reinterpret_cast<int*>(smem_raw + kUlOff);
+  for (int base = 0; base < units; base += NTHR) {
+    const int u = base + tid;
+    int n0 = 0, n1 = 0;
+    if (u < units) unit_lens(d, u, n0, n1);
+    const int nc0 = chunks_of(n0);
+    const int nc = nc0 + chunks_of(n1);
+    const int ne = nc > 0 ? 1 : 0;
+    int sc = nc, sn = ne;  // warp inclusive scans
 #pragma unroll
-      for (int off = 1; off < 32; off <<= 1) {
-        const int y = __shfl_up_sync(kFull, sc, off), z = __shfl_up_sync(kFull, sn, off);
-        if (lane >= off) { sc += y; sn += z; }
-      }
-      if (lane == 31) { s_wsum[warp] = sc; s_wsum[16 + warp] = sn; }
-      named_barrier(kBarCons, NCONS);
-      int wc = 0, wn = 0, tc = 0, tn = 0;
-      for (int w = 0; w < CW; ++w) {
-        if (w < warp) { wc += s_wsum[w]; wn += s_wsum[16 + w]; }
-        tc += s_wsum[w]; tn += s_wsum[16 + w];
-      }
-      const int cb = s_carry_c + wc + sc - nc;
-      const int ne_idx = s_carry_n + wn + sn - ne;
-      if (ne && cb <= k0 && k0 < cb + nc) s_e0 = ne_idx;
-      named_barrier(kBarCons, NCONS);
-      if (ne && cb < k1 && cb + nc > k0) {
-        const int idx = ne_idx - s_e0;
-        int* rec = ulist + (long long)idx * kRec;
+    for (int off = 1; off < 32; off <<= 1) {
+      const int y = __shfl_up_sync(kFull, sc, off), z = __shfl_up_sync(kFull, sn, off);
+      if (lane >= off) { sc += y; sn += z; }
+    }
+    if (lane == 31) { s_wsum[warp] = sc; s_wsum[16 + warp] = sn; }
+    __syncthreads();
+    int wc = 0, wn = 0, tc = 0, tn = 0;
+    for (int w = 0; w < CW; ++w) {
+      if (w < warp) { wc += s_wsum[w]; wn += s_wsum[16 + w]; }
+      tc += s_wsum[w]; tn += s_wsum[16 + w];
+    }
+    const int cb = s_carry_c + wc + sc - nc;
+    const int ne_idx = s_carry_n + wn + sn - ne;
+    if (ne && cb <= k0 && k0 < cb + nc) s_e0 = ne_idx;
+    __syncthreads();
+    if (ne && cb < k1 && cb + nc > k0) {
+      const int idx = ne_idx - s_e0;
+      // the list lives in shared memory when it fits, else in the workspace
+      int* recs[2] = {ulist_g + (long long)idx * kRec, idx < kUlCap ? ulist_s + idx * kRec : nullptr};
+      for (int c = 0; c < 2; ++c) {
+        int* rec = recs[c];
+        if (rec == nullptr) continue;
         rec[0] = u; rec[1] = cb; rec[2] = nc; rec[3] = n0; rec[4] = n1;
         rec[5] = (cb >= k0 && cb + nc <= k1) ? 1 : 0;
         rec[6] = nc0;
-        atomicMax(&s_nent, idx + 1);
       }
-      named_barrier(kBarCons, NCONS);
-      if (tid == 0) { s_carry_c += tc; s_carry_n += tn; }
-      named_barrier(kBarCons, NCONS);
+      atomicMax(&s_nent, idx + 1);
     }
+    __syncthreads();
+    if (tid == 0) { s_carry_c += tc; s_carry_n += tn; }
+    __syncthreads();
   }
   // tile statistics (max, sum, factor per head): shared memory unless many tiles
   float* tsm;
@@ -443,251 +520,249 @@ __global__ void __launch_bounds__(Geo<D, KB>::kThreads, 1) fused_decode_kernel(F
   for (int i = tid; i < ntile * H; i += NTHR) { tsm[i] = -INFINITY; tsl[i] = 0.0f; }
   __syncthreads();  // list complete
   const int nent = s_nent;
-  // prescaled q of the CTA's units and its per-group sums (one warp per (unit, head))
-  if (consumer) {
+  int* const ulist = nent <= kUlCap ? ulist_s : ulist_g;
+  // q of the CTA's units (one warp per (unit, head)): scaled by 2^E so that
+  // its largest magnitude lies in [2^14, 2^15), stored as fp16 (exact for
+  // the bf16 inputs), with A = q_scale * 2^-E and Z[g] = q_scale * sum of
+  // the group's q for the fold after the MMA.
+  {
     constexpr int DPL = D / 32;  // channels per lane
     for (int task = warp; task < nent * H; task += CW) {
       const int e = task / H, h = task % H;
-      const Unit x = load_unit(ulist + (long long)e * kRec);
+      const Unit x = load_unit(ulist + e * kRec);
       const int b = x.u / d.Hkv, g = x.u % d.Hkv;
       const uint16_t* qs = d.q + ((long long)b * d.Hq + g * H + h) * D + lane * DPL;
-      float* qd = (e < kQSlots ? reinterpret_cast<float*>(smem_raw + kQOff) + e * H * D
-                               : a.qbuf + (long long)x.u * H * D) + h * D + lane * DPL;
-      float s = 0.0f;
+      float v[DPL];
+      float amax = 0.0f, s = 0.0f;
 #pragma unroll
       for (int i = 0; i < DPL; ++i) {
-        const float v = __uint_as_float(((uint32_t)qs[i]) << 16) * d.q_scale;
-        qd[i] = v;
-        s += v;
+        v[i] = __uint_as_float(((uint32_t)qs[i]) << 16);
+        amax = fmaxf(amax, fabsf(v[i]));
+        s += v[i];
       }
+#pragma unroll
+      for (int off = 16; off >= 1; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(kFull, amax, off));
+      int ex = 0;
+      const bool fin = amax > 0.0f && amax <= FLT_MAX;
+      if (fin) frexpf(amax, &ex);
+      const int E = fin ? 15 - ex : 0;
+      __half* qd = (e < kQSlots ? reinterpret_cast<__half*>(smem_raw + kQOff) + e * H * D
+                                : reinterpret_cast<__half*>(a.qbuf) + (long long)x.u * H * D) +
+                   h * D + lane * DPL;
+#pragma unroll
+      for (int i = 0; i < DPL; ++i) qd[i] = __float2half_rn(ldexpf(v[i], E));
       const int lpg = d.G / DPL;  // lanes per quantization group
       for (int off = 1; off < lpg; off <<= 1) s += __shfl_xor_sync(kFull, s, off);
-      if (lane % lpg == 0) {
-        a.qgsum[((long long)x.u * H + h) * 4 + lane / lpg] = s;
-        if (e < kQSlots) reinterpret_cast<float*>(smem_raw + kQgOff)[(e * H + h) * 4 + lane / lpg] = s;
-      }
+      float* az = e < kQSlots ? reinterpret_cast<float*>(smem_raw + kAzOff) + (e * H + h) * 8
+                              : a.qgsum + ((long long)x.u * H + h) * 8;
+      if (lane % lpg == 0) az[lane / lpg] = d.q_scale * s;
+      if (lane == 0) az[4] = ldexpf(d.q_scale, -E);
     }
   }
   __syncthreads();  // q ready; phase 1 starts
 
-  float* lg = a.glogits + (long long)cta * a.cpc_max * kChunk * H;  // [slot][H], slot = kk * kChunk + row
+  float* lg = a.glogits + (long long)cta * a.cpc_max * kChunk * H;  // [tile * TR + row][H]
 
   // ------------------------------------------------------------ phase 1
-  // Warp w takes tiles w, w + CW, ... of the CTA (tile t = chunk t / TPC,
-  // rows (t % TPC) * TR ...) and keeps two of them in flight in its own two
-  // ring stages, issuing each bulk copy itself.
-  {
-    Magic<KB> mg;
-    mg.load(s_magic);
-    const uint64_t pol = policy_evict_first();
-    volatile int* abort_flag = &s_abort;
-    int nt = warp, ent = 0;
-    // next non-empty tile of this warp, or false
-    auto next_tile = [&](TileDesc& td) -> bool {
-      while (nt < ntile) {
-        const int t = nt;
-        nt += CW;
-        const int g = k0 + t / TPC, sub = t % TPC;
-        while (ent + 1 < nent && ulist[(long long)(ent + 1) * kRec + 1] <= g) ++ent;
-        const Unit x = load_unit(ulist + (long long)ent * kRec);
-        const ChunkRows cr = chunk_rows(x, g - x.cb);
-        const int rows = min(TR, cr.rows - sub * TR);
-        if (rows > 0) {
-          td.slot = t; td.seg = cr.seg; td.row0 = cr.row0 + sub * TR; td.rows = rows; td.entry = ent;
-          td.u = x.u;
-          return true;
+  // The producer warp streams the CTA's chunks in order into a ring of S
+  // stages (chunk c -> stage c % S) with two 1-D bulk copies each; consumer
+  // warp w takes tiles w, w + kConsumers, ... (tile t = quarter t % 4 of
+  // chunk t / 4).  "full" completes when a chunk has landed, "empty" when
+  // the consumers of its four tiles have read it.
+  volatile int* abort_flag = &s_abort;
+  if (warp == kProducer) {
+    if (lane == 0) {
+      const uint64_t pol = policy_evict_first();
+      int ent = 0, c = 0;
+      for (; c < nck; ++c) {
+        const int s = c % S, k = c / S;
+        if (k > 0 && !mbar_wait(&empty[s], (k - 1) & 1, limit_ns)) {
+          atomicExch(d.status, kStatusTimeout);
+          *abort_flag = 1;
+          break;
         }
+        if (*abort_flag) break;
+        const int g = k0 + c;
+        while (ent + 1 < nent && ulist[(ent + 1) * kRec + 1] <= g) ++ent;
+        const Unit x = load_unit(ulist + ent * kRec);
+        const ChunkRows cr = chunk_rows(x, g - x.cb);
+        const int row = cr.row0, rows = max(0, cr.rows);
+        int* dd = desc + s * 8;
+        dd[0] = cr.seg; dd[1] = row; dd[2] = rows; dd[3] = ent; dd[4] = x.u;
+        if (rows > 0) {
+          const int r0 = (ng == 1) ? (row & ~1) : row;
+          const int r1 = (ng == 1) ? ((row + rows + 1) & ~1) : row + rows;
+          const uint32_t cbytes = (uint32_t)rows * Gk::RB;
+          const uint32_t sbytes = (uint32_t)(r1 - r0) * ng * 8;
+          uint8_t* dst = ring + (size_t)s * Gk::kStageBytes;
+          mbar_arrive_expect_tx(&full[s], cbytes + sbytes);
+          // a chunk is one page of a paged cache
+          const long long ubase = (long long)x.u * d.T_cap;
+          const long long pr = PAGED ? unit_row<PAGED>(a, x.u, row) : ubase + row;
+          const long long pr0 = PAGED ? unit_row<PAGED>(a, x.u, r0) : ubase + r0;
+          bulk_g2s(dst, d.kc[cr.seg] + pr * Gk::RB, cbytes, &full[s], pol);
+          bulk_g2s(dst + Gk::kStageCodes, d.ksz[cr.seg] + pr0 * ng * 2, sbytes, &full[s], pol);
+        } else {
+          mbar_arrive(&full[s]);
+        }
+        // chunk c's phase of full[s] is now the current one; a consumer that
+        // waited on the parity before this could match an older phase
+        __threadfence_block();
+        *static_cast<volatile int*>(&s_issued) = c + 1;
       }
-      return false;
-    };
-    auto issue = [&](const TileDesc& td, int stage) {
-      if (lane == 0) {
-        const long long ubase = (long long)td.u * d.T_cap;
-        const int row = td.row0, rows = td.rows;
-        const int r0 = (ng == 1) ? (row & ~1) : row;
-        const int r1 = (ng == 1) ? ((row + rows + 1) & ~1) : row + rows;
-        const uint32_t cbytes = (uint32_t)rows * Gk::RB;
-        const uint32_t sbytes = (uint32_t)(r1 - r0) * ng * 8;
-        uint8_t* dst = ring + (size_t)stage * Gk::kStageBytes;
-        mbar_arrive_expect_tx(&full[stage], cbytes + sbytes);
-        // a tile lies in one chunk, which is one page of a paged cache
-        const long long pr = PAGED ? unit_row<PAGED>(a, td.u, row) : ubase + row;
-        const long long pr0 = PAGED ? unit_row<PAGED>(a, td.u, r0) : ubase + r0;
-        bulk_g2s(dst, d.kc[td.seg] + pr * Gk::RB, cbytes, &full[stage], pol);
-        bulk_g2s(dst + Gk::kStageCodes, d.ksz[td.seg] + pr0 * ng * 2, sbytes, &full[stage], pol);
-      }
-    };
-    TileDesc p0, p1;
-    int issued = 0, consumed = 0;
-    if (next_tile(p0)) { issue(p0, warp * kSlotsPerWarp + 0); ++issued; }
-    if (issued == 1 && next_tile(p1)) { issue(p1, warp * kSlotsPerWarp + 1); ++issued; }
-    while (consumed < issued) {
-      const int slotw = consumed % kSlotsPerWarp;
-      const int stage = warp * kSlotsPerWarp + slotw;
+      // never leave copies in flight: the last use of every stage has landed
+      for (int s = 0; s < S && s < c; ++s) mbar_wait(&full[s], ((c - 1 - s) / S) & 1, limit_ns);
+    }
+  } else {
+    int bf_ent = -1;               // unit entry whose B fragments are loaded
+    uint32_t bf[2][D / 8];
+    float azA = 0.0f, azZ[2] = {0.0f, 0.0f};
+    float azA2[2] = {0.0f, 0.0f}, azZ2[2][2] = {{0.0f, 0.0f}, {0.0f, 0.0f}};
+    for (int t = warp; t < ntile; t += kConsumers) {
+      const int c = t / TPC, sub = t % TPC;
+      const int s = c % S, k = c / S;
       if (*abort_flag) break;
-      if (!mbar_wait(&full[stage], (consumed / kSlotsPerWarp) & 1, limit_ns)) {
-        atomicExch(d.status, kStatusTimeout);
-        atomicExch(&s_abort, 1);
+      if (!wait_issued(&s_issued, c + 1, abort_flag, limit_ns) || !mbar_wait(&full[s], k & 1, limit_ns)) {
+        if (!*abort_flag) atomicExch(d.status, kStatusTimeout);
+        *abort_flag = 1;
         break;
       }
-      const TileDesc td = slotw ? p1 : p0;
-      const uint8_t* codes = ring + (size_t)stage * Gk::kStageBytes;
-      const float* szs = reinterpret_cast<const float*>(codes + Gk::kStageCodes) +
-                         ((ng == 1) ? (td.row0 & 1) : 0) * ng * 2;
-      bool valid[RPL];
-      const uint4* src[RPL];
-#pragma unroll
-      for (int r = 0; r < RPL; ++r) {
-        const int i = lane + 32 * r;
-        valid[r] = i < td.rows;
-        src[r] = reinterpret_cast<const uint4*>(codes + (valid[r] ? i : 0) * Gk::RB);
+      const int* dd = desc + s * 8;
+      const int rows = max(0, min(TR, dd[2] - sub * TR));
+      if (rows == 0) {
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&empty[s]);
+        continue;
       }
-      float dot[RPL][H];
-      // The dot products of the tile's rows with the unit's prescaled q (qv)
-      // and its per-group sums (qg).  Called with shared-memory pointers for
-      // the CTA's first kQSlots units (shared loads) and with global ones
-      // otherwise.
-      // SPG (16-channel slices per quantization group) is G / 16 when known at
-      // compile time, so the group folds sit at fixed places in the unrolled
-      // loop, or 0 to read G at run time.
-      auto k_rows = [&](auto spg, const float* __restrict__ qv, const float* __restrict__ qg) {
-      constexpr int SPG = decltype(spg)::value;
-      float2 acc[RPL][H];
+      const int entry = dd[3];
+      if (entry != bf_ent) {
+        // B fragments and fold constants of the tile's unit
+        bf_ent = entry;
+        const int u = dd[4];
+        const __half* q16 = entry < kQSlots ? reinterpret_cast<const __half*>(smem_raw + kQOff) + entry * H * D
+                                            : reinterpret_cast<const __half*>(a.qbuf) + (long long)u * H * D;
+        const float* azb = entry < kQSlots ? reinterpret_cast<const float*>(smem_raw + kAzOff) + entry * H * 8
+                                           : a.qgsum + (long long)u * H * 8;
+        build_bfrags<D, KB, H>(q16, ng, d.G, tig, gid, bf);
+        // fold constants of the heads this lane's C columns belong to
+        if (ng == 2) {
+          const int h = tig < H ? tig : 0;
+          azA = tig < H ? azb[h * 8 + 4] : 0.0f;
+          azZ[0] = azb[h * 8 + 0]; azZ[1] = azb[h * 8 + 1];
+        } else if (ng == 1) {
 #pragma unroll
-      for (int r = 0; r < RPL; ++r)
-#pragma unroll
-        for (int h = 0; h < H; ++h) { dot[r][h] = 0.0f; acc[r][h] = make_float2(0.0f, 0.0f); }
-      // q of the next 4-channel block, fetched one block ahead
-      float4 qn[H];
-#pragma unroll
-      for (int h = 0; h < H; ++h) qn[h] = *reinterpret_cast<const float4*>(qv + h * D);
-      constexpr int SW = 2 * KB;  // words of 64 channels of a row
-#pragma unroll
-      for (int sgm = 0; sgm < D / 64; ++sgm) {
-        uint32_t w[RPL][SW];
-#pragma unroll
-        for (int r = 0; r < RPL; ++r)
-#pragma unroll
-          for (int q4 = 0; q4 < SW / 4; ++q4) {
-            const uint4 v = src[r][sgm * (SW / 4) + q4];
-            w[r][4 * q4] = v.x; w[r][4 * q4 + 1] = v.y; w[r][4 * q4 + 2] = v.z; w[r][4 * q4 + 3] = v.w;
+          for (int c = 0; c < 2; ++c) {
+            const int h = 2 * tig + c < H ? 2 * tig + c : 0;
+            azA2[c] = 2 * tig + c < H ? azb[h * 8 + 4] : 0.0f;
+            azZ2[c][0] = azb[h * 8 + 0];
           }
+        } else {
 #pragma unroll
-        for (int cc = 0; cc < 4; ++cc) {
-          const int c = sgm * 4 + cc;
-          LaneWords<KB> lw[RPL];
-#pragma unroll
-          for (int r = 0; r < RPL; ++r)
-#pragma unroll
-            for (int k2 = 0; k2 < NW; ++k2) lw[r].w[k2] = w[r][cc * NW + k2];
-#pragma unroll
-          for (int b4 = 0; b4 < 4; ++b4) {
-            const int blk = c * 4 + b4;
-            float4 qc[H];
-#pragma unroll
-            for (int h = 0; h < H; ++h) qc[h] = qn[h];
-            if (blk + 1 < D / 4) {
-#pragma unroll
-              for (int h = 0; h < H; ++h) qn[h] = *reinterpret_cast<const float4*>(qv + h * D + (blk + 1) * 4);
-            }
-            float2 cp[RPL][2];
-#pragma unroll
-            for (int r = 0; r < RPL; ++r) {
-              cp[r][0] = code_pair_at<KB>(lw[r], mg, 2 * b4);
-              cp[r][1] = code_pair_at<KB>(lw[r], mg, 2 * b4 + 1);
-            }
-#pragma unroll
-            for (int h = 0; h < H; ++h)
-#pragma unroll
-              for (int r = 0; r < RPL; ++r) {
-                acc[r][h] = __ffma2_rn(make_float2(qc[h].x, qc[h].y), cp[r][0], acc[r][h]);
-                acc[r][h] = __ffma2_rn(make_float2(qc[h].z, qc[h].w), cp[r][1], acc[r][h]);
-              }
-          }
-          if (SPG ? ((c + 1) % SPG == 0) : (((c + 1) * 16) % d.G == 0)) {  // end of a group: fold (scale, zero)
-            const int gidx = SPG ? c / SPG : (c * 16) / d.G;
-            float qsum[H];
-#pragma unroll
-            for (int h = 0; h < H; ++h) qsum[h] = qg[h * 4 + gidx];
-#pragma unroll
-            for (int r = 0; r < RPL; ++r) {
-              const int i = valid[r] ? lane + 32 * r : 0;
-              const float2 sz = *reinterpret_cast<const float2*>(szs + (i * ng + gidx) * 2);
-#pragma unroll
-              for (int h = 0; h < H; ++h) {
-                dot[r][h] = fmaf(sz.x, acc[r][h].x + acc[r][h].y, fmaf(sz.y, qsum[h], dot[r][h]));
-                acc[r][h] = make_float2(0.0f, 0.0f);
-              }
-            }
+          for (int n2 = 0; n2 < 2; ++n2) {
+            const int hh = 2 * n2 + tig / 2;
+            const int h = hh < H ? hh : 0;
+            azA2[n2] = hh < H ? azb[h * 8 + 4] : 0.0f;
+            azZ2[n2][0] = azb[h * 8 + 2 * (tig & 1)];
+            azZ2[n2][1] = azb[h * 8 + 2 * (tig & 1) + 1];
           }
         }
       }
+      const uint8_t* stg = ring + (size_t)s * Gk::kStageBytes;
+      const uint8_t* codes = stg + sub * TR * Gk::RB;
+      const float* szs = reinterpret_cast<const float*>(stg + Gk::kStageCodes) +
+                         (((ng == 1) ? (dd[1] & 1) : 0) + sub * TR) * ng * 2;
+      // logits of head tig (base 2) for rows 16 mt + gid + 8 hf
+      float sv[4][2];
+      auto fold_pair = [&](auto mc) {
+        constexpr int MT0 = decltype(mc)::value;
+        float acc[2][2][4];
+        if (NT == 2) mma_pair<D, KB, 2, MT0>(codes, tig, gid, bf, acc);
+        else mma_pair<D, KB, 1, MT0>(codes, tig, gid, bf, acc);
+#pragma unroll
+        for (int m = 0; m < 2; ++m)
+#pragma unroll
+          for (int hf = 0; hf < 2; ++hf) {
+            const int r = 16 * (MT0 + m) + gid + 8 * hf;
+            const float c0 = acc[m][0][2 * hf], c1 = acc[m][0][2 * hf + 1];
+            float val;
+            if (ng == 2) {
+              const float4 s4 = *reinterpret_cast<const float4*>(szs + r * 4);
+              val = fmaf(azA, fmaf(s4.z, c1, s4.x * c0), fmaf(s4.w, azZ[1], s4.y * azZ[0]));
+            } else if (ng == 1) {
+              const float2 s2 = *reinterpret_cast<const float2*>(szs + r * 2);
+              const float v0 = fmaf(azA2[0] * s2.x, c0, s2.y * azZ2[0][0]);
+              const float v1 = fmaf(azA2[1] * s2.x, c1, s2.y * azZ2[1][0]);
+              const int src = (lane & ~3) | (tig >> 1);
+              const float u0 = __shfl_sync(kFull, v0, src), u1 = __shfl_sync(kFull, v1, src);
+              val = (tig & 1) ? u1 : u0;
+            } else {
+              const float4 s4 = *reinterpret_cast<const float4*>(szs + r * ng * 2 + 4 * (tig & 1));
+              float f[2];
+#pragma unroll
+              for (int n2 = 0; n2 < 2; ++n2) {
+                const float e0 = acc[m][n2][2 * hf], e1 = acc[m][n2][2 * hf + 1];
+                float pv = fmaf(azA2[n2], fmaf(s4.z, e1, s4.x * e0), fmaf(s4.w, azZ2[n2][1], s4.y * azZ2[n2][0]));
+                pv += __shfl_xor_sync(kFull, pv, 1);
+                f[n2] = pv;
+              }
+              const int src = (lane & ~3) | (2 * (tig & 1));
+              const float u0 = __shfl_sync(kFull, f[0], src), u1 = __shfl_sync(kFull, f[1], src);
+              val = (tig >> 1) ? u1 : u0;
+            }
+            sv[MT0 + m][hf] = val;
+          }
       };
-      if (td.entry < kQSlots) {
-        const float* qv_s = reinterpret_cast<const float*>(smem_raw + kQOff) + td.entry * H * D;
-        const float* qg_s = reinterpret_cast<const float*>(smem_raw + kQgOff) + td.entry * H * 4;
-        if (d.G == 32) k_rows(std::integral_constant<int, 2>{}, qv_s, qg_s);
-        else if (d.G == 64) k_rows(std::integral_constant<int, 4>{}, qv_s, qg_s);
-        else k_rows(std::integral_constant<int, 8>{}, qv_s, qg_s);
-      } else {
-        k_rows(std::integral_constant<int, 0>{}, a.qbuf + (long long)td.u * H * D, a.qgsum + (long long)td.u * H * 4);
-      }
-      // The stage's data is in registers now: refill it with this warp's next tile.
-      ++consumed;
+      fold_pair(std::integral_constant<int, 0>{});
+      fold_pair(std::integral_constant<int, 2>{});
+      // the stage's data is in registers: hand it back to the producer
       fence_proxy_async_smem();
       __syncwarp();
-      {
-        TileDesc tn;
-        if (next_tile(tn)) {
-          if (slotw) p1 = tn; else p0 = tn;
-          issue(tn, stage);
-          ++issued;
-        }
-      }
-      // tile statistics: per-head maximum and sum of exp2 over the tile's rows
-      float tm[H], tl[H];
+      if (lane == 0) mbar_arrive(&empty[s]);
+      // tile statistics of head tig: maximum and sum of exp2 over the valid rows
+      float m = -INFINITY;
 #pragma unroll
-      for (int h = 0; h < H; ++h) {
-        float m = -INFINITY;
+      for (int mt = 0; mt < 4; ++mt)
 #pragma unroll
-        for (int r = 0; r < RPL; ++r) m = valid[r] ? fmaxf(m, dot[r][h]) : m;
+        for (int hf = 0; hf < 2; ++hf)
+          if (16 * mt + gid + 8 * hf < rows) m = fmaxf(m, sv[mt][hf]);
 #pragma unroll
-        for (int off = 16; off >= 1; off >>= 1) m = fmaxf(m, __shfl_xor_sync(kFull, m, off));
-        tm[h] = m;
-        float l = 0.0f;
+      for (int off = 4; off < 32; off <<= 1) m = fmaxf(m, __shfl_xor_sync(kFull, m, off));
+      float l = 0.0f;
 #pragma unroll
-        for (int r = 0; r < RPL; ++r) {
-          dot[r][h] = exp2f(dot[r][h] - m);
-          l += valid[r] ? dot[r][h] : 0.0f;
+      for (int mt = 0; mt < 4; ++mt)
+#pragma unroll
+        for (int hf = 0; hf < 2; ++hf) {
+          const bool ok = 16 * mt + gid + 8 * hf < rows;
+          sv[mt][hf] = ok ? exp2f(sv[mt][hf] - m) : 0.0f;
+          l += sv[mt][hf];
         }
 #pragma unroll
-        for (int off = 16; off >= 1; off >>= 1) l += __shfl_xor_sync(kFull, l, off);
-        tl[h] = l;
-      }
+      for (int off = 4; off < 32; off <<= 1) l += __shfl_xor_sync(kFull, l, off);
+      if (tig < H) {
 #pragma unroll
-      for (int r = 0; r < RPL; ++r)
-        if (valid[r]) store_heads<H>(lg + ((long long)td.slot * TR + lane + 32 * r) * H, dot[r]);
-      if (lane < H) {
-        float mv = tm[0], lv = tl[0];
+        for (int mt = 0; mt < 4; ++mt)
 #pragma unroll
-        for (int h = 1; h < H; ++h) if (lane == h) { mv = tm[h]; lv = tl[h]; }
-        tsm[td.slot * H + lane] = mv;
-        tsl[td.slot * H + lane] = lv;
+          for (int hf = 0; hf < 2; ++hf) {
+            const int r = 16 * mt + gid + 8 * hf;
+            if (r < rows) lg[((long long)t * TR + r) * H + tig] = sv[mt][hf];
+          }
+        if (gid == 0) {
+          tsm[t * H + tig] = m;
+          tsl[t * H + tig] = l;
+        }
       }
     }
-    // Never leave copies in flight (only after an abort can any be pending).
-    for (; consumed < issued; ++consumed)
-      mbar_wait(&full[warp * kSlotsPerWarp + consumed % kSlotsPerWarp], (consumed / kSlotsPerWarp) & 1, limit_ns);
   }
-  named_barrier(kBarCons, NCONS);
+  __syncthreads();
   // After a timed-out wait a bulk copy may still land in the ring, which
   // phase 2 reuses: skip straight to the end (the status word says why).
-  const bool aborted = *static_cast<volatile int*>(&s_abort) != 0;
+  const bool aborted = *abort_flag != 0;
   const int n_work = aborted ? 0 : nent;
 
-  // ------------------------------------------------------------ piece statistics
+  // ------------------------------------------------------------ statistics
+  // piece statistics: the CTA's tiles of each unit, merged
   for (int e = warp; e < n_work; e += CW) {
-    int* rec = ulist + (long long)e * kRec;
+    int* rec = ulist + e * kRec;
     const Unit x = load_unit(rec);
     const int ta = (max(x.cb, k0) - k0) * TPC, tb = (min(x.cb + x.nc, k1) - k0) * TPC;
 #pragma unroll 1
@@ -715,190 +790,364 @@ __global__ void __launch_bounds__(Geo<D, KB>::kThreads, 1) fused_decode_kernel(F
       }
     }
   }
-  named_barrier(kBarCons, NCONS);
+  __syncthreads();
   if (tid == 0 && n_work > 0) {
-    __threadfence();  // orders every consumer's statistics before the arrivals
+    __threadfence();  // orders every warp's statistics before the arrivals
     const Unit x0 = load_unit(ulist);
     if (!x0.owned) atomicAdd(a.arrive1 + x0.u, 1);
     if (nent > 1) {
-      const Unit x1 = load_unit(ulist + (long long)(nent - 1) * kRec);
+      const Unit x1 = load_unit(ulist + (nent - 1) * kRec);
       if (!x1.owned) atomicAdd(a.arrive1 + x1.u, 1);
     }
   }
+  // global statistics of every piece's unit: (max, 1 / sum) per head replace
+  // the piece's own in its record; a unit shared with other CTAs waits
+  // (bounded) for their pieces
+  for (int e = warp; e < n_work; e += CW) {
+    int* rec = ulist + e * kRec;
+    const Unit x = load_unit(rec);
+    float* st = reinterpret_cast<float*>(rec + 8);
+    if (x.owned) {
+      if (lane < H) {
+        const float l = st[2 * lane + 1];
+        st[2 * lane + 1] = l > 0.0f ? 1.0f / l : 0.0f;
+      }
+    } else {
+      const int i_first = x.cb / cpc, i_last = (x.cb + x.nc - 1) / cpc;
+      bool ok = true;
+      if (lane == 0) ok = wait_counter(a.arrive1 + x.u, i_last - i_first + 1, limit_ns);
+      ok = __shfl_sync(kFull, ok ? 1 : 0, 0) != 0;
+      if (!ok) {
+        if (lane == 0) atomicExch(d.status, kStatusTimeout);
+        if (lane < H) { st[2 * lane] = -INFINITY; st[2 * lane + 1] = 0.0f; }
+      } else if (lane < H) {
+        __threadfence();
+        float m = -INFINITY, l = 0.0f;
+        for (int i = i_first; i <= i_last; ++i) {
+          const int slot = (i == i_first) ? 1 : 0;
+          const float* ps = a.pstats + ((long long)i * 2 + slot) * H * 2;
+          merge_ml(m, l, __ldcg(ps + 2 * lane), __ldcg(ps + 2 * lane + 1));
+        }
+        st[2 * lane] = m;
+        st[2 * lane + 1] = l > 0.0f ? 1.0f / l : 0.0f;
+      }
+    }
+  }
+  __syncthreads();
+  // per-tile factors exp2(max_tile - max) / sum
+  for (int q = tid; q < (n_work > 0 ? ntile * H : 0); q += NTHR) {
+    const int t2 = q / H, h = q % H;
+    const int g = k0 + t2 / TPC;
+    int lo = 0, hi = nent - 1;  // entry holding chunk g
+    while (lo < hi) { const int mid = (lo + hi + 1) >> 1; if (ulist[mid * kRec + 1] <= g) lo = mid; else hi = mid - 1; }
+    const float* st = reinterpret_cast<const float*>(ulist + lo * kRec + 8);
+    const float M = st[2 * h], il = st[2 * h + 1];
+    const float mt = tsm[t2 * H + h];
+    tsf[t2 * H + h] = (il > 0.0f && mt > -INFINITY) ? exp2f(mt - M) * il : 0.0f;
+  }
+  __syncthreads();
 
   // ------------------------------------------------------------ phase 2
-  // phase-2 shared memory (in the ring): kept-row lists [CW][kListCap], their
-  // per-head weights [CW][kListCap][H] and the warps' partial outputs [CW][H][D]
-  int* lists = reinterpret_cast<int*>(ring);
-  float* wts = reinterpret_cast<float*>(ring + kMaxConsumerWarps * kListCap * 4);
-  constexpr int kListsBytes = kMaxConsumerWarps * kListCap * 4 * (1 + H);
-  float* red = reinterpret_cast<float*>(ring + (kListsBytes > kDenseStaging ? kListsBytes : kDenseStaging));
+  // phase-2 shared memory (in the ring).  Sparse mode: per warp its kept
+  // rows [lcap] and their weights [lcap][H], then one staging slot per kept
+  // V row.  Scan mode: kept-row lists [CW][kListCap] and weights; dense
+  // mode: the V staging buffers.  The warps' partial outputs [CW][H][D]
+  // are last.
+  const int red_off = a.ring_bytes - CW * H * D * 4;
+  float* red = reinterpret_cast<float*>(ring + red_off);
   // the dense V pass applies when every row is kept and the V rows fit its buffers
   const bool dense = d.tau <= 0.0f && VB0 <= 6 && VB1 <= 6;
-  int dense_uses[2] = {0, 0};
-  Magic<VB0> mg0;
-  mg0.load(s_magic);
-  Magic<VB1> mg1;
-  mg1.load(s_magic);
+  const int lcap = a.cand_cap;
+  const bool sparse_try = !dense && lcap > 0;
   unsigned long long cnt_heads = 0, cnt_rows = 0;
   uint8_t* const smask = d.skip_mask;
   float* const mass_out = d.mass;
-  for (int pass = 0; pass < 2; ++pass) {
-    for (int e = 0; e < n_work; ++e) {
-      int* rec = ulist + (long long)e * kRec;
-      const Unit x = load_unit(rec);
-      if ((pass == 0) != (x.owned != 0)) continue;  // owned pieces first, shared ones after
-      const int b = x.u / d.Hkv, g = x.u % d.Hkv;
-      const int i_first = x.cb / cpc, i_last = (x.cb + x.nc - 1) / cpc;
-      // global statistics of the unit
-      if (x.owned) {
-        if (tid < H) {
-          const float m = reinterpret_cast<float*>(rec + 8)[2 * tid];
-          const float l = reinterpret_cast<float*>(rec + 8)[2 * tid + 1];
-          s_glob[2 * tid] = m;
-          s_glob[2 * tid + 1] = l > 0.0f ? 1.0f / l : 0.0f;
-        }
-      } else if (warp == 0) {
-        bool ok = true;
-        if (lane == 0) ok = wait_counter(a.arrive1 + x.u, i_last - i_first + 1, limit_ns);
-        ok = __shfl_sync(kFull, ok ? 1 : 0, 0) != 0;
-        if (!ok) {
-          if (lane == 0) atomicExch(d.status, kStatusTimeout);
-          if (lane < H) { s_glob[2 * lane] = -INFINITY; s_glob[2 * lane + 1] = 0.0f; }
-        } else if (lane < H) {
-          __threadfence();
-          float m = -INFINITY, l = 0.0f;
-          for (int i = i_first; i <= i_last; ++i) {
-            const int slot = (i == i_first) ? 1 : 0;
-            const float* ps = a.pstats + ((long long)i * 2 + slot) * H * 2;
-            merge_ml(m, l, __ldcg(ps + 2 * lane), __ldcg(ps + 2 * lane + 1));
-          }
-          s_glob[2 * lane] = m;
-          s_glob[2 * lane + 1] = l > 0.0f ? 1.0f / l : 0.0f;
-        }
-      }
-      named_barrier(kBarCons, NCONS);
-      const int ga = max(x.cb, k0), gb = min(x.cb + x.nc, k1);
-      // per-tile factors exp2(max_tile - max) / sum
-      for (int q = tid; q < (gb - ga) * TPC * H; q += NCONS) {
-        const int t2 = (ga - k0) * TPC + q / H, h = q % H;
-        const float M = s_glob[2 * h], il = s_glob[2 * h + 1];
-        const float mt = tsm[t2 * H + h];
-        tsf[t2 * H + h] = (il > 0.0f && mt > -INFINITY) ? exp2f(mt - M) * il : 0.0f;
-      }
-      named_barrier(kBarCons, NCONS);
-
-      const float* lgu = lg + (long long)(x.cb - k0) * kChunk * H;   // row v of the unit at lgu[v * H]
-      const float* tfu = tsf + (x.cb - k0) * TPC * H;                 // tile v / TR at tfu[(v / TR) * H]
-      const long long ubase = (long long)x.u * d.T_cap;
-      const int v_lo = (ga - x.cb) * kChunk, v_hi = (gb - x.cb) * kChunk;  // chunk-aligned (padded) rows
-      float2 acc[H][8];
-      float Z[H];
+  constexpr int kSzSlot = 8 * ((D / 32) > 2 ? (D / 32) : 2);
+  constexpr int kVRowMax = D * (VB0 > VB1 ? VB0 : VB1) / 8;
+  constexpr int kSlotBytes = kVRowMax + kSzSlot;
+  int* const lrows = reinterpret_cast<int*>(ring) + warp * lcap * (1 + H);   // this warp's kept rows
+  float* const lw = reinterpret_cast<float*>(lrows + lcap);                   // ... and their weights
+  const int lists_bytes = CW * lcap * (1 + H) * 4;
+  int n_kept = 0;
+  if (sparse_try && n_work > 0) {
+    // 1. every row of the CTA: p = e * factor; the skip decision, the skip
+    //    mask, the attention mass and the counts; rows some head keeps go to
+    //    the warp's list with their weights, in row order.  Warp w scans a
+    //    contiguous run of the CTA's tiles, kScanTiles tiles in flight.
+    const int t_lo = (ntile * warp) / CW, t_hi = (ntile * (warp + 1)) / CW;
+    int ent = 0;
+    for (int t0 = t_lo; t0 < t_hi; t0 += kScanTiles) {
+      float ev[kScanTiles][2][H];
+      int nrow[kScanTiles], tent[kScanTiles], tpos[kScanTiles];
 #pragma unroll
-      for (int h = 0; h < H; ++h) {
-        Z[h] = 0.0f;
+      for (int u = 0; u < kScanTiles; ++u) {
+        const int t = t0 + u;
+        nrow[u] = 0;
+        tent[u] = 0;
+        tpos[u] = 0;
+        if (t < t_hi) {
+          const int g = k0 + t / TPC;
+          while (ent + 1 < nent && ulist[(ent + 1) * kRec + 1] <= g) ++ent;
+          const Unit x = load_unit(ulist + ent * kRec);
+          const ChunkRows cr = chunk_rows(x, g - x.cb);
+          nrow[u] = max(0, min(TR, cr.rows - (t % TPC) * TR));
+          tent[u] = ent;
+          tpos[u] = cr.row0 + (t % TPC) * TR;  // position of the tile's first row (plain decode)
 #pragma unroll
-        for (int i = 0; i < 8; ++i) acc[h][i] = make_float2(0.0f, 0.0f);
+          for (int hf = 0; hf < 2; ++hf)
+            if (hf * 32 + lane < nrow[u]) ldcg_heads<H>(lg + ((long long)t * TR + hf * 32 + lane) * H, ev[u][hf]);
+        }
       }
-      if (dense) {
-        // Dense V pass: every valid row is kept, so the warp streams its
-        // 32-row blocks (round robin over warps) into shared memory with bulk
-        // copies, two blocks in flight, and accumulates them from there.
-        uint8_t* stg = ring + (size_t)warp * 2 * kDenseBuf;
-        const int nblk = (v_hi - v_lo) / 32;
-        const uint64_t pol = policy_evict_first();
-        int rows_of[2] = {0, 0};
-        auto issue = [&](int k, int buf) {
-          rows_of[buf] = 0;
-          const int blk = warp + k * CW;
-          if (blk >= nblk) return;
-          const int v0 = v_lo + blk * 32;
-          const ChunkRows cr = chunk_rows(x, v0 / kChunk);
-          const int rows = min(32, cr.rows - v0 % kChunk);
-          if (rows <= 0) return;
-          rows_of[buf] = rows;
-          if (lane == 0) {
-            const int seg = cr.seg, row = cr.row0 + v0 % kChunk;
-            const int rbv = seg ? D * VB1 / 8 : D * VB0 / 8;
-            const int r0 = (ng == 1) ? (row & ~1) : row;
-            const int r1 = (ng == 1) ? ((row + rows + 1) & ~1) : row + rows;
-            const uint32_t cbytes = (uint32_t)rows * rbv, sbytes = (uint32_t)(r1 - r0) * ng * 8;
-            const uint32_t lbytes = 32u * H * 4u;
-            uint8_t* dst = stg + buf * kDenseBuf;
-            uint64_t* bar = &full[kDenseBar + warp * 2 + buf];
-            mbar_arrive_expect_tx(bar, cbytes + sbytes + lbytes);
-            const long long pr = PAGED ? unit_row<PAGED>(a, x.u, row) : ubase + row;
-            const long long pr0 = PAGED ? unit_row<PAGED>(a, x.u, r0) : ubase + r0;
-            bulk_g2s(dst, d.vc[seg] + pr * rbv, cbytes, bar, pol);
-            bulk_g2s(dst + kDenseCodes, d.vsz[seg] + pr0 * ng * 2, sbytes, bar, pol);
-            bulk_g2s(dst + kDenseCodes + kDenseSz, lgu + (long long)v0 * H, lbytes, bar, pol);
-          }
-        };
-        issue(0, 0);
-        issue(1, 1);
-        bool stalled = false;
-        for (int k = 0; warp + k * CW < nblk && !stalled; ++k) {
-          const int buf = k & 1;
-          const int rows = rows_of[buf];
-          if (rows > 0) {
-            if (!mbar_wait(&full[kDenseBar + warp * 2 + buf], dense_uses[buf] & 1, limit_ns)) {
-              atomicExch(d.status, kStatusTimeout);
-              stalled = true;  // leave the copy pending: it is drained below
-              break;
+#pragma unroll
+      for (int u = 0; u < kScanTiles; ++u) {
+        if (nrow[u] == 0) continue;  // the same for the whole warp
+        const int t = t0 + u;
+        float f[H];
+        lds_heads<H>(tsf + t * H, f);
+        const Unit x = load_unit(ulist + tent[u] * kRec);
+        const int b = x.u / d.Hkv, g = x.u % d.Hkv;
+#pragma unroll
+        for (int hf = 0; hf < 2; ++hf) {
+          const int r = hf * 32 + lane;
+          bool need = false;
+          float wgt[H];
+          if (r < nrow[u]) {
+            float ms = 0.0f;
+#pragma unroll
+            for (int h = 0; h < H; ++h) {
+              const float p = ev[u][hf][h] * f[h];
+              const bool keep = !(p < d.tau);
+              wgt[h] = keep ? p : 0.0f;
+              need |= keep;
+              cnt_heads += keep ? 0u : 1u;
+              ms += p;
+              if (smask) smask[((long long)b * d.Hq + g * H + h) * d.T_cap + tpos[u] + r] = keep ? 0 : 1;
             }
-            ++dense_uses[buf];
-            rows_of[buf] = 0;
-            {
-              const int v0 = v_lo + (warp + k * CW) * 32;
-              const ChunkRows cr = chunk_rows(x, v0 / kChunk);
-              const int row = cr.row0 + v0 % kChunk;
-              const int sz_skip = (ng == 1) ? (row & 1) : 0;
-              const uint8_t* src = stg + buf * kDenseBuf;
-              const float* lgs = reinterpret_cast<const float*>(src + kDenseCodes + kDenseSz);
-              const float* szs = reinterpret_cast<const float*>(src + kDenseCodes);
-              float f[H];
-              lds_heads<H>(tfu + (v0 / TR) * H, f);
-              for (int s2 = 0; s2 < 32 / RPW; ++s2) {
-                const int i = s2 * RPW + lane / LPR;
-                if (i >= rows) continue;  // the lanes of a row agree
-                float e[H], wgt[H];
-                lds_heads<H>(lgs + i * H, e);
-                float ms = 0.0f;
+            cnt_rows += need ? 0u : 1u;
+            if (mass_out) mass_out[((long long)b * d.Hkv + g) * d.T_cap + tpos[u] + r] = ms * (1.0f / H);
+          }
+          const unsigned bal = __ballot_sync(kFull, need);
+          const int o = n_kept + __popc(bal & ((1u << lane) - 1u));
+          if (need && o < lcap) {
+            lrows[o] = (t * TR + r) | (tent[u] << kCandRowBits);
+            store_heads<H>(lw + o * H, wgt);
+          }
+          n_kept += __popc(bal);
+        }
+      }
+    }
+    if (n_kept > lcap) s_ovf = 1;
+  }
+  __syncthreads();
+  const bool sparse = sparse_try && n_work > 0 && !*static_cast<volatile int*>(&s_ovf);
+  if (sparse_try && !sparse) { cnt_heads = 0; cnt_rows = 0; }  // the scan mode below counts again
+  const int stage_slots = sparse ? (red_off - lists_bytes) / kSlotBytes : 0;
+  if (sparse) {
+    // 2. kept V rows into their staging slots with 16-byte asynchronous
+    //    copies (warp w's rows take slots [off_w, off_w + n_w)); rows past
+    //    the capacity are read from global memory when accumulated
+    if (lane == 0) s_nw[warp] = n_kept;
+    __syncthreads();
+    int off_w = 0;
+    for (int w2 = 0; w2 < warp; ++w2) off_w += s_nw[w2];
+    if (lane == 0) s_coff[warp] = off_w;
+    const int n_stage = max(0, min(n_kept, stage_slots - off_w));
+    constexpr int kMaxChunks = kVRowMax / 16 + kSzSlot / 16;
+    for (int q = lane; q < n_stage * kMaxChunks; q += 32) {
+      const int i = q / kMaxChunks, c = q % kMaxChunks;
+      const int rowe = lrows[i];
+      const int ent = rowe >> kCandRowBits, row = rowe & ((1 << kCandRowBits) - 1);
+      const Unit x = load_unit(ulist + ent * kRec);
+      const ChunkRows cr = chunk_rows(x, (k0 + row / kChunk) - x.cb);
+      const int vr = cr.row0 + row % kChunk;
+      const int rbv = cr.seg ? D * VB1 / 8 : D * VB0 / 8;
+      const int szb = ng == 1 ? 16 : ng * 8;
+      uint8_t* slot = ring + lists_bytes + (size_t)(off_w + i) * kSlotBytes;
+      if (c * 16 < rbv) {
+        const long long pr = PAGED ? unit_row<PAGED>(a, x.u, vr) : (long long)x.u * d.T_cap + vr;
+        cp_async16(slot + c * 16, d.vc[cr.seg] + pr * rbv + c * 16);
+      } else if ((c - kVRowMax / 16) * 16 < szb && c >= kVRowMax / 16) {
+        const int cz = c - kVRowMax / 16;
+        const int vr0 = ng == 1 ? (vr & ~1) : vr;
+        const long long pr0 = PAGED ? unit_row<PAGED>(a, x.u, vr0) : (long long)x.u * d.T_cap + vr0;
+        cp_async16(slot + kVRowMax + cz * 16, reinterpret_cast<const uint8_t*>(d.vsz[cr.seg] + pr0 * ng * 2) + cz * 16);
+      }
+    }
+    cp_async_wait_all();
+    __syncthreads();
+  }
+  int* lists = reinterpret_cast<int*>(ring);
+  float* wts = reinterpret_cast<float*>(ring + kWarps * kListCap * 4);
+  int dense_uses[2] = {0, 0};
+  for (int e = 0; e < n_work; ++e) {
+    int* rec = ulist + e * kRec;
+    const Unit x = load_unit(rec);
+    const int b = x.u / d.Hkv, g = x.u % d.Hkv;
+    const int i_first = x.cb / cpc, i_last = (x.cb + x.nc - 1) / cpc;
+    const int ga = max(x.cb, k0), gb = min(x.cb + x.nc, k1);
+    const float* lgu = lg + (long long)(x.cb - k0) * kChunk * H;   // row v of the unit at lgu[v * H]
+    const float* tfu = tsf + (x.cb - k0) * TPC * H;                 // tile v / TR at tfu[(v / TR) * H]
+    const long long ubase = (long long)x.u * d.T_cap;
+    const int v_lo = (ga - x.cb) * kChunk, v_hi = (gb - x.cb) * kChunk;  // chunk-aligned (padded) rows
+    float2 acc[H][8];
+    float Z[H];
 #pragma unroll
-                for (int h = 0; h < H; ++h) { wgt[h] = e[h] * f[h]; ms += wgt[h]; }
-                if (j == 0) {
-                  if (smask) {
+    for (int h = 0; h < H; ++h) {
+      Z[h] = 0.0f;
 #pragma unroll
-                    for (int h = 0; h < H; ++h) smask[((long long)b * d.Hq + g * H + h) * d.T_cap + v0 + i] = 0;
-                  }
-                  if (mass_out) mass_out[((long long)b * d.Hkv + g) * d.T_cap + v0 + i] = ms * (1.0f / H);
+      for (int i = 0; i < 8; ++i) acc[h][i] = make_float2(0.0f, 0.0f);
+    }
+    if (sparse) {
+      // this warp's kept rows of the piece: a contiguous run of its list
+      int lo, hi;
+      {
+        const int nk = min(n_kept, lcap);
+        int a0 = 0, a1 = nk;  // first entry of unit entry >= e
+        while (a0 < a1) { const int mid = (a0 + a1) >> 1; if ((lrows[mid] >> kCandRowBits) < e) a0 = mid + 1; else a1 = mid; }
+        lo = a0;
+        a1 = nk;              // first entry of unit entry > e
+        while (a0 < a1) { const int mid = (a0 + a1) >> 1; if ((lrows[mid] >> kCandRowBits) <= e) a0 = mid + 1; else a1 = mid; }
+        hi = a0;
+      }
+      if (lane == 0) { s_cs[2 * warp] = lo; s_cs[2 * warp + 1] = hi - lo; }
+      __syncthreads();
+      // the piece's kept rows of all warps, split evenly over the warps
+      int n_all = 0;
+#pragma unroll
+      for (int w2 = 0; w2 < CW; ++w2) n_all += s_cs[2 * w2 + 1];
+      const int per = ((n_all + CW - 1) / CW + RPW - 1) / RPW * RPW;
+      const int g_lo = min(n_all, warp * per), g_hi = min(n_all, g_lo + per);
+      int sw = 0, sbase = 0;
+      for (int i0 = g_lo; i0 < g_hi; i0 += RPW) {
+        const int gidx = i0 + lane / LPR;
+        if (gidx >= g_hi) continue;  // the lanes of a row agree
+        while (gidx >= sbase + s_cs[2 * sw + 1]) { sbase += s_cs[2 * sw + 1]; ++sw; }
+        const int li = s_cs[2 * sw] + gidx - sbase;   // entry of warp sw's list
+        const int* lr = reinterpret_cast<const int*>(ring) + sw * lcap * (1 + H);
+        const float* lwt = reinterpret_cast<const float*>(lr + lcap);
+        float wgt[H];
+        lds_heads<H>(lwt + li * H, wgt);
+        const int row = lr[li] & ((1 << kCandRowBits) - 1);
+        const int v = (k0 - x.cb) * kChunk + row;
+        const ChunkRows cr = chunk_rows(x, v / kChunk);
+        const int vr = cr.row0 + v % kChunk;
+        const int slot = s_coff[sw] + li;
+        LaneWords<VB0> w0;
+        LaneWords<(VB0 == VB1) ? 2 : VB1> w1;
+        float2 sz;
+        if (slot < stage_slots) {
+          const uint8_t* src = ring + lists_bytes + (size_t)slot * kSlotBytes;
+          const float* szp = reinterpret_cast<const float*>(src + kVRowMax) + (ng == 1 ? (vr & 1) * 2 : gi * 2);
+          sz = *reinterpret_cast<const float2*>(szp);
+          if (cr.seg == 0 || VB0 == VB1) lds_lane_words<VB0>(src + j * 2 * VB0, w0);
+          else if constexpr (VB0 != VB1) lds_lane_words<VB1>(src + j * 2 * VB1, w1);
+        } else {
+          const long long pr = PAGED ? unit_row<PAGED>(a, x.u, vr) : ubase + vr;
+          if (cr.seg == 0 || VB0 == VB1) ldg_v<VB0>(d.vc[cr.seg] + pr * (D * VB0 / 8), d.vsz[cr.seg] + pr * ng * 2, j, gi, w0, sz);
+          else if constexpr (VB0 != VB1) ldg_v<VB1>(d.vc[1] + pr * (D * VB1 / 8), d.vsz[1] + pr * ng * 2, j, gi, w1, sz);
+        }
+        if (cr.seg == 0 || VB0 == VB1) accumulate_v<H, VB0>(w0, sz, wgt, acc, Z);
+        else if constexpr (VB0 != VB1) accumulate_v<H, VB1>(w1, sz, wgt, acc, Z);
+      }
+    } else if (dense) {
+      // Dense V pass: every valid row is kept, so the warp streams its
+      // 32-row blocks (round robin over warps) into shared memory with bulk
+      // copies, two blocks in flight, and accumulates them from there.
+      uint8_t* stg = ring + (size_t)warp * 2 * kDenseBuf;
+      const int nblk = (v_hi - v_lo) / 32;
+      const uint64_t pol = policy_evict_first();
+      int rows_of[2] = {0, 0};
+      auto issue = [&](int k, int buf) {
+        rows_of[buf] = 0;
+        const int blk = warp + k * CW;
+        if (blk >= nblk) return;
+        const int v0 = v_lo + blk * 32;
+        const ChunkRows cr = chunk_rows(x, v0 / kChunk);
+        const int rows = min(32, cr.rows - v0 % kChunk);
+        if (rows <= 0) return;
+        rows_of[buf] = rows;
+        if (lane == 0) {
+          const int seg = cr.seg, row = cr.row0 + v0 % kChunk;
+          const int rbv = seg ? D * VB1 / 8 : D * VB0 / 8;
+          const int r0 = (ng == 1) ? (row & ~1) : row;
+          const int r1 = (ng == 1) ? ((row + rows + 1) & ~1) : row + rows;
+          const uint32_t cbytes = (uint32_t)rows * rbv, sbytes = (uint32_t)(r1 - r0) * ng * 8;
+          const uint32_t lbytes = 32u * H * 4u;
+          uint8_t* dst = stg + buf * kDenseBuf;
+          uint64_t* bar = &dbar[warp * 2 + buf];
+          mbar_arrive_expect_tx(bar, cbytes + sbytes + lbytes);
+          const long long pr = PAGED ? unit_row<PAGED>(a, x.u, row) : ubase + row;
+          const long long pr0 = PAGED ? unit_row<PAGED>(a, x.u, r0) : ubase + r0;
+          bulk_g2s(dst, d.vc[seg] + pr * rbv, cbytes, bar, pol);
+          bulk_g2s(dst + kDenseCodes, d.vsz[seg] + pr0 * ng * 2, sbytes, bar, pol);
+          bulk_g2s(dst + kDenseCodes + kDenseSz, lgu + (long long)v0 * H, lbytes, bar, pol);
+        }
+      };
+      issue(0, 0);
+      issue(1, 1);
+      bool stalled = false;
+      for (int k = 0; warp + k * CW < nblk && !stalled; ++k) {
+        const int buf = k & 1;
+        const int rows = rows_of[buf];
+        if (rows > 0) {
+          if (!mbar_wait(&dbar[warp * 2 + buf], dense_uses[buf] & 1, limit_ns)) {
+            atomicExch(d.status, kStatusTimeout);
+            stalled = true;  // leave the copy pending: it is drained below
+            break;
+          }
+          ++dense_uses[buf];
+          rows_of[buf] = 0;
+          {
+            const int v0 = v_lo + (warp + k * CW) * 32;
+            const ChunkRows cr = chunk_rows(x, v0 / kChunk);
+            const int row = cr.row0 + v0 % kChunk;
+            const int sz_skip = (ng == 1) ? (row & 1) : 0;
+            const uint8_t* src = stg + buf * kDenseBuf;
+            const float* lgs = reinterpret_cast<const float*>(src + kDenseCodes + kDenseSz);
+            const float* szs = reinterpret_cast<const float*>(src + kDenseCodes);
+            float f[H];
+            lds_heads<H>(tfu + (v0 / TR) * H, f);
+            for (int s2 = 0; s2 < 32 / RPW; ++s2) {
+              const int i = s2 * RPW + lane / LPR;
+              if (i >= rows) continue;  // the lanes of a row agree
+              float ev[H], wgt[H];
+              lds_heads<H>(lgs + i * H, ev);
+              float ms = 0.0f;
+#pragma unroll
+              for (int h = 0; h < H; ++h) { wgt[h] = ev[h] * f[h]; ms += wgt[h]; }
+              if (j == 0) {
+                if (smask) {
+#pragma unroll
+                  for (int h = 0; h < H; ++h) smask[((long long)b * d.Hq + g * H + h) * d.T_cap + v0 + i] = 0;
                 }
-                const float2 sz = *reinterpret_cast<const float2*>(szs + ((sz_skip + i) * ng + gi) * 2);
-                if (cr.seg == 0) {
-                  LaneWords<VB0> lw;
-                  lds_lane_words<VB0>(src + i * (D * VB0 / 8) + j * 2 * VB0, lw);
-                  accumulate_v<H, VB0>(lw, mg0, sz, wgt, acc, Z);
-                } else {
-                  LaneWords<VB1> lw;
-                  lds_lane_words<VB1>(src + i * (D * VB1 / 8) + j * 2 * VB1, lw);
-                  accumulate_v<H, VB1>(lw, mg1, sz, wgt, acc, Z);
-                }
+                if (mass_out) mass_out[((long long)b * d.Hkv + g) * d.T_cap + v0 + i] = ms * (1.0f / H);
+              }
+              const float2 sz = *reinterpret_cast<const float2*>(szs + ((sz_skip + i) * ng + gi) * 2);
+              if (cr.seg == 0) {
+                LaneWords<VB0> lwd;
+                lds_lane_words<VB0>(src + i * (D * VB0 / 8) + j * 2 * VB0, lwd);
+                accumulate_v<H, VB0>(lwd, sz, wgt, acc, Z);
+              } else {
+                LaneWords<VB1> lwd;
+                lds_lane_words<VB1>(src + i * (D * VB1 / 8) + j * 2 * VB1, lwd);
+                accumulate_v<H, VB1>(lwd, sz, wgt, acc, Z);
               }
             }
           }
-          // the buffer's data is in registers: refill it
-          fence_proxy_async_smem();
-          __syncwarp();
-          issue(k + 2, buf);
         }
-        // never leave copies in flight (only a timed-out wait leaves one)
-        for (int buf = 0; buf < 2; ++buf)
-          if (rows_of[buf] > 0) {
-            mbar_wait(&full[kDenseBar + warp * 2 + buf], dense_uses[buf] & 1, limit_ns);
-            ++dense_uses[buf];
-          }
-      } else
-      for (int vb = v_lo; vb < v_hi; vb += NCONS * kBatchBlocks) {
+        // the buffer's data is in registers: refill it
+        fence_proxy_async_smem();
+        __syncwarp();
+        issue(k + 2, buf);
+      }
+      // never leave copies in flight (only a timed-out wait leaves one)
+      for (int buf = 0; buf < 2; ++buf)
+        if (rows_of[buf] > 0) {
+          mbar_wait(&dbar[warp * 2 + buf], dense_uses[buf] & 1, limit_ns);
+          ++dense_uses[buf];
+        }
+    } else {
+      for (int vb = v_lo; vb < v_hi; vb += CW * 32 * kBatchBlocks) {
         // scan: 32-row blocks round robin over warps, row order kept per warp;
         // the logits of kScanBlocks blocks are loaded before any is used.  A
         // block lies in one chunk and one tile, so its valid-row count and
@@ -962,10 +1211,9 @@ __global__ void __launch_bounds__(Geo<D, KB>::kThreads, 1) fused_decode_kernel(F
         cnt_rows += my_rows;
         __syncwarp();
         // gather: the CTA's kept rows (warp 0's list, then warp 1's, ...) are
-        // split evenly over the warps, in order, so every warp waits for about
-        // the same number of HBM round trips
+        // split evenly over the warps, in order
         if (lane == 0) s_nw[warp] = n_w;
-        named_barrier(kBarCons, NCONS);
+        __syncthreads();
         int n_all = 0;
 #pragma unroll
         for (int w2 = 0; w2 < CW; ++w2) n_all += s_nw[w2];
@@ -1007,84 +1255,76 @@ __global__ void __launch_bounds__(Geo<D, KB>::kThreads, 1) fused_decode_kernel(F
             float wgt[H];
             lds_heads<H>(wts + li[s2] * H, wgt);
             if constexpr (kOneWidth) {
-              accumulate_v<H, VB0>(w0[s2], mg0, szv[s2], wgt, acc, Z);
+              accumulate_v<H, VB0>(w0[s2], szv[s2], wgt, acc, Z);
             } else {
-              if (v / kChunk < x.nc0) accumulate_v<H, VB0>(w0[s2], mg0, szv[s2], wgt, acc, Z);
-              else accumulate_v<H, VB1>(w1[s2], mg1, szv[s2], wgt, acc, Z);
+              if (v / kChunk < x.nc0) accumulate_v<H, VB0>(w0[s2], szv[s2], wgt, acc, Z);
+              else accumulate_v<H, VB1>(w1[s2], szv[s2], wgt, acc, Z);
             }
           }
         }
-        named_barrier(kBarCons, NCONS);  // other warps read this batch's lists
+        __syncthreads();  // other warps read this batch's lists
       }
-      // fold the per-group constant, reduce the row slots of the warp
-      // (code that runs once per piece is kept short: loops stay rolled)
+    }
+    // fold the per-group constant, add the warp's row slots with shuffles
+#pragma unroll
+    for (int h = 0; h < H; ++h)
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        float2 v2 = make_float2(acc[h][i].x + Z[h], acc[h][i].y + Z[h]);
+#pragma unroll
+        for (int off = LPR; off < 32; off <<= 1) {
+          v2.x += __shfl_xor_sync(kFull, v2.x, off);
+          v2.y += __shfl_xor_sync(kFull, v2.y, off);
+        }
+        acc[h][i] = v2;
+      }
+    if (lane < LPR) {
 #pragma unroll
       for (int h = 0; h < H; ++h)
 #pragma unroll
-        for (int i = 0; i < 8; ++i) { acc[h][i].x += Z[h]; acc[h][i].y += Z[h]; }
-      if (lane < LPR) {
-#pragma unroll
-        for (int h = 0; h < H; ++h)
-#pragma unroll
-          for (int i = 0; i < 8; ++i)
-            *reinterpret_cast<float2*>(red + (warp * H + h) * D + j * kDimsPerLane + 2 * i) = make_float2(0.0f, 0.0f);
-      }
-      __syncwarp();
-      // the RPW row slots of the warp add their partial sums in shared memory
-#pragma unroll 1
-      for (int slot = 0; slot < RPW; ++slot) {
-        if (lane / LPR == slot) {
-#pragma unroll
-          for (int h = 0; h < H; ++h)
-#pragma unroll
-            for (int i = 0; i < 8; ++i) {
-              float2* o = reinterpret_cast<float2*>(red + (warp * H + h) * D + j * kDimsPerLane + 2 * i);
-              const float2 pv = *o;
-              *o = make_float2(pv.x + acc[h][i].x, pv.y + acc[h][i].y);
-            }
-        }
-        __syncwarp();
-      }
-      named_barrier(kBarCons, NCONS);
-      for (int o = tid; o < H * D; o += NCONS) {
-        float s2 = 0.0f;
-#pragma unroll
-        for (int w2 = 0; w2 < CW; ++w2) s2 += red[w2 * H * D + o];
-        const int h = o / D, dd = o % D;
-        if (x.owned) {
-          d.out[((long long)b * d.Hq + g * H + h) * D + dd] = s2;
-        } else {
-          if (e == 0) a.ppart[(((long long)cta * 2 + 0) * H + h) * D + dd] = s2;
-          if (e == nent - 1) a.ppart[(((long long)cta * 2 + 1) * H + h) * D + dd] = s2;
-        }
-      }
-      if (!x.owned) {
-        named_barrier(kBarCons, NCONS);
-        if (tid == 0) {
-          __threadfence();  // every thread's partial before the arrival
-          const int old = atomicAdd(a.arrive2 + x.u, 1);
-          s_last = (old == i_last - i_first) ? 1 : 0;
-        }
-        named_barrier(kBarCons, NCONS);
-        if (s_last) {
-          __threadfence();
-          for (int o = tid; o < H * D; o += NCONS) {
-            float s2 = 0.0f;
-            for (int i = i_first; i <= i_last; ++i) {
-              const int slot = (i == i_first) ? 1 : 0;
-              s2 += __ldcg(a.ppart + (((long long)i * 2 + slot) * H) * D + o);
-            }
-            const int h = o / D, dd = o % D;
-            d.out[((long long)b * d.Hq + g * H + h) * D + dd] = s2;
-          }
-          if (tid == 0) {
-            a.arrive1[x.u] = 0;
-            a.arrive2[x.u] = 0;
-          }
-        }
-      }
-      named_barrier(kBarCons, NCONS);
+        for (int i = 0; i < 8; i += 2)
+          *reinterpret_cast<float4*>(red + (warp * H + h) * D + j * kDimsPerLane + 2 * i) =
+              make_float4(acc[h][i].x, acc[h][i].y, acc[h][i + 1].x, acc[h][i + 1].y);
     }
+    __syncthreads();
+    for (int o = tid; o < H * D; o += NTHR) {
+      float s2 = 0.0f;
+#pragma unroll
+      for (int w2 = 0; w2 < CW; ++w2) s2 += red[w2 * H * D + o];
+      const int h = o / D, dd = o % D;
+      if (x.owned) {
+        d.out[((long long)b * d.Hq + g * H + h) * D + dd] = s2;
+      } else {
+        if (e == 0) a.ppart[(((long long)cta * 2 + 0) * H + h) * D + dd] = s2;
+        if (e == nent - 1) a.ppart[(((long long)cta * 2 + 1) * H + h) * D + dd] = s2;
+      }
+    }
+    if (!x.owned) {
+      __syncthreads();
+      if (tid == 0) {
+        __threadfence();  // every thread's partial before the arrival
+        const int old = atomicAdd(a.arrive2 + x.u, 1);
+        s_last = (old == i_last - i_first) ? 1 : 0;
+      }
+      __syncthreads();
+      if (s_last) {
+        __threadfence();
+        for (int o = tid; o < H * D; o += NTHR) {
+          float s2 = 0.0f;
+          for (int i = i_first; i <= i_last; ++i) {
+            const int slot = (i == i_first) ? 1 : 0;
+            s2 += __ldcg(a.ppart + (((long long)i * 2 + slot) * H) * D + o);
+          }
+          const int h = o / D, dd = o % D;
+          d.out[((long long)b * d.Hq + g * H + h) * D + dd] = s2;
+        }
+        if (tid == 0) {
+          a.arrive1[x.u] = 0;
+          a.arrive2[x.u] = 0;
+        }
+      }
+    }
+    __syncthreads();
   }
 
   // ------------------------------------------------------------ skip counts
@@ -1099,7 +1339,7 @@ __global__ void __launch_bounds__(Geo<D, KB>::kThreads, 1) fused_decode_kernel(F
       atomicAdd(a.wcounts + 1, cnt_rows);
     }
   }
-  named_barrier(kBarCons, NCONS);
+  __syncthreads();
   if (tid == 0) {
     __threadfence();
     const int old = atomicAdd(a.done, 1);

@@ -13,7 +13,7 @@ cudaError_t launch_one(const FusedArgs& a, size_t smem, int grid, cudaStream_t s
   if (e != cudaSuccess) return e;
   FusedArgs args = a;
   void* params[] = {&args};
-  return cudaLaunchCooperativeKernel((const void*)kern, dim3(grid), dim3(Geo<D, KB>::kThreads), params, smem, s);
+  return cudaLaunchCooperativeKernel((const void*)kern, dim3(grid), dim3(kThreads), params, smem, s);
 }
 
 // PAGED instantiations exist for plain decode only (one V width).

@@ -76,6 +76,7 @@ struct FusedArgs {
   int cpc_max;                   // upper bound of chunks per CTA
   int stages;                    // ring stages in use
   int ring_bytes;                // shared-memory ring size
+  int cand_cap;                  // candidate-list entries per warp (0: candidate mode off)
   long long smem_logit_floats;   // logits that fit in shared memory per CTA
   const unsigned long long* timeout_ns;  // workspace word: wait limit override (0 = default)
   int* arrive1;                  // [units] piece statistics published
@@ -86,8 +87,8 @@ struct FusedArgs {
   int* ulist;                    // [grid][cpc_max][16]
   float* glogits;                // [grid][cpc_max * chunk][H] (when shared memory is short)
   float* gstats;                 // [grid][cpc_max * 8][12] tile statistics (when there are many tiles)
-  float* qbuf;                   // [units][H][D] q * softmax_scale * log2(e)
-  float* qgsum;                  // [units][H][4] sums of qbuf per quantization group
+  float* qbuf;                   // [units][H][D] fp16 q scaled by a power of two (units past the shared slots)
+  float* qgsum;                  // [units][H][8] fold constants: q_scale * group sums of q [4], q_scale * 2^-E
   unsigned long long* wcounts;   // [2] skip-count accumulators
   int* done;                     // CTAs finished
   // paged cache (plain decode only): block table [B][pages_per_seq], T_cap = pages_per_seq * kPageTokens
