@@ -83,15 +83,15 @@ FusedLayout fused_layout(int B, int Hq, int Hkv, int T_cap, int D, int KB) {
   const long long chunks_max = units * per_unit > 0 ? units * per_unit : 1;
   L.cpc_max = (int)((chunks_max + L.grid - 1) / L.grid);
   // phase 1: as many ring stages as shared memory holds (at most kMaxStages);
-  // phase 2 reuses the ring: sparse-mode lists of kept rows (256 per warp)
-  // and V staging slots, the fallback scan's lists, or the dense-mode
+  // phase 2 reuses the ring: the sparse-mode list of kept rows (2048 per
+  // CTA), two partial outputs per warp and V staging slots, the fallback scan's lists, or the dense-mode
   // buffers, each followed by the warps' partial outputs
   const int sb = fused::stage_bytes_host(D, KB);
   const int red = fused::kWarps * L.H * D * 4;
   const int slot = D * 8 / 8 + 8 * std::max(2, D / 32);  // widest V row plus (scale, zero)
-  int lcap = 256;
+  int lcap = 2048;  // kept rows one CTA can list (more fall back to a per-piece scan)
   if ((long long)L.cpc_max * kChunk >= (1ll << fused::kCandRowBits) || L.cpc_max >= 2048) lcap = 0;
-  const int sparse = fused::kWarps * lcap * (1 + L.H) * 4 + 128 * slot + red;
+  const int sparse = (lcap * (1 + L.H) * 4 + 127) / 128 * 128 + 2 * red + 128 * slot;
   const int scan_fb = fused::kWarps * fused::kListCap * 4 * (1 + L.H) + red;
   const int dense = fused::kDenseStaging + red;
   const int phase2 = std::max(sparse, std::max(scan_fb, dense));

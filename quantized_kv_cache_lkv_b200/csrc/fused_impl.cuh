@@ -55,12 +55,12 @@ constexpr int kMaxStages = 24;   // ring stages, one chunk each
 constexpr int kListCap = 256;  // fallback scan: V-row list entries per warp per batch
 constexpr int kBatchBlocks = kListCap / 32;
 constexpr int kRec = 16;       // ints per unit-list record
-constexpr int kGatherUnroll = 4;
+constexpr int kGatherUnroll = 2;
 constexpr int kScanBlocks = 4;  // 32-row blocks whose logits one warp loads at once
 constexpr int kTsCap = 128;    // tile statistics kept in shared memory up to this many tiles
 constexpr int kQSlots = 4;     // units whose q is staged in shared memory
 constexpr int kCandRowBits = 20;  // kept-row entry: CTA-local row | unit entry << 20
-constexpr int kScanTiles = 4;      // tiles whose e-values one warp loads at once in the sparse scan
+constexpr int kScanTiles = 1;      // tiles whose e-values one warp loads at once in the sparse scan
 // Dense V pass (tau <= 0): per warp two buffers of one 32-row block each:
 // V codes (up to 6 bits), (scale, zero) of 34 rows and the block's logits.
 constexpr int kDenseCodes = 32 * 96;
@@ -73,7 +73,8 @@ constexpr unsigned kFull = 0xFFFFFFFFu;
 // per warp for the dense pass), per q slot and head A and Z[4] [1024, 1536),
 // misc ints [1536, 2560), tile statistics [2560, 8704), fp16 q of up to
 // kQSlots units [8704, 12800), unit list [12800, 16896), stage descriptors
-// [16896, 17664).
+// [16896, 17664), tile descriptors [17664, 18688), piece slot ranges
+// [18688, 19200).
 constexpr int kBarOff = 0;
 constexpr int kAzOff = 1024;
 constexpr int kMiscOff = 1536;
@@ -82,9 +83,12 @@ constexpr int kQOff = 8704;
 constexpr int kUlOff = 12800;
 constexpr int kUlCap = 64;
 constexpr int kDescOff = 16896;
-constexpr int kHeader = 17664;
+constexpr int kTinfoOff = 17664;  // per tile (valid rows | segment << 7 | unit entry << 8, first row)
+constexpr int kPrangeOff = 18688; // sparse mode: per piece the range of partial-output slots
+constexpr int kHeader = 19200;
 static_assert(2 * kMaxStages + 2 * kWarps <= 128, "barriers fit their 1024 bytes");
-static_assert(kDescOff + kMaxStages * 32 <= kHeader, "stage descriptors fit");
+static_assert(kDescOff + kMaxStages * 32 <= kTinfoOff, "stage descriptors fit");
+static_assert(kTinfoOff + kTsCap * 8 <= kPrangeOff && kPrangeOff + kUlCap * 8 <= kHeader, "tile and piece tables fit");
 static_assert(kHeader % 128 == 0, "the ring starts 128-byte aligned");
 
 // Compile-time geometry of one instantiation.
@@ -181,6 +185,14 @@ __device__ __forceinline__ bool wait_counter(const int* p, int target, uint64_t 
   }
 }
 
+// 2^x with the hardware approximation (relative error about 2^-22; flushes
+// subnormal results to zero, which only ever meets weights of 2^-126 or less).
+__device__ __forceinline__ float fast_exp2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
 // Bounded wait until the producer has issued `target` chunks (or the CTA
 // aborted); false after a timeout.
 __device__ __forceinline__ bool wait_issued(const int* issued, int target, const volatile int* abort_flag,
@@ -189,7 +201,7 @@ __device__ __forceinline__ bool wait_issued(const int* issued, int target, const
   if (*p >= target) { __threadfence_block(); return true; }
   const uint64_t t0 = global_ns();
   while (true) {
-    __nanosleep(32);
+    __nanosleep(64);
     if (*p >= target) { __threadfence_block(); return true; }
     if (*abort_flag) return false;
     if (global_ns() - t0 > limit_ns) return false;
@@ -390,7 +402,6 @@ __global__ void __launch_bounds__(kThreads, 1) fused_decode_kernel(FusedArgs a) 
   const DecodeArgs& d = a.d;
   const int units = d.B * d.Hkv;
   const int ng = D / d.G;
-  const int NT = (H * ng > 8) ? 2 : 1;
   const int S = a.stages;
   const uint64_t limit_ns = (a.timeout_ns && *a.timeout_ns) ? *a.timeout_ns : 2000000000ull;
   const int j = lane % LPR;                 // phase 2: lane's 16-channel slice of a row
@@ -413,18 +424,22 @@ __global__ void __launch_bounds__(kThreads, 1) fused_decode_kernel(FusedArgs a) 
   int& s_last = misc[6];
   int& s_ovf = misc[7];
   int& s_issued = misc[8];                            // chunks the producer has issued
+  int* s_kept = misc + 10;                            // sparse mode: kept (row, head) pairs, kept rows
+  int* s_lastu = misc + 12;                           // sparse mode: shared pieces this CTA combines
+  int* s_spiece = misc + 128;                         // sparse mode: piece in each warp's two slots
+  int* s_pdone = misc + 160;                          // sparse mode: pieces written straight out (kUlCap)
+  int* s_pref = misc + 224;                           // sparse mode: first list position of each warp (17)
   int* s_wsum = misc + 16;                            // 2 x 16 warp partials
-  int* s_coff = misc + 72;                            // sparse mode: staging offset per warp
   int* s_nw = misc + 88;                              // sparse mode: list length per warp
-  int* s_cs = misc + 104;                             // sparse mode: per warp (start, count) in a piece
 
   if (tid == 0) {
     for (int s = 0; s < kMaxStages; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], kTilesPerChunk); }
     for (int s = 0; s < 2 * kWarps; ++s) mbar_init(&dbar[s], 1);
     fence_mbar_init();
     s_total = 0; s_e0 = 0; s_nent = 0; s_abort = 0; s_carry_c = 0; s_carry_n = 0; s_last = 0; s_ovf = 0;
-    s_issued = 0;
+    s_issued = 0; s_kept[0] = 0; s_kept[1] = 0;
   }
+  for (int i = tid; i < kUlCap; i += kThreads) s_pdone[i] = 0;
   __syncthreads();
 
   // ------------------------------------------------------------ unit list
@@ -518,6 +533,8 @@ __global__ void __launch_bounds__(kThreads, 1) fused_decode_kernel(FusedArgs a) 
     tsf = tsl + a.cpc_max * 8 * 4;
   }
   for (int i = tid; i < ntile * H; i += NTHR) { tsm[i] = -INFINITY; tsl[i] = 0.0f; }
+  int2* const tinfo = reinterpret_cast<int2*>(smem_raw + kTinfoOff);  // when ntile <= kTsCap
+  for (int i = tid; i < min(ntile, kTsCap); i += NTHR) tinfo[i] = make_int2(0, 0);
   __syncthreads();  // list complete
   const int nent = s_nent;
   int* const ulist = nent <= kUlCap ? ulist_s : ulist_g;
@@ -573,9 +590,8 @@ __global__ void __launch_bounds__(kThreads, 1) fused_decode_kernel(FusedArgs a) 
   if (warp == kProducer) {
     if (lane == 0) {
       const uint64_t pol = policy_evict_first();
-      int ent = 0, c = 0;
-      for (; c < nck; ++c) {
-        const int s = c % S, k = c / S;
+      int ent = 0, c = 0, s = 0, k = 0;
+      for (; c < nck; ++c, s = (s + 1 == S) ? 0 : s + 1, k += (s == 0) ? 1 : 0) {
         if (k > 0 && !mbar_wait(&empty[s], (k - 1) & 1, limit_ns)) {
           atomicExch(d.status, kStatusTimeout);
           *abort_flag = 1;
@@ -614,144 +630,161 @@ __global__ void __launch_bounds__(kThreads, 1) fused_decode_kernel(FusedArgs a) 
       for (int s = 0; s < S && s < c; ++s) mbar_wait(&full[s], ((c - 1 - s) / S) & 1, limit_ns);
     }
   } else {
-    int bf_ent = -1;               // unit entry whose B fragments are loaded
-    uint32_t bf[2][D / 8];
-    float azA = 0.0f, azZ[2] = {0.0f, 0.0f};
-    float azA2[2] = {0.0f, 0.0f}, azZ2[2][2] = {{0.0f, 0.0f}, {0.0f, 0.0f}};
-    for (int t = warp; t < ntile; t += kConsumers) {
-      const int c = t / TPC, sub = t % TPC;
-      const int s = c % S, k = c / S;
-      if (*abort_flag) break;
-      if (!wait_issued(&s_issued, c + 1, abort_flag, limit_ns) || !mbar_wait(&full[s], k & 1, limit_ns)) {
-        if (!*abort_flag) atomicExch(d.status, kStatusTimeout);
-        *abort_flag = 1;
-        break;
-      }
-      const int* dd = desc + s * 8;
-      const int rows = max(0, min(TR, dd[2] - sub * TR));
-      if (rows == 0) {
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&empty[s]);
-        continue;
-      }
-      const int entry = dd[3];
-      if (entry != bf_ent) {
-        // B fragments and fold constants of the tile's unit
-        bf_ent = entry;
-        const int u = dd[4];
-        const __half* q16 = entry < kQSlots ? reinterpret_cast<const __half*>(smem_raw + kQOff) + entry * H * D
-                                            : reinterpret_cast<const __half*>(a.qbuf) + (long long)u * H * D;
-        const float* azb = entry < kQSlots ? reinterpret_cast<const float*>(smem_raw + kAzOff) + entry * H * 8
-                                           : a.qgsum + (long long)u * H * 8;
-        build_bfrags<D, KB, H>(q16, ng, d.G, tig, gid, bf);
-        // fold constants of the heads this lane's C columns belong to
-        if (ng == 2) {
-          const int h = tig < H ? tig : 0;
-          azA = tig < H ? azb[h * 8 + 4] : 0.0f;
-          azZ[0] = azb[h * 8 + 0]; azZ[1] = azb[h * 8 + 1];
-        } else if (ng == 1) {
-#pragma unroll
-          for (int c = 0; c < 2; ++c) {
-            const int h = 2 * tig + c < H ? 2 * tig + c : 0;
-            azA2[c] = 2 * tig + c < H ? azb[h * 8 + 4] : 0.0f;
-            azZ2[c][0] = azb[h * 8 + 0];
-          }
-        } else {
-#pragma unroll
-          for (int n2 = 0; n2 < 2; ++n2) {
-            const int hh = 2 * n2 + tig / 2;
-            const int h = hh < H ? hh : 0;
-            azA2[n2] = hh < H ? azb[h * 8 + 4] : 0.0f;
-            azZ2[n2][0] = azb[h * 8 + 2 * (tig & 1)];
-            azZ2[n2][1] = azb[h * 8 + 2 * (tig & 1) + 1];
-          }
+    // consumer warps, specialised on the number of quantization groups per
+    // row (NG): tile t = quarter t % 4 of chunk t / 4, stage (t / 4) % S
+    auto consume = [&](auto ngc) {
+      constexpr int NG = decltype(ngc)::value;
+      constexpr int NTC = (H * NG > 8) ? 2 : 1;
+      int bf_ent = -1;               // unit entry whose B fragments are loaded
+      uint32_t bf[2][D / 8];
+      // fold constants of the head(s) whose C columns this lane holds:
+      // NG 2: head tig (groups 0, 1); NG 1: heads 2 tig, 2 tig + 1;
+      // NG 4: heads tig / 2 and 2 + tig / 2 (groups 2 (tig & 1), + 1)
+      float fA[2] = {0.0f, 0.0f}, fZ[2][2] = {{0.0f, 0.0f}, {0.0f, 0.0f}};
+      int t = warp, c = warp / TPC;
+      int s = c % S, k = c / S;
+      while (t < ntile) {
+        const int sub = t % TPC;
+        if (*abort_flag) break;
+        if (!wait_issued(&s_issued, c + 1, abort_flag, limit_ns) || !mbar_wait(&full[s], k & 1, limit_ns)) {
+          if (!*abort_flag) atomicExch(d.status, kStatusTimeout);
+          *abort_flag = 1;
+          break;
         }
-      }
-      const uint8_t* stg = ring + (size_t)s * Gk::kStageBytes;
-      const uint8_t* codes = stg + sub * TR * Gk::RB;
-      const float* szs = reinterpret_cast<const float*>(stg + Gk::kStageCodes) +
-                         (((ng == 1) ? (dd[1] & 1) : 0) + sub * TR) * ng * 2;
-      // logits of head tig (base 2) for rows 16 mt + gid + 8 hf
-      float sv[4][2];
-      auto fold_pair = [&](auto mc) {
-        constexpr int MT0 = decltype(mc)::value;
-        float acc[2][2][4];
-        if (NT == 2) mma_pair<D, KB, 2, MT0>(codes, tig, gid, bf, acc);
-        else mma_pair<D, KB, 1, MT0>(codes, tig, gid, bf, acc);
+        const int* dd = desc + s * 8;
+        const int rows = max(0, min(TR, dd[2] - sub * TR));
+        const int dseg = dd[0], drow = dd[1];  // read before the stage is handed back
+        if (rows > 0) {
+          const int entry = dd[3];
+          if (entry != bf_ent) {
+            // B fragments and fold constants of the tile's unit
+            bf_ent = entry;
+            const int u = dd[4];
+            const __half* q16 = entry < kQSlots ? reinterpret_cast<const __half*>(smem_raw + kQOff) + entry * H * D
+                                                : reinterpret_cast<const __half*>(a.qbuf) + (long long)u * H * D;
+            const float* azb = entry < kQSlots ? reinterpret_cast<const float*>(smem_raw + kAzOff) + entry * H * 8
+                                               : a.qgsum + (long long)u * H * 8;
+            build_bfrags<D, KB, H>(q16, NG, d.G, tig, gid, bf);
 #pragma unroll
-        for (int m = 0; m < 2; ++m)
-#pragma unroll
-          for (int hf = 0; hf < 2; ++hf) {
-            const int r = 16 * (MT0 + m) + gid + 8 * hf;
-            const float c0 = acc[m][0][2 * hf], c1 = acc[m][0][2 * hf + 1];
-            float val;
-            if (ng == 2) {
-              const float4 s4 = *reinterpret_cast<const float4*>(szs + r * 4);
-              val = fmaf(azA, fmaf(s4.z, c1, s4.x * c0), fmaf(s4.w, azZ[1], s4.y * azZ[0]));
-            } else if (ng == 1) {
-              const float2 s2 = *reinterpret_cast<const float2*>(szs + r * 2);
-              const float v0 = fmaf(azA2[0] * s2.x, c0, s2.y * azZ2[0][0]);
-              const float v1 = fmaf(azA2[1] * s2.x, c1, s2.y * azZ2[1][0]);
-              const int src = (lane & ~3) | (tig >> 1);
-              const float u0 = __shfl_sync(kFull, v0, src), u1 = __shfl_sync(kFull, v1, src);
-              val = (tig & 1) ? u1 : u0;
-            } else {
-              const float4 s4 = *reinterpret_cast<const float4*>(szs + r * ng * 2 + 4 * (tig & 1));
-              float f[2];
-#pragma unroll
-              for (int n2 = 0; n2 < 2; ++n2) {
-                const float e0 = acc[m][n2][2 * hf], e1 = acc[m][n2][2 * hf + 1];
-                float pv = fmaf(azA2[n2], fmaf(s4.z, e1, s4.x * e0), fmaf(s4.w, azZ2[n2][1], s4.y * azZ2[n2][0]));
-                pv += __shfl_xor_sync(kFull, pv, 1);
-                f[n2] = pv;
-              }
-              const int src = (lane & ~3) | (2 * (tig & 1));
-              const float u0 = __shfl_sync(kFull, f[0], src), u1 = __shfl_sync(kFull, f[1], src);
-              val = (tig >> 1) ? u1 : u0;
+            for (int c2 = 0; c2 < 2; ++c2) {
+              const int hh = NG == 2 ? tig : (NG == 1 ? 2 * tig + c2 : 2 * c2 + tig / 2);
+              const int h = hh < H ? hh : 0;
+              const int g0 = NG == 4 ? 2 * (tig & 1) : 0;
+              fA[c2] = hh < H ? azb[h * 8 + 4] : 0.0f;
+              fZ[c2][0] = azb[h * 8 + g0];
+              fZ[c2][1] = azb[h * 8 + g0 + 1];
             }
-            sv[MT0 + m][hf] = val;
           }
-      };
-      fold_pair(std::integral_constant<int, 0>{});
-      fold_pair(std::integral_constant<int, 2>{});
-      // the stage's data is in registers: hand it back to the producer
-      fence_proxy_async_smem();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&empty[s]);
-      // tile statistics of head tig: maximum and sum of exp2 over the valid rows
-      float m = -INFINITY;
+          const uint8_t* stg = ring + (size_t)s * Gk::kStageBytes;
+          const uint8_t* codes = stg + sub * TR * Gk::RB;
+          const float* szs = reinterpret_cast<const float*>(stg + Gk::kStageCodes) +
+                             (((NG == 1) ? (drow & 1) : 0) + sub * TR) * NG * 2;
+          // logits of head tig (base 2) for rows 16 mt + gid + 8 hf
+          float sv[4][2];
+          auto fold_pair = [&](auto mc) {
+            constexpr int MT0 = decltype(mc)::value;
+            float acc[2][2][4];
+            mma_pair<D, KB, NTC, MT0>(codes, tig, gid, bf, acc);
 #pragma unroll
-      for (int mt = 0; mt < 4; ++mt)
+            for (int m = 0; m < 2; ++m)
 #pragma unroll
-        for (int hf = 0; hf < 2; ++hf)
-          if (16 * mt + gid + 8 * hf < rows) m = fmaxf(m, sv[mt][hf]);
+              for (int hf = 0; hf < 2; ++hf) {
+                const int r = 16 * (MT0 + m) + gid + 8 * hf;
+                float val;
+                if constexpr (NG == 2) {
+                  const float c0 = acc[m][0][2 * hf], c1 = acc[m][0][2 * hf + 1];
+                  const float4 s4 = *reinterpret_cast<const float4*>(szs + r * 4);
+                  val = fmaf(fA[0], fmaf(s4.z, c1, s4.x * c0), fmaf(s4.w, fZ[0][1], s4.y * fZ[0][0]));
+                } else if constexpr (NG == 1) {
+                  const float c0 = acc[m][0][2 * hf], c1 = acc[m][0][2 * hf + 1];
+                  const float2 s2 = *reinterpret_cast<const float2*>(szs + r * 2);
+                  const float v0 = fmaf(fA[0] * s2.x, c0, s2.y * fZ[0][0]);
+                  const float v1 = fmaf(fA[1] * s2.x, c1, s2.y * fZ[1][0]);
+                  const int src = (lane & ~3) | (tig >> 1);
+                  const float u0 = __shfl_sync(kFull, v0, src), u1 = __shfl_sync(kFull, v1, src);
+                  val = (tig & 1) ? u1 : u0;
+                } else {
+                  const float4 s4 = *reinterpret_cast<const float4*>(szs + r * NG * 2 + 4 * (tig & 1));
+                  float f[2];
 #pragma unroll
-      for (int off = 4; off < 32; off <<= 1) m = fmaxf(m, __shfl_xor_sync(kFull, m, off));
-      float l = 0.0f;
+                  for (int n2 = 0; n2 < 2; ++n2) {
+                    const float e0 = acc[m][n2][2 * hf], e1 = acc[m][n2][2 * hf + 1];
+                    float pv = fmaf(fA[n2], fmaf(s4.z, e1, s4.x * e0), fmaf(s4.w, fZ[n2][1], s4.y * fZ[n2][0]));
+                    pv += __shfl_xor_sync(kFull, pv, 1);
+                    f[n2] = pv;
+                  }
+                  const int src = (lane & ~3) | (2 * (tig & 1));
+                  const float u0 = __shfl_sync(kFull, f[0], src), u1 = __shfl_sync(kFull, f[1], src);
+                  val = (tig >> 1) ? u1 : u0;
+                }
+                sv[MT0 + m][hf] = val;
+              }
+          };
+          fold_pair(std::integral_constant<int, 0>{});
+          fold_pair(std::integral_constant<int, 2>{});
+          // the stage's data is in registers: hand it back to the producer
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&empty[s]);
+          // tile statistics of head tig: maximum and sum of exp2 over the valid rows
+          float m = -INFINITY, l = 0.0f;
+          if (rows == TR) {
 #pragma unroll
-      for (int mt = 0; mt < 4; ++mt)
+            for (int mt = 0; mt < 4; ++mt) m = fmaxf(m, fmaxf(sv[mt][0], sv[mt][1]));
+          } else {
 #pragma unroll
-        for (int hf = 0; hf < 2; ++hf) {
-          const bool ok = 16 * mt + gid + 8 * hf < rows;
-          sv[mt][hf] = ok ? exp2f(sv[mt][hf] - m) : 0.0f;
-          l += sv[mt][hf];
-        }
+            for (int mt = 0; mt < 4; ++mt)
 #pragma unroll
-      for (int off = 4; off < 32; off <<= 1) l += __shfl_xor_sync(kFull, l, off);
-      if (tig < H) {
-#pragma unroll
-        for (int mt = 0; mt < 4; ++mt)
-#pragma unroll
-          for (int hf = 0; hf < 2; ++hf) {
-            const int r = 16 * mt + gid + 8 * hf;
-            if (r < rows) lg[((long long)t * TR + r) * H + tig] = sv[mt][hf];
+              for (int hf = 0; hf < 2; ++hf)
+                if (16 * mt + gid + 8 * hf < rows) m = fmaxf(m, sv[mt][hf]);
           }
-        if (gid == 0) {
-          tsm[t * H + tig] = m;
-          tsl[t * H + tig] = l;
+#pragma unroll
+          for (int off = 4; off < 32; off <<= 1) m = fmaxf(m, __shfl_xor_sync(kFull, m, off));
+#pragma unroll
+          for (int mt = 0; mt < 4; ++mt)
+#pragma unroll
+            for (int hf = 0; hf < 2; ++hf) {
+              const float e = fast_exp2(sv[mt][hf] - m);
+              sv[mt][hf] = (rows == TR || 16 * mt + gid + 8 * hf < rows) ? e : 0.0f;
+              l += sv[mt][hf];
+            }
+#pragma unroll
+          for (int off = 4; off < 32; off <<= 1) l += __shfl_xor_sync(kFull, l, off);
+          if (tig < H) {
+            float* lgt = lg + (size_t)t * TR * H + gid * H + tig;
+            if (rows == TR) {
+#pragma unroll
+              for (int mt = 0; mt < 4; ++mt)
+#pragma unroll
+                for (int hf = 0; hf < 2; ++hf) lgt[(16 * mt + 8 * hf) * H] = sv[mt][hf];
+            } else {
+#pragma unroll
+              for (int mt = 0; mt < 4; ++mt)
+#pragma unroll
+                for (int hf = 0; hf < 2; ++hf)
+                  if (16 * mt + gid + 8 * hf < rows) lgt[(16 * mt + 8 * hf) * H] = sv[mt][hf];
+            }
+            if (gid == 0) {
+              tsm[t * H + tig] = m;
+              tsl[t * H + tig] = l;
+            }
+          }
+          if (lane == 0 && t < kTsCap) tinfo[t] = make_int2(rows | (dseg << 7) | (entry << 8), drow + sub * TR);
+        } else {
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&empty[s]);
         }
+        // this warp's next tile: the chunk index advances by 3 or 4
+        t += kConsumers;
+        const int c2 = t / TPC;
+        s += c2 - c;
+        while (s >= S) { s -= S; ++k; }
+        c = c2;
       }
-    }
+    };
+    if (ng == 2) consume(std::integral_constant<int, 2>{});
+    else if (ng == 1) consume(std::integral_constant<int, 1>{});
+    else if constexpr (D == 128) consume(std::integral_constant<int, 4>{});
   }
   __syncthreads();
   // After a timed-out wait a bulk copy may still land in the ring, which
@@ -760,20 +793,26 @@ __global__ void __launch_bounds__(kThreads, 1) fused_decode_kernel(FusedArgs a) 
   const int n_work = aborted ? 0 : nent;
 
   // ------------------------------------------------------------ statistics
-  // piece statistics: the CTA's tiles of each unit, merged
-  for (int e = warp; e < n_work; e += CW) {
+  // piece statistics: the CTA's tiles of each unit, merged -- one warp per
+  // (piece, head): the maximum first, then the rescaled sum
+  for (int task = warp; task < n_work * H; task += CW) {
+    const int e = task / H, h = task % H;
     int* rec = ulist + e * kRec;
     const Unit x = load_unit(rec);
     const int ta = (max(x.cb, k0) - k0) * TPC, tb = (min(x.cb + x.nc, k1) - k0) * TPC;
-#pragma unroll 1
-    for (int h = 0; h < H; ++h) {
+    {
       float m = -INFINITY, l = 0.0f;
-      for (int t2 = ta + lane; t2 < tb; t2 += 32) merge_ml(m, l, tsm[t2 * H + h], tsl[t2 * H + h]);
+      for (int t2 = ta + lane; t2 < tb; t2 += 32) m = fmaxf(m, tsm[t2 * H + h]);
 #pragma unroll
-      for (int off = 16; off >= 1; off >>= 1) {
-        const float m2 = __shfl_xor_sync(kFull, m, off), l2 = __shfl_xor_sync(kFull, l, off);
-        merge_ml(m, l, m2, l2);
+      for (int off = 16; off >= 1; off >>= 1) m = fmaxf(m, __shfl_xor_sync(kFull, m, off));
+      if (m > -INFINITY) {
+        for (int t2 = ta + lane; t2 < tb; t2 += 32) {
+          const float mt = tsm[t2 * H + h];
+          if (mt > -INFINITY) l = fmaf(tsl[t2 * H + h], exp2f(mt - m), l);
+        }
       }
+#pragma unroll
+      for (int off = 16; off >= 1; off >>= 1) l += __shfl_xor_sync(kFull, l, off);
       if (lane == 0) {
         reinterpret_cast<float*>(rec + 8)[2 * h] = m;
         reinterpret_cast<float*>(rec + 8)[2 * h + 1] = l;
@@ -849,124 +888,197 @@ __global__ void __launch_bounds__(kThreads, 1) fused_decode_kernel(FusedArgs a) 
 
   // ------------------------------------------------------------ phase 2
   // phase-2 shared memory (in the ring).  Sparse mode: per warp its kept
-  // rows [lcap] and their weights [lcap][H], then one staging slot per kept
-  // V row.  Scan mode: kept-row lists [CW][kListCap] and weights; dense
-  // mode: the V staging buffers.  The warps' partial outputs [CW][H][D]
+  // rows [lcap], their weights [lcap][H] and staging slots [lcap]; the
+  // warps' partial outputs [CW][2][H][D]; then one staging slot per kept V
+  // row.  Scan mode: kept-row lists [CW][kListCap] and weights; dense mode:
+  // the V staging buffers; for both, the warps' partial outputs [CW][H][D]
   // are last.
   const int red_off = a.ring_bytes - CW * H * D * 4;
   float* red = reinterpret_cast<float*>(ring + red_off);
   // the dense V pass applies when every row is kept and the V rows fit its buffers
   const bool dense = d.tau <= 0.0f && VB0 <= 6 && VB1 <= 6;
   const int lcap = a.cand_cap;
-  const bool sparse_try = !dense && lcap > 0;
+  const bool sparse_try = !dense && lcap > 0 && n_work > 0 && nent <= kUlCap;
   unsigned long long cnt_heads = 0, cnt_rows = 0;
   uint8_t* const smask = d.skip_mask;
   float* const mass_out = d.mass;
   constexpr int kSzSlot = 8 * ((D / 32) > 2 ? (D / 32) : 2);
   constexpr int kVRowMax = D * (VB0 > VB1 ? VB0 : VB1) / 8;
   constexpr int kSlotBytes = kVRowMax + kSzSlot;
-  int* const lrows = reinterpret_cast<int*>(ring) + warp * lcap * (1 + H);   // this warp's kept rows
-  float* const lw = reinterpret_cast<float*>(lrows + lcap);                   // ... and their weights
-  const int lists_bytes = CW * lcap * (1 + H) * 4;
-  int n_kept = 0;
-  if (sparse_try && n_work > 0) {
-    // 1. every row of the CTA: p = e * factor; the skip decision, the skip
-    //    mask, the attention mass and the counts; rows some head keeps go to
-    //    the warp's list with their weights, in row order.  Warp w scans a
-    //    contiguous run of the CTA's tiles, kScanTiles tiles in flight.
-    const int t_lo = (ntile * warp) / CW, t_hi = (ntile * (warp + 1)) / CW;
-    int ent = 0;
-    for (int t0 = t_lo; t0 < t_hi; t0 += kScanTiles) {
-      float ev[kScanTiles][2][H];
-      int nrow[kScanTiles], tent[kScanTiles], tpos[kScanTiles];
-#pragma unroll
-      for (int u = 0; u < kScanTiles; ++u) {
-        const int t = t0 + u;
-        nrow[u] = 0;
-        tent[u] = 0;
-        tpos[u] = 0;
-        if (t < t_hi) {
+  // sparse mode layout in the ring: the CTA's kept-row list [lcap] rows and
+  // [lcap][H] weights first; behind it the e-values of a round of tiles
+  // during the scan, then the warps' partial outputs [CW][2][H][D] and the
+  // V staging slots during the accumulation
+  int* const krow = reinterpret_cast<int*>(ring);             // CTA-local row | unit entry << 20
+  float* const kw = reinterpret_cast<float*>(krow + lcap);    // weights p (0 for a skipping head)
+  const int lists_bytes = (lcap * (1 + H) * 4 + 127) / 128 * 128;
+  float* const ebuf = reinterpret_cast<float*>(ring + lists_bytes);
+  const int round_tiles = sparse_try ? (a.ring_bytes - lists_bytes) / (TR * H * 4) : 0;
+  float* const red2 = reinterpret_cast<float*>(ring + lists_bytes);      // [CW][2][H][D]
+  const int red2_bytes = CW * 2 * H * D * 4;
+  uint8_t* const stage0 = ring + lists_bytes + red2_bytes;
+  const int stage_slots = sparse_try ? max(0, (a.ring_bytes - lists_bytes - red2_bytes) / kSlotBytes) : 0;
+  uint32_t kh_lane = 0, kr_lane = 0;  // kept (row, head) pairs and kept rows seen by this lane
+  if (sparse_try) {
+    // 1. every row of the CTA, in rounds of round_tiles tiles: the round's
+    //    e-values come into shared memory in one go (each warp copies its
+    //    own contiguous run of tiles); pass A takes every skip decision,
+    //    writes the skip mask and attention mass and counts the kept rows;
+    //    pass B lists them, in row order, in the CTA-wide list at offsets
+    //    from the counts, with their weights, and starts bringing their V
+    //    rows into L2.
+    int kbase = 0;
+    const int wcap = lcap / CW;  // list entries of one warp
+    int n_w = 0;                 // this warp's kept rows so far
+    for (int T0 = 0; T0 < ntile; T0 += round_tiles) {
+      const int T1 = min(ntile, T0 + round_tiles);
+      const int t_lo = T0 + ((T1 - T0) * warp) / CW, t_hi = T0 + ((T1 - T0) * (warp + 1)) / CW;
+      // tile t: valid rows, entry, segment, position
+      auto tile_info = [&](int t, int& nrow, int& ent, int& seg, int& pos) {
+        if (t < kTsCap) {
+          const int2 ti = tinfo[t];
+          nrow = ti.x & 127; seg = (ti.x >> 7) & 1; ent = ti.x >> 8; pos = ti.y;
+        } else {
           const int g = k0 + t / TPC;
-          while (ent + 1 < nent && ulist[(ent + 1) * kRec + 1] <= g) ++ent;
-          const Unit x = load_unit(ulist + ent * kRec);
+          int lo2 = 0, hi2 = nent - 1;
+          while (lo2 < hi2) { const int mid = (lo2 + hi2 + 1) >> 1; if (ulist[mid * kRec + 1] <= g) lo2 = mid; else hi2 = mid - 1; }
+          const Unit x = load_unit(ulist + lo2 * kRec);
           const ChunkRows cr = chunk_rows(x, g - x.cb);
-          nrow[u] = max(0, min(TR, cr.rows - (t % TPC) * TR));
-          tent[u] = ent;
-          tpos[u] = cr.row0 + (t % TPC) * TR;  // position of the tile's first row (plain decode)
-#pragma unroll
-          for (int hf = 0; hf < 2; ++hf)
-            if (hf * 32 + lane < nrow[u]) ldcg_heads<H>(lg + ((long long)t * TR + hf * 32 + lane) * H, ev[u][hf]);
+          nrow = max(0, min(TR, cr.rows - (t % TPC) * TR)); ent = lo2; seg = cr.seg; pos = cr.row0 + (t % TPC) * TR;
         }
+      };
+      // copy: the e-values of this warp's tiles (a tile's rows are one run
+      // of nrow * H floats in the workspace, 16-byte aligned)
+#pragma unroll 1
+      for (int t = t_lo; t < t_hi; ++t) {
+        int nrow, ent, seg, pos;
+        tile_info(t, nrow, ent, seg, pos);
+        const int nchk = (nrow * H * 4 + 15) / 16;
+        const uint8_t* src = reinterpret_cast<const uint8_t*>(lg + (long long)t * TR * H);
+        uint8_t* dst = reinterpret_cast<uint8_t*>(ebuf + (t - T0) * TR * H);
+        for (int q = lane; q < nchk; q += 32) cp_async16(dst + q * 16, src + q * 16);
       }
-#pragma unroll
-      for (int u = 0; u < kScanTiles; ++u) {
-        if (nrow[u] == 0) continue;  // the same for the whole warp
-        const int t = t0 + u;
+      cp_async_wait_all();
+      __syncwarp();
+      // one pass: the skip decisions; kept rows (with their weights p, 0 for
+      // a head that skips) go to the warp's list, in row order
+      const float tau = d.tau;
+#pragma unroll 1
+      for (int t = t_lo; t < t_hi; ++t) {
+        int nrow, ent, seg, pos;
+        tile_info(t, nrow, ent, seg, pos);
+        if (nrow == 0) continue;  // the same for the whole warp
         float f[H];
         lds_heads<H>(tsf + t * H, f);
-        const Unit x = load_unit(ulist + tent[u] * kRec);
-        const int b = x.u / d.Hkv, g = x.u % d.Hkv;
+        const float* et = ebuf + (t - T0) * TR * H;
 #pragma unroll
         for (int hf = 0; hf < 2; ++hf) {
           const int r = hf * 32 + lane;
-          bool need = false;
-          float wgt[H];
-          if (r < nrow[u]) {
-            float ms = 0.0f;
+          float ev[H];
 #pragma unroll
-            for (int h = 0; h < H; ++h) {
-              const float p = ev[u][hf][h] * f[h];
-              const bool keep = !(p < d.tau);
-              wgt[h] = keep ? p : 0.0f;
-              need |= keep;
-              cnt_heads += keep ? 0u : 1u;
-              ms += p;
-              if (smask) smask[((long long)b * d.Hq + g * H + h) * d.T_cap + tpos[u] + r] = keep ? 0 : 1;
-            }
-            cnt_rows += need ? 0u : 1u;
-            if (mass_out) mass_out[((long long)b * d.Hkv + g) * d.T_cap + tpos[u] + r] = ms * (1.0f / H);
+          for (int h = 0; h < H; ++h) ev[h] = 0.0f;
+          if (r < nrow) lds_heads<H>(et + r * H, ev);
+          float wgt[H];
+          bool need = false;
+          uint32_t kh = 0, kbits = 0;
+#pragma unroll
+          const bool valid = r < nrow;
+          for (int h = 0; h < H; ++h) {
+            const float p = ev[h] * f[h];
+            const bool keep = valid && !(p < tau);
+            wgt[h] = keep ? p : 0.0f;
+            need |= keep;
+            kh += keep ? 1u : 0u;
+            kbits |= keep ? (1u << h) : 0u;
           }
+          kh_lane += kh;
+          kr_lane += need ? 1u : 0u;
           const unsigned bal = __ballot_sync(kFull, need);
-          const int o = n_kept + __popc(bal & ((1u << lane) - 1u));
-          if (need && o < lcap) {
-            lrows[o] = (t * TR + r) | (tent[u] << kCandRowBits);
-            store_heads<H>(lw + o * H, wgt);
+          if (need) {
+            const int o = n_w + __popc(bal & ((1u << lane) - 1u));
+            if (o < wcap) {
+              krow[warp * wcap + o] = (t * TR + r) | (ent << kCandRowBits);
+              store_heads<H>(kw + (warp * wcap + o) * H, wgt);
+              const int uu = ulist[ent * kRec];
+              const int vr = pos + r;
+              const int rbv = seg ? D * VB1 / 8 : D * VB0 / 8;
+              const long long pr = PAGED ? unit_row<PAGED>(a, uu, vr) : (long long)uu * d.T_cap + vr;
+              prefetch_l2(d.vc[seg] + pr * rbv);
+              prefetch_l2(d.vsz[seg] + pr * ng * 2);
+            }
           }
-          n_kept += __popc(bal);
+          n_w += __popc(bal);
+          if (smask != nullptr || mass_out != nullptr) {
+            // the optional outputs: skip mask and the group's mean attention
+            const int uu = ulist[ent * kRec];
+            const int b = uu / d.Hkv, g = uu % d.Hkv;
+            if (r < nrow) {
+              float ms = 0.0f;
+#pragma unroll
+              for (int h = 0; h < H; ++h) {
+                ms += ev[h] * f[h];
+                if (smask) smask[((long long)b * d.Hq + g * H + h) * d.T_cap + pos + r] = ((kbits >> h) & 1u) ? 0 : 1;
+              }
+              if (mass_out) mass_out[((long long)b * d.Hkv + g) * d.T_cap + pos + r] = ms * (1.0f / H);
+            }
+          }
         }
       }
+      __syncthreads();  // the next round reuses the e-value buffer
     }
-    if (n_kept > lcap) s_ovf = 1;
+    if (n_w > wcap) s_ovf = 1;
+    if (lane == 0) s_nw[warp] = min(n_w, wcap);
+    (void)kbase;
   }
   __syncthreads();
-  const bool sparse = sparse_try && n_work > 0 && !*static_cast<volatile int*>(&s_ovf);
-  if (sparse_try && !sparse) { cnt_heads = 0; cnt_rows = 0; }  // the scan mode below counts again
-  const int stage_slots = sparse ? (red_off - lists_bytes) / kSlotBytes : 0;
+  const bool sparse = sparse_try && !*static_cast<volatile int*>(&s_ovf);
   if (sparse) {
-    // 2. kept V rows into their staging slots with 16-byte asynchronous
-    //    copies (warp w's rows take slots [off_w, off_w + n_w)); rows past
-    //    the capacity are read from global memory when accumulated
-    if (lane == 0) s_nw[warp] = n_kept;
+    if (tid == 0) {
+      int acc_n = 0;
+      for (int w2 = 0; w2 < CW; ++w2) { s_pref[w2] = acc_n; acc_n += s_nw[w2]; }
+      s_pref[CW] = acc_n;
+    }
+    // counts: every valid (row, head) of the CTA minus the kept ones
+#pragma unroll
+    for (int off = 16; off >= 1; off >>= 1) {
+      kh_lane += __shfl_xor_sync(kFull, kh_lane, off);
+      kr_lane += __shfl_xor_sync(kFull, kr_lane, off);
+    }
+    if (lane == 0) { atomicAdd(&s_kept[0], (int)kh_lane); atomicAdd(&s_kept[1], (int)kr_lane); }
+    if (tid < CW * 2) s_spiece[tid] = -1;
+    // 2. the CTA's kept rows are split evenly over the warps; each warp
+    //    brings its rows' V codes and (scale, zero) into its staging slots
+    //    (slot = list position; rows past the slots are read from global
+    //    memory), then accumulates.  A warp's share is cut where the unit
+    //    piece changes; the first and last pieces of the share go to the
+    //    warp's two partial-output slots, pieces in between (whole pieces,
+    //    owned by this CTA) straight to the output.
     __syncthreads();
-    int off_w = 0;
-    for (int w2 = 0; w2 < warp; ++w2) off_w += s_nw[w2];
-    if (lane == 0) s_coff[warp] = off_w;
-    const int n_stage = max(0, min(n_kept, stage_slots - off_w));
+    const int n_all = s_pref[CW];
+    const int wcap = lcap / CW;
+    // physical list index of CTA list position gidx (warp lists in warp order)
+    auto pidx = [&](int gidx) {
+      int lo2 = 0, hi2 = CW - 1;
+      while (lo2 < hi2) { const int mid = (lo2 + hi2 + 1) >> 1; if (s_pref[mid] <= gidx) lo2 = mid; else hi2 = mid - 1; }
+      return lo2 * wcap + gidx - s_pref[lo2];
+    };
+    const int per = ((n_all + CW - 1) / CW + RPW - 1) / RPW * RPW;
+    const int g_lo = min(n_all, warp * per), g_hi = min(n_all, g_lo + per);
     constexpr int kMaxChunks = kVRowMax / 16 + kSzSlot / 16;
-    for (int q = lane; q < n_stage * kMaxChunks; q += 32) {
-      const int i = q / kMaxChunks, c = q % kMaxChunks;
-      const int rowe = lrows[i];
+    for (int q = lane; q < (min(g_hi, stage_slots) - g_lo) * kMaxChunks; q += 32) {
+      const int i = g_lo + q / kMaxChunks, c = q % kMaxChunks;
+      const int rowe = krow[pidx(i)];
       const int ent = rowe >> kCandRowBits, row = rowe & ((1 << kCandRowBits) - 1);
       const Unit x = load_unit(ulist + ent * kRec);
       const ChunkRows cr = chunk_rows(x, (k0 + row / kChunk) - x.cb);
       const int vr = cr.row0 + row % kChunk;
       const int rbv = cr.seg ? D * VB1 / 8 : D * VB0 / 8;
       const int szb = ng == 1 ? 16 : ng * 8;
-      uint8_t* slot = ring + lists_bytes + (size_t)(off_w + i) * kSlotBytes;
+      uint8_t* slot = stage0 + (size_t)i * kSlotBytes;
       if (c * 16 < rbv) {
         const long long pr = PAGED ? unit_row<PAGED>(a, x.u, vr) : (long long)x.u * d.T_cap + vr;
         cp_async16(slot + c * 16, d.vc[cr.seg] + pr * rbv + c * 16);
-      } else if ((c - kVRowMax / 16) * 16 < szb && c >= kVRowMax / 16) {
+      } else if (c >= kVRowMax / 16 && (c - kVRowMax / 16) * 16 < szb) {
         const int cz = c - kVRowMax / 16;
         const int vr0 = ng == 1 ? (vr & ~1) : vr;
         const long long pr0 = PAGED ? unit_row<PAGED>(a, x.u, vr0) : (long long)x.u * d.T_cap + vr0;
@@ -974,12 +1086,181 @@ __global__ void __launch_bounds__(kThreads, 1) fused_decode_kernel(FusedArgs a) 
       }
     }
     cp_async_wait_all();
+    __syncwarp();
+    int seg_lo = g_lo;
+    while (seg_lo < g_hi) {
+      // the segment [seg_lo, seg_hi): the share's rows of one piece
+      const int pc = krow[pidx(seg_lo)] >> kCandRowBits;
+      int seg_hi;
+      {
+        int lo2 = seg_lo + 1, hi2 = g_hi;  // first index of a later piece
+        while (lo2 < hi2) { const int mid = (lo2 + hi2) >> 1; if ((krow[pidx(mid)] >> kCandRowBits) == pc) lo2 = mid + 1; else hi2 = mid; }
+        seg_hi = lo2;
+      }
+      const Unit x = load_unit(ulist + pc * kRec);
+      float2 acc[H][8];
+      float Z[H];
+#pragma unroll
+      for (int h = 0; h < H; ++h) {
+        Z[h] = 0.0f;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) acc[h][i] = make_float2(0.0f, 0.0f);
+      }
+      int sw = 0;
+      {
+        const int g0 = min(seg_lo + lane / LPR, n_all - 1);
+        int lo2 = 0, hi2 = CW - 1;
+        while (lo2 < hi2) { const int mid = (lo2 + hi2 + 1) >> 1; if (s_pref[mid] <= g0) lo2 = mid; else hi2 = mid - 1; }
+        sw = lo2;
+      }
+      for (int i0 = seg_lo; i0 < seg_hi; i0 += RPW) {
+        const int gidx = i0 + lane / LPR;
+        if (gidx >= seg_hi) break;  // the lanes of a row agree
+        while (gidx >= s_pref[sw + 1]) ++sw;
+        float wgt[H];
+        const int pi = sw * wcap + gidx - s_pref[sw];
+        lds_heads<H>(kw + pi * H, wgt);
+        const int row = krow[pi] & ((1 << kCandRowBits) - 1);
+        const int v = (k0 - x.cb) * kChunk + row;
+        const ChunkRows cr = chunk_rows(x, v / kChunk);
+        const int vr = cr.row0 + v % kChunk;
+        LaneWords<VB0> w0;
+        LaneWords<(VB0 == VB1) ? 2 : VB1> w1;
+        float2 sz;
+        if (gidx < stage_slots) {
+          const uint8_t* src = stage0 + (size_t)gidx * kSlotBytes;
+          const float* szp = reinterpret_cast<const float*>(src + kVRowMax) + (ng == 1 ? (vr & 1) * 2 : gi * 2);
+          sz = *reinterpret_cast<const float2*>(szp);
+          if (cr.seg == 0 || VB0 == VB1) lds_lane_words<VB0>(src + j * 2 * VB0, w0);
+          else if constexpr (VB0 != VB1) lds_lane_words<VB1>(src + j * 2 * VB1, w1);
+        } else {
+          const long long pr = PAGED ? unit_row<PAGED>(a, x.u, vr) : (long long)x.u * d.T_cap + vr;
+          if (cr.seg == 0 || VB0 == VB1) ldg_v<VB0>(d.vc[cr.seg] + pr * (D * VB0 / 8), d.vsz[cr.seg] + pr * ng * 2, j, gi, w0, sz);
+          else if constexpr (VB0 != VB1) ldg_v<VB1>(d.vc[1] + pr * (D * VB1 / 8), d.vsz[1] + pr * ng * 2, j, gi, w1, sz);
+        }
+        if (cr.seg == 0 || VB0 == VB1) accumulate_v<H, VB0>(w0, sz, wgt, acc, Z);
+        else if constexpr (VB0 != VB1) accumulate_v<H, VB1>(w1, sz, wgt, acc, Z);
+      }
+      // add the warp's row slots with shuffles
+#pragma unroll
+      for (int h = 0; h < H; ++h)
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          float2 v2 = make_float2(acc[h][i].x + Z[h], acc[h][i].y + Z[h]);
+#pragma unroll
+          for (int off = LPR; off < 32; off <<= 1) {
+            v2.x += __shfl_xor_sync(kFull, v2.x, off);
+            v2.y += __shfl_xor_sync(kFull, v2.y, off);
+          }
+          acc[h][i] = v2;
+        }
+      const bool first = seg_lo == g_lo, last = seg_hi == g_hi;
+      if (first || last) {
+        const int k = first ? 0 : 1;
+        if (lane < LPR) {
+#pragma unroll
+          for (int h = 0; h < H; ++h)
+#pragma unroll
+            for (int i = 0; i < 8; i += 2)
+              *reinterpret_cast<float4*>(red2 + ((warp * 2 + k) * H + h) * D + j * kDimsPerLane + 2 * i) =
+                  make_float4(acc[h][i].x, acc[h][i].y, acc[h][i + 1].x, acc[h][i + 1].y);
+        }
+        if (lane == 0) s_spiece[warp * 2 + k] = pc;
+      } else if (lane < LPR) {
+        // a whole piece between two others: owned by this CTA, and only this warp holds its rows
+        const int b = x.u / d.Hkv, g = x.u % d.Hkv;
+#pragma unroll
+        for (int h = 0; h < H; ++h)
+#pragma unroll
+          for (int i = 0; i < 8; i += 2)
+            *reinterpret_cast<float4*>(d.out + ((long long)b * d.Hq + g * H + h) * D + j * kDimsPerLane + 2 * i) =
+                make_float4(acc[h][i].x, acc[h][i].y, acc[h][i + 1].x, acc[h][i + 1].y);
+        if (lane == 0) s_pdone[pc] = 1;
+      }
+      seg_lo = seg_hi;
+    }
     __syncthreads();
+    // 3. the output of every piece not yet written: the sum of the slots
+    //    that hold it, in warp order (zero when no head kept any row); a
+    //    piece's slots lie in one range of the warp-ordered slot list
+    int2* const prange = reinterpret_cast<int2*>(smem_raw + kPrangeOff);
+    for (int e = tid; e < n_work; e += NTHR) {
+      int k_lo = CW * 2, k_hi = 0;
+      for (int k2 = 0; k2 < CW * 2; ++k2)
+        if (s_spiece[k2] == e) { k_lo = min(k_lo, k2); k_hi = k2 + 1; }
+      prange[e] = make_int2(k_lo, k_hi);
+    }
+    __syncthreads();
+    for (int e = 0; e < n_work; ++e) {
+      if (s_pdone[e]) continue;
+      const int2 kr = prange[e];
+      const Unit x = load_unit(ulist + e * kRec);
+      const int b = x.u / d.Hkv, g = x.u % d.Hkv;
+      for (int o = tid; o < H * D; o += NTHR) {
+        float s2 = 0.0f;
+        for (int k2 = kr.x; k2 < kr.y; ++k2)
+          if (s_spiece[k2] == e) s2 += red2[k2 * H * D + o];
+        const int h = o / D, dd = o % D;
+        if (x.owned) {
+          d.out[((long long)b * d.Hq + g * H + h) * D + dd] = s2;
+        } else {
+          if (e == 0) a.ppart[(((long long)cta * 2 + 0) * H + h) * D + dd] = s2;
+          if (e == nent - 1) a.ppart[(((long long)cta * 2 + 1) * H + h) * D + dd] = s2;
+        }
+      }
+    }
+    __syncthreads();
+    // 4. shared units: publish the partial; the last CTA to arrive adds them
+    if (tid == 0) {
+      __threadfence();  // every thread's partial before the arrivals
+      for (int c = 0; c < 2; ++c) {
+        const int e = c == 0 ? 0 : nent - 1;
+        if (c == 1 && nent == 1) break;
+        const Unit x = load_unit(ulist + e * kRec);
+        s_lastu[c] = -1;
+        if (x.owned) continue;
+        const int i_first = x.cb / cpc, i_last = (x.cb + x.nc - 1) / cpc;
+        const int old = atomicAdd(a.arrive2 + x.u, 1);
+        if (old == i_last - i_first) s_lastu[c] = e;
+      }
+    }
+    __syncthreads();
+    for (int c = 0; c < 2; ++c) {
+      const int e = s_lastu[c];
+      if (e < 0 || (c == 1 && nent == 1)) continue;
+      __threadfence();
+      const Unit x = load_unit(ulist + e * kRec);
+      const int i_first = x.cb / cpc, i_last = (x.cb + x.nc - 1) / cpc;
+      const int b = x.u / d.Hkv, g = x.u % d.Hkv;
+      for (int o = tid; o < H * D; o += NTHR) {
+        float s2 = 0.0f;
+        for (int i = i_first; i <= i_last; ++i) {
+          const int slot = (i == i_first) ? 1 : 0;
+          s2 += __ldcg(a.ppart + (((long long)i * 2 + slot) * H) * D + o);
+        }
+        d.out[((long long)b * d.Hq + g * H + o / D) * D + o % D] = s2;
+      }
+      if (tid == 0) {
+        a.arrive1[x.u] = 0;
+        a.arrive2[x.u] = 0;
+      }
+    }
+    __syncthreads();
+    if (tid == 0) {
+      long long valid = 0;
+      for (int e = 0; e < n_work; ++e) {
+        const Unit x = load_unit(ulist + e * kRec);
+        const int ga = max(x.cb, k0), gb = min(x.cb + x.nc, k1);
+        for (int c = ga; c < gb; ++c) valid += chunk_rows(x, c - x.cb).rows;
+      }
+      cnt_heads = (unsigned long long)(valid * H - s_kept[0]);
+      cnt_rows = (unsigned long long)(valid - s_kept[1]);
+    }
   }
   int* lists = reinterpret_cast<int*>(ring);
   float* wts = reinterpret_cast<float*>(ring + kWarps * kListCap * 4);
   int dense_uses[2] = {0, 0};
-  for (int e = 0; e < n_work; ++e) {
+  for (int e = 0; e < (sparse ? 0 : n_work); ++e) {
     int* rec = ulist + e * kRec;
     const Unit x = load_unit(rec);
     const int b = x.u / d.Hkv, g = x.u % d.Hkv;
@@ -997,59 +1278,7 @@ __global__ void __launch_bounds__(kThreads, 1) fused_decode_kernel(FusedArgs a) 
 #pragma unroll
       for (int i = 0; i < 8; ++i) acc[h][i] = make_float2(0.0f, 0.0f);
     }
-    if (sparse) {
-      // this warp's kept rows of the piece: a contiguous run of its list
-      int lo, hi;
-      {
-        const int nk = min(n_kept, lcap);
-        int a0 = 0, a1 = nk;  // first entry of unit entry >= e
-        while (a0 < a1) { const int mid = (a0 + a1) >> 1; if ((lrows[mid] >> kCandRowBits) < e) a0 = mid + 1; else a1 = mid; }
-        lo = a0;
-        a1 = nk;              // first entry of unit entry > e
-        while (a0 < a1) { const int mid = (a0 + a1) >> 1; if ((lrows[mid] >> kCandRowBits) <= e) a0 = mid + 1; else a1 = mid; }
-        hi = a0;
-      }
-      if (lane == 0) { s_cs[2 * warp] = lo; s_cs[2 * warp + 1] = hi - lo; }
-      __syncthreads();
-      // the piece's kept rows of all warps, split evenly over the warps
-      int n_all = 0;
-#pragma unroll
-      for (int w2 = 0; w2 < CW; ++w2) n_all += s_cs[2 * w2 + 1];
-      const int per = ((n_all + CW - 1) / CW + RPW - 1) / RPW * RPW;
-      const int g_lo = min(n_all, warp * per), g_hi = min(n_all, g_lo + per);
-      int sw = 0, sbase = 0;
-      for (int i0 = g_lo; i0 < g_hi; i0 += RPW) {
-        const int gidx = i0 + lane / LPR;
-        if (gidx >= g_hi) continue;  // the lanes of a row agree
-        while (gidx >= sbase + s_cs[2 * sw + 1]) { sbase += s_cs[2 * sw + 1]; ++sw; }
-        const int li = s_cs[2 * sw] + gidx - sbase;   // entry of warp sw's list
-        const int* lr = reinterpret_cast<const int*>(ring) + sw * lcap * (1 + H);
-        const float* lwt = reinterpret_cast<const float*>(lr + lcap);
-        float wgt[H];
-        lds_heads<H>(lwt + li * H, wgt);
-        const int row = lr[li] & ((1 << kCandRowBits) - 1);
-        const int v = (k0 - x.cb) * kChunk + row;
-        const ChunkRows cr = chunk_rows(x, v / kChunk);
-        const int vr = cr.row0 + v % kChunk;
-        const int slot = s_coff[sw] + li;
-        LaneWords<VB0> w0;
-        LaneWords<(VB0 == VB1) ? 2 : VB1> w1;
-        float2 sz;
-        if (slot < stage_slots) {
-          const uint8_t* src = ring + lists_bytes + (size_t)slot * kSlotBytes;
-          const float* szp = reinterpret_cast<const float*>(src + kVRowMax) + (ng == 1 ? (vr & 1) * 2 : gi * 2);
-          sz = *reinterpret_cast<const float2*>(szp);
-          if (cr.seg == 0 || VB0 == VB1) lds_lane_words<VB0>(src + j * 2 * VB0, w0);
-          else if constexpr (VB0 != VB1) lds_lane_words<VB1>(src + j * 2 * VB1, w1);
-        } else {
-          const long long pr = PAGED ? unit_row<PAGED>(a, x.u, vr) : ubase + vr;
-          if (cr.seg == 0 || VB0 == VB1) ldg_v<VB0>(d.vc[cr.seg] + pr * (D * VB0 / 8), d.vsz[cr.seg] + pr * ng * 2, j, gi, w0, sz);
-          else if constexpr (VB0 != VB1) ldg_v<VB1>(d.vc[1] + pr * (D * VB1 / 8), d.vsz[1] + pr * ng * 2, j, gi, w1, sz);
-        }
-        if (cr.seg == 0 || VB0 == VB1) accumulate_v<H, VB0>(w0, sz, wgt, acc, Z);
-        else if constexpr (VB0 != VB1) accumulate_v<H, VB1>(w1, sz, wgt, acc, Z);
-      }
-    } else if (dense) {
+    if (dense) {
       // Dense V pass: every valid row is kept, so the warp streams its
       // 32-row blocks (round robin over warps) into shared memory with bulk
       // copies, two blocks in flight, and accumulates them from there.

@@ -76,7 +76,7 @@ struct FusedArgs {
   int cpc_max;                   // upper bound of chunks per CTA
   int stages;                    // ring stages in use
   int ring_bytes;                // shared-memory ring size
-  int cand_cap;                  // candidate-list entries per warp (0: candidate mode off)
+  int cand_cap;                  // sparse mode: kept rows one CTA can list (0: sparse mode off)
   long long smem_logit_floats;   // logits that fit in shared memory per CTA
   const unsigned long long* timeout_ns;  // workspace word: wait limit override (0 = default)
   int* arrive1;                  // [units] piece statistics published
