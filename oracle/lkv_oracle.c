@@ -29,6 +29,7 @@
  * through this file alone (closed forms, brute force, a float64 library
  * softmax, values the pages print).
  */
+#include <float.h>
 #include <math.h>
 #include <stdint.h>
 #include <stdlib.h>
@@ -67,6 +68,17 @@ long long lkv_oracle_row_bytes(int bits, int D)
  *   5. the record is (scale, zero) with zero = mn (+0.0 makes a minus zero
  *      into plus zero, so the stored bits do not depend on which of two
  *      equal zeros was found first).
+ * Two ranges of finite values leave fp32 in steps 3-4 and take the same
+ * formula on exactly rescaled values (each step rounded on its own):
+ *   - d so small that qmax / d overflows: the differences and d are
+ *     scaled by 2^64 first, inv = qmax / (d * 2^64) and
+ *     code_i = round((x_i - mn) * 2^64 * inv); scale = d / qmax as above;
+ *   - d itself overflowing (mx - mn above the largest float): the group is
+ *     quantized at half size, d_h = mx/2 - mn/2, inv = qmax / d_h,
+ *     code_i = round((x_i/2 - mn/2) * inv), and scale = (d_h / qmax) * 2.
+ * Both keep |x - xhat| <= scale / 2 (up to the fp32 rounding of the
+ * formula) and the group minimum's exact reconstruction for every finite
+ * group.
  */
 void lkv_oracle_quantize_group(const float *x, int n, int bits,
                                uint32_t *codes, float *scale_out, float *zero_out)
@@ -79,16 +91,39 @@ void lkv_oracle_quantize_group(const float *x, int n, int bits,
     const float qmax = (float)((1u << bits) - 1u);
     const float d = mx - mn;
     float scale = 0.0f, inv = 0.0f;
+    int regime = 0;              /* 0: as written; 1: tiny range; 2: huge range */
+    const float two64 = 18446744073709551616.0f;
+    float mnh = 0.0f;
     if (d != 0.0f) {
         scale = d / qmax;
         inv = qmax / d;
+        if (d > FLT_MAX) {               /* mx - mn overflowed */
+            const float dh = mx * 0.5f - mn * 0.5f;
+            mnh = mn * 0.5f;
+            scale = (dh / qmax) * 2.0f;
+            inv = qmax / dh;
+            regime = 2;
+        } else if (inv > FLT_MAX) {      /* qmax / d overflowed */
+            inv = qmax / (d * two64);
+            regime = 1;
+        }
     }
     for (int i = 0; i < n; ++i) {
-        float diff = x[i] - mn;
-        float y = diff * inv;
+        float y;
+        if (regime == 1) {
+            float diff = x[i] - mn;
+            float big = diff * two64;
+            y = big * inv;
+        } else if (regime == 2) {
+            float half = x[i] * 0.5f;
+            float diff = half - mnh;
+            y = diff * inv;
+        } else {
+            float diff = x[i] - mn;
+            y = diff * inv;
+        }
         float r = nearbyintf(y); /* default rounding mode: half to even */
-        if (!(r >= 0.0f)) r = 0.0f; /* also NaN: 0 * inf when d is tiny enough
-                                       that qmax / d overflows */
+        if (!(r >= 0.0f)) r = 0.0f; /* also NaN (inputs outside the contract) */
         if (r > qmax) r = qmax;
         codes[i] = (uint32_t)r;
     }
@@ -96,11 +131,12 @@ void lkv_oracle_quantize_group(const float *x, int n, int bits,
     *zero_out = mn + 0.0f;
 }
 
-/* Reconstruction of one code: (float)code * scale, then + zero, each rounded. */
+/* Reconstruction of one code: code * scale + zero, rounded once to fp32
+ * (a product that does not fit fp32 on its own -- the group maximum of a
+ * range wider than the largest float -- still gives a finite value). */
 float lkv_oracle_dequant(uint32_t code, float scale, float zero)
 {
-    float a = (float)code * scale;
-    return a + zero;
+    return fmaf((float)code, scale, zero);
 }
 
 /*

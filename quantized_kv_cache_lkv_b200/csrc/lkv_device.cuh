@@ -171,6 +171,46 @@ __device__ __forceinline__ void pack16_magic(const uint32_t (&rb)[16], LaneWords
   }
 }
 
+// The scalar path of the group quantizer for the two ranges of finite
+// values whose formula leaves fp32 (each step rounded on its own):
+//   tiny d, qmax / d overflowing: inv = qmax / (d * 2^64),
+//     code = rint(((x - mn) * 2^64) * inv), scale = d / qmax unchanged;
+//   huge d, mx - mn overflowing: dh = mx/2 - mn/2, inv = qmax / dh,
+//     code = rint((x/2 - mn/2) * inv), scale = (dh / qmax) * 2.
+// Every other group (and a NaN d) keeps code = rint((x - mn) * inv).
+// Codes are clamped to [0, qmax]; a NaN code is 0.
+struct WideQuant {
+  int mode;   // 0: plain, 1: tiny d, 2: huge d
+  float mnh;  // mn / 2 (mode 2)
+  float inv;
+};
+
+__device__ __forceinline__ WideQuant wide_quant_setup(float mn, float mx, float d, float qmax, float inv,
+                                                      float& scale) {
+  WideQuant q{0, 0.0f, inv};
+  if (d > 3.4028234663852886e38f) {
+    const float dh = __fsub_rn(__fmul_rn(mx, 0.5f), __fmul_rn(mn, 0.5f));
+    q.mode = 2;
+    q.mnh = __fmul_rn(mn, 0.5f);
+    scale = __fmul_rn(__fdiv_rn(dh, qmax), 2.0f);
+    q.inv = __fdiv_rn(qmax, dh);
+  } else if (inv > 3.4028234663852886e38f) {
+    q.mode = 1;
+    q.inv = __fdiv_rn(qmax, __fmul_rn(d, 18446744073709551616.0f));
+  }
+  return q;
+}
+
+__device__ __forceinline__ uint32_t wide_quant_code(const WideQuant& q, float x, float mn, int cmask) {
+  float y;
+  if (q.mode == 2) y = __fmul_rn(__fsub_rn(__fmul_rn(x, 0.5f), q.mnh), q.inv);
+  else if (q.mode == 1) y = __fmul_rn(__fmul_rn(__fsub_rn(x, mn), 18446744073709551616.0f), q.inv);
+  else y = __fmul_rn(__fsub_rn(x, mn), q.inv);
+  int ci = __float2int_rn(y);  // NaN gives 0
+  ci = ci < 0 ? 0 : ci;
+  return static_cast<uint32_t>(ci > cmask ? cmask : ci);
+}
+
 // Quantize the 16 bf16 values a lane holds (raw words w, value 2i in the low
 // half of w[i]), sharing min/max with the other lanes of its group (LPG =
 // G / 16 consecutive lanes), and pack the codes into lw.  The formula is the
@@ -182,7 +222,7 @@ __device__ __forceinline__ void pack16_magic(const uint32_t (&rb)[16], LaneWords
 // (two values per packed fp32 operation) and read from the low mantissa bits.
 // `one` must be 1.0f, passed in at run time (see the rounding step).
 // Otherwise (inv overflowing for a tiny d, or d overflowing) every value takes
-// the clamped scalar path.  `mask` names the lanes of the calling row.
+// the scalar path of wide_quant_code.  `mask` names the lanes of the calling row.
 template <int BITS>
 __device__ __forceinline__ void quantize16(const uint32_t (&w)[8], int lpg, unsigned mask, float one,
                                            LaneWords<BITS>& lw, float& scale, float& zero) {
@@ -236,13 +276,12 @@ __device__ __forceinline__ void quantize16(const uint32_t (&w)[8], int lpg, unsi
     }
     pack16_magic<BITS>(rb, lw);
   } else {
+    const WideQuant wq = wide_quant_setup(mn, mx, d, qmax, inv, scale);
     uint32_t c[16];
 #pragma unroll
     for (int i = 0; i < 16; ++i) {
       const float x = (i & 1) ? bf16_hi(w[i / 2]) : bf16_lo(w[i / 2]);
-      int ci = __float2int_rn(__fmul_rn(__fsub_rn(x, mn), inv));  // NaN gives 0
-      ci = ci < 0 ? 0 : ci;
-      c[i] = static_cast<uint32_t>(ci > (int)cmask ? (int)cmask : ci);
+      c[i] = wide_quant_code(wq, x, mn, (int)cmask);
     }
     pack16<BITS>(c, lw);
   }

@@ -152,13 +152,12 @@ __device__ __forceinline__ void quantize32(const uint32_t (&w)[16], unsigned mas
     }
     pack32_magic<BITS>(rb, out);
   } else {
+    const WideQuant wq = wide_quant_setup(mn, mx, d, qmax, inv, scale);
     uint32_t c[32];
 #pragma unroll
     for (int i = 0; i < 32; ++i) {
       const float x = (i & 1) ? bf16_hi(w[i / 2]) : bf16_lo(w[i / 2]);
-      int ci = __float2int_rn(__fmul_rn(__fsub_rn(x, mn), inv));  // NaN gives 0
-      ci = ci < 0 ? 0 : ci;
-      c[i] = static_cast<uint32_t>(ci > (int)cmask ? (int)cmask : ci);
+      c[i] = wide_quant_code(wq, x, mn, (int)cmask);
     }
     pack32<BITS>(c, out);
   }

@@ -45,6 +45,14 @@ def special_rows(inp):
     # that d = mx - mn overflows: both take the clamped path of the formula
     v[0, 0, 4] = torch.linspace(0.0, 1e-38, 16, dtype=torch.float64).repeat(D // 16).to(torch.bfloat16)
     k[0, 0, 4] = torch.linspace(-3e38, 3e38, 16, dtype=torch.float64).repeat(D // 16).to(torch.bfloat16)
+    # random spans of +-1e38..3e38, random subnormal values, and a few
+    # near-subnormal steps around 2^-120
+    g = torch.Generator().manual_seed(D)
+    k[0, 0, 5] = ((torch.rand(D, generator=g, dtype=torch.float64) * 6 - 3) * 1e38).to(torch.bfloat16)
+    v[0, 0, 5] = (torch.randn(D, generator=g, dtype=torch.float64) * 1e-39).to(torch.bfloat16)
+    k[0, 0, 6] = (2.0 ** -120 + torch.randint(-2, 3, (D,), generator=g).double() * 2.0 ** -127).to(torch.bfloat16)
+    v[0, 0, 6] = ((torch.rand(D, generator=g, dtype=torch.float64) * 2 + 1) * 1e38).to(torch.bfloat16)
+    v[0, 0, 6, ::3] *= -1
     return inp
 
 
@@ -106,6 +114,11 @@ def test_append_equals_quantize_of_the_longer_sequence(orc, D, G, kb, vb):
     cfg = W.Config("append", B=4, Hq=4, Hkv=2, D=D, T_cap=T_cap, G=G, bits=[(kb, vb)], seed=90 + D + G + kb)
     full = torch.tensor([50, 96, 1, 20], dtype=torch.int32)
     inp = W.make_inputs(cfg, seq_lens=full)
+    # two appended rows carry the extreme ranges: a span whose d overflows fp32
+    # and subnormal values whose qmax / d overflows
+    g = torch.Generator().manual_seed(D + kb)
+    inp["k"][0, :, 49] = ((torch.rand(2, D, generator=g, dtype=torch.float64) * 6 - 3) * 1e38).to(torch.bfloat16)
+    inp["v"][1, :, 95] = (torch.randn(2, D, generator=g, dtype=torch.float64) * 1e-39).to(torch.bfloat16)
     before = torch.tensor([49, 95, 0, 20], dtype=torch.int32)   # sequence 3 appends at an invalid slot below
     cache = gpu_quantize(kb, vb, G, dict(inp, seq_lens=before))
     pos = torch.tensor([49, 95, 0, T_cap], dtype=torch.int32)    # T_cap: nothing written

@@ -35,10 +35,12 @@ def bf16_round(a):
 
 
 def random_groups(rng, n, G):
-    """Groups with varied ranges: normal, scaled, outliers, tiny spread, large magnitude."""
+    """Groups with varied ranges: normal, scaled, outliers, tiny spread, large
+    magnitude, spreads so small that qmax / d overflows fp32 (subnormal and
+    near-subnormal values), and spans of +-1e38..3e38 whose d overflows."""
     out = []
     for i in range(n):
-        kind = i % 5
+        kind = i % 7
         x = rng.standard_normal(G).astype(np.float32)
         if kind == 1:
             x *= np.float32(rng.uniform(0.01, 100))
@@ -48,8 +50,26 @@ def random_groups(rng, n, G):
             x = np.float32(rng.uniform(-50, 50)) + x * np.float32(0.3)
         elif kind == 4:
             x = x * np.float32(1e20)
+        elif kind == 5:
+            if i % 2:  # subnormal values
+                x = x * np.float32(10.0 ** rng.uniform(-40, -37.5))
+            else:  # a few steps around a near-subnormal base
+                x = np.float32(2.0 ** -120) + rng.integers(-2, 3, G).astype(np.float32) * np.float32(2.0 ** -127)
+        elif kind == 6:
+            x = rng.uniform(-3.0, 3.0, G).astype(np.float32) * np.float32(1e38)
+            x[0] = np.float32(rng.uniform(1.0, 3.0) * 1e38)
+            x[1] = -np.float32(rng.uniform(1.0, 3.0) * 1e38)
         out.append(bf16_round(x))
     return out
+
+
+def p1_bound(x, s, bits):
+    """P1: scale/2, plus the storage precision of the scale (a subnormal scale
+    keeps few bits: code * scale may miss code * d/qmax by (qmax/2) ulp(scale)),
+    plus the fp32 rounding of the formula, 2 ulp(max(|mn|, |mx|))."""
+    qmax = (1 << bits) - 1
+    mag = max(abs(float(x.min())), abs(float(x.max())))
+    return float(s) / 2 + (qmax / 2 + 1) * float(ulp(s)) + 2 * float(ulp(mag))
 
 
 # ---------------------------------------------------------------- bit layout
@@ -93,16 +113,17 @@ def test_pack_roundtrip_bruteforce(orc, bits, D):
 
 @pytest.mark.parametrize("bits", BITS)
 def test_quantize_error_bound(orc, bits):
-    """|x - xhat| <= scale/2 + 2 ulp(max(|mn|, |mx|)) for every element
-    (the quantization error bound the tier thresholds are derived from,
-    Super KV Compression §第二层)."""
+    """P1: |x - xhat| <= scale/2 + (qmax/2 + 1) ulp(scale) + 2 ulp(max(|mn|,
+    |mx|)) for every element, and every reconstruction finite (the
+    quantization error bound the tier thresholds are derived from, Super KV
+    Compression §第二层), for every kind of finite group."""
     rng = np.random.default_rng(bits)
     for x in random_groups(rng, 200, 64):
         codes, s, z = orc.quantize_group(x, bits)
         assert codes.max() <= (1 << bits) - 1
         xh = np.array([orc.dequant(c, s, z) for c in codes], np.float32)
-        mag = max(abs(float(x.min())), abs(float(x.max())))
-        bound = float(s) / 2 + 2 * float(ulp(mag))
+        assert np.all(np.isfinite(xh)) and np.isfinite(s)
+        bound = p1_bound(x, s, bits)
         assert np.all(np.abs(x.astype(np.float64) - xh.astype(np.float64)) <= bound), (bits, s)
 
 
@@ -115,18 +136,19 @@ def test_quantize_is_nearest_level(orc, bits):
     for x in random_groups(rng, 60, 32):
         codes, s, z = orc.quantize_group(x, bits)
         levels = np.array([orc.dequant(c, s, z) for c in range(qmax + 1)], np.float64)
+        mag = max(abs(float(x.min())), abs(float(x.max())))
+        slack = 4 * float(ulp(mag)) + 1e-7 * float(s) + qmax * float(ulp(s))
         for xi, c in zip(x.astype(np.float64), codes):
             best = np.min(np.abs(levels - xi))
-            mag = max(abs(float(x.min())), abs(float(x.max())))
-            assert abs(levels[c] - xi) <= best + 4 * float(ulp(mag)) + 1e-7 * float(s)
+            assert abs(levels[c] - xi) <= best + slack
 
 
 @pytest.mark.parametrize("bits", BITS)
 def test_group_min_and_max(orc, bits):
-    """The group minimum reconstructs bit-exactly (code 0 -> zero = mn); the
-    maximum gets code qmax and reconstructs exactly up to the fp32 rounding
-    of scale = d/qmax, of qmax*scale and of the final add: within
-    4 ulp(max(|mn|, |mx|)), since d <= 2 max(|mn|, |mx|)."""
+    """P2: the group minimum reconstructs bit-exactly (code 0 -> zero = mn);
+    the maximum gets code qmax and reconstructs exactly up to the fp32
+    rounding of scale = d/qmax and of the final fused multiply-add: within
+    (qmax/2) ulp(scale) + 4 ulp(max(|mn|, |mx|)), since d <= 2 max(|mn|, |mx|)."""
     rng = np.random.default_rng(200 + bits)
     qmax = (1 << bits) - 1
     for x in random_groups(rng, 100, 64):
@@ -139,7 +161,8 @@ def test_group_min_and_max(orc, bits):
             continue  # a constant group has no separate maximum
         assert codes[i_mx] == qmax
         mag = max(abs(float(x.min())), abs(float(x.max())))
-        assert abs(float(orc.dequant(codes[i_mx], s, z)) - float(x[i_mx])) <= 4 * float(ulp(mag))
+        xm = float(orc.dequant(codes[i_mx], s, z))
+        assert abs(xm - float(x[i_mx])) <= qmax / 2 * float(ulp(s)) + 4 * float(ulp(mag))
 
 
 @pytest.mark.parametrize("bits", BITS)
@@ -166,6 +189,71 @@ def test_arithmetic_progression_exact(orc, bits):
         codes, s, z = orc.quantize_group(x, bits)
         assert s == np.float32(step) and z == np.float32(base)
         assert codes.tolist() == k.tolist()
+
+
+@pytest.mark.parametrize("bits", BITS)
+def test_tiny_range_progression_exact(orc, bits):
+    """A spread so small that qmax / d overflows fp32: x_k = mn + k * 2^-140
+    (fp32 subnormal steps), d = qmax * 2^-140.  The rescaled formula gives
+    code k exactly, scale = 2^-140 exactly, and every x_k reconstructs."""
+    qmax = (1 << bits) - 1
+    step = np.float32(2.0 ** -140)
+    for base in (0.0, -(2.0 ** -135), 2.0 ** -130):
+        k = np.arange(qmax + 1)[::-1].copy()
+        x = (np.float32(base) + k.astype(np.float32) * step).astype(np.float32)
+        d = float(x.max()) - float(x.min())
+        with np.errstate(over="ignore"):
+            assert np.isinf(np.float32(qmax) / np.float32(d))  # the formula as written overflows
+        codes, s, z = orc.quantize_group(x, bits)
+        assert s == step and z == np.float32(base)
+        assert codes.tolist() == k.tolist()
+        assert [orc.dequant(c, s, z) for c in codes] == x.tolist()
+
+
+@pytest.mark.parametrize("bits", BITS)
+def test_huge_range_progression_exact(orc, bits):
+    """A span whose d = mx - mn overflows fp32: x_k = (2k - qmax) * 2^(128-bits),
+    so d = 2^129 - 2^(129-bits) > FLT_MAX while every x_k is a finite bf16
+    value.  Quantized at half size, code k comes out exactly, scale is
+    2^(129-bits), zero = mn, and every x_k reconstructs exactly."""
+    qmax = (1 << bits) - 1
+    e = 128 - bits
+    k = np.arange(qmax + 1)
+    x = ((2 * k - qmax).astype(np.float64) * 2.0 ** e).astype(np.float32)
+    assert np.all(np.isfinite(x)) and np.array_equal(bf16_round(x), x)
+    with np.errstate(over="ignore"):
+        assert np.isinf(np.float32(x.max()) - np.float32(x.min()))
+    codes, s, z = orc.quantize_group(x, bits)
+    assert s == np.float32(2.0 ** (e + 1)) and z == x.min()
+    assert codes.tolist() == k.tolist()
+    assert [orc.dequant(c, s, z) for c in codes] == x.tolist()
+
+
+@pytest.mark.parametrize("bits", BITS)
+def test_wide_ranges_match_fp64_quantizer(orc, bits):
+    """Against the same quantizer evaluated in float64 (where neither range
+    overflows): for groups of both extreme kinds the fp32 codes differ from
+    the exact ones only where the fp64 value of (x - mn) * qmax / d lies
+    within 1e-4 of a rounding boundary."""
+    rng = np.random.default_rng(900 + bits)
+    qmax = (1 << bits) - 1
+    n = 0
+    for x in random_groups(rng, 140, 64):
+        x64 = x.astype(np.float64)
+        d = x64.max() - x64.min()
+        with np.errstate(over="ignore", divide="ignore"):
+            wide = d > np.finfo(np.float32).max or np.isinf(np.float32(qmax) / np.float32(d))
+        if not wide:
+            continue
+        n += 1
+        codes, s, z = orc.quantize_group(x, bits)
+        y = (x64 - x64.min()) * qmax / d
+        exact = np.clip(np.rint(y), 0, qmax)
+        frac = np.abs(y - np.floor(y) - 0.5)
+        differ = codes != exact
+        assert np.all(frac[differ] < 1e-4), (bits, y[differ], codes[differ])
+        assert np.all(np.abs(codes.astype(np.int64) - exact) <= 1)
+    assert n >= 20
 
 
 def test_round_half_to_even(orc):
