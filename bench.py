@@ -1,23 +1,47 @@
 """Benchmark of the quantized-KV decode path on B200.
 
-One step = one pass of the whole path over one batch of the
+Headline (`value`): the decode call, lkv_decode_attention, on the
 Llama-3.1-8B-shaped workload (B16, 32 query / 8 KV heads, head_dim 128,
-context 8192, group 64, K6V4, 1% heavy hitters):
+context 8192, group 64, K6V4, 1% heavy hitters, sparse-V skip at tau 1e-4):
+its algorithmic HBM bytes (every K row and (scale, zero) row, the V rows some
+head keeps, q and out) over the median of its device times, in GB/s.
 
-  quantize   lkv_quantize_kv     bf16 K, V -> K6 / V4 codes + (scale, zero)
-  decode     lkv_decode_attention  sparse-V skip at tau = 1e-4 (one launch)
-  classify   lkv_tier_classify   Zipf(1.1) previous-step mass, tau_low 1e-4, tau_high 1e-2
-  repack     lkv_tier_repack     kept tokens -> K6/V6 and K6/V4 segments
+Each timed step runs the whole path once on that workload, with L2 flushed
+(a 512 MiB write) before every kernel, outside the kernel's event pair:
+
+  quantize   lkv_quantize_kv       bf16 K, V -> K6 / V4 codes + (scale, zero)
+  decode     lkv_decode_attention  one launch, sparse-V skip at tau = 1e-4
+  classify   lkv_tier_classify     Zipf(1.1) previous-step mass, tau_low 1e-4, tau_high 1e-2
+  repack     lkv_tier_repack       kept tokens -> K6/V6 and K6/V4 segments
   tiered     lkv_tiered_attention  decode over the kept tokens (one launch)
 
-value = algorithmic HBM bytes of the step / step time (GB/s), timed with CUDA
-events on the launching stream with L2 flushed before every step; each
-kernel is also timed on its own for the roofline.  Multi-GPU: one process per
-GPU, every rank runs its own batch (weak scaling, no collective on the data
-path), value = all ranks' bytes / max-over-ranks time.
+and the step's figures sit under "step".  At one GPU the other workloads
+follow under their own keys, each timed the same way (median over the timed
+steps, L2 flushed before every launch):
 
---impl reference times the CPU oracle (the reference arm) on a bounded sample
-of the same workload.
+  long_context  B1, context 131072, tau 1e-5, 0.1% heavy hitters: decode, and
+                quantize of the full 131072-token bf16 K/V;
+  bit_sweep     B64, ragged context uniform in [512, 4096], group 32: decode
+                per (k_bits, v_bits) in K8V8, K6V4, K4V4, K4V2, with the
+                measured compression ratio against the bit-count formula and
+                the rel-L2 error against fp64 attention over the unquantized
+                bf16 cache (computed with torch in float64 on the device);
+  tiered        B32, context log-uniform in [1024, 32768], Zipf(1.1) mass:
+                classify, repack and tiered decode, with the tiered cache's
+                compression ratio.
+
+e2e is a decode loop through the public API with host buffers: every step
+copies q and the new token's K/V (plus positions and lengths) host->device,
+appends the token (lkv_append_kv), decodes, and reads out and the skip counts
+back device->host; value = the decode + append algorithmic bytes over the
+loop's device time.
+
+Multi-GPU: one process per GPU, every rank decodes its own batch (weak
+scaling, no collective on the data path), value = all ranks' decode bytes /
+the max-over-ranks median time.
+
+--impl reference times the CPU oracle (the reference arm) on the same
+workload and metric.
 """
 import argparse
 import hashlib
@@ -38,7 +62,7 @@ import torch  # noqa: E402
 
 from quantized_kv_cache_lkv_b200 import workloads as W  # noqa: E402
 
-CFG_ID = 2
+CFG_MAIN, CFG_LONG, CFG_SWEEP, CFG_TIER = 2, 3, 4, 5
 KB, VB = 6, 4
 TAU_LOW, TAU_HIGH = 1e-4, 1e-2       # tier thresholds of the tiered-cache workload
 METRIC = "quantized-KV decode attention: HBM GB/s (% of peak), KV tokens/s"
@@ -75,12 +99,13 @@ def traffic_table():
 # Sources each timed kernel is compiled from (an ncu traffic figure only
 # counts while these files are unchanged).
 CSRC = "quantized_kv_cache_lkv_b200/csrc/"
+FUSED = [CSRC + "fused_impl.cuh", CSRC + "mma_k.cuh", CSRC + "fused_k6.cu", CSRC + "lkv_device.cuh"]
 KERNEL_SOURCES = {
     "quantize": [CSRC + "quantize.cu", CSRC + "lkv_device.cuh"],
     "repack": [CSRC + "quantize.cu", CSRC + "lkv_device.cuh"],
     "classify": [CSRC + "tier.cu"],
-    "decode": [CSRC + "fused_impl.cuh", CSRC + "fused_k6.cu", CSRC + "lkv_device.cuh"],
-    "tiered": [CSRC + "fused_impl.cuh", CSRC + "fused_k6.cu", CSRC + "lkv_device.cuh"],
+    "decode": FUSED,
+    "tiered": FUSED,
 }
 
 
@@ -149,44 +174,63 @@ class ClockSampler:
                 "reasons": sorted(reasons), "samples": len(sm)}
 
 
-def path_bytes(cfg, seq_lens, counts, skipped_rows, skipped_rows_tiered):
-    """Algorithmic HBM bytes of each kernel of one step.
+# ----------------------------------------------------------------- algorithmic bytes
 
-    quantize  per valid row: bf16 K and V read, K6 + V4 codes and both
-              (scale, zero) rows written;
-    decode    every K row (codes + sz), the V rows some head keeps, q and out;
-    classify  mass of valid tokens read, the tier byte of every slot written,
-              4 bytes per kept position, the counts;
-    repack    per kept token: bf16 K and V read, its position, codes + sz written;
-    tiered    K rows of the kept tokens, their V rows unless every head
-              skips them, q and out, the counts.
-    """
-    D, ng, Hkv = cfg.D, cfg.D // cfg.G, cfg.Hkv
-    B, Hq, T_cap = cfg.B if seq_lens is None else len(seq_lens), cfg.Hq, cfg.T_cap
-    rows = int(np.asarray(seq_lens, np.int64).sum()) * Hkv
-    k_row, v_row, sz = D * KB // 8, D * VB // 8, 8 * ng
-    r6, r4 = D * 6 // 8, D * 4 // 8
-    qo = B * Hq * D * (2 + 4)
-    n2, n1 = int(np.asarray(counts)[..., 0].sum()), int(np.asarray(counts)[..., 1].sum())
+def sz_bytes(D, G):
+    return 8 * (D // G)
+
+
+def quantize_bytes(rows, D, G, kb, vb):
+    """bf16 K and V read, K and V codes and both (scale, zero) rows written."""
+    return rows * (2 * D * 2 + D * kb // 8 + D * vb // 8 + 2 * sz_bytes(D, G))
+
+
+def decode_bytes(rows, v_rows_kept, B, Hq, D, G, kb, vb):
+    """Every K row and its (scale, zero), the V rows some head keeps, q and out."""
+    return rows * (D * kb // 8 + sz_bytes(D, G)) + v_rows_kept * (D * vb // 8 + sz_bytes(D, G)) + B * Hq * D * 6
+
+
+def classify_bytes(rows, B, Hkv, T_cap, kept):
+    """Mass of valid tokens read, the tier byte of every slot, 4 bytes per kept position, the counts."""
+    return rows * 4 + B * Hkv * T_cap + kept * 4 + B * Hkv * 8
+
+
+def repack_bytes(n2, n1, D, G):
+    """Per kept token: bf16 K and V read, its position, codes + (scale, zero) written."""
+    r6, r4, sz = D * 6 // 8, D * 4 // 8, sz_bytes(D, G)
+    return (n2 + n1) * (2 * D * 2 + 4 + r6 + sz) + n2 * (r6 + sz) + n1 * (r4 + sz)
+
+
+def tiered_bytes(n2, n1, skipped_rows, B, Hq, Hkv, D, G):
+    """K rows of the kept tokens, their V rows unless every head skips them, q, out, the counts."""
+    r6, r4, sz = D * 6 // 8, D * 4 // 8, sz_bytes(D, G)
     kept = n2 + n1
-    by = {
-        "quantize": rows * (2 * D * 2 + k_row + v_row + 2 * sz),
-        "decode": rows * (k_row + sz) + (rows - skipped_rows) * (v_row + sz) + qo,
-        "classify": rows * 4 + B * Hkv * T_cap + kept * 4 + B * Hkv * 8,
-        "repack": kept * (2 * D * 2 + 4 + r6 + sz) + n2 * (r6 + sz) + n1 * (r4 + sz),
-    }
     v_kept = n2 * (r6 + sz) + n1 * (r4 + sz)
-    keep_frac = 1.0 - skipped_rows_tiered / kept if kept else 0.0
-    by["tiered"] = kept * (r6 + sz) + int(round(v_kept * keep_frac)) + qo + B * Hkv * 8
-    return by
+    keep_frac = 1.0 - skipped_rows / kept if kept else 0.0
+    return kept * (r6 + sz) + int(round(v_kept * keep_frac)) + B * Hq * D * 6 + B * Hkv * 8
 
 
-# ----------------------------------------------------------------- ranks
+def path_bytes(cfg, seq_lens, counts, skipped_rows, skipped_rows_tiered):
+    """Algorithmic HBM bytes of each kernel of one step of the main workload."""
+    D, G, Hkv, Hq = cfg.D, cfg.G, cfg.Hkv, cfg.Hq
+    B, T_cap = len(seq_lens), cfg.T_cap
+    rows = int(np.asarray(seq_lens, np.int64).sum()) * Hkv
+    n2, n1 = int(np.asarray(counts)[..., 0].sum()), int(np.asarray(counts)[..., 1].sum())
+    return {
+        "quantize": quantize_bytes(rows, D, G, KB, VB),
+        "decode": decode_bytes(rows, rows - skipped_rows, B, Hq, D, G, KB, VB),
+        "classify": classify_bytes(rows, B, Hkv, T_cap, n2 + n1),
+        "repack": repack_bytes(n2, n1, D, G),
+        "tiered": tiered_bytes(n2, n1, skipped_rows_tiered, B, Hq, Hkv, D, G),
+    }
+
+
+# ----------------------------------------------------------------- ranks and timing
 
 def rank_workload(rank):
-    """The batch rank `rank` decodes: the bench workload with its own seed, so
+    """The batch rank `rank` decodes: the main workload with its own seed, so
     the ranks process distinct, independent batches (weak scaling)."""
-    base = W.CONFIGS[CFG_ID]
+    base = W.CONFIGS[CFG_MAIN]
     return W.scaled(base, seed=base.seed + 1000 * rank)
 
 
@@ -201,15 +245,50 @@ def max_over_ranks(x, device=None):
     return float(t.item())
 
 
-def job_throughput(bytes_per_rank_step, world, steps, max_ms):
+def job_throughput(bytes_per_rank, world, seconds):
     """Whole-job GB/s: the bytes all ranks moved over the slowest rank's time."""
-    return bytes_per_rank_step * world * steps / (max_ms * 1e-3) / 1e9
+    return bytes_per_rank * world / seconds / 1e9
 
 
-# ----------------------------------------------------------------- the step
+class Timed:
+    """Runs named launches in order, steps times, with L2 flushed before each
+    launch outside its event pair; keeps every launch's device time (ms)."""
+
+    def __init__(self, device, stream):
+        self.stream = stream
+        self.flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=device)
+
+    def run(self, launches, steps, warmup, on_step=None):
+        for _ in range(warmup):
+            for _, fn in launches:
+                self.flush.zero_()
+                fn()
+        torch.cuda.synchronize()
+        ev = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in launches] for _ in range(steps)]
+        for i in range(steps):
+            for j, (_, fn) in enumerate(launches):
+                self.flush.zero_()
+                ev[i][j][0].record(self.stream)
+                fn()
+                ev[i][j][1].record(self.stream)
+            if on_step is not None:
+                on_step(i)
+        torch.cuda.synchronize()
+        return {name: [ev[i][j][0].elapsed_time(ev[i][j][1]) for i in range(steps)]
+                for j, (name, _) in enumerate(launches)}
+
+
+def kernel_line(ms_list, nbytes, peak):
+    ms = statistics.median(ms_list)
+    gbs = nbytes / (ms * 1e-3) / 1e9
+    return {"us": round(ms * 1e3, 2), "bytes": int(nbytes), "gbs": round(gbs, 1), "frac": round(gbs / peak, 4)}
+
+
+# ----------------------------------------------------------------- the main step
 
 class Step:
-    """Device buffers and the launches of one step of the path."""
+    """Device buffers and the five launches of one step of the main workload."""
 
     def __init__(self, cfg, inp, device):
         from quantized_kv_cache_lkv_b200 import buffers, lkv
@@ -217,8 +296,7 @@ class Step:
         self.cfg = cfg
         B, Hq, Hkv, D, T, G = cfg.B, cfg.Hq, cfg.Hkv, cfg.D, cfg.T_cap, cfg.G
         self.shape = (B, Hq, Hkv, D, T, G)
-        d = {k: v.to(device) for k, v in inp.items()}
-        self.d = d
+        self.d = {k: v.to(device) for k, v in inp.items()}
         self.cache = buffers.alloc_cache(KB, VB, G, B, Hkv, T, D, device, zero=True)
         self.out = torch.empty(B, Hq, D, device=device)
         self.out2 = torch.empty(B, Hq, D, device=device)
@@ -228,52 +306,247 @@ class Step:
         self.ws2 = buffers.alloc_workspace(lkv.lkv_tiered_workspace_bytes(B, Hq, Hkv, T, D, G), device)
         self.tiers = buffers.alloc_tiers(B, Hkv, T, device, zero=True)
         self.A, self.Bs = buffers.alloc_segments(G, B, Hkv, T, D, device, zero=True)
-        self.names = ["quantize", "decode", "classify", "repack", "tiered"]
 
-    def launches(self, stream, events=None):
-        L, c, d = self.lkv, self.cfg, self.d
+    def quantize(self, s=None):
         B, Hq, Hkv, D, T, G = self.shape
-        s = stream.cuda_stream
+        d, c = self.d, self.cache
+        self.lkv.lkv_quantize_kv((KB, VB, G), B, Hkv, T, D, d["seq_lens"], d["k"], d["v"], c["k_codes"],
+                                 c["k_sz"], c["v_codes"], c["v_sz"], s)
 
-        def mark(i):
-            if events is not None:
-                events[i].record(stream)
-        mark(0)
-        L.lkv_quantize_kv((KB, VB, G), B, Hkv, T, D, d["seq_lens"], d["k"], d["v"], self.cache["k_codes"],
-                          self.cache["k_sz"], self.cache["v_codes"], self.cache["v_sz"], s)
-        mark(1)
-        L.lkv_decode_attention((KB, VB, G), B, Hq, Hkv, T, D, d["seq_lens"], d["q"], self.cache["k_codes"],
-                               self.cache["k_sz"], self.cache["v_codes"], self.cache["v_sz"],
-                               c.softmax_scale, c.tau, self.out, None, self.cnt, self.ws, self.ws.numel(), s)
-        mark(2)
-        t = self.tiers
-        L.lkv_tier_classify(B, Hkv, T, d["seq_lens"], d["mass"], TAU_LOW, TAU_HIGH, t["tier"], t["counts"],
-                            t["pos_a"], t["pos_b"], s)
-        mark(3)
-        L.lkv_tier_repack(B, Hkv, T, D, G, d["k"], d["v"], t["counts"], t["pos_a"], t["pos_b"], self.A,
-                          self.Bs, s)
-        mark(4)
-        L.lkv_tiered_attention(B, Hq, Hkv, T, D, G, t["counts"], d["q"], self.A, self.Bs, c.softmax_scale,
-                               0.0, self.out2, self.cnt2, self.ws2, self.ws2.numel(), s)
-        mark(5)
+    def decode(self, s=None, seq_lens=None, q=None):
+        B, Hq, Hkv, D, T, G = self.shape
+        d, c = self.d, self.cache
+        self.lkv.lkv_decode_attention((KB, VB, G), B, Hq, Hkv, T, D,
+                                      d["seq_lens"] if seq_lens is None else seq_lens,
+                                      d["q"] if q is None else q, c["k_codes"], c["k_sz"], c["v_codes"],
+                                      c["v_sz"], self.cfg.softmax_scale, self.cfg.tau, self.out, None, self.cnt,
+                                      self.ws, self.ws.numel(), s)
+
+    def classify(self, s=None):
+        B, Hq, Hkv, D, T, G = self.shape
+        t, d = self.tiers, self.d
+        self.lkv.lkv_tier_classify(B, Hkv, T, d["seq_lens"], d["mass"], TAU_LOW, TAU_HIGH, t["tier"],
+                                   t["counts"], t["pos_a"], t["pos_b"], s)
+
+    def repack(self, s=None):
+        B, Hq, Hkv, D, T, G = self.shape
+        t, d = self.tiers, self.d
+        self.lkv.lkv_tier_repack(B, Hkv, T, D, G, d["k"], d["v"], t["counts"], t["pos_a"], t["pos_b"], self.A,
+                                 self.Bs, s)
+
+    def tiered(self, s=None):
+        B, Hq, Hkv, D, T, G = self.shape
+        self.lkv.lkv_tiered_attention(B, Hq, Hkv, T, D, G, self.tiers["counts"], self.d["q"], self.A, self.Bs,
+                                      self.cfg.softmax_scale, 0.0, self.out2, self.cnt2, self.ws2,
+                                      self.ws2.numel(), s)
+
+    def launches(self, stream):
+        s = stream.cuda_stream
+        return [("quantize", lambda: self.quantize(s)), ("decode", lambda: self.decode(s)),
+                ("classify", lambda: self.classify(s)), ("repack", lambda: self.repack(s)),
+                ("tiered", lambda: self.tiered(s))]
 
     LAUNCHES_PER_STEP = 5    # quantize, decode, classify, repack, tiered: one kernel each
 
     def algorithmic_bytes(self):
         """Bytes each kernel must move, from the step's device results."""
-        B, Hq, Hkv, D, T, G = self.shape
         sl = self.d["seq_lens"].cpu().numpy()
         counts = self.tiers["counts"].cpu().numpy()
         self.skipped_rows = int(self.cnt[1].item())
         by = path_bytes(self.cfg, sl, counts, self.skipped_rows, int(self.cnt2[1].item()))
-        self.kept = (int(counts[..., 0].sum()), int(counts[..., 1].sum()), int(sl.astype(np.int64).sum()) * Hkv)
+        self.kept = (int(counts[..., 0].sum()), int(counts[..., 1].sum()),
+                     int(sl.astype(np.int64).sum()) * self.cfg.Hkv)
         return by
 
-    def dense_decode_bytes(self):
-        B, Hq, Hkv, D, T, G = self.shape
-        rows = int(self.d["seq_lens"].sum().item()) * Hkv
-        return rows * (D * (KB + VB) // 8 + 16 * (D // G)) + B * Hq * D * 6
 
+def run_e2e(step, inp, device, stream, steps):
+    """Decode loop through the public API with host buffers.  The cache holds
+    the workload's tokens; the loop starts `steps` tokens short of the full
+    context and, every step, copies q, the new token's K/V, its position and
+    the new lengths host->device, appends the token (lkv_append_kv), decodes
+    over the longer sequences, and copies out and the skip counts back."""
+    cfg = step.cfg
+    B, Hq, Hkv, D, T, G = step.shape
+    L = step.lkv
+    s = stream.cuda_stream
+    full = inp["seq_lens"].to(torch.int64)
+    start = torch.clamp(full - steps, min=0)
+    h_pos = torch.stack([torch.clamp(start + i, max=T - 1) for i in range(steps)]).to(torch.int32)
+    h_len = torch.stack([torch.minimum(start + i + 1, full) for i in range(steps)]).to(torch.int32)
+    idx = h_pos.to(torch.int64)
+    h_k = torch.stack([inp["k"][torch.arange(B), :, idx[i]] for i in range(steps)]).contiguous().pin_memory()
+    h_v = torch.stack([inp["v"][torch.arange(B), :, idx[i]] for i in range(steps)]).contiguous().pin_memory()
+    h_pos, h_len = h_pos.pin_memory(), h_len.pin_memory()
+    h_q = inp["q"].contiguous().pin_memory()
+    d_pos = torch.empty(B, dtype=torch.int32, device=device)
+    d_len = torch.empty(B, dtype=torch.int32, device=device)
+    d_q = torch.empty_like(step.d["q"])
+    d_k = torch.empty(B, Hkv, D, dtype=torch.bfloat16, device=device)
+    d_v = torch.empty(B, Hkv, D, dtype=torch.bfloat16, device=device)
+    h_out = torch.empty(steps, B, Hq, D, dtype=torch.float32).pin_memory()
+    h_cnt = torch.empty(steps, 2, dtype=torch.int64).pin_memory()
+    c = step.cache
+
+    def one(i):
+        d_q.copy_(h_q, non_blocking=True)
+        d_k.copy_(h_k[i], non_blocking=True)
+        d_v.copy_(h_v[i], non_blocking=True)
+        d_pos.copy_(h_pos[i], non_blocking=True)
+        d_len.copy_(h_len[i], non_blocking=True)
+        L.lkv_append_kv((KB, VB, G), B, Hkv, T, D, d_pos, d_k, d_v, c["k_codes"], c["k_sz"], c["v_codes"],
+                        c["v_sz"], s)
+        step.decode(s, seq_lens=d_len, q=d_q)
+        h_out[i].copy_(step.out, non_blocking=True)
+        h_cnt[i].copy_(step.cnt, non_blocking=True)
+
+    one(0)                                   # warm-up (rewrites the same row)
+    torch.cuda.synchronize(device)
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for i in range(steps):
+        one(i)
+    t1.record(stream)
+    torch.cuda.synchronize(device)
+    sec = t0.elapsed_time(t1) * 1e-3
+    by = 0
+    for i in range(steps):
+        rows = int(h_len[i].to(torch.int64).sum()) * Hkv
+        by += decode_bytes(rows, rows - int(h_cnt[i, 1]), B, Hq, D, G, KB, VB)
+        by += quantize_bytes(B * Hkv, D, G, KB, VB)           # the appended rows
+    h2d = (h_q.numel() + h_k[0].numel() + h_v[0].numel()) * 2 + (h_pos[0].numel() + h_len[0].numel()) * 4
+    d2h = h_out[0].numel() * 4 + h_cnt[0].numel() * 8
+    return {"value": round(by / sec / 1e9, 2), "unit": "GB/s", "h2d_bytes_per_step": int(h2d),
+            "d2h_bytes_per_step": int(d2h), "seconds": sec, "bytes": by, "steps": steps,
+            "us_per_step": round(sec / steps * 1e6, 2),
+            "loop": "H2D q + new K/V + pos + lengths, lkv_append_kv, lkv_decode_attention, D2H out + counts"}
+
+
+# ----------------------------------------------------------------- other workloads (1 GPU)
+
+def bench_long(device, stream, timer, args, peak):
+    from quantized_kv_cache_lkv_b200 import buffers, lkv
+    cfg = W.CONFIGS[CFG_LONG]
+    B, Hq, Hkv, D, T, G = cfg.B, cfg.Hq, cfg.Hkv, cfg.D, cfg.T_cap, cfg.G
+    inp = {k: v.to(device) for k, v in W.make_inputs(cfg).items()}
+    cache = buffers.alloc_cache(KB, VB, G, B, Hkv, T, D, device, zero=True)
+    out = torch.empty(B, Hq, D, device=device)
+    cnt = torch.zeros(2, dtype=torch.int64, device=device)
+    ws = buffers.alloc_workspace(lkv.lkv_decode_workspace_bytes((KB, VB, G), B, Hq, Hkv, T, D), device)
+    s = stream.cuda_stream
+    quant = lambda: lkv.lkv_quantize_kv((KB, VB, G), B, Hkv, T, D, inp["seq_lens"], inp["k"], inp["v"],
+                                        cache["k_codes"], cache["k_sz"], cache["v_codes"], cache["v_sz"], s)
+    dec = lambda: lkv.lkv_decode_attention((KB, VB, G), B, Hq, Hkv, T, D, inp["seq_lens"], inp["q"],
+                                           cache["k_codes"], cache["k_sz"], cache["v_codes"], cache["v_sz"],
+                                           cfg.softmax_scale, cfg.tau, out, None, cnt, ws, ws.numel(), s)
+    t = timer.run([("quantize", quant), ("decode", dec)], args.steps, args.warmup)
+    rows = int(inp["seq_lens"].sum()) * Hkv
+    skipped = int(cnt[1].item())
+    dline = kernel_line(t["decode"], decode_bytes(rows, rows - skipped, B, Hq, D, G, KB, VB), peak)
+    dline["v_rows_skipped_frac"] = round(skipped / rows, 4)
+    dline["kv_tokens_per_s"] = round(rows / Hkv / (dline["us"] * 1e-6), 1)
+    res = {"workload": cfg.name, "decode": dline,
+           "quantize": kernel_line(t["quantize"], quantize_bytes(rows, D, G, KB, VB), peak)}
+    del inp, cache, ws
+    torch.cuda.empty_cache()
+    return res
+
+
+def fp64_reference(inp, cfg):
+    """fp64 softmax attention over the unquantized bf16 K/V, with torch on the
+    device (the quality yardstick of the bit-width sweep)."""
+    B, Hq, Hkv, D = cfg.B, cfg.Hq, cfg.Hkv, cfg.D
+    r = Hq // Hkv
+    out = torch.zeros(B, Hq, D, dtype=torch.float64, device=inp["q"].device)
+    for b in range(B):
+        T = int(inp["seq_lens"][b])
+        if T == 0:
+            continue
+        K = inp["k"][b, :, :T].double()                                  # [Hkv, T, D]
+        V = inp["v"][b, :, :T].double()
+        q = inp["q"][b].double().view(Hkv, r, D)
+        s = torch.einsum("grd,gtd->grt", q, K) * cfg.softmax_scale
+        out[b] = torch.einsum("grt,gtd->grd", torch.softmax(s, dim=-1), V).reshape(Hq, D)
+    return out
+
+
+def bench_sweep(device, stream, timer, args, peak):
+    from quantized_kv_cache_lkv_b200 import buffers, lkv
+    cfg = W.CONFIGS[CFG_SWEEP]
+    B, Hq, Hkv, D, T, G = cfg.B, cfg.Hq, cfg.Hkv, cfg.D, cfg.T_cap, cfg.G
+    inp = {k: v.to(device) for k, v in W.make_inputs(cfg).items()}
+    ref = fp64_reference(inp, cfg)
+    rows = int(inp["seq_lens"].sum()) * Hkv
+    out = torch.empty(B, Hq, D, device=device)
+    cnt = torch.zeros(2, dtype=torch.int64, device=device)
+    s = stream.cuda_stream
+    res = {"workload": cfg.name}
+    for kb, vb in cfg.bits:
+        cache = buffers.alloc_cache(kb, vb, G, B, Hkv, T, D, device, zero=True)
+        ws = buffers.alloc_workspace(lkv.lkv_decode_workspace_bytes((kb, vb, G), B, Hq, Hkv, T, D), device)
+        lkv.lkv_quantize_kv((kb, vb, G), B, Hkv, T, D, inp["seq_lens"], inp["k"], inp["v"], cache["k_codes"],
+                            cache["k_sz"], cache["v_codes"], cache["v_sz"], s)
+        dec = (lambda kb=kb, vb=vb, cache=cache, ws=ws: lkv.lkv_decode_attention(
+            (kb, vb, G), B, Hq, Hkv, T, D, inp["seq_lens"], inp["q"], cache["k_codes"], cache["k_sz"],
+            cache["v_codes"], cache["v_sz"], cfg.softmax_scale, cfg.tau, out, None, cnt, ws, ws.numel(), s))
+        t = timer.run([("decode", dec)], args.steps, args.warmup)
+        skipped = int(cnt[1].item())
+        line = kernel_line(t["decode"], decode_bytes(rows, rows - skipped, B, Hq, D, G, kb, vb), peak)
+        # compression: bytes the buffers give one valid row, against bf16 K + V
+        row_q = (cache["k_codes"].shape[-1] + cache["v_codes"].shape[-1]
+                 + (cache["k_sz"][0, 0, 0].numel() + cache["v_sz"][0, 0, 0].numel()) * 4)
+        formula = (2 * 16 * D) / ((kb + vb) * D + 2 * 64 * (D // G))
+        err = (out.double() - ref).norm() / ref.norm()
+        line.update({"compression": {"measured": round(2 * D * 2 / row_q, 4), "formula": round(formula, 4)},
+                     "rel_l2_vs_bf16_fp64": float(f"{err.item():.4e}")})
+        res[f"K{kb}V{vb}"] = line
+        del cache, ws
+    del inp, ref
+    torch.cuda.empty_cache()
+    return res
+
+
+def bench_tiered(device, stream, timer, args, peak):
+    from quantized_kv_cache_lkv_b200 import buffers, lkv
+    cfg = W.CONFIGS[CFG_TIER]
+    B, Hq, Hkv, D, T, G = cfg.B, cfg.Hq, cfg.Hkv, cfg.D, cfg.T_cap, cfg.G
+    inp = {k: v.to(device) for k, v in W.make_inputs(cfg, with_mass=True).items()}
+    tiers = buffers.alloc_tiers(B, Hkv, T, device, zero=True)
+    A, Bs = buffers.alloc_segments(G, B, Hkv, T, D, device, zero=True)
+    out = torch.empty(B, Hq, D, device=device)
+    cnt = torch.zeros(2, dtype=torch.int64, device=device)
+    ws = buffers.alloc_workspace(lkv.lkv_tiered_workspace_bytes(B, Hq, Hkv, T, D, G), device)
+    s = stream.cuda_stream
+    lo, hi = cfg.tau_low, cfg.tau_high
+    launches = [
+        ("classify", lambda: lkv.lkv_tier_classify(B, Hkv, T, inp["seq_lens"], inp["mass"], lo, hi, tiers["tier"],
+                                                   tiers["counts"], tiers["pos_a"], tiers["pos_b"], s)),
+        ("repack", lambda: lkv.lkv_tier_repack(B, Hkv, T, D, G, inp["k"], inp["v"], tiers["counts"],
+                                               tiers["pos_a"], tiers["pos_b"], A, Bs, s)),
+        ("tiered", lambda: lkv.lkv_tiered_attention(B, Hq, Hkv, T, D, G, tiers["counts"], inp["q"], A, Bs,
+                                                    cfg.softmax_scale, cfg.tau, out, cnt, ws, ws.numel(), s)),
+    ]
+    t = timer.run(launches, args.steps, args.warmup)
+    counts = tiers["counts"].cpu().numpy()
+    n2, n1 = int(counts[..., 0].sum()), int(counts[..., 1].sum())
+    rows = int(inp["seq_lens"].sum()) * Hkv
+    r6, r4, sz = D * 6 // 8, D * 4 // 8, sz_bytes(D, G)
+    tiered_cache = n2 * (2 * r6 + 2 * sz) + n1 * (r6 + r4 + 2 * sz)
+    k6v4_cache = rows * (r6 + r4 + 2 * sz)
+    res = {
+        "workload": cfg.name,
+        "classify": kernel_line(t["classify"], classify_bytes(rows, B, Hkv, T, n2 + n1), peak),
+        "repack": kernel_line(t["repack"], repack_bytes(n2, n1, D, G), peak),
+        "tiered_decode": kernel_line(t["tiered"], tiered_bytes(n2, n1, int(cnt[1].item()), B, Hq, Hkv, D, G), peak),
+        "tiers": {"v6": n2, "v4": n1, "evicted": rows - n2 - n1, "rows": rows},
+        "compression": {"vs_bf16": round(rows * 2 * D * 2 / max(tiered_cache, 1), 3),
+                        "vs_k6v4_cache": round(k6v4_cache / max(tiered_cache, 1), 3)},
+    }
+    del inp, tiers, A, Bs, ws
+    torch.cuda.empty_cache()
+    return res
+
+
+# ----------------------------------------------------------------- the GPU arm
 
 def run_lkv(args):
     rank = int(os.environ.get("RANK", "0"))
@@ -297,138 +570,111 @@ def run_lkv(args):
     inp = W.make_inputs(cfg, with_mass=True)
     step = Step(cfg, inp, device)
     stream = torch.cuda.current_stream(device)
-    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=device)
+    timer = Timed(device, stream)
+    peak, peak_kind = peaks()
 
     def barrier():
         if dist:
             torch.distributed.barrier()
         torch.cuda.synchronize(device)
 
+    launches = step.launches(stream)
     for _ in range(args.warmup):
-        flush.zero_()
-        step.launches(stream)
+        for _, fn in launches:
+            timer.flush.zero_()
+            fn()
     barrier()
-    n = len(step.names)
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(n + 1)] for _ in range(args.steps)]
     with ClockSampler(local) as clocks:
         barrier()
-        for i in range(args.steps):
-            flush.zero_()                      # L2 flush, outside the timed region
-            step.launches(stream, ev[i])
+        times = timer.run(launches, args.steps, 0)
         barrier()
-    per_kernel = {name: [] for name in step.names}
-    step_ms = []
-    for i in range(args.steps):
-        for j, name in enumerate(step.names):
-            per_kernel[name].append(ev[i][j].elapsed_time(ev[i][j + 1]))
-        step_ms.append(ev[i][0].elapsed_time(ev[i][n]))
-    total_ms = max_over_ranks(sum(step_ms), device)
     by = step.algorithmic_bytes()
-    step_bytes = sum(by.values())
-    value = job_throughput(step_bytes, world, args.steps, total_ms)
-    kv_tokens = int(inp["seq_lens"].sum()) * world
-    peak, peak_kind = peaks()
-
-    # per-kernel roofline (algorithmic bytes / mean launch time)
+    dec_ms = max_over_ranks(statistics.median(times["decode"]), device)
+    value = job_throughput(by["decode"], world, dec_ms * 1e-3)
+    step_ms_list = [sum(times[n][i] for n, _ in launches) for i in range(args.steps)]
+    step_ms = max_over_ranks(statistics.median(step_ms_list), device)
     kern = {}
-    for name in step.names:
-        ms = statistics.mean(per_kernel[name])
-        gbs = by[name] / (ms * 1e-3) / 1e9
-        kern[name] = {"us": round(ms * 1e3, 2), "bytes": by[name], "gbs": round(gbs, 1),
-                      "frac": round(gbs / peak, 4), "share": round(ms / statistics.mean(step_ms), 4)}
-    dominant = max(step.names, key=lambda k: kern[k]["us"])
+    for name, _ in launches:
+        kern[name] = kernel_line(times[name], by[name], peak)
+        kern[name]["share"] = round(statistics.median(times[name]) / statistics.median(step_ms_list), 4)
     traffic = traffic_table()
 
     def roofline(name):
         tr = traffic.get(name)
-        t_bytes = None
-        if tr and tr[0] == source_hash(name):
-            t_bytes = tr[1]
+        t_bytes = tr[1] if tr and tr[0] == source_hash(name) else None
         return {"bound": "hbm", "achieved": kern[name]["gbs"], "peak": peak, "unit": "GB/s",
                 "frac": kern[name]["frac"], "traffic": t_bytes, "kernel": name,
-                "peak_source": f"{peak_kind} hbm_gbs"}
+                "algorithmic_bytes": by[name], "peak_source": f"{peak_kind} hbm_gbs (of {peak_kind})"}
 
     e2e = None
     if not args.no_e2e:   # every rank runs it; the job's time is the slowest rank's
-        e2e = run_e2e(step, inp, device, stream, args)
+        e2e = run_e2e(step, inp, device, stream, max(args.steps, 20))
         sec = max_over_ranks(e2e["seconds"], device)
-        e2e["value"] = round(job_throughput(e2e["bytes"], world, e2e["steps"], sec * 1e3), 2)
+        e2e["value"] = round(job_throughput(e2e["bytes"], world, sec), 2)
+    extras = {}
+    if world == 1 and not args.no_extras:
+        del step.d["k"], step.d["v"]
+        torch.cuda.empty_cache()
+        extras["long_context"] = bench_long(device, stream, timer, args, peak)
+        extras["bit_sweep"] = bench_sweep(device, stream, timer, args, peak)
+        extras["tiered"] = bench_tiered(device, stream, timer, args, peak)
     cpu = cpu_baseline(cfg, inp, args) if rank == 0 and world == 1 and not args.no_cpu else None
 
     if rank == 0:
         clk = clocks.summary()
+        rows = step.kept[2]
         line = {
             "metric": METRIC, "value": round(value, 1), "unit": "GB/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup,
-            "ms_per_step": round(total_ms / args.steps, 4),
+            "ms_per_step": round(dec_ms, 5),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "f32", "data": "synthetic",
             "config": {"workload": cfg.name, "B": cfg.B, "Hq": cfg.Hq, "Hkv": cfg.Hkv, "head_dim": cfg.D,
                        "context": cfg.T_cap, "group": cfg.G, "k_bits": KB, "v_bits": VB, "tau": cfg.tau,
-                       "heavy_hitters": cfg.hh_frac, "tier_tau_low": TAU_LOW, "tier_tau_high": TAU_HIGH,
+                       "heavy_hitters": cfg.hh_frac,
                        "parallelism": f"dp{world}" if world > 1 else "single",
-                       "l2": "flushed before every step (512 MiB write)",
-                       "step": "quantize + decode + tier classify + repack + tiered decode"},
-            "kv_tokens_per_s": round(kv_tokens * args.steps / (total_ms * 1e-3), 1),
-            "roofline": roofline(dominant),
-            "roofline_decode": roofline("decode"),
-            "kernels": kern,
-            "decode_skip": {"v_rows_skipped": step.skipped_rows, "rows": step.kept[2],
-                            "frac": round(step.skipped_rows / max(step.kept[2], 1), 4),
-                            "dense_bytes": step.dense_decode_bytes()},
-            "tiers": {"v6": step.kept[0], "v4": step.kept[1], "rows": step.kept[2]},
+                       "value": "lkv_decode_attention algorithmic GB/s, median over the timed steps",
+                       "l2": "flushed (512 MiB write) before every kernel, outside its events"},
+            "kv_tokens_per_s": round(rows / cfg.Hkv * world / (dec_ms * 1e-3), 1),
+            "roofline": roofline("decode"),
+            "decode_skip": {"v_rows_skipped": step.skipped_rows, "rows": rows,
+                            "frac": round(step.skipped_rows / max(rows, 1), 4),
+                            "dense_bytes": decode_bytes(rows, rows, cfg.B, cfg.Hq, cfg.D, cfg.G, KB, VB)},
+            "step": {"ms": round(step_ms, 5), "gbs": round(job_throughput(sum(by.values()), world, step_ms * 1e-3), 1),
+                     "kernels": kern, "dominant_roofline": roofline(max(kern, key=lambda k: kern[k]["us"])),
+                     "tiers": {"v6": step.kept[0], "v4": step.kept[1], "rows": rows,
+                               "tau_low": TAU_LOW, "tau_high": TAU_HIGH},
+                     "what": "quantize + decode + tier classify + repack + tiered decode"},
             "gpu_launches": Step.LAUNCHES_PER_STEP * args.steps,
             "clocks": {k: clk[k] for k in ("sm_mhz", "sm_max_mhz", "reasons")},
-            "e2e": {k: e2e[k] for k in ("value", "unit", "h2d_bytes_per_step", "d2h_bytes_per_step")}
-            if e2e else None,
+            "e2e": {k: e2e[k] for k in ("value", "unit", "h2d_bytes_per_step", "d2h_bytes_per_step",
+                                        "us_per_step", "steps", "loop")} if e2e else None,
             "cpu_baseline": cpu,
         }
+        line.update(extras)
         print(json.dumps(line), flush=True)
     if dist:
         torch.distributed.barrier()
         torch.distributed.destroy_process_group()
 
 
-def run_e2e(step, inp, device, stream, args):
-    """The same step through the public API from pinned host memory: every
-    step copies its inputs host->device and reads both outputs back."""
-    host = {k: v.pin_memory() for k, v in inp.items()}
-    h_out = torch.empty(step.out.shape, dtype=torch.float32).pin_memory()
-    h_out2 = torch.empty(step.out2.shape, dtype=torch.float32).pin_memory()
-    n = max(1, min(args.e2e_steps, args.steps))
-    h2d = sum(v.numel() * v.element_size() for v in host.values())
-    d2h = 2 * h_out.numel() * 4
-    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    for i in range(n + 1):
-        if i == 1:
-            torch.cuda.synchronize(device)
-            start.record(stream)
-        for k in host:
-            step.d[k].copy_(host[k], non_blocking=True)
-        step.launches(stream)
-        h_out.copy_(step.out, non_blocking=True)
-        h_out2.copy_(step.out2, non_blocking=True)
-    end.record(stream)
-    torch.cuda.synchronize(device)
-    sec = start.elapsed_time(end) * 1e-3
-    by = sum(step.algorithmic_bytes().values())
-    return {"value": round(by * n / sec / 1e9, 2), "unit": "GB/s", "h2d_bytes_per_step": h2d,
-            "d2h_bytes_per_step": d2h, "seconds": sec, "bytes": by, "steps": n}
-
-
 # ----------------------------------------------------------------- CPU oracle
 
-def oracle_step(orc, cfg, sub):
-    """One pass of the oracle over a sample: quantize, decode, tiers, repack,
-    tiered attention.  Returns the algorithmic bytes of the sample."""
+def oracle_decode_gbs(orc, cfg, sub, passes_seconds):
+    """The oracle's decode over a sample, repeated for about passes_seconds:
+    (GB/s of the decode metric, passes, seconds)."""
     k, v, q = W.bf16_bits(sub["k"]), W.bf16_bits(sub["v"]), W.bf16_bits(sub["q"])
-    sl, mass = sub["seq_lens"].numpy(), sub["mass"].numpy()
+    sl = sub["seq_lens"].numpy()
     cache = orc.quantize_kv(KB, VB, cfg.G, k, v, sl)
-    _, _, cnt = orc.decode_attention(KB, VB, cfg.G, sl, q, cache, cfg.softmax_scale, cfg.tau, want_mask=False)
-    tier, counts, p2, p1 = orc.tier_classify(sl, mass, TAU_LOW, TAU_HIGH)
-    A, Bs = orc.tier_repack(cfg.G, k, v, counts, p2, p1)
-    _, cnt2 = orc.tiered_attention(cfg.G, counts, q, A, Bs, cfg.softmax_scale, 0.0)
-    return sum(path_bytes(cfg, sl, counts, int(cnt[1]), int(cnt2[1])).values())
+    rows = int(sl.astype(np.int64).sum()) * cfg.Hkv
+    total_by, total_dt, passes = 0, 0.0, 0
+    while total_dt < passes_seconds or passes == 0:
+        t0 = time.perf_counter()
+        _, _, cnt = orc.decode_attention(KB, VB, cfg.G, sl, q, cache, cfg.softmax_scale, cfg.tau, want_mask=False)
+        total_dt += time.perf_counter() - t0
+        total_by += decode_bytes(rows, rows - int(cnt[1]), len(sl), cfg.Hq, cfg.D, cfg.G, KB, VB)
+        passes += 1
+    return total_by / total_dt / 1e9, passes, total_dt
 
 
 def oracle_sample(cfg, inp, n_seq):
@@ -436,30 +682,20 @@ def oracle_sample(cfg, inp, n_seq):
 
 
 def cpu_baseline(cfg, inp, args):
+    """The oracle's decode on the host cores (all of them, then one), on
+    samples of the main workload sized to about --cpu-seconds each."""
     import oracle
     oracle.lib()
-    target = args.cpu_seconds
-    n_seq = 1
-    t0 = time.perf_counter()
-    by = oracle_step(oracle, cfg, oracle_sample(cfg, inp, n_seq))
-    dt = time.perf_counter() - t0
-    if dt < target / 2 and n_seq < cfg.B:
-        n_seq = int(min(cfg.B, max(1, math.floor(target / max(dt, 1e-3)))))
-        t0 = time.perf_counter()
-        by = oracle_step(oracle, cfg, oracle_sample(cfg, inp, n_seq))
-        dt = time.perf_counter() - t0
-    # the whole batch may still be quick on a large host: repeat the pass
-    sample = oracle_sample(cfg, inp, n_seq)
-    passes, total_by, total_dt = 1, by, dt
-    while total_dt < target:
-        t0 = time.perf_counter()
-        total_by += oracle_step(oracle, cfg, sample)
-        total_dt += time.perf_counter() - t0
-        passes += 1
-    return {"value": round(total_by / total_dt / 1e9, 4), "unit": "GB/s", "cores": oracle.threads(),
-            "kind": "oracle",
-            "sample": f"first {n_seq} of {cfg.B} sequences of {cfg.name}, {passes} oracle pass(es) "
-                      f"(quantize + decode + tiers + repack + tiered), {total_dt:.1f} s"}
+    all_cores = oracle.threads()
+    gbs, passes, dt = oracle_decode_gbs(oracle, cfg, oracle_sample(cfg, inp, cfg.B), args.cpu_seconds)
+    oracle.set_threads(1)
+    n1 = 1
+    gbs1, passes1, dt1 = oracle_decode_gbs(oracle, cfg, oracle_sample(cfg, inp, n1), args.cpu_seconds)
+    oracle.set_threads(all_cores)
+    return {"value": round(gbs, 4), "unit": "GB/s", "cores": all_cores, "kind": "oracle",
+            "sample": f"all {cfg.B} sequences of {cfg.name}, oracle decode (fp64), {passes} pass(es) in {dt:.1f} s",
+            "one_thread": {"value": round(gbs1, 4), "unit": "GB/s", "cores": 1,
+                           "sample": f"first {n1} of {cfg.B} sequences, {passes1} pass(es) in {dt1:.1f} s"}}
 
 
 def run_reference(args):
@@ -468,30 +704,34 @@ def run_reference(args):
         return
     import oracle
     oracle.lib()
-    cfg = W.CONFIGS[CFG_ID]
+    cfg = W.CONFIGS[CFG_MAIN]
     inp = W.make_inputs(cfg, with_mass=True)
-    # bounded sample per step so the whole run stays within a few minutes
-    n_seq = 1
-    sub = oracle_sample(cfg, inp, n_seq)
-    for _ in range(args.warmup):
-        oracle_step(oracle, cfg, sub)
+    k, v, q = W.bf16_bits(inp["k"]), W.bf16_bits(inp["v"]), W.bf16_bits(inp["q"])
+    sl = inp["seq_lens"].numpy()
+    cache = oracle.quantize_kv(KB, VB, cfg.G, k, v, sl)
+    rows = int(sl.astype(np.int64).sum()) * cfg.Hkv
     times, by = [], 0
-    for _ in range(args.steps):
+    for i in range(args.warmup + args.steps):
         t0 = time.perf_counter()
-        by = oracle_step(oracle, cfg, sub)
-        times.append(time.perf_counter() - t0)
-    total = sum(times)
-    value = by * args.steps / total / 1e9
+        _, _, cnt = oracle.decode_attention(KB, VB, cfg.G, sl, q, cache, cfg.softmax_scale, cfg.tau,
+                                            want_mask=False)
+        dt = time.perf_counter() - t0
+        if i >= args.warmup:
+            times.append(dt)
+            by = decode_bytes(rows, rows - int(cnt[1]), cfg.B, cfg.Hq, cfg.D, cfg.G, KB, VB)
+    med = statistics.median(times)
+    value = by / med / 1e9
     line = {
         "impl": "reference", "metric": METRIC, "value": round(value, 4), "unit": "GB/s", "n_gpus": 1,
-        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(total / args.steps * 1e3, 3),
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(med * 1e3, 3),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic",
         "config": {"workload": cfg.name, "B": cfg.B, "Hq": cfg.Hq, "Hkv": cfg.Hkv, "head_dim": cfg.D,
                    "context": cfg.T_cap, "group": cfg.G, "k_bits": KB, "v_bits": VB, "tau": cfg.tau,
-                   "parallelism": "single", "sample_sequences": n_seq},
+                   "parallelism": "single",
+                   "value": "oracle decode algorithmic GB/s, median over the timed steps"},
         "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": oracle.threads(), "kind": "oracle",
-                         "sample": f"first {n_seq} of {cfg.B} sequences per step"},
+                         "sample": f"all {cfg.B} sequences per step, oracle decode (fp64)"},
         "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
@@ -503,10 +743,10 @@ def main():
     ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["lkv", "reference"], default="lkv")
-    ap.add_argument("--e2e-steps", type=int, default=3)
-    ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--no-cpu", action="store_true", help="skip the CPU-oracle baseline leg")
     ap.add_argument("--no-e2e", action="store_true", help="skip the end-to-end (host buffers) leg")
+    ap.add_argument("--no-extras", action="store_true", help="skip the long-context, sweep and tiered workloads")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)   # at least 3 untimed warm-up steps
     if args.impl == "reference":

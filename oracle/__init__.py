@@ -59,6 +59,12 @@ def lib():
         L.lkv_oracle_tiered_attention.argtypes = [_I, _I, _I, _I, _I, _I, _P, _P,
                                                   _P, _P, _P, _P, _P, _P, _P, _P,
                                                   _F, _F, _P, _P, _P]
+        L.lkv_oracle_attention_bf16.restype = _I
+        L.lkv_oracle_attention_bf16.argtypes = [_I, _I, _I, _I, _I, _P, _P, _P, _P, _F, _P]
+        L.lkv_oracle_set_threads.restype = None
+        L.lkv_oracle_set_threads.argtypes = [_I]
+        L.lkv_oracle_get_threads.restype = _I
+        L.lkv_oracle_get_threads.argtypes = []
         _lib = L
     return _lib
 
@@ -250,7 +256,23 @@ def tiered_attention(G, counts, q_bf16, seg_a, seg_b, softmax_scale, tau, want_p
     return out, sc
 
 
+def attention_bf16(seq_lens, q_bf16, k_bf16, v_bf16, softmax_scale):
+    """fp64 softmax attention over the unquantized bf16 K/V (raw uint16 bits,
+    [B][Hkv][T_cap][D]); q bf16 bits [B][Hq][D].  Returns f32 [B][Hq][D]."""
+    B, Hq, D = q_bf16.shape
+    Hkv, T_cap = k_bf16.shape[1], k_bf16.shape[2]
+    q, k, v = _c(q_bf16, np.uint16), _c(k_bf16, np.uint16), _c(v_bf16, np.uint16)
+    out = np.zeros((B, Hq, D), np.float32)
+    _check(lib().lkv_oracle_attention_bf16(B, Hq, Hkv, T_cap, D, _ptr(_c(seq_lens, np.int32)), _ptr(q), _ptr(k),
+                                           _ptr(v), float(softmax_scale), _ptr(out)), "attention_bf16")
+    return out
+
+
+def set_threads(n):
+    """Run the oracle's parallel loops on n threads."""
+    lib().lkv_oracle_set_threads(int(n))
+
+
 def threads():
-    """Number of OpenMP threads the oracle's parallel loops use."""
-    n = os.environ.get("OMP_NUM_THREADS")
-    return int(n) if n else (os.cpu_count() or 1)
+    """Number of threads the oracle's parallel loops use."""
+    return int(lib().lkv_oracle_get_threads())

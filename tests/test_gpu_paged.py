@@ -1,12 +1,13 @@
 """Paged caches: the pool-and-block-table calls give exactly what the
-contiguous calls give on the same tokens, with the pages scattered over a
-pool in random order ("TurboQuant" §与其他优化技术的对比: the quantized
+contiguous calls give on the same tokens, and what the CPU oracle gives,
+with the pages scattered over a pool in random order ("TurboQuant" §与其他优化技术的对比: the quantized
 cache is meant to combine with paged KV management)."""
 import numpy as np
 import pytest
 import torch
 
-from gpu_helpers import dev, gpu_decode, gpu_quantize
+from gpu_helpers import (assert_attention_close, assert_masks_match, dev, gpu_decode, gpu_quantize, oracle_inputs,
+                         vmax)
 from quantized_kv_cache_lkv_b200 import buffers, lkv
 from quantized_kv_cache_lkv_b200 import workloads as W
 
@@ -49,20 +50,24 @@ def setup(kb=6, vb=4, G=64, r=4, seed=3, lens=(768, 300, 1)):
 
 
 @pytest.mark.parametrize("kb,vb,G", [(6, 4, 64), (8, 8, 32), (4, 2, 128)])
-def test_paged_quantize_equals_contiguous(kb, vb, G):
+def test_paged_quantize_equals_contiguous(orc, kb, vb, G):
     cfg, inp, table, pool, _ = setup(kb, vb, G)
     want = gpu_quantize(kb, vb, G, inp)
     got = gather_pool(pool, table, cfg.B, cfg.T_cap)
+    k, v, _, sl = oracle_inputs(inp)
+    o = orc.quantize_kv(kb, vb, G, k, v, sl)
     for key in want:
         for b in range(cfg.B):
             T = int(inp["seq_lens"][b])
             assert torch.equal(got[key][b, :, :T], want[key][b, :, :T]), (key, b)
+            g = np.ascontiguousarray(got[key][b, :, :T].cpu().numpy())
+            assert np.array_equal(g.view(np.uint8), np.ascontiguousarray(o[key][b, :, :T]).view(np.uint8)), (key, b)
 
 
 @pytest.mark.parametrize("r,tau", [(4, 1e-3), (2, 0.0), (1, 1e-4)])
-def test_paged_decode_equals_contiguous(r, tau):
+def test_paged_decode_equals_contiguous(orc, r, tau):
     """Same work partition, same arithmetic: outputs, masks and counts are
-    bit-identical to the contiguous decode."""
+    bit-identical to the contiguous decode, and match the oracle."""
     cfg, inp, table, pool, num_pages = setup(r=r, seed=10 + r)
     cache = gpu_quantize(6, 4, 64, inp)
     want_out, want_mask, want_counts = gpu_decode(6, 4, 64, inp, cache, cfg.softmax_scale, tau)
@@ -80,9 +85,15 @@ def test_paged_decode_equals_contiguous(r, tau):
     np.testing.assert_array_equal(out.cpu().numpy(), want_out)
     np.testing.assert_array_equal(mask.cpu().numpy(), want_mask)
     assert counts.cpu().tolist() == want_counts.tolist()
+    k, v, q, sl = oracle_inputs(inp)
+    o_out, o_mask, o_counts, p = orc.decode_attention(6, 4, 64, sl, q, orc.quantize_kv(6, 4, 64, k, v, sl),
+                                                      cfg.softmax_scale, tau, want_p=True)
+    assert_attention_close(out.cpu().numpy(), o_out, vmax(inp), "paged vs oracle")
+    if assert_masks_match(mask.cpu().numpy(), o_mask, p, np.float32(tau), sl, "paged vs oracle") == 0:
+        assert counts.cpu().tolist() == o_counts.tolist()
 
 
-def test_paged_append_equals_contiguous():
+def test_paged_append_equals_contiguous(orc):
     cfg, inp, table, pool, num_pages = setup(lens=(767, 299, 0))
     pos = torch.tensor([767, 299, 0], dtype=torch.int32)
     k_new = torch.stack([inp["k"][b, :, int(pos[b])] for b in range(3)]).contiguous()
@@ -93,10 +104,14 @@ def test_paged_append_equals_contiguous():
     full = dict(inp, seq_lens=torch.tensor([768, 300, 1], dtype=torch.int32))
     want = gpu_quantize(6, 4, 64, full)
     got = gather_pool(pool, table, 3, cfg.T_cap)
+    k, v, _, sl = oracle_inputs(full)
+    o = orc.quantize_kv(6, 4, 64, k, v, sl)
     for key in want:
         for b in range(3):
             T = int(full["seq_lens"][b])
             assert torch.equal(got[key][b, :, :T], want[key][b, :, :T]), (key, b)
+            g = np.ascontiguousarray(got[key][b, :, :T].cpu().numpy())
+            assert np.array_equal(g.view(np.uint8), np.ascontiguousarray(o[key][b, :, :T]).view(np.uint8)), (key, b)
 
 
 def test_paged_decode_bad_page_is_reported():
@@ -118,10 +133,11 @@ def test_paged_decode_bad_page_is_reported():
 
 
 @pytest.mark.slow
-def test_paged_decode_full_size_equals_contiguous():
+def test_paged_decode_full_size_equals_contiguous(orc):
     """The Llama-3.1-8B-shaped decode (B16, 32 q / 8 kv heads, T8192 = 32
     pages per sequence, tau 1e-4) over a shuffled pool of 520 pages is
-    bit-identical to the contiguous decode."""
+    bit-identical to the contiguous decode, and every sequence matches the
+    oracle."""
     cfg = W.CONFIGS[2]
     B, Hq, Hkv, D, T, G = cfg.B, cfg.Hq, cfg.Hkv, cfg.D, cfg.T_cap, cfg.G
     pps = T // P
@@ -146,3 +162,9 @@ def test_paged_decode_full_size_equals_contiguous():
     assert lkv.lkv_workspace_status(ws) == lkv.LKV_OK
     np.testing.assert_array_equal(out.cpu().numpy(), want_out)
     assert counts.cpu().tolist() == want_counts.tolist()
+    k, v, q, sl = oracle_inputs(inp)
+    o_out, _, o_counts, p = orc.decode_attention(6, 4, G, sl, q, orc.quantize_kv(6, 4, G, k, v, sl),
+                                                 cfg.softmax_scale, cfg.tau, want_p=True)
+    assert_attention_close(out.cpu().numpy(), o_out, vmax(inp), "paged full size vs oracle")
+    if not (np.abs(p - np.float32(cfg.tau)) < 1e-7).any():
+        assert counts.cpu().tolist() == o_counts.tolist()

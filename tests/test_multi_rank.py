@@ -35,7 +35,7 @@ def _rank_main(rank, world, port, out):
         inp = bench.W.make_inputs(small)
         local_ms = 10.0 + 5.0 * rank                      # rank 1 is the slower one
         job_ms = bench.max_over_ranks(local_ms)
-        value = bench.job_throughput(1_000_000, world, 4, job_ms)
+        value = bench.job_throughput(1_000_000, world, job_ms * 1e-3)
         out[rank] = {"seed": cfg.seed, "k_sum": float(inp["k"].float().sum()), "job_ms": job_ms, "value": value}
     finally:
         dist.destroy_process_group()
@@ -51,12 +51,21 @@ def test_two_ranks_shard_batches_and_agree_on_time():
     assert res[0]["seed"] != res[1]["seed"]
     assert res[0]["k_sum"] != res[1]["k_sum"]                    # distinct batches
     assert res[0]["job_ms"] == res[1]["job_ms"] == 15.0          # slowest rank
-    # 2 ranks x 4 steps x 1 MB over 15 ms
-    assert res[0]["value"] == pytest.approx(2 * 4 * 1e6 / 15e-3 / 1e9)
+    # 2 ranks x 1 MB over the slowest rank's 15 ms
+    assert res[0]["value"] == pytest.approx(2 * 1e6 / 15e-3 / 1e9)
 
 
 def test_single_process_needs_no_group():
     assert bench.max_over_ranks(3.5) == 3.5
-    assert bench.job_throughput(2e9, 1, 1, 1000.0) == pytest.approx(2.0)
+    assert bench.job_throughput(2e9, 1, 1.0) == pytest.approx(2.0)
     a, b = bench.rank_workload(0), bench.rank_workload(0)
     assert a.seed == b.seed                                       # reproducible
+
+
+def test_decode_bytes_per_row():
+    """Algorithmic bytes of the decode metric: for the Llama-3.1-8B-shaped
+    K6V4 rows (D 128, group 64) a K row is 96 code bytes + 16 bytes of
+    (scale, zero), a kept V row 64 + 16, and q (bf16) + out (f32) 6 bytes
+    per (b, h, d)."""
+    assert bench.decode_bytes(10, 4, 2, 32, 128, 64, 6, 4) == 10 * 112 + 4 * 80 + 2 * 32 * 128 * 6
+    assert bench.quantize_bytes(3, 128, 64, 6, 4) == 3 * (512 + 96 + 64 + 32)

@@ -480,6 +480,46 @@ def test_attention_mass_is_group_mean_of_torch_softmax(orc):
 
 # ---------------------------------------------------------------- tiers
 
+# ---------------------------------------------------------------- bf16-cache attention
+
+def _bf16_f32(a_bits):
+    return torch.from_numpy(np.ascontiguousarray(a_bits).view(np.int16)).view(torch.bfloat16).float().numpy()
+
+
+def test_attention_bf16_vs_torch_fp64(orc):
+    """The unquantized-cache attention (the reference the quantized decode's
+    quality is measured against) matches torch float64 softmax over the same
+    bf16 values, ragged lengths and GQA included, T = 0 giving zeros."""
+    cfg = W.scaled(W.CONFIGS[4], B=5, T_cap=150, seq_lo=1, seq_hi=150, seed=31)
+    inp = W.make_inputs(cfg, seq_lens=torch.tensor([150, 1, 0, 77, 149], dtype=torch.int32))
+    k, v, q, sl = (W.bf16_bits(inp["k"]), W.bf16_bits(inp["v"]), W.bf16_bits(inp["q"]), inp["seq_lens"].numpy())
+    got = orc.attention_bf16(sl, q, k, v, cfg.softmax_scale)
+    want = _torch_attention(q, _bf16_f32(k), _bf16_f32(v), sl, cfg.softmax_scale, 0.0)
+    assert np.abs(got - want).max() <= 1e-6 * max(1.0, np.abs(want).max())
+    assert np.all(got[2] == 0)
+    # T = 1: the output is that row's V exactly (p = 1)
+    r = cfg.Hq // cfg.Hkv
+    assert np.array_equal(got[1], np.repeat(_bf16_f32(v)[1, :, 0], r, axis=0))
+
+
+def test_attention_bf16_closed_forms(orc):
+    """q = 0 gives the mean of V; a key far along q returns its V row."""
+    B, Hq, Hkv, T, D = 1, 4, 2, 33, 64
+    rng = np.random.default_rng(5)
+    v = bf16_round(rng.standard_normal((B, Hkv, T, D)).astype(np.float32))
+    k = bf16_round(rng.standard_normal((B, Hkv, T, D)).astype(np.float32))
+    tob = lambda a: torch.from_numpy(np.asarray(a, np.float32)).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    sl = np.array([T], np.int32)
+    out = orc.attention_bf16(sl, tob(np.zeros((B, Hq, D))), tob(k), tob(v), 0.125)
+    mean = v.astype(np.float64).mean(axis=2)
+    assert np.abs(out[0] - np.repeat(mean[0], 2, axis=0)).max() <= 1e-6
+    q = bf16_round(rng.standard_normal((B, Hq, D)).astype(np.float32))
+    k2 = k.copy()
+    k2[0, 1, 7] = bf16_round(q[0, 2] * 40)   # KV head 1 serves query heads 2 and 3
+    out = orc.attention_bf16(sl, tob(q), tob(k2), tob(v), 1.0)
+    assert np.abs(out[0, 2] - v[0, 1, 7]).max() <= 1e-6
+
+
 def test_tier_boundaries(orc):
     """Super KV Compression §第二层: above tau_high -> 6-bit V (2), within
     [tau_low, tau_high] -> 4-bit V (1), below tau_low -> evicted (0)."""

@@ -8,7 +8,8 @@ import numpy as np
 import pytest
 import torch
 
-from gpu_helpers import assert_attention_close, dev, gpu_decode, gpu_quantize, vmax
+from gpu_helpers import (assert_attention_close, assert_masks_match, dev, gpu_decode, gpu_quantize, oracle_inputs,
+                         vmax)
 from quantized_kv_cache_lkv_b200 import lkv
 from quantized_kv_cache_lkv_b200 import workloads as W
 
@@ -37,7 +38,7 @@ def static_decode(kb, vb, G, inp, cache, softmax_scale, tau, seq_lens=None):
     ("ragged_r8", W.Config("ragged_r8", B=3, Hq=16, Hkv=2, D=128, T_cap=700, G=64, bits=[(6, 4)],
                            hh_frac=0.01, seed=91), 1e-3),
 ])
-def test_static_matches_workspace_entry_point_twice(name, cfg, tau):
+def test_static_matches_workspace_entry_point_twice(orc, name, cfg, tau):
     inp = W.make_inputs(cfg)
     need = lkv.lkv_decode_workspace_bytes((6, 4, cfg.G), cfg.B, cfg.Hq, cfg.Hkv, cfg.T_cap, cfg.D)
     assert 0 < need <= lkv.LKV_STATIC_WORKSPACE_BYTES
@@ -50,9 +51,16 @@ def test_static_matches_workspace_entry_point_twice(name, cfg, tau):
         assert_attention_close(out, want_out, vmax(inp), what)
         np.testing.assert_array_equal(mask, want_mask, err_msg=what)
         assert counts.tolist() == want_counts.tolist(), what
+    # and against the oracle, which quantizes from bf16 itself: every sequence
+    k, v, q, sl = oracle_inputs(inp)
+    o_out, o_mask, o_counts, p = orc.decode_attention(6, 4, cfg.G, sl, q, orc.quantize_kv(6, 4, cfg.G, k, v, sl),
+                                                      cfg.softmax_scale, tau, want_p=True)
+    assert_attention_close(out, o_out, vmax(inp), f"{name} vs oracle")
+    if assert_masks_match(mask, o_mask, p, np.float32(tau), sl, f"{name} vs oracle") == 0:
+        assert counts.tolist() == o_counts.tolist()
 
 
-def test_static_failed_call_leaves_nothing_behind():
+def test_static_failed_call_leaves_nothing_behind(orc):
     """A length beyond T_cap is reported in the status word of that call only;
     the next call on the same scratch is clean and correct."""
     cfg = W.Config("bad", B=2, Hq=8, Hkv=2, D=128, T_cap=512, G=64, bits=[(6, 4)], seed=17)
@@ -67,3 +75,8 @@ def test_static_failed_call_leaves_nothing_behind():
     assert status == lkv.LKV_OK
     assert_attention_close(out, want_out, vmax(inp), "after a failed call")
     assert counts.tolist() == want_counts.tolist()
+    k, v, q, sl = oracle_inputs(inp)
+    o_out, _, o_counts = orc.decode_attention(6, 4, 64, sl, q, orc.quantize_kv(6, 4, 64, k, v, sl),
+                                              cfg.softmax_scale, 0.0)
+    assert_attention_close(out, o_out, vmax(inp), "after a failed call, vs oracle")
+    assert counts.tolist() == o_counts.tolist()
