@@ -50,9 +50,12 @@ static float bf16_to_float(uint16_t h)
     return f;
 }
 
+/* 16 is the passthrough width of [SKV] §第一层 "异常层处理" (outlier layers
+ * kept in 16-bit floating point): the row holds the bf16 values unchanged,
+ * with no (scale, zero). */
 static int bits_supported(int bits)
 {
-    return bits == 2 || bits == 4 || bits == 6 || bits == 8;
+    return bits == 2 || bits == 4 || bits == 6 || bits == 8 || bits == 16;
 }
 
 /* Bytes of one packed token row: D codes of `bits` bits each. */
@@ -174,12 +177,19 @@ void lkv_oracle_unpack_row(const uint8_t *row, int D, int bits, uint32_t *codes)
     }
 }
 
-/* Quantize and pack one token row of D bf16 values in groups of G. */
+/* Quantize and pack one token row of D bf16 values in groups of G.  At the
+ * passthrough width the "code" of a value is its own bf16 bit pattern and
+ * sz_row is not touched. */
 static void quantize_row(const uint16_t *src, int D, int G, int bits,
                          uint8_t *codes_row, float *sz_row)
 {
     float xs[256];
     uint32_t cs[256];
+    if (bits == 16) {
+        for (int d = 0; d < D; ++d) cs[d] = src[d];
+        lkv_oracle_pack_row(cs, D, bits, codes_row);
+        return;
+    }
     for (int d = 0; d < D; ++d) xs[d] = bf16_to_float(src[d]);
     for (int g = 0; g < D / G; ++g) {
         lkv_oracle_quantize_group(xs + g * G, G, bits, cs + g * G,
@@ -194,6 +204,10 @@ static void dequant_row(const uint8_t *codes_row, const float *sz_row, int D, in
 {
     uint32_t cs[256];
     lkv_oracle_unpack_row(codes_row, D, bits, cs);
+    if (bits == 16) {  /* passthrough: the bf16 value itself */
+        for (int d = 0; d < D; ++d) out[d] = bf16_to_float((uint16_t)cs[d]);
+        return;
+    }
     for (int d = 0; d < D; ++d) {
         int g = d / G;
         out[d] = lkv_oracle_dequant(cs[d], sz_row[2 * g], sz_row[2 * g + 1]);

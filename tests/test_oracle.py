@@ -311,9 +311,54 @@ def test_compression_ratios_match_pages(orc):
         n_t = 2 if vb else 1
         src = n_t * x.size * 2
         packed = cache["k_codes"].nbytes + (cache["v_codes"].nbytes if vb else 0)
-        if meta:
-            packed += cache["k_sz"].nbytes + (cache["v_sz"].nbytes if vb else 0)
+        if meta:  # a 16-bit (passthrough) tensor has no (scale, zero)
+            packed += (cache["k_sz"].nbytes if kb < 16 else 0) + (cache["v_sz"].nbytes if 0 < vb < 16 else 0)
         assert src / packed == pytest.approx(want, rel=1e-12), label
+
+
+def test_passthrough_width_keeps_the_values(orc):
+    """16 bits (Super KV Compression §第一层, outlier layers kept in 16-bit
+    floating point): the row is the bf16 values themselves, byte for byte,
+    with no (scale, zero) written, and reconstructs every value exactly --
+    NaN and infinity included; K and V can take different widths."""
+    rng = np.random.default_rng(3)
+    B, H, T, D, G = 2, 2, 9, 64, 32
+    x = rng.standard_normal((B, H, T, D)).astype(np.float32) * np.float32(100)
+    x[0, 0, 0, :4] = [np.inf, -np.inf, np.nan, 3e38]
+    kb16 = W.bf16_bits(torch.from_numpy(x).to(torch.bfloat16))
+    vb16 = W.bf16_bits(torch.from_numpy(-x).to(torch.bfloat16))
+    sl = np.array([9, 4], np.int32)
+    cache = orc.quantize_kv(16, 4, G, kb16, vb16, sl)
+    assert orc.row_bytes(16, D) == 2 * D
+    for b in range(B):
+        n = int(sl[b])
+        assert np.array_equal(cache["k_codes"][b, :, :n].reshape(-1), kb16[b, :, :n].reshape(-1).view(np.uint8))
+        assert not cache["k_codes"][b, :, n:].any()
+        kh = orc.dequant_rows(cache["k_codes"][b, :, :n].copy(), cache["k_sz"][b, :, :n].copy(), D, G, 16)
+        want = torch.from_numpy(kb16[b, :, :n].view(np.int16)).view(torch.bfloat16).float().numpy()
+        assert np.array_equal(kh.view(np.uint32), want.view(np.uint32))  # bit-exact, NaN included
+    assert not cache["k_sz"].any()                 # nothing written for the 16-bit tensor
+    assert cache["v_sz"][0, :, :9].any()          # the 4-bit tensor has its (scale, zero)
+
+
+@pytest.mark.parametrize("kb,vb", [(16, 16), (16, 4), (6, 16)])
+def test_decode_passthrough_vs_torch(orc, kb, vb):
+    """Decode over caches with a 16-bit tensor against torch float64 softmax
+    over the reconstructed values; K16V16 at tau 0 is plain attention over
+    the bf16 cache."""
+    cfg = W.scaled(W.CONFIGS[1], seed=70 + kb + vb)
+    inp = W.make_inputs(cfg, seq_lens=torch.tensor([200], dtype=torch.int32))
+    k, v, q, sl = (W.bf16_bits(inp["k"]), W.bf16_bits(inp["v"]), W.bf16_bits(inp["q"]), inp["seq_lens"].numpy())
+    cache = orc.quantize_kv(kb, vb, cfg.G, k, v, sl)
+    kh, vh = _dequant_cache(orc, cache, kb, vb, cfg.D, cfg.G)
+    for tau in (0.0, 1e-3):
+        out, _, _ = orc.decode_attention(kb, vb, cfg.G, sl, q, cache, cfg.softmax_scale, tau)
+        want = _torch_attention(q, kh, vh, sl, cfg.softmax_scale, tau)
+        assert np.abs(out - want).max() <= 1e-6 * max(1.0, np.abs(want).max())
+    if kb == vb == 16:
+        bf = _torch_attention(q, _bf16_f32(k), _bf16_f32(v), sl, cfg.softmax_scale, 0.0)
+        out, _, _ = orc.decode_attention(kb, vb, cfg.G, sl, q, cache, cfg.softmax_scale, 0.0)
+        assert np.abs(out - bf).max() <= 1e-6
 
 
 # ---------------------------------------------------------------- attention
