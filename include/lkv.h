@@ -33,7 +33,12 @@
  *   G contiguous head_dim channels of one token share one (scale, zero);
  *   G in {32, 64, 128}, G divides D, ng = D / G.  T_cap cache capacity
  *   in tokens; T_b = seq_lens[b] valid tokens of sequence b.  bits in
- *   {2, 4, 6, 8}.
+ *   {2, 4, 6, 8, 16}.  16 is the passthrough width of outlier layers
+ *   ([SKV] §第一层 "异常层处理": kept in 16-bit floating point): the row
+ *   holds the bf16 values unchanged (the codes below with bits = 16 are the
+ *   bf16 bit patterns), and that tensor has no (scale, zero) -- its sz
+ *   pointer is ignored and may be NULL.  A per-layer width policy is a
+ *   table on the caller's side: each layer's cache has its own lkv_qspec.
  *
  *   K, V (bf16)  [B][Hkv][T_cap][D]
  *   codes (u8)   [B][Hkv][T_cap][D*bits/8]   one packed row per token:
@@ -73,8 +78,8 @@ enum lkv_status {
 
 /* Quantizer settings: bit widths of K and V codes and the group size. */
 typedef struct {
-    int32_t k_bits; /* 2, 4, 6 or 8 */
-    int32_t v_bits; /* 2, 4, 6 or 8 */
+    int32_t k_bits; /* 2, 4, 6, 8, or 16 (passthrough bf16, no scale/zero) */
+    int32_t v_bits; /* 2, 4, 6, 8, or 16 (passthrough bf16, no scale/zero) */
     int32_t group;  /* 32, 64 or 128; divides D */
 } lkv_qspec;
 
@@ -171,7 +176,7 @@ LKV_API int lkv_append_kv_paged(lkv_qspec spec, int B, int Hkv, int pages_per_se
 
 /*
  * lkv_decode_attention over a paged cache.  Groups of 1, 2 or 4 query heads
- * (LKV_ERR_UNSUPPORTED otherwise).  The workspace is that of
+ * and widths below 16 bits (LKV_ERR_UNSUPPORTED otherwise).  The workspace is that of
  * lkv_decode_attention with T_cap = pages_per_seq * LKV_PAGE_TOKENS; the
  * skip mask is [B][Hq][T_cap] over logical positions.
  */

@@ -34,7 +34,8 @@ constexpr size_t kHeaderBytes = 256;  // status, wait limit, done counter, skip-
 
 size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
 
-bool bits_ok(int b) { return b == 2 || b == 4 || b == 6 || b == 8; }
+// 16 is the passthrough width: the row holds the bf16 values, with no (scale, zero)
+bool bits_ok(int b) { return b == 2 || b == 4 || b == 6 || b == 8 || b == 16; }
 bool dim_ok(int D) { return D == 64 || D == 128; }
 bool group_ok(int G, int D) { return (G == 32 || G == 64 || G == 128) && G <= D && D % G == 0; }
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -165,7 +166,7 @@ int run_attention(DecodeArgs& a, int D, int kb, int vb0, int vb1, void* ws, size
   f.num_pages = num_pages;
   cudaError_t e;
   if (block_table != nullptr) {
-    if (vb0 != vb1) return LKV_ERR_UNSUPPORTED;
+    if (vb0 != vb1 || kb == 16 || vb0 == 16) return LKV_ERR_UNSUPPORTED;
     switch (kb) {
       case 2: e = launch_fused_paged_k2(f, D, L.H, vb0, L.smem_bytes, L.grid, s); break;
       case 4: e = launch_fused_paged_k4(f, D, L.H, vb0, L.smem_bytes, L.grid, s); break;
@@ -180,6 +181,7 @@ int run_attention(DecodeArgs& a, int D, int kb, int vb0, int vb1, void* ws, size
     case 4: e = launch_fused_k4(f, D, L.H, vb0, vb1, L.smem_bytes, L.grid, s); break;
     case 6: e = launch_fused_k6(f, D, L.H, vb0, vb1, L.smem_bytes, L.grid, s); break;
     case 8: e = launch_fused_k8(f, D, L.H, vb0, vb1, L.smem_bytes, L.grid, s); break;
+    case 16: e = launch_fused_k16(f, D, L.H, vb0, vb1, L.smem_bytes, L.grid, s); break;
     default: return LKV_ERR_UNSUPPORTED;
   }
   return from_cuda(e);
@@ -281,8 +283,8 @@ int quantize_impl(lkv_qspec spec, int B, int Hkv, int T_cap, int D, const int32_
   int rc = check_cache_shape(B, Hkv, T_cap, D, spec.group);
   if (rc) return rc;
   const bool ne = (long long)B * Hkv * T_cap > 0;
-  if (!ptr_ok(seq_lens, B > 0) || !ptr_ok(k, ne) || !ptr_ok(v, ne) || !ptr_ok(k_codes, ne) || !ptr_ok(k_sz, ne) ||
-      !ptr_ok(v_codes, ne) || !ptr_ok(v_sz, ne))
+  if (!ptr_ok(seq_lens, B > 0) || !ptr_ok(k, ne) || !ptr_ok(v, ne) || !ptr_ok(k_codes, ne) || !ptr_ok(k_sz, ne && spec.k_bits < 16) ||
+      !ptr_ok(v_codes, ne) || !ptr_ok(v_sz, ne && spec.v_bits < 16))
     return LKV_ERR_INVALID_ARG;
   if (!ne) return LKV_OK;
   QuantizeArgs a{};
@@ -305,8 +307,8 @@ int append_impl(lkv_qspec spec, int B, int Hkv, int T_cap, int D, const int32_t*
   int rc = check_cache_shape(B, Hkv, T_cap, D, spec.group);
   if (rc) return rc;
   const bool ne = (long long)B * Hkv * T_cap > 0;
-  if (!ptr_ok(pos, ne) || !ptr_ok(k_new, ne) || !ptr_ok(v_new, ne) || !ptr_ok(k_codes, ne) || !ptr_ok(k_sz, ne) ||
-      !ptr_ok(v_codes, ne) || !ptr_ok(v_sz, ne))
+  if (!ptr_ok(pos, ne) || !ptr_ok(k_new, ne) || !ptr_ok(v_new, ne) || !ptr_ok(k_codes, ne) || !ptr_ok(k_sz, ne && spec.k_bits < 16) ||
+      !ptr_ok(v_codes, ne) || !ptr_ok(v_sz, ne && spec.v_bits < 16))
     return LKV_ERR_INVALID_ARG;
   if (!ne) return LKV_OK;
   QuantizeArgs a{};
@@ -438,7 +440,7 @@ int decode_impl(lkv_qspec spec, int B, int Hq, int Hkv, int T_cap, int D, const 
   if (!std::isfinite(softmax_scale) || std::isnan(tau)) return LKV_ERR_INVALID_ARG;
   const bool ne = (long long)B * Hkv * T_cap > 0;
   if (!ptr_ok(seq_lens, B > 0) || !ptr_ok(q, B > 0) || !ptr_ok(out, B > 0) || !ptr_ok(k_codes, ne) ||
-      !ptr_ok(k_sz, ne) || !ptr_ok(v_codes, ne) || !ptr_ok(v_sz, ne))
+      !ptr_ok(k_sz, ne && spec.k_bits < 16) || !ptr_ok(v_codes, ne) || !ptr_ok(v_sz, ne && spec.v_bits < 16))
     return LKV_ERR_INVALID_ARG;
   if (skip_counts && !aligned16(skip_counts)) return LKV_ERR_INVALID_ARG;
   if (mass && (reinterpret_cast<uintptr_t>(mass) & 3u) != 0) return LKV_ERR_INVALID_ARG;
@@ -481,7 +483,7 @@ int lkv_decode_attention_static(lkv_qspec spec, int B, int Hq, int Hkv, int T_ca
   if (!std::isfinite(softmax_scale) || std::isnan(tau)) return LKV_ERR_INVALID_ARG;
   const bool ne = (long long)B * Hkv * T_cap > 0;
   if (!ptr_ok(seq_lens, B > 0) || !ptr_ok(q, B > 0) || !ptr_ok(out, B > 0) || !ptr_ok(k_codes, ne) ||
-      !ptr_ok(k_sz, ne) || !ptr_ok(v_codes, ne) || !ptr_ok(v_sz, ne))
+      !ptr_ok(k_sz, ne && spec.k_bits < 16) || !ptr_ok(v_codes, ne) || !ptr_ok(v_sz, ne && spec.v_bits < 16))
     return LKV_ERR_INVALID_ARG;
   if (skip_counts && !aligned16(skip_counts)) return LKV_ERR_INVALID_ARG;
   if (status && (reinterpret_cast<uintptr_t>(status) & 3u) != 0) return LKV_ERR_INVALID_ARG;

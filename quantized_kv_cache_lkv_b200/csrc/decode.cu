@@ -146,16 +146,29 @@ __global__ void __launch_bounds__(kThreads) k_phase_kernel(DecodeArgs a) {
       const long long row = (long long)bg * a.T_cap + (seg ? v - sl.n0 : v);
       LaneWords<KB> lw;
       load_lane_words<KB>(a.kc[seg] + row * (D * KB / 8) + j * (2 * KB), lw);
-      const float2 sz = __ldg(reinterpret_cast<const float2*>(a.ksz[seg] + (row * ng + gi) * 2));
-      float2 f[8];
-      unpack16_f<KB>(lw, f);
-      const float u = sz.x * (float)(1 << KB);
+      if constexpr (KB == 16) {
+        // passthrough width: the bf16 K values themselves
 #pragma unroll
-      for (int h = 0; h < H; ++h) {
-        float2 acc = make_float2(0.0f, 0.0f);
+        for (int h = 0; h < H; ++h) {
+          float2 acc = make_float2(0.0f, 0.0f);
 #pragma unroll
-        for (int i = 0; i < 8; ++i) acc = __ffma2_rn(qf[h][i], f[i], acc);
-        dot[h] = fmaf(u, (acc.x + acc.y) - Q[h], sz.y * Q[h]);
+          for (int i = 0; i < 8; ++i)
+            acc = __ffma2_rn(qf[h][i], make_float2(__uint_as_float(lw.w[i] << 16), __uint_as_float(lw.w[i] & 0xFFFF0000u)),
+                             acc);
+          dot[h] = acc.x + acc.y;
+        }
+      } else {
+        const float2 sz = __ldg(reinterpret_cast<const float2*>(a.ksz[seg] + (row * ng + gi) * 2));
+        float2 f[8];
+        unpack16_f<KB>(lw, f);
+        const float u = sz.x * (float)(1 << KB);
+#pragma unroll
+        for (int h = 0; h < H; ++h) {
+          float2 acc = make_float2(0.0f, 0.0f);
+#pragma unroll
+          for (int i = 0; i < 8; ++i) acc = __ffma2_rn(qf[h][i], f[i], acc);
+          dot[h] = fmaf(u, (acc.x + acc.y) - Q[h], sz.y * Q[h]);
+        }
       }
     }
     hidx = 0;
@@ -203,18 +216,30 @@ __device__ __forceinline__ void v_row_accumulate(const uint8_t* __restrict__ cod
                                                  float2 (&acc)[H][8], float (&Z)[H]) {
   LaneWords<VB> lw;
   load_lane_words<VB>(codes + j * (2 * VB), lw);
-  const float2 sz = __ldg(reinterpret_cast<const float2*>(sz_row + gi * 2));
-  float2 f[8];
-  unpack16_f<VB>(lw, f);
-  const float u = sz.x * (float)(1 << VB);
-  const float zu = sz.y - u;
+  if constexpr (VB == 16) {
+    // passthrough width: the bf16 V values themselves
 #pragma unroll
-  for (int h = 0; h < H; ++h) {
-    const float w = keep[h] ? p[h] : 0.0f;
-    const float wu = w * u;
+    for (int h = 0; h < H; ++h) {
+      const float w = keep[h] ? p[h] : 0.0f;
 #pragma unroll
-    for (int i = 0; i < 8; ++i) acc[h][i] = __ffma2_rn(f2(wu), f[i], acc[h][i]);
-    Z[h] = fmaf(w, zu, Z[h]);
+      for (int i = 0; i < 8; ++i)
+        acc[h][i] = __ffma2_rn(f2(w), make_float2(__uint_as_float(lw.w[i] << 16), __uint_as_float(lw.w[i] & 0xFFFF0000u)),
+                               acc[h][i]);
+    }
+  } else {
+    const float2 sz = __ldg(reinterpret_cast<const float2*>(sz_row + gi * 2));
+    float2 f[8];
+    unpack16_f<VB>(lw, f);
+    const float u = sz.x * (float)(1 << VB);
+    const float zu = sz.y - u;
+#pragma unroll
+    for (int h = 0; h < H; ++h) {
+      const float w = keep[h] ? p[h] : 0.0f;
+      const float wu = w * u;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) acc[h][i] = __ffma2_rn(f2(wu), f[i], acc[h][i]);
+      Z[h] = fmaf(w, zu, Z[h]);
+    }
   }
 }
 
@@ -383,6 +408,7 @@ cudaError_t launch_k_bits(const DecodeArgs& a, int kb, dim3 grid, cudaStream_t s
     case 4: return launch_k<D, H, 4>(a, grid, s);
     case 6: return launch_k<D, H, 6>(a, grid, s);
     case 8: return launch_k<D, H, 8>(a, grid, s);
+    case 16: return launch_k<D, H, 16>(a, grid, s);
   }
   return cudaErrorInvalidValue;
 }
@@ -395,6 +421,7 @@ cudaError_t launch_v_bits(const DecodeArgs& a, int vb0, int vb1, dim3 grid, cuda
       case 4: v_phase_kernel<D, H, 4, 4><<<grid, kThreads, 0, s>>>(a); return cudaGetLastError();
       case 6: v_phase_kernel<D, H, 6, 6><<<grid, kThreads, 0, s>>>(a); return cudaGetLastError();
       case 8: v_phase_kernel<D, H, 8, 8><<<grid, kThreads, 0, s>>>(a); return cudaGetLastError();
+      case 16: v_phase_kernel<D, H, 16, 16><<<grid, kThreads, 0, s>>>(a); return cudaGetLastError();
     }
   } else if (vb0 == 6 && vb1 == 4) {
     v_phase_kernel<D, H, 6, 4><<<grid, kThreads, 0, s>>>(a);

@@ -99,14 +99,15 @@ struct Geo {
   static constexpr int SWB = SW * 4;
   static constexpr int KS = D / 16;                // MMA k-steps per row
   static constexpr int kStageCodes = kChunk * RB;             // a stage holds one chunk
-  static constexpr int kStageSz = (kChunk + 2) * (D / 32) * 8;  // ng <= D/32, plus alignment rows
+  // (scale, zero) rows: ng <= D/32, plus alignment rows; none at the 16-bit width
+  static constexpr int kStageSz = KB == 16 ? 0 : (kChunk + 2) * (D / 32) * 8;
   static constexpr int kStageBytes = (kStageCodes + kStageSz + 127) / 128 * 128;
 };
 
 // Host-side view of the geometry (the same formulas as Geo).
 inline int stage_bytes_host(int D, int KB) {
   const int rb = D * KB / 8;
-  return (kChunk * rb + (kChunk + 2) * (D / 32) * 8 + 127) / 128 * 128;
+  return (kChunk * rb + (KB == 16 ? 0 : (kChunk + 2) * (D / 32) * 8) + 127) / 128 * 128;
 }
 
 // Unit-list record (ints): u, first chunk, chunks, n0, n1, owned, chunks of
@@ -281,21 +282,34 @@ template <int VB>
 __device__ __forceinline__ void ldg_v(const uint8_t* codes_row, const float* sz_row, int j, int gi,
                                       LaneWords<VB>& lw, float2& sz) {
   load_lane_words<VB>(codes_row + j * (2 * VB), lw);
-  sz = __ldg(reinterpret_cast<const float2*>(sz_row + gi * 2));
+  if constexpr (VB == 16) sz = make_float2(0.0f, 0.0f);  // passthrough width: no (scale, zero)
+  else sz = __ldg(reinterpret_cast<const float2*>(sz_row + gi * 2));
 }
 
 template <int H, int VB>
 __device__ __forceinline__ void accumulate_v(const LaneWords<VB>& lw, float2 sz, const float (&w)[H],
                                              float2 (&acc)[H][8], float (&Z)[H]) {
   float2 c[8];
-  unpack16_int_r<VB>(lw, c);
+  if constexpr (VB == 16) {
+    // passthrough width: the lane's 16 bf16 values, weighted as they are
 #pragma unroll
-  for (int h = 0; h < H; ++h) {
-    const float ws = w[h] * sz.x;
-    const float2 w2 = make_float2(ws, ws);
+    for (int i = 0; i < 8; ++i) c[i] = make_float2(__uint_as_float(lw.w[i] << 16), __uint_as_float(lw.w[i] & 0xFFFF0000u));
 #pragma unroll
-    for (int i = 0; i < 8; ++i) acc[h][i] = __ffma2_rn(w2, c[i], acc[h][i]);
-    Z[h] = fmaf(w[h], sz.y, Z[h]);
+    for (int h = 0; h < H; ++h) {
+      const float2 w2 = make_float2(w[h], w[h]);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) acc[h][i] = __ffma2_rn(w2, c[i], acc[h][i]);
+    }
+  } else {
+    unpack16_int_r<VB>(lw, c);
+#pragma unroll
+    for (int h = 0; h < H; ++h) {
+      const float ws = w[h] * sz.x;
+      const float2 w2 = make_float2(ws, ws);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) acc[h][i] = __ffma2_rn(w2, c[i], acc[h][i]);
+      Z[h] = fmaf(w[h], sz.y, Z[h]);
+    }
   }
 }
 
@@ -354,8 +368,13 @@ __device__ __forceinline__ void mma_pair(const uint8_t* codes, int tig, int gid,
     for (int m = 0; m < 2; ++m) {
       const uint32_t a0 = a_reg<KB, 2 * s>(w[m][0]), a1 = a_reg<KB, 2 * s>(w[m][1]);
       const uint32_t a2 = a_reg<KB, 2 * s + 1>(w[m][0]), a3 = a_reg<KB, 2 * s + 1>(w[m][1]);
-      hmma16816(acc[m][0], a0, a1, a2, a3, bf[0][2 * s], bf[0][2 * s + 1]);
-      if constexpr (NT == 2) hmma16816(acc[m][1], a0, a1, a2, a3, bf[1][2 * s], bf[1][2 * s + 1]);
+      if constexpr (KB == 16) {
+        hmma16816_bf16(acc[m][0], a0, a1, a2, a3, bf[0][2 * s], bf[0][2 * s + 1]);
+        if constexpr (NT == 2) hmma16816_bf16(acc[m][1], a0, a1, a2, a3, bf[1][2 * s], bf[1][2 * s + 1]);
+      } else {
+        hmma16816(acc[m][0], a0, a1, a2, a3, bf[0][2 * s], bf[0][2 * s + 1]);
+        if constexpr (NT == 2) hmma16816(acc[m][1], a0, a1, a2, a3, bf[1][2 * s], bf[1][2 * s + 1]);
+      }
     }
   };
   step(std::integral_constant<int, 0>{});
@@ -562,12 +581,18 @@ __global__ void __launch_bounds__(kThreads, 1) fused_decode_kernel(FusedArgs a) 
       int ex = 0;
       const bool fin = amax > 0.0f && amax <= FLT_MAX;
       if (fin) frexpf(amax, &ex);
-      const int E = fin ? 15 - ex : 0;
+      // 16-bit K meets q in a bf16 MMA: q stays as it is (E = 0)
+      const int E = (fin && KB != 16) ? 15 - ex : 0;
       __half* qd = (e < kQSlots ? reinterpret_cast<__half*>(smem_raw + kQOff) + e * H * D
                                 : reinterpret_cast<__half*>(a.qbuf) + (long long)x.u * H * D) +
                    h * D + lane * DPL;
+      if constexpr (KB == 16) {
 #pragma unroll
-      for (int i = 0; i < DPL; ++i) qd[i] = __float2half_rn(ldexpf(v[i], E));
+        for (int i = 0; i < DPL; ++i) reinterpret_cast<uint16_t*>(qd)[i] = qs[i];
+      } else {
+#pragma unroll
+        for (int i = 0; i < DPL; ++i) qd[i] = __float2half_rn(ldexpf(v[i], E));
+      }
       const int lpg = d.G / DPL;  // lanes per quantization group
       for (int off = 1; off < lpg; off <<= 1) s += __shfl_xor_sync(kFull, s, off);
       float* az = e < kQSlots ? reinterpret_cast<float*>(smem_raw + kAzOff) + (e * H + h) * 8
@@ -609,7 +634,7 @@ __global__ void __launch_bounds__(kThreads, 1) fused_decode_kernel(FusedArgs a) 
           const int r0 = (ng == 1) ? (row & ~1) : row;
           const int r1 = (ng == 1) ? ((row + rows + 1) & ~1) : row + rows;
           const uint32_t cbytes = (uint32_t)rows * Gk::RB;
-          const uint32_t sbytes = (uint32_t)(r1 - r0) * ng * 8;
+          const uint32_t sbytes = KB == 16 ? 0u : (uint32_t)(r1 - r0) * ng * 8;  // none at the 16-bit width
           uint8_t* dst = ring + (size_t)s * Gk::kStageBytes;
           mbar_arrive_expect_tx(&full[s], cbytes + sbytes);
           // a chunk is one page of a paged cache
@@ -617,7 +642,7 @@ __global__ void __launch_bounds__(kThreads, 1) fused_decode_kernel(FusedArgs a) 
           const long long pr = PAGED ? unit_row<PAGED>(a, x.u, row) : ubase + row;
           const long long pr0 = PAGED ? unit_row<PAGED>(a, x.u, r0) : ubase + r0;
           bulk_g2s(dst, d.kc[cr.seg] + pr * Gk::RB, cbytes, &full[s], pol);
-          bulk_g2s(dst + Gk::kStageCodes, d.ksz[cr.seg] + pr0 * ng * 2, sbytes, &full[s], pol);
+          if (sbytes > 0) bulk_g2s(dst + Gk::kStageCodes, d.ksz[cr.seg] + pr0 * ng * 2, sbytes, &full[s], pol);
         } else {
           mbar_arrive(&full[s]);
         }
@@ -664,7 +689,7 @@ __global__ void __launch_bounds__(kThreads, 1) fused_decode_kernel(FusedArgs a) 
                                                 : reinterpret_cast<const __half*>(a.qbuf) + (long long)u * H * D;
             const float* azb = entry < kQSlots ? reinterpret_cast<const float*>(smem_raw + kAzOff) + entry * H * 8
                                                : a.qgsum + (long long)u * H * 8;
-            build_bfrags<D, KB, H>(q16, NG, d.G, tig, gid, bf);
+            build_bfrags<D, KB, H>(q16, NG, KB == 16 ? D : d.G, tig, gid, bf);
 #pragma unroll
             for (int c2 = 0; c2 < 2; ++c2) {
               const int hh = NG == 2 ? tig : (NG == 1 ? 2 * tig + c2 : 2 * c2 + tig / 2);
@@ -697,9 +722,15 @@ __global__ void __launch_bounds__(kThreads, 1) fused_decode_kernel(FusedArgs a) 
                   val = fmaf(fA[0], fmaf(s4.z, c1, s4.x * c0), fmaf(s4.w, fZ[0][1], s4.y * fZ[0][0]));
                 } else if constexpr (NG == 1) {
                   const float c0 = acc[m][0][2 * hf], c1 = acc[m][0][2 * hf + 1];
-                  const float2 s2 = *reinterpret_cast<const float2*>(szs + r * 2);
-                  const float v0 = fmaf(fA[0] * s2.x, c0, s2.y * fZ[0][0]);
-                  const float v1 = fmaf(fA[1] * s2.x, c1, s2.y * fZ[1][0]);
+                  float v0, v1;
+                  if constexpr (KB == 16) {  // bf16 K: no (scale, zero) to fold
+                    v0 = fA[0] * c0;
+                    v1 = fA[1] * c1;
+                  } else {
+                    const float2 s2 = *reinterpret_cast<const float2*>(szs + r * 2);
+                    v0 = fmaf(fA[0] * s2.x, c0, s2.y * fZ[0][0]);
+                    v1 = fmaf(fA[1] * s2.x, c1, s2.y * fZ[1][0]);
+                  }
                   const int src = (lane & ~3) | (tig >> 1);
                   const float u0 = __shfl_sync(kFull, v0, src), u1 = __shfl_sync(kFull, v1, src);
                   val = (tig & 1) ? u1 : u0;
@@ -782,7 +813,8 @@ __global__ void __launch_bounds__(kThreads, 1) fused_decode_kernel(FusedArgs a) 
         c = c2;
       }
     };
-    if (ng == 2) consume(std::integral_constant<int, 2>{});
+    if constexpr (KB == 16) consume(std::integral_constant<int, 1>{});  // one "group": the whole row
+    else if (ng == 2) consume(std::integral_constant<int, 2>{});
     else if (ng == 1) consume(std::integral_constant<int, 1>{});
     else if constexpr (D == 128) consume(std::integral_constant<int, 4>{});
   }
@@ -1004,7 +1036,7 @@ __global__ void __launch_bounds__(kThreads, 1) fused_decode_kernel(FusedArgs a) 
               const int rbv = seg ? D * VB1 / 8 : D * VB0 / 8;
               const long long pr = PAGED ? unit_row<PAGED>(a, uu, vr) : (long long)uu * d.T_cap + vr;
               prefetch_l2(d.vc[seg] + pr * rbv);
-              prefetch_l2(d.vsz[seg] + pr * ng * 2);
+              if ((seg ? VB1 : VB0) < 16) prefetch_l2(d.vsz[seg] + pr * ng * 2);
             }
           }
           n_w += __popc(bal);
@@ -1073,7 +1105,7 @@ __global__ void __launch_bounds__(kThreads, 1) fused_decode_kernel(FusedArgs a) 
       const ChunkRows cr = chunk_rows(x, (k0 + row / kChunk) - x.cb);
       const int vr = cr.row0 + row % kChunk;
       const int rbv = cr.seg ? D * VB1 / 8 : D * VB0 / 8;
-      const int szb = ng == 1 ? 16 : ng * 8;
+      const int szb = (cr.seg ? VB1 : VB0) == 16 ? 0 : (ng == 1 ? 16 : ng * 8);
       uint8_t* slot = stage0 + (size_t)i * kSlotBytes;
       if (c * 16 < rbv) {
         const long long pr = PAGED ? unit_row<PAGED>(a, x.u, vr) : (long long)x.u * d.T_cap + vr;
@@ -1130,7 +1162,7 @@ __global__ void __launch_bounds__(kThreads, 1) fused_decode_kernel(FusedArgs a) 
         if (gidx < stage_slots) {
           const uint8_t* src = stage0 + (size_t)gidx * kSlotBytes;
           const float* szp = reinterpret_cast<const float*>(src + kVRowMax) + (ng == 1 ? (vr & 1) * 2 : gi * 2);
-          sz = *reinterpret_cast<const float2*>(szp);
+          sz = (cr.seg ? VB1 : VB0) == 16 ? make_float2(0.0f, 0.0f) : *reinterpret_cast<const float2*>(szp);
           if (cr.seg == 0 || VB0 == VB1) lds_lane_words<VB0>(src + j * 2 * VB0, w0);
           else if constexpr (VB0 != VB1) lds_lane_words<VB1>(src + j * 2 * VB1, w1);
         } else {

@@ -16,7 +16,8 @@ cudaError_t launch_one(const FusedArgs& a, size_t smem, int grid, cudaStream_t s
   return cudaLaunchCooperativeKernel((const void*)kern, dim3(grid), dim3(kThreads), params, smem, s);
 }
 
-// PAGED instantiations exist for plain decode only (one V width).
+// PAGED instantiations exist for plain decode only (one V width, not the
+// 16-bit passthrough width).
 template <int D, int H, int KB, bool PAGED>
 cudaError_t launch_v(const FusedArgs& a, int vb0, int vb1, size_t smem, int grid, cudaStream_t s) {
   if (vb0 == vb1) {
@@ -25,6 +26,9 @@ cudaError_t launch_v(const FusedArgs& a, int vb0, int vb1, size_t smem, int grid
       case 4: return launch_one<D, H, KB, 4, 4, PAGED>(a, smem, grid, s);
       case 6: return launch_one<D, H, KB, 6, 6, PAGED>(a, smem, grid, s);
       case 8: return launch_one<D, H, KB, 8, 8, PAGED>(a, smem, grid, s);
+      case 16:
+        if constexpr (!PAGED) return launch_one<D, H, KB, 16, 16, false>(a, smem, grid, s);
+        break;
     }
   }
   if constexpr (KB == 6 && !PAGED) {

@@ -53,8 +53,12 @@ struct LaneWords {
 
 template <int BITS>
 __device__ __forceinline__ void load_lane_words(const uint8_t* __restrict__ p, LaneWords<BITS>& lw) {
-  // p is 4-byte aligned; 8- and 16-byte alignment hold for 4- and 8-bit rows.
-  if constexpr (BITS == 8) {
+  // p is 4-byte aligned; 8- and 16-byte alignment hold for 4-, 8- and 16-bit rows.
+  if constexpr (BITS == 16) {
+    const uint4 v = __ldg(reinterpret_cast<const uint4*>(p)), u = __ldg(reinterpret_cast<const uint4*>(p) + 1);
+    lw.w[0] = v.x; lw.w[1] = v.y; lw.w[2] = v.z; lw.w[3] = v.w;
+    lw.w[4] = u.x; lw.w[5] = u.y; lw.w[6] = u.z; lw.w[7] = u.w;
+  } else if constexpr (BITS == 8) {
     uint4 v = __ldg(reinterpret_cast<const uint4*>(p));
     lw.w[0] = v.x; lw.w[1] = v.y; lw.w[2] = v.z; lw.w[3] = v.w;
   } else if constexpr (BITS == 4) {
@@ -103,7 +107,10 @@ __device__ __forceinline__ void pack16(const uint32_t (&c)[16], LaneWords<BITS>&
 
 template <int BITS>
 __device__ __forceinline__ void store_lane_words(uint8_t* p, const LaneWords<BITS>& lw) {
-  if constexpr (BITS == 8) {
+  if constexpr (BITS == 16) {
+    *reinterpret_cast<uint4*>(p) = make_uint4(lw.w[0], lw.w[1], lw.w[2], lw.w[3]);
+    *reinterpret_cast<uint4*>(p + 16) = make_uint4(lw.w[4], lw.w[5], lw.w[6], lw.w[7]);
+  } else if constexpr (BITS == 8) {
     *reinterpret_cast<uint4*>(p) = make_uint4(lw.w[0], lw.w[1], lw.w[2], lw.w[3]);
   } else if constexpr (BITS == 4) {
     *reinterpret_cast<uint2*>(p) = make_uint2(lw.w[0], lw.w[1]);
@@ -373,7 +380,11 @@ __device__ __forceinline__ void unpack16_int(const LaneWords<BITS>& lw, float2 (
 // Lane words from shared memory (4-byte aligned; wider when the width allows).
 template <int BITS>
 __device__ __forceinline__ void lds_lane_words(const uint8_t* p, LaneWords<BITS>& lw) {
-  if constexpr (BITS == 8) {
+  if constexpr (BITS == 16) {
+    const uint4 v = *reinterpret_cast<const uint4*>(p), u = *reinterpret_cast<const uint4*>(p + 16);
+    lw.w[0] = v.x; lw.w[1] = v.y; lw.w[2] = v.z; lw.w[3] = v.w;
+    lw.w[4] = u.x; lw.w[5] = u.y; lw.w[6] = u.z; lw.w[7] = u.w;
+  } else if constexpr (BITS == 8) {
     const uint4 v = *reinterpret_cast<const uint4*>(p);
     lw.w[0] = v.x; lw.w[1] = v.y; lw.w[2] = v.z; lw.w[3] = v.w;
   } else if constexpr (BITS == 4) {

@@ -101,6 +101,7 @@ cudaError_t launch_fused_k2(const FusedArgs& a, int D, int H, int vb0, int vb1, 
 cudaError_t launch_fused_k4(const FusedArgs& a, int D, int H, int vb0, int vb1, size_t smem, int grid, cudaStream_t s);
 cudaError_t launch_fused_k6(const FusedArgs& a, int D, int H, int vb0, int vb1, size_t smem, int grid, cudaStream_t s);
 cudaError_t launch_fused_k8(const FusedArgs& a, int D, int H, int vb0, int vb1, size_t smem, int grid, cudaStream_t s);
+cudaError_t launch_fused_k16(const FusedArgs& a, int D, int H, int vb0, int vb1, size_t smem, int grid, cudaStream_t s);
 // The same over a paged cache (plain decode: one V width).
 cudaError_t launch_fused_paged_k2(const FusedArgs& a, int D, int H, int vb, size_t smem, int grid, cudaStream_t s);
 cudaError_t launch_fused_paged_k4(const FusedArgs& a, int D, int H, int vb, size_t smem, int grid, cudaStream_t s);

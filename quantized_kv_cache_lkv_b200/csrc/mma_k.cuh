@@ -110,7 +110,7 @@ __device__ __forceinline__ uint32_t hsub2_u32(uint32_t a, uint32_t b) {
 // Register J (0 .. D/8 - 1) of a lane slice held in words w (the slice's
 // D*KB/128 words): two codes as exact fp16 values c * 2^off.
 template <int KB, int J, int SW>
-__device__ __forceinline__ uint32_t a_reg(const uint32_t (&w)[SW]) {
+__device__ __forceinline__ uint32_t a_reg_codes(const uint32_t (&w)[SW]) {
   constexpr PlanEntry pe = Plan<KB>::e[J % 8];
   constexpr int p = pe.p + (J / 8) * 16 * KB;  // first bit of the window in the slice
   constexpr int wi = p / 32, sh = p % 32;
@@ -135,6 +135,17 @@ __device__ __forceinline__ uint32_t a_reg(const uint32_t (&w)[SW]) {
   return hsub2_u32(r, kF16Magic2);
 }
 
+// At the 16-bit passthrough width the slice holds bf16 values: register J
+// is word J, channels (2J, 2J + 1), used as it is by the bf16 MMA.
+template <int KB, int J, int SW>
+__device__ __forceinline__ uint32_t a_reg(const uint32_t (&w)[SW]) {
+  if constexpr (KB == 16) {
+    return w[J];
+  } else {
+    return a_reg_codes<KB, J, SW>(w);
+  }
+}
+
 // Slice channels (0 .. D/4 - 1) and power-of-two offsets of register J.
 template <int KB, int J>
 struct RegChannels {
@@ -143,6 +154,10 @@ struct RegChannels {
   static constexpr int hi = (J / 8) * 16 + pe.hi;
   static constexpr int lo_off = pe.lo_off;
   static constexpr int hi_off = pe.hi_off;
+};
+template <int J>
+struct RegChannels<16, J> {
+  static constexpr int lo = 2 * J, hi = 2 * J + 1, lo_off = 0, hi_off = 0;
 };
 
 __device__ __forceinline__ void hmma16816(float (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
@@ -154,7 +169,19 @@ __device__ __forceinline__ void hmma16816(float (&c)[4], uint32_t a0, uint32_t a
       : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
-// fp16 pair (x, y), each scaled by its exact power of two.
+// The same with bf16 operands (the 16-bit passthrough width: bf16 K rows
+// against the bf16 q; every product is exact in the fp32 accumulator).
+__device__ __forceinline__ void hmma16816_bf16(float (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                               uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%0,%1,%2,%3};"
+      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// fp16 pair (x, y), each scaled by its exact power of two (offsets 0: the
+// two 16-bit patterns side by side, whatever their type).
 template <int OFF_LO, int OFF_HI>
 __device__ __forceinline__ uint32_t q_pair(__half x, __half y) {
   __half2 v = __halves2half2(x, y);
@@ -168,7 +195,8 @@ __device__ __forceinline__ uint32_t q_pair(__half x, __half y) {
 // B fragments of one n-tile for lane (gid, tig): column n = 8 * nt + gid is
 // (head n / ng, group n % ng); it is nonzero only on the channels of the
 // lane's slice when they belong to that group.  qh points at the scaled
-// fp16 q of the column's head (D values); bf[J] for J = 0 .. D/8 - 1.
+// fp16 q of the column's head (D values; for 16-bit K the raw bf16 q);
+// bf[J] for J = 0 .. D/8 - 1.
 template <int KB, int D, int J>
 __device__ __forceinline__ void bfrag_one(const __half* qh, int base, bool on, uint32_t* bf) {
   using R = RegChannels<KB, J>;

@@ -39,12 +39,17 @@ __device__ __forceinline__ void fetch_lane_rows(const uint16_t* k, const uint16_
 template <int BITS>
 __device__ __forceinline__ void quantize_lane(const uint4& w0, const uint4& w1, uint8_t* __restrict__ codes,
                                               float* __restrict__ sz, int j, int lpg, unsigned mask, float one) {
-  const uint32_t w[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
-  LaneWords<BITS> lw;
-  float scale, zero;
-  quantize16<BITS>(w, lpg, mask, one, lw, scale, zero);
-  store_lane_words<BITS>(codes + j * (2 * BITS), lw);
-  if (j % lpg == 0) *reinterpret_cast<float2*>(sz + 2 * (j / lpg)) = make_float2(scale, zero);
+  if constexpr (BITS == 16) {  // passthrough width: the bf16 values themselves, no (scale, zero)
+    *reinterpret_cast<uint4*>(codes + j * 32) = w0;
+    *reinterpret_cast<uint4*>(codes + j * 32 + 16) = w1;
+  } else {
+    const uint32_t w[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
+    LaneWords<BITS> lw;
+    float scale, zero;
+    quantize16<BITS>(w, lpg, mask, one, lw, scale, zero);
+    store_lane_words<BITS>(codes + j * (2 * BITS), lw);
+    if (j % lpg == 0) *reinterpret_cast<float2*>(sz + 2 * (j / lpg)) = make_float2(scale, zero);
+  }
 }
 
 // ------------------------------------------------------------ 32 channels per lane
@@ -178,14 +183,19 @@ __device__ __forceinline__ void store_words32(uint8_t* p, const uint32_t (&w)[BI
 template <int BITS, int LPG>
 __device__ __forceinline__ void quantize_lane32(const uint4 (&w4)[4], uint8_t* __restrict__ codes,
                                                 float* __restrict__ sz, int j, unsigned mask, float one) {
-  uint32_t w[16];
+  if constexpr (BITS == 16) {  // passthrough width: the bf16 values themselves, no (scale, zero)
 #pragma unroll
-  for (int i = 0; i < 4; ++i) { w[4 * i] = w4[i].x; w[4 * i + 1] = w4[i].y; w[4 * i + 2] = w4[i].z; w[4 * i + 3] = w4[i].w; }
-  uint32_t out[BITS];
-  float scale, zero;
-  quantize32<BITS, LPG>(w, mask, one, out, scale, zero);
-  store_words32<BITS>(codes + j * (4 * BITS), out);
-  if (j % LPG == 0) *reinterpret_cast<float2*>(sz + 2 * (j / LPG)) = make_float2(scale, zero);
+    for (int i = 0; i < 4; ++i) *reinterpret_cast<uint4*>(codes + j * 64 + 16 * i) = w4[i];
+  } else {
+    uint32_t w[16];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) { w[4 * i] = w4[i].x; w[4 * i + 1] = w4[i].y; w[4 * i + 2] = w4[i].z; w[4 * i + 3] = w4[i].w; }
+    uint32_t out[BITS];
+    float scale, zero;
+    quantize32<BITS, LPG>(w, mask, one, out, scale, zero);
+    store_words32<BITS>(codes + j * (4 * BITS), out);
+    if (j % LPG == 0) *reinterpret_cast<float2*>(sz + 2 * (j / LPG)) = make_float2(scale, zero);
+  }
 }
 
 // Row batches: batch (b, g, tb) covers tokens tb * RPW ... of KV head g of
@@ -354,34 +364,50 @@ __global__ void __launch_bounds__(256, 2) tier_repack_flat_kernel(RepackArgs a) 
   if (tid == (int)blockDim.x - 1) s_first[pairs] = run;  // the last thread's inclusive prefix: every row
   __syncthreads();
   const int total = s_first[pairs];
-  // row r lies in the last pair whose first row is <= r (empty pairs are passed over)
-  auto fetch = [&](int r, LaneRows32& x, int& seg, long long& slot) -> bool {
-    if (r >= total) return false;
+  // Row r: its pair (segment, unit) is the last whose first row is <= r
+  // (empty pairs are passed over), its slot in the segment, and where its
+  // position lives.  The position is loaded two rows ahead of use and the
+  // bf16 rows one ahead, so the two dependent loads of a row never meet on
+  // the critical path.
+  struct Loc {
+    bool ok;
+    int seg;
+    long long bg, slot;
+    int t;  // position (loaded ahead)
+  };
+  auto locate = [&](int r) {
+    Loc l{false, 0, 0, 0, 0};
+    if (r >= total) return l;
     int lo = 0, hi = pairs - 1;
     while (lo < hi) {
       const int mid = (lo + hi + 1) >> 1;
       if (s_first[mid] <= r) lo = mid; else hi = mid - 1;
     }
-    seg = lo / units;
-    const long long bg = lo % units;
+    l.ok = true;
+    l.seg = lo / units;
+    l.bg = lo % units;
     const int i = r - s_first[lo];
-    int t = __ldg((seg == 0 ? a.pos_a : a.pos_b) + bg * a.T_cap + i);
-    t = t < 0 ? 0 : (t >= a.T_cap ? a.T_cap - 1 : t);
-    const long long src = bg * a.T_cap + t;
+    l.slot = l.bg * a.T_cap + i;
+    l.t = __ldg((l.seg == 0 ? a.pos_a : a.pos_b) + l.slot);
+    return l;
+  };
+  auto fetch = [&](const Loc& l, LaneRows32& x) {
+    if (!l.ok) return;
+    const int t = l.t < 0 ? 0 : (l.t >= a.T_cap ? a.T_cap - 1 : l.t);
+    const long long src = l.bg * a.T_cap + t;
     fetch_lane_rows32(a.k + src * D + j * kLaneDims32, a.v + src * D + j * kLaneDims32, x);
-    slot = bg * a.T_cap + i;
-    return true;
   };
   const int stride = (int)gridDim.x * nw * RPW;
   int r = ((int)blockIdx.x * nw + warp) * RPW + sub;
   LaneRows32 cur, nxt;
-  int seg = 0, seg_n = 0;
-  long long slot = 0, slot_n = 0;
-  bool ok = fetch(r, cur, seg, slot);
+  Loc l0 = locate(r), l1 = locate(r + stride);
+  fetch(l0, cur);
   for (; r - sub < total; r += stride) {  // r - sub is the same for the whole warp
-    const bool ok_n = fetch(r + stride, nxt, seg_n, slot_n);
-    if (ok) {
-      if (seg == 0) {
+    const Loc l2 = locate(r + 2 * stride);
+    fetch(l1, nxt);
+    if (l0.ok) {
+      const long long slot = l0.slot;
+      if (l0.seg == 0) {
         quantize_lane32<6, LPG>(cur.k, a.a_kc + slot * (D * 6 / 8), a.a_ksz + slot * ng * 2, j, mask, a.one);
         quantize_lane32<6, LPG>(cur.v, a.a_vc + slot * (D * 6 / 8), a.a_vsz + slot * ng * 2, j, mask, a.one);
       } else {
@@ -389,7 +415,7 @@ __global__ void __launch_bounds__(256, 2) tier_repack_flat_kernel(RepackArgs a) 
         quantize_lane32<4, LPG>(cur.v, a.b_vc + slot * (D * 4 / 8), a.b_vsz + slot * ng * 2, j, mask, a.one);
       }
     }
-    cur = nxt; ok = ok_n; seg = seg_n; slot = slot_n;
+    cur = nxt; l0 = l1; l1 = l2;
   }
 }
 
@@ -441,6 +467,7 @@ static cudaError_t launch_quantize_vb(const QuantizeArgs& a, int vb, bool append
     case 4: return append ? launch_append_t<D, KB, 4>(a, s) : launch_quantize_t<D, KB, 4>(a, s);
     case 6: return append ? launch_append_t<D, KB, 6>(a, s) : launch_quantize_t<D, KB, 6>(a, s);
     case 8: return append ? launch_append_t<D, KB, 8>(a, s) : launch_quantize_t<D, KB, 8>(a, s);
+    case 16: return append ? launch_append_t<D, KB, 16>(a, s) : launch_quantize_t<D, KB, 16>(a, s);
     default: return cudaErrorInvalidValue;
   }
 }
@@ -452,6 +479,7 @@ static cudaError_t launch_quantize_d(const QuantizeArgs& a, int kb, int vb, bool
     case 4: return launch_quantize_vb<D, 4>(a, vb, append, s);
     case 6: return launch_quantize_vb<D, 6>(a, vb, append, s);
     case 8: return launch_quantize_vb<D, 8>(a, vb, append, s);
+    case 16: return launch_quantize_vb<D, 16>(a, vb, append, s);
     default: return cudaErrorInvalidValue;
   }
 }

@@ -55,11 +55,54 @@ def test_decode_gqa_ratios_ragged(orc, r, D):
         assert np.all(out[2] == 0.0)
 
 
-@pytest.mark.parametrize("kb,vb", [(8, 8), (6, 4), (4, 4), (4, 2), (2, 2), (2, 8), (8, 6)])
+@pytest.mark.parametrize("kb,vb", [(8, 8), (6, 4), (4, 4), (4, 2), (2, 2), (2, 8), (8, 6),
+                                   (16, 16), (16, 4), (6, 16), (16, 8)])
 def test_decode_bit_widths(orc, kb, vb):
     cfg = W.scaled(W.CONFIGS[4], B=3, T_cap=520, seq_lo=100, seq_hi=520, seed=40 + kb + vb)
     run_case(orc, cfg, kb, vb, 0.0)
     run_case(orc, cfg, kb, vb, 2e-3)
+
+
+@pytest.mark.parametrize("r", [1, 2, 4, 8])
+@pytest.mark.parametrize("kb,vb", [(16, 16), (16, 4), (6, 16)])
+def test_decode_passthrough_width_gqa(orc, r, kb, vb):
+    """The 16-bit width through every GQA ratio (groups of 8 take the
+    three-launch path), D 64 and 128, ragged lengths with 0 and 1."""
+    for D, G in ((128, 64), (64, 32)):
+        cfg = W.Config("pass", B=4, Hq=2 * r, Hkv=2, D=D, T_cap=600, G=G, bits=[(kb, vb)], hh_frac=0.01,
+                       seed=7 * r + kb + vb + D)
+        sl = torch.tensor([600, 1, 0, 333], dtype=torch.int32)
+        for tau in (0.0, 1e-3):
+            out, _, _ = run_case(orc, cfg, kb, vb, tau, seq_lens=sl)
+            assert np.all(out[2] == 0.0)
+
+
+def test_per_layer_bit_policy_two_layers(orc):
+    """A per-layer width policy is a table on the caller's side: an outlier
+    layer kept at 16 bits (K16V16) and an ordinary layer at K6V4, each with
+    its own cache, decoded one after the other with one workspace sized for
+    the larger of the two; each layer matches the oracle at its own width
+    ("Super KV Compression" §第一层: outlier layers stay in 16-bit floating
+    point, the others take K6V4)."""
+    policy = {0: (16, 16), 1: (6, 4)}
+    base = W.scaled(W.CONFIGS[2], B=2, T_cap=1024)
+    layers = {layer: W.make_inputs(W.scaled(base, seed=200 + layer)) for layer in policy}
+    B, Hq, Hkv, D, T, G = base.B, base.Hq, base.Hkv, base.D, base.T_cap, base.G
+    nb = max(lkv.lkv_decode_workspace_bytes((kb, vb, G), B, Hq, Hkv, T, D) for kb, vb in policy.values())
+    ws = buffers.alloc_workspace(nb)
+    caches = {layer: gpu_quantize(kb, vb, G, layers[layer]) for layer, (kb, vb) in policy.items()}
+    for step in range(2):
+        for layer, (kb, vb) in policy.items():
+            inp = layers[layer]
+            got, _, counts = gpu_decode(kb, vb, G, inp, caches[layer], base.softmax_scale, base.tau,
+                                        want_mask=False, ws=ws)
+            k, v, q, sl = oracle_inputs(inp)
+            want, _, o_counts = orc.decode_attention(kb, vb, G, sl, q, orc.quantize_kv(kb, vb, G, k, v, sl),
+                                                     base.softmax_scale, base.tau, want_mask=False)
+            assert_attention_close(got, want, vmax(inp), f"layer {layer} K{kb}V{vb} step {step}")
+    # the outlier layer's cache is the bf16 cache itself; the other is 3.2x smaller in codes
+    c0, c1 = caches[0], caches[1]
+    assert c0["k_codes"].shape[-1] == 2 * D and c1["k_codes"].shape[-1] + c1["v_codes"].shape[-1] == 10 * D // 8
 
 
 @pytest.mark.parametrize("tau", [1e-4, 1e-2, 0.5])

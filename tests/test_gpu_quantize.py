@@ -57,7 +57,8 @@ def special_rows(inp):
 
 
 @pytest.mark.parametrize("D,G", [(64, 32), (64, 64), (128, 32), (128, 64), (128, 128)])
-@pytest.mark.parametrize("kb,vb", [(6, 4), (8, 8), (4, 4), (4, 2), (2, 8), (8, 6), (2, 2), (6, 6)])
+@pytest.mark.parametrize("kb,vb", [(6, 4), (8, 8), (4, 4), (4, 2), (2, 8), (8, 6), (2, 2), (6, 6),
+                                   (16, 4), (6, 16), (16, 16)])
 def test_quantize_bit_exact_small(orc, D, G, kb, vb):
     cfg = W.Config("q", B=3, Hq=4, Hkv=2, D=D, T_cap=80, G=G, bits=[(kb, vb)], seed=D + G + kb * 7 + vb)
     inp = special_rows(W.make_inputs(cfg, seq_lens=torch.tensor([80, 37, 0], dtype=torch.int32)))
@@ -104,7 +105,8 @@ def test_quantize_out_of_range_lengths_are_clamped(orc):
     assert int(gpu["k_codes"][1].abs().sum()) == 0
 
 
-@pytest.mark.parametrize("D,G,kb,vb", [(128, 64, 6, 4), (64, 32, 8, 8), (128, 128, 4, 2), (128, 32, 2, 6)])
+@pytest.mark.parametrize("D,G,kb,vb", [(128, 64, 6, 4), (64, 32, 8, 8), (128, 128, 4, 2), (128, 32, 2, 6),
+                                       (128, 64, 16, 4), (64, 32, 16, 16)])
 def test_append_equals_quantize_of_the_longer_sequence(orc, D, G, kb, vb):
     """lkv_append_kv writes the new token's row exactly as lkv_quantize_kv
     would (bit-exact vs the oracle), and touches no other row; positions
@@ -137,3 +139,26 @@ def test_append_equals_quantize_of_the_longer_sequence(orc, D, G, kb, vb):
         for b in range(4):
             keep = [t for t in range(T_cap) if not (b < 3 and t == int(pos[b]))]
             assert torch.equal(g[b, :, keep], s0[b, :, keep]), (key, b)
+
+
+@pytest.mark.parametrize("kb,vb", [(16, 16), (16, 4), (6, 16)])
+def test_passthrough_width_rows_are_the_bf16_values(kb, vb):
+    """At 16 bits the cache row is the bf16 row itself, byte for byte, and
+    the (scale, zero) of that tensor is never written (it may be omitted)."""
+    from quantized_kv_cache_lkv_b200 import buffers, lkv
+    from gpu_helpers import dev
+    cfg = W.Config("pass", B=2, Hq=4, Hkv=2, D=128, T_cap=64, G=64, bits=[(kb, vb)], seed=8)
+    inp = W.make_inputs(cfg, seq_lens=torch.tensor([64, 10], dtype=torch.int32))
+    cache = buffers.alloc_cache(kb, vb, 64, 2, 2, 64, 128, zero=True)
+    lkv.lkv_quantize_kv((kb, vb, 64), 2, 2, 64, 128, dev(inp["seq_lens"]), dev(inp["k"]), dev(inp["v"]),
+                        cache["k_codes"], None if kb == 16 else cache["k_sz"], cache["v_codes"],
+                        None if vb == 16 else cache["v_sz"])
+    torch.cuda.synchronize()
+    for bits, key, src in ((kb, "k", inp["k"]), (vb, "v", inp["v"])):
+        if bits != 16:
+            continue
+        got = cache[key + "_codes"].cpu()
+        for b, T in enumerate((64, 10)):
+            assert torch.equal(got[b, :, :T].view(torch.bfloat16), src[b, :, :T])
+            assert int(got[b, :, T:].abs().sum()) == 0
+        assert int(cache[key + "_sz"].abs().sum()) == 0
