@@ -79,6 +79,11 @@ FusedLayout fused_layout(int B, int Hq, int Hkv, int T_cap, int D, int KB) {
   L.grid = num_sms();
   L.H = Hq / Hkv;
   const long long units = (long long)B * Hkv;
+  // A little fewer units than SMs: one CTA per unit instead of all SMs.  With
+  // equal lengths every unit is then owned by one CTA, which saves the
+  // exchange of statistics and partial outputs between CTAs (worth more
+  // than the idle SMs cost the bandwidth-bound first phase).
+  if (units >= (3 * L.grid) / 4 && units < L.grid) L.grid = (int)units;
   // each segment rounds up to whole chunks: at most one more chunk per unit
   const long long per_unit = T_cap > 0 ? (T_cap + kChunk - 1) / kChunk + 1 : 1;
   const long long chunks_max = units * per_unit > 0 ? units * per_unit : 1;

@@ -557,13 +557,15 @@ __global__ void __launch_bounds__(kThreads, 1) fused_decode_kernel(FusedArgs a) 
   __syncthreads();  // list complete
   const int nent = s_nent;
   int* const ulist = nent <= kUlCap ? ulist_s : ulist_g;
-  // q of the CTA's units (one warp per (unit, head)): scaled by 2^E so that
-  // its largest magnitude lies in [2^14, 2^15), stored as fp16 (exact for
-  // the bf16 inputs), with A = q_scale * 2^-E and Z[g] = q_scale * sum of
-  // the group's q for the fold after the MMA.
-  {
+  // q of the CTA's units (one consumer warp per (unit, head)): scaled by
+  // 2^E so that its largest magnitude lies in [2^14, 2^15), stored as fp16
+  // (exact for the bf16 inputs), with A = q_scale * 2^-E and Z[g] = q_scale
+  // * sum of the group's q for the fold after the MMA.  The producer warp
+  // does not take part: it starts streaming K meanwhile, and the consumers
+  // meet at a barrier of their own before the first tile.
+  if (warp != kProducer) {
     constexpr int DPL = D / 32;  // channels per lane
-    for (int task = warp; task < nent * H; task += CW) {
+    for (int task = warp; task < nent * H; task += kConsumers) {
       const int e = task / H, h = task % H;
       const Unit x = load_unit(ulist + e * kRec);
       const int b = x.u / d.Hkv, g = x.u % d.Hkv;
@@ -601,7 +603,7 @@ __global__ void __launch_bounds__(kThreads, 1) fused_decode_kernel(FusedArgs a) 
       if (lane == 0) az[4] = ldexpf(d.q_scale, -E);
     }
   }
-  __syncthreads();  // q ready; phase 1 starts
+  if (warp != kProducer) named_barrier(1, kConsumers * 32);  // q ready; the producer is already streaming
 
   float* lg = a.glogits + (long long)cta * a.cpc_max * kChunk * H;  // [tile * TR + row][H]
 
@@ -1013,8 +1015,8 @@ __global__ void __launch_bounds__(kThreads, 1) fused_decode_kernel(FusedArgs a) 
           float wgt[H];
           bool need = false;
           uint32_t kh = 0, kbits = 0;
-#pragma unroll
           const bool valid = r < nrow;
+#pragma unroll
           for (int h = 0; h < H; ++h) {
             const float p = ev[h] * f[h];
             const bool keep = valid && !(p < tau);
@@ -1368,6 +1370,8 @@ __global__ void __launch_bounds__(kThreads, 1) fused_decode_kernel(FusedArgs a) 
             const float* szs = reinterpret_cast<const float*>(src + kDenseCodes);
             float f[H];
             lds_heads<H>(tfu + (v0 / TR) * H, f);
+            // not unrolled: the body is large and the instruction cache small
+#pragma unroll 1
             for (int s2 = 0; s2 < 32 / RPW; ++s2) {
               const int i = s2 * RPW + lane / LPR;
               if (i >= rows) continue;  // the lanes of a row agree
