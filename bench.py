@@ -279,6 +279,14 @@ class Timed:
                 for j, (name, _) in enumerate(launches)}
 
 
+def launch_floor_us(timer, steps):
+    """Device time of a trivial kernel (zeroing 4 KB) timed exactly like the
+    library's kernels: the floor under every small launch of this harness."""
+    small = torch.empty(1024, device=timer.flush.device)
+    t = timer.run([("floor", lambda: small.zero_())], max(steps, 10), 3)
+    return round(statistics.median(t["floor"]) * 1e3, 2)
+
+
 def kernel_line(ms_list, nbytes, peak):
     ms = statistics.median(ms_list)
     gbs = nbytes / (ms * 1e-3) / 1e9
@@ -611,7 +619,7 @@ def run_lkv(args):
         e2e = run_e2e(step, inp, device, stream, max(args.steps, 20))
         sec = max_over_ranks(e2e["seconds"], device)
         e2e["value"] = round(job_throughput(e2e["bytes"], world, sec), 2)
-    extras = {}
+    extras = {"launch_floor_us": launch_floor_us(timer, args.steps)}
     if world == 1 and not args.no_extras:
         del step.d["k"], step.d["v"]
         torch.cuda.empty_cache()

@@ -3,15 +3,17 @@
 // tokens keep a 6-bit V, medium ones a 4-bit V, low ones are evicted).
 //
 // Each (b, kv head) unit is split into P contiguous parts (P <= 8), one CTA
-// per part, and the P CTAs of a unit form one thread-block cluster.  Pass 1:
-// a CTA classifies its part (the mass of positions inside the sequence read
-// once, 16 bytes per thread-load),
-// writes the tier bytes and counts its tier-2 and tier-1 tokens.  The CTAs
-// then exchange their counts through distributed shared memory across one
-// cluster barrier, so each knows how many kept tokens precede its part.
-// Pass 2: the CTA reads its tier bytes back (from L2) and a block-wide
-// exclusive scan gives every kept token its output slot, so positions come
-// out in ascending order.
+// of 256 threads per part, each thread taking 32 consecutive positions; the
+// P CTAs of a unit form one thread-block cluster.  Pass 1: a CTA classifies
+// its part (the mass of positions inside the sequence read once, 16 bytes
+// per load), writes every tier byte of the part and counts its tier-2 and
+// tier-1 tokens.  The CTAs then exchange their counts through distributed
+// shared memory across one cluster barrier, so each knows how many kept
+// tokens precede its part.  Pass 2: a block-wide exclusive scan of the
+// threads' counts gives every kept token its output slot, so positions come
+// out in ascending order.  A part of one tile (8192 positions, the usual
+// case) keeps its tiers in registers between the passes; longer parts read
+// their tier bytes back.
 #include <algorithm>
 
 #include "lkv_kernels.cuh"
@@ -21,12 +23,12 @@ namespace lkv {
 namespace {
 
 constexpr int kThreads = 256;
-constexpr int kPerThread = 8;
+constexpr int kPerThread = 32;                // consecutive positions of one thread
 constexpr int kTile = kThreads * kPerThread;  // positions one pass of a CTA covers
 constexpr int kMaxParts = 8;                  // CTAs per unit (portable cluster size)
 
 // Exclusive scan of two counters packed in one 32-bit word (16 bits each; a
-// tile holds at most 2048 positions, so neither overflows).
+// tile holds at most 8192 positions, so neither overflows).
 __device__ __forceinline__ uint32_t block_exclusive_scan(uint32_t x, uint32_t* warp_tot, uint32_t& total) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   uint32_t incl = x;
@@ -75,12 +77,39 @@ __device__ __forceinline__ uint32_t ld_dsmem(const uint32_t* local, uint32_t ran
   return v;
 }
 
-// Classification of position t with mass m (t beyond the sequence: tier 0).
-__device__ __forceinline__ int8_t classify(float m, bool valid, float lo, float hi) {
-  if (!valid) return 0;
-  if (m > hi) return 2;
-  if (m >= lo && m <= hi) return 1;
-  return 0;  // below tau_low, or NaN
+// Tiers of the thread's kPerThread positions [tb, tb + 32) as two bit masks
+// (bit i: position tb + i is tier 2, resp. tier 1); positions at or beyond
+// `lim` (the end of the part or of the sequence) are tier 0 and their mass
+// is not read.  NaN masses are tier 0.
+__device__ __forceinline__ void classify32(const float* mass, int tb, int lim, bool vec, float lo, float hi,
+                                           uint32_t& is2, uint32_t& is1) {
+  float m[kPerThread];
+  if (vec && tb + kPerThread <= lim) {
+#pragma unroll
+    for (int q = 0; q < kPerThread / 4; ++q) {
+      const float4 x = __ldg(reinterpret_cast<const float4*>(mass + tb) + q);
+      m[4 * q] = x.x; m[4 * q + 1] = x.y; m[4 * q + 2] = x.z; m[4 * q + 3] = x.w;
+    }
+  } else {
+#pragma unroll
+    for (int i = 0; i < kPerThread; ++i) m[i] = tb + i < lim ? __ldg(mass + tb + i) : 0.0f;
+  }
+  is2 = 0u;
+  is1 = 0u;
+#pragma unroll
+  for (int i = 0; i < kPerThread; ++i) {
+    const bool in = tb + i < lim;
+    is2 |= (in && m[i] > hi) ? (1u << i) : 0u;
+    is1 |= (in && m[i] >= lo && m[i] <= hi) ? (1u << i) : 0u;
+  }
+}
+
+// Tier bytes of 4 consecutive positions starting at bit i of the masks.
+__device__ __forceinline__ uint32_t tier_word(uint32_t is2, uint32_t is1, int i) {
+  uint32_t w = 0u;
+#pragma unroll
+  for (int k = 0; k < 4; ++k) w |= ((((is2 >> (i + k)) & 1u) << 1) | ((is1 >> (i + k)) & 1u)) << (8 * k);
+  return w;
 }
 
 // Grid: units * P CTAs, clusters of P along x; CTA rank p of unit u covers
@@ -89,54 +118,41 @@ __global__ void __launch_bounds__(kThreads) tier_classify_kernel(ClassifyArgs a,
   __shared__ uint32_t warp_tot[kThreads / 32 + 1];
   __shared__ uint32_t part_n[2];  // this CTA's tier-2 and tier-1 counts
   __shared__ int base[2];         // kept tokens of the unit's earlier parts
-  const int p = (int)cluster_rank();
+  const int p = P > 1 ? (int)cluster_rank() : 0;
   const long long bg = blockIdx.x / P;
   const int b = (int)(bg / a.Hkv);
   const int T = clamp_len(a.seq_lens[b], a.T_cap);
   const float* mass = a.mass + bg * a.T_cap;
   int8_t* tier = a.tier + bg * a.T_cap;
   const int t_lo = min(a.T_cap, p * L), t_hi = min(a.T_cap, t_lo + L);
-  // rows start 32-byte aligned for the masses and 8-byte aligned for the tiers
-  const bool vec = (a.T_cap % 8) == 0 && (reinterpret_cast<uintptr_t>(a.mass) & 31u) == 0 &&
-                   (reinterpret_cast<uintptr_t>(a.tier) & 7u) == 0;
+  const int lim = min(t_hi, T);  // positions of the part inside the sequence
+  // rows start 32-byte aligned for the masses and 16-byte aligned for the tiers
+  const bool vec = (a.T_cap % 16) == 0 && (reinterpret_cast<uintptr_t>(a.mass) & 31u) == 0 &&
+                   (reinterpret_cast<uintptr_t>(a.tier) & 15u) == 0;
+  const bool one_tile = t_hi - t_lo <= kTile;
 
-  // pass 1: classify, write the tier bytes, count
-  uint32_t n2 = 0, n1 = 0;
+  // pass 1: classify (masses read once), write every tier byte of the part, count
+  uint32_t n2 = 0, n1 = 0, keep2 = 0, keep1 = 0;
   for (int t0 = t_lo; t0 < t_hi; t0 += kTile) {
     const int tb = t0 + threadIdx.x * kPerThread;
-    // masses are read for positions inside the sequence only (t >= T_b is tier 0)
-    float m8[kPerThread];
-    const bool full = vec && tb + kPerThread <= t_hi;
-    if (full && tb + kPerThread <= T) {
-      const float4 x0 = __ldg(reinterpret_cast<const float4*>(mass + tb));
-      const float4 x1 = __ldg(reinterpret_cast<const float4*>(mass + tb + 4));
-      m8[0] = x0.x; m8[1] = x0.y; m8[2] = x0.z; m8[3] = x0.w;
-      m8[4] = x1.x; m8[5] = x1.y; m8[6] = x1.z; m8[7] = x1.w;
+    uint32_t is2 = 0, is1 = 0;
+    if (tb < t_hi) classify32(mass, tb, lim, vec, a.tau_low, a.tau_high, is2, is1);
+    n2 += __popc(is2);
+    n1 += __popc(is1);
+    keep2 = is2;  // the part's only tile stays in registers for pass 2
+    keep1 = is1;
+    if (vec && tb + kPerThread <= t_hi) {
+#pragma unroll
+      for (int q = 0; q < kPerThread / 16; ++q)
+        *reinterpret_cast<uint4*>(tier + tb + 16 * q) =
+            make_uint4(tier_word(is2, is1, 16 * q), tier_word(is2, is1, 16 * q + 4), tier_word(is2, is1, 16 * q + 8),
+                       tier_word(is2, is1, 16 * q + 12));
     } else {
-#pragma unroll
-      for (int i = 0; i < kPerThread; ++i) m8[i] = (tb + i < t_hi && tb + i < T) ? __ldg(mass + tb + i) : 0.0f;
-    }
-    int8_t c[kPerThread];
-#pragma unroll
-    for (int i = 0; i < kPerThread; ++i) {
-      c[i] = classify(m8[i], tb + i < T && tb + i < t_hi, a.tau_low, a.tau_high);
-      n2 += c[i] == 2;
-      n1 += c[i] == 1;
-    }
-    if (full) {
-      uint2 w;
-      w.x = (uint32_t)(uint8_t)c[0] | ((uint32_t)(uint8_t)c[1] << 8) | ((uint32_t)(uint8_t)c[2] << 16) |
-            ((uint32_t)(uint8_t)c[3] << 24);
-      w.y = (uint32_t)(uint8_t)c[4] | ((uint32_t)(uint8_t)c[5] << 8) | ((uint32_t)(uint8_t)c[6] << 16) |
-            ((uint32_t)(uint8_t)c[7] << 24);
-      *reinterpret_cast<uint2*>(tier + tb) = w;
-    } else {
-#pragma unroll
-      for (int i = 0; i < kPerThread; ++i)
-        if (tb + i < t_hi) tier[tb + i] = c[i];
+      for (int i = 0; i < kPerThread && tb + i < t_hi; ++i)
+        tier[tb + i] = (int8_t)((((is2 >> i) & 1u) << 1) | ((is1 >> i) & 1u));
     }
   }
-  // the part's counts (a part may exceed 65535 kept tokens: two words)
+  // the part's counts
 #pragma unroll
   for (int off = 16; off >= 1; off >>= 1) {
     n2 += __shfl_xor_sync(0xFFFFFFFFu, n2, off);
@@ -145,48 +161,53 @@ __global__ void __launch_bounds__(kThreads) tier_classify_kernel(ClassifyArgs a,
   if (threadIdx.x == 0) { part_n[0] = 0u; part_n[1] = 0u; }
   __syncthreads();
   if ((threadIdx.x & 31) == 0) { atomicAdd(&part_n[0], n2); atomicAdd(&part_n[1], n1); }
-  // exchange: every CTA of the unit reads the counts of the parts before it
-  cluster_sync();
-  if (threadIdx.x < 2) {
-    uint32_t s = 0, all = 0;
-    for (int q = 0; q < P; ++q) {
-      const uint32_t v = ld_dsmem(&part_n[threadIdx.x], (uint32_t)q);
-      if (q < p) s += v;
-      all += v;
+  if (P > 1) {
+    // exchange: every CTA of the unit reads the counts of the parts before it
+    cluster_sync();
+    if (threadIdx.x < 2) {
+      uint32_t s = 0, all = 0;
+      for (int q = 0; q < P; ++q) {
+        const uint32_t v = ld_dsmem(&part_n[threadIdx.x], (uint32_t)q);
+        if (q < p) s += v;
+        all += v;
+      }
+      base[threadIdx.x] = (int)s;
+      if (p == P - 1) a.counts[2 * bg + threadIdx.x] = (int)all;
     }
-    base[threadIdx.x] = (int)s;
-    if (p == P - 1) a.counts[2 * bg + threadIdx.x] = (int)all;
+    // no CTA leaves while another may still read its counts
+    cluster_sync();
+  } else {
+    __syncthreads();
+    if (threadIdx.x < 2) {
+      base[threadIdx.x] = 0;
+      a.counts[2 * bg + threadIdx.x] = (int)part_n[threadIdx.x];
+    }
+    __syncthreads();
   }
-  // no CTA leaves while another may still read its counts
-  cluster_sync();
 
-  // pass 2: the tier bytes back (this CTA wrote them; visible after the
-  // barriers above), a scan per tile, the positions
+  // pass 2: per tile a scan of the threads' counts gives every kept token
+  // its slot; a part of more than one tile reads its tier bytes back (this
+  // CTA wrote them, each thread its own)
   int32_t* pos_a = a.pos_a + bg * a.T_cap;
   int32_t* pos_b = a.pos_b + bg * a.T_cap;
   int base2 = base[0], base1 = base[1];
   for (int t0 = t_lo; t0 < t_hi; t0 += kTile) {
     const int tb = t0 + threadIdx.x * kPerThread;
-    int8_t c[kPerThread];
-    if (vec && tb + kPerThread <= t_hi) {
-      const uint2 w = *reinterpret_cast<const uint2*>(tier + tb);
-#pragma unroll
-      for (int i = 0; i < 4; ++i) { c[i] = (int8_t)(w.x >> (8 * i)); c[4 + i] = (int8_t)(w.y >> (8 * i)); }
-    } else {
-#pragma unroll
-      for (int i = 0; i < kPerThread; ++i) c[i] = tb + i < t_hi ? tier[tb + i] : 0;
+    uint32_t is2 = keep2, is1 = keep1;
+    if (!one_tile) {
+      is2 = 0u;
+      is1 = 0u;
+      for (int i = 0; i < kPerThread && tb + i < t_hi; ++i) {
+        const int c = tier[tb + i];
+        is2 |= (c == 2) ? (1u << i) : 0u;
+        is1 |= (c == 1) ? (1u << i) : 0u;
+      }
     }
-    uint32_t m2 = 0, m1 = 0;
-#pragma unroll
-    for (int i = 0; i < kPerThread; ++i) { m2 += c[i] == 2; m1 += c[i] == 1; }
     uint32_t total;
-    const uint32_t excl = block_exclusive_scan(m2 | (m1 << 16), warp_tot, total);
+    const uint32_t excl = block_exclusive_scan((uint32_t)__popc(is2) | ((uint32_t)__popc(is1) << 16), warp_tot, total);
     int o2 = base2 + (int)(excl & 0xFFFFu), o1 = base1 + (int)(excl >> 16);
-#pragma unroll
-    for (int i = 0; i < kPerThread; ++i) {
-      if (c[i] == 2) pos_a[o2++] = tb + i;
-      else if (c[i] == 1) pos_b[o1++] = tb + i;
-    }
+    while (is2) { const int i = __ffs(is2) - 1; pos_a[o2++] = tb + i; is2 &= is2 - 1u; }
+    while (is1) { const int i = __ffs(is1) - 1; pos_b[o1++] = tb + i; is1 &= is1 - 1u; }
     base2 += (int)(total & 0xFFFFu);
     base1 += (int)(total >> 16);
   }
@@ -200,11 +221,15 @@ cudaError_t launch_tier_classify(const ClassifyArgs& a, cudaStream_t s) {
     if (units > 0) return cudaMemsetAsync(a.counts, 0, (size_t)units * 2 * sizeof(int32_t), s);
     return cudaSuccess;
   }
-  // parts of at least one tile each, at most kMaxParts per unit
+  // parts of at most one tile each while kMaxParts suffice
   const int P = (int)std::min<long long>(kMaxParts, ((long long)a.T_cap + kTile - 1) / kTile);
   const long long per = ((long long)a.T_cap + P - 1) / P;
   const int L = (int)((per + kPerThread - 1) / kPerThread * kPerThread);
   if (units * P >= (1ll << 31)) return cudaErrorInvalidValue;
+  if (P == 1) {
+    tier_classify_kernel<<<(unsigned)units, kThreads, 0, s>>>(a, 1, L);
+    return cudaGetLastError();
+  }
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)(units * P));
   cfg.blockDim = dim3(kThreads);
