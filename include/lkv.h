@@ -255,8 +255,11 @@ LKV_API int lkv_decode_attention_mass(lkv_qspec spec, int B, int Hq, int Hkv, in
 
 /*
  * Size of the fixed device scratch that lkv_decode_attention_static uses:
- * 32 MiB per device, enough for e.g. B = 16, Hkv = 8, T_cap = 8192, D = 128
- * with groups of 4 query heads (about 18 MiB on 148 SMs).
+ * 32 MiB on each device.  Whether a shape fits depends on the device, since
+ * the decode's scratch layout scales with the SM count: the test is
+ * lkv_decode_workspace_bytes(...) <= LKV_STATIC_WORKSPACE_BYTES, called with
+ * the target device current.  On a 148-SM B200, B = 16, Hkv = 8,
+ * T_cap = 8192, D = 128 with groups of 4 query heads needs about 18 MiB.
  */
 #define LKV_STATIC_WORKSPACE_BYTES (32u << 20)
 
@@ -278,9 +281,10 @@ LKV_API int lkv_decode_attention_mass(lkv_qspec spec, int B, int Hq, int Hkv, in
  * needs more than LKV_STATIC_WORKSPACE_BYTES (lkv_decode_workspace_bytes
  * gives the need).  Nothing is allocated or freed.  Each call first clears,
  * on `stream`, the part of the scratch that must start at zero, so an
- * earlier failed call leaves nothing behind.  The first call on a device
- * looks up the scratch's address (which may load the library's device
- * code); make it before any stream capture.  All calls on one device share
+ * earlier failed call leaves nothing behind.  Every call looks up the
+ * scratch's address in the current context (so a device reset or another
+ * context is safe); the first one on a device may load the library's device
+ * code, so make it before any stream capture.  All calls on one device share
  * the one scratch: calls that overlap on the GPU (other streams, other host
  * threads) race and give wrong results, so order them (one stream, or
  * events).

@@ -21,6 +21,15 @@ LIB = os.path.join(PKG, "liblkv.so")
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 NVCC_FLAGS = ["-O3", "-std=c++17", "-lineinfo", "--expt-relaxed-constexpr", "-Xcompiler", "-fPIC",
               "-Xcompiler", "-fvisibility=hidden", "-I", os.path.join(ROOT, "include")]
+# Translation units whose results must be bit-exact with the oracle (codes,
+# (scale, zero), tiers and positions): no multiply-add contraction, so a
+# plain a * b + c there can never turn into one fused operation.  The
+# decode's deliberate fused operations live in other files.
+NO_FMAD = ("quantize.cu", "tier.cu")
+
+
+def extra_flags(src):
+    return ["--fmad=false"] if os.path.basename(src) in NO_FMAD else []
 
 
 def nvcc():
@@ -41,7 +50,7 @@ def _headers():
 
 def _compile(src, verbose):
     obj = os.path.join(BUILD, os.path.basename(src) + ".o")
-    cmd = [nvcc(), *ARCH, *NVCC_FLAGS, "-c", src, "-o", obj]
+    cmd = [nvcc(), *ARCH, *NVCC_FLAGS, *extra_flags(src), "-c", src, "-o", obj]
     if verbose:
         cmd.insert(1, "-Xptxas=-v")
     p = subprocess.run(cmd, capture_output=True, text=True)

@@ -7,7 +7,6 @@
 
 #include "../../include/lkv.h"
 #include <algorithm>
-#include <mutex>
 
 #include "fused_impl.cuh"
 #include "lkv_kernels.cuh"
@@ -229,28 +228,18 @@ using namespace lkv;
 // cudaMalloc would fail and a cudaFree would synchronize the whole device.
 // Its size is fixed at LKV_STATIC_WORKSPACE_BYTES; larger decodes are
 // rejected.  Host code never uses the array's name as a device address: the
-// address comes from cudaGetSymbolAddress, looked up once per device.
+// address comes from cudaGetSymbolAddress, looked up on every call.
 static __device__ __align__(256) unsigned char g_static_ws[LKV_STATIC_WORKSPACE_BYTES];
 
 namespace {
 
-constexpr int kMaxDevices = 64;
-std::mutex g_static_mu;
-void* g_static_ptr[kMaxDevices] = {};
-
-// Device address of g_static_ws on the current device; the first call for a
-// device looks it up (with that device current, as it is here).
+// Device address of g_static_ws in the current context, looked up on every
+// call (cheap once the module is loaded): after a device reset, or in
+// another context, the array can sit at another address.
 int static_scratch(void** ptr) {
-  int dev = -1;
-  if (cudaGetDevice(&dev) != cudaSuccess) return LKV_ERR_CUDA;
-  if (dev < 0 || dev >= kMaxDevices) return LKV_ERR_UNSUPPORTED;
-  std::lock_guard<std::mutex> lock(g_static_mu);
-  if (g_static_ptr[dev] == nullptr) {
-    void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_static_ws) != cudaSuccess || p == nullptr) return LKV_ERR_CUDA;
-    g_static_ptr[dev] = p;
-  }
-  *ptr = g_static_ptr[dev];
+  void* p = nullptr;
+  if (cudaGetSymbolAddress(&p, g_static_ws) != cudaSuccess || p == nullptr) return LKV_ERR_CUDA;
+  *ptr = p;
   return LKV_OK;
 }
 
