@@ -30,6 +30,16 @@ steps, L2 flushed before every launch):
                 classify, repack and tiered decode, with the tiered cache's
                 compression ratio.
 
+stream: the same decode call back to back, rotating over four copies of the
+quantized cache (inputs larger than L2 instead of a flush between calls);
+events around each block of calls, per-call time = block time / calls, median
+over the blocks.  It is the call's throughput in a decode loop, where the
+launch latency overlaps the previous call and the code stays resident; the
+headline keeps the isolated, flushed figure.
+
+--call NAME times only one call of the step (after one untimed pass of the
+whole step), the way the ncu commands under profiles/ capture it.
+
 e2e is a decode loop through the public API with host buffers: every step
 copies q and the new token's K/V (plus positions and lengths) host->device,
 appends the token (lkv_append_kv), decodes, and reads out and the skip counts
@@ -429,6 +439,51 @@ def run_e2e(step, inp, device, stream, steps):
             "loop": "H2D q + new K/V + pos + lengths, lkv_append_kv, lkv_decode_attention, D2H out + counts"}
 
 
+def bench_stream(step, device, stream, args, peak, nbytes, copies=4, blocks=5):
+    """The decode call back to back over `copies` copies of the cache (the
+    step's quantized cache plus copies), one event pair per block of calls."""
+    caches = [step.cache] + [{k: t.clone() for k, t in step.cache.items()} for _ in range(copies - 1)]
+    B, Hq, Hkv, D, T, G = step.shape
+    L, s, cfg, d = step.lkv, stream.cuda_stream, step.cfg, step.d
+
+    def call(c):
+        L.lkv_decode_attention((KB, VB, G), B, Hq, Hkv, T, D, d["seq_lens"], d["q"], c["k_codes"], c["k_sz"],
+                               c["v_codes"], c["v_sz"], cfg.softmax_scale, cfg.tau, step.out, None, step.cnt,
+                               step.ws, step.ws.numel(), s)
+
+    per_block = max(args.steps, 4 * copies) // copies * copies
+    for i in range(2 * copies):
+        call(caches[i % copies])
+    torch.cuda.synchronize(device)
+    ms = []
+    for _ in range(blocks):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for i in range(per_block):
+            call(caches[i % copies])
+        e1.record(stream)
+        torch.cuda.synchronize(device)
+        ms.append(e0.elapsed_time(e1) / per_block)
+    line = kernel_line(ms, nbytes, peak)
+    line.update({"calls_per_block": per_block, "blocks": blocks, "cache_copies": copies,
+                 "l2": f"inputs larger than L2: {copies} cache copies of "
+                       f"{sum(t.numel() * t.element_size() for t in step.cache.values()) >> 20} MiB rotated, no flush"})
+    del caches
+    torch.cuda.empty_cache()
+    return line
+
+
+def run_one_call(args, step, timer, stream):
+    """--call: one untimed pass of the whole step, then only the named call,
+    warm-up + timed steps with L2 flushed before each; prints its median."""
+    launches = dict(step.launches(stream))
+    for fn in launches.values():
+        fn()
+    t = timer.run([(args.call, launches[args.call])], args.steps, args.warmup)
+    print(json.dumps({"call": args.call, "workload": step.cfg.name, "steps": args.steps,
+                      "us_median": round(statistics.median(t[args.call]) * 1e3, 2)}), flush=True)
+
+
 # ----------------------------------------------------------------- other workloads (1 GPU)
 
 def bench_long(device, stream, timer, args, peak):
@@ -586,6 +641,10 @@ def run_lkv(args):
             torch.distributed.barrier()
         torch.cuda.synchronize(device)
 
+    if args.call:
+        run_one_call(args, step, timer, stream)
+        return
+
     launches = step.launches(stream)
     for _ in range(args.warmup):
         for _, fn in launches:
@@ -620,6 +679,9 @@ def run_lkv(args):
         sec = max_over_ranks(e2e["seconds"], device)
         e2e["value"] = round(job_throughput(e2e["bytes"], world, sec), 2)
     extras = {"launch_floor_us": launch_floor_us(timer, args.steps)}
+    if world == 1 and not args.no_extras:
+        extras["stream"] = bench_stream(step, device, stream, args, peak, by["decode"])
+        extras["stream"]["kv_tokens_per_s"] = round(step.kept[2] / cfg.Hkv / (extras["stream"]["us"] * 1e-6), 1)
     if world == 1 and not args.no_extras:
         del step.d["k"], step.d["v"]
         torch.cuda.empty_cache()
@@ -755,6 +817,8 @@ def main():
     ap.add_argument("--no-cpu", action="store_true", help="skip the CPU-oracle baseline leg")
     ap.add_argument("--no-e2e", action="store_true", help="skip the end-to-end (host buffers) leg")
     ap.add_argument("--no-extras", action="store_true", help="skip the long-context, sweep and tiered workloads")
+    ap.add_argument("--call", choices=["quantize", "decode", "classify", "repack", "tiered"],
+                    help="time only this call of the step (for profiling)")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)   # at least 3 untimed warm-up steps
     if args.impl == "reference":

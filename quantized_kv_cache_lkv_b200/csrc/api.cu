@@ -67,7 +67,7 @@ bool fused_ok(int r) { return r == 1 || r == 2 || r == 4; }
 struct FusedLayout {
   int grid, H, cpc_max, ring_bytes, stages, cand_cap;
   size_t smem_bytes;
-  size_t arrive1, arrive2, pstats, ppart, ulist, glogits, gstats, qbuf, qgsum, total;
+  size_t arrive1, arrive2, pstats, ppart, wslot, ulist, glogits, gstats, qbuf, qgsum, total;
   bool need_gstats;
 };
 
@@ -89,14 +89,15 @@ FusedLayout fused_layout(int B, int Hq, int Hkv, int T_cap, int D, int KB) {
   L.cpc_max = (int)((chunks_max + L.grid - 1) / L.grid);
   // phase 1: as many ring stages as shared memory holds (at most kMaxStages);
   // phase 2 reuses the ring: the sparse-mode list of kept rows (2048 per
-  // CTA), two partial outputs per warp and V staging slots, the fallback scan's lists, or the dense-mode
-  // buffers, each followed by the warps' partial outputs
+  // CTA), one partial output per warp and V staging slots, the fallback
+  // scan's lists, or the dense-mode buffers, each followed by the warps'
+  // partial outputs
   const int sb = fused::stage_bytes_host(D, KB);
   const int red = fused::kWarps * L.H * D * 4;
   const int slot = D * 8 / 8 + 8 * std::max(2, D / 32);  // widest V row plus (scale, zero)
   int lcap = 2048;  // kept rows one CTA can list (more fall back to a per-piece scan)
   if ((long long)L.cpc_max * kChunk >= (1ll << fused::kCandRowBits) || L.cpc_max >= 2048) lcap = 0;
-  const int sparse = (lcap * (1 + L.H) * 4 + 127) / 128 * 128 + 2 * red + 128 * slot;
+  const int sparse = (lcap * (1 + L.H) * 4 + 127) / 128 * 128 + red + 128 * slot;
   const int scan_fb = fused::kWarps * fused::kListCap * 4 * (1 + L.H) + red;
   const int dense = fused::kDenseStaging + red;
   const int phase2 = std::max(sparse, std::max(scan_fb, dense));
@@ -111,6 +112,7 @@ FusedLayout fused_layout(int B, int Hq, int Hkv, int T_cap, int D, int KB) {
   L.arrive2 = off; off = align_up(off + units * 4);
   L.pstats = off; off = align_up(off + (size_t)L.grid * 2 * L.H * 2 * 4);
   L.ppart = off; off = align_up(off + (size_t)L.grid * 2 * L.H * D * 4);
+  L.wslot = off; off = align_up(off + (size_t)L.grid * fused::kWarps * L.H * D * 4);
   L.ulist = off; off = align_up(off + (size_t)L.grid * L.cpc_max * fused::kRec * 4);
   L.glogits = off; off = align_up(off + (size_t)L.grid * L.cpc_max * kChunk * L.H * 4);
   L.gstats = off;
@@ -159,6 +161,7 @@ int run_attention(DecodeArgs& a, int D, int kb, int vb0, int vb1, void* ws, size
   f.arrive2 = reinterpret_cast<int*>(base + L.arrive2);
   f.pstats = reinterpret_cast<float*>(base + L.pstats);
   f.ppart = reinterpret_cast<float*>(base + L.ppart);
+  f.wslot = reinterpret_cast<float*>(base + L.wslot);
   f.cstats = nullptr;
   f.ulist = reinterpret_cast<int*>(base + L.ulist);
   f.glogits = reinterpret_cast<float*>(base + L.glogits);

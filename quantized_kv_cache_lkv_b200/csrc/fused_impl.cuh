@@ -921,10 +921,9 @@ __global__ void __launch_bounds__(kThreads, 1) fused_decode_kernel(FusedArgs a) 
   __syncthreads();
 
   // ------------------------------------------------------------ phase 2
-  // phase-2 shared memory (in the ring).  Sparse mode: per warp its kept
-  // rows [lcap], their weights [lcap][H] and staging slots [lcap]; the
-  // warps' partial outputs [CW][2][H][D]; then one staging slot per kept V
-  // row.  Scan mode: kept-row lists [CW][kListCap] and weights; dense mode:
+  // phase-2 shared memory (in the ring).  Sparse mode: the kept rows
+  // [lcap] and their weights [lcap][H]; the warps' partial outputs
+  // [CW][H][D]; then one staging slot per kept V row.  Scan mode: kept-row lists [CW][kListCap] and weights; dense mode:
   // the V staging buffers; for both, the warps' partial outputs [CW][H][D]
   // are last.
   const int red_off = a.ring_bytes - CW * H * D * 4;
@@ -941,15 +940,16 @@ __global__ void __launch_bounds__(kThreads, 1) fused_decode_kernel(FusedArgs a) 
   constexpr int kSlotBytes = kVRowMax + kSzSlot;
   // sparse mode layout in the ring: the CTA's kept-row list [lcap] rows and
   // [lcap][H] weights first; behind it the e-values of a round of tiles
-  // during the scan, then the warps' partial outputs [CW][2][H][D] and the
-  // V staging slots during the accumulation
+  // during the scan, then the warps' last-piece partial outputs [CW][H][D]
+  // and the V staging slots during the accumulation (a warp's first piece,
+  // when its share holds more than one, goes to its workspace slot)
   int* const krow = reinterpret_cast<int*>(ring);             // CTA-local row | unit entry << 20
   float* const kw = reinterpret_cast<float*>(krow + lcap);    // weights p (0 for a skipping head)
   const int lists_bytes = (lcap * (1 + H) * 4 + 127) / 128 * 128;
   float* const ebuf = reinterpret_cast<float*>(ring + lists_bytes);
   const int round_tiles = sparse_try ? (a.ring_bytes - lists_bytes) / (TR * H * 4) : 0;
-  float* const red2 = reinterpret_cast<float*>(ring + lists_bytes);      // [CW][2][H][D]
-  const int red2_bytes = CW * 2 * H * D * 4;
+  float* const red2 = reinterpret_cast<float*>(ring + lists_bytes);      // [CW][H][D]
+  const int red2_bytes = CW * H * D * 4;
   uint8_t* const stage0 = ring + lists_bytes + red2_bytes;
   const int stage_slots = sparse_try ? max(0, (a.ring_bytes - lists_bytes - red2_bytes) / kSlotBytes) : 0;
   uint32_t kh_lane = 0, kr_lane = 0;  // kept (row, head) pairs and kept rows seen by this lane
@@ -1098,9 +1098,8 @@ __global__ void __launch_bounds__(kThreads, 1) fused_decode_kernel(FusedArgs a) 
     };
     const int per = ((n_all + CW - 1) / CW + RPW - 1) / RPW * RPW;
     const int g_lo = min(n_all, warp * per), g_hi = min(n_all, g_lo + per);
-    constexpr int kMaxChunks = kVRowMax / 16 + kSzSlot / 16;
-    for (int q = lane; q < (min(g_hi, stage_slots) - g_lo) * kMaxChunks; q += 32) {
-      const int i = g_lo + q / kMaxChunks, c = q % kMaxChunks;
+    // one row per lane: its codes and (scale, zero) in 16-byte copies
+    for (int i = g_lo + lane; i < min(g_hi, stage_slots); i += 32) {
       const int rowe = krow[pidx(i)];
       const int ent = rowe >> kCandRowBits, row = rowe & ((1 << kCandRowBits) - 1);
       const Unit x = load_unit(ulist + ent * kRec);
@@ -1109,14 +1108,13 @@ __global__ void __launch_bounds__(kThreads, 1) fused_decode_kernel(FusedArgs a) 
       const int rbv = cr.seg ? D * VB1 / 8 : D * VB0 / 8;
       const int szb = (cr.seg ? VB1 : VB0) == 16 ? 0 : (ng == 1 ? 16 : ng * 8);
       uint8_t* slot = stage0 + (size_t)i * kSlotBytes;
-      if (c * 16 < rbv) {
-        const long long pr = PAGED ? unit_row<PAGED>(a, x.u, vr) : (long long)x.u * d.T_cap + vr;
-        cp_async16(slot + c * 16, d.vc[cr.seg] + pr * rbv + c * 16);
-      } else if (c >= kVRowMax / 16 && (c - kVRowMax / 16) * 16 < szb) {
-        const int cz = c - kVRowMax / 16;
-        const int vr0 = ng == 1 ? (vr & ~1) : vr;
-        const long long pr0 = PAGED ? unit_row<PAGED>(a, x.u, vr0) : (long long)x.u * d.T_cap + vr0;
-        cp_async16(slot + kVRowMax + cz * 16, reinterpret_cast<const uint8_t*>(d.vsz[cr.seg] + pr0 * ng * 2) + cz * 16);
+      const long long pr = PAGED ? unit_row<PAGED>(a, x.u, vr) : (long long)x.u * d.T_cap + vr;
+      for (int c = 0; c < rbv; c += 16) cp_async16(slot + c, d.vc[cr.seg] + pr * rbv + c);
+      if (szb > 0) {
+        // ng == 1: the 16 bytes of the even/odd row pair (T_cap is even then)
+        const long long pr0 = ng == 1 ? (pr & ~1ll) : pr;
+        const uint8_t* zs = reinterpret_cast<const uint8_t*>(d.vsz[cr.seg] + pr0 * ng * 2);
+        for (int c = 0; c < szb; c += 16) cp_async16(slot + kVRowMax + c, zs + c);
       }
     }
     cp_async_wait_all();
@@ -1190,13 +1188,16 @@ __global__ void __launch_bounds__(kThreads, 1) fused_decode_kernel(FusedArgs a) 
         }
       const bool first = seg_lo == g_lo, last = seg_hi == g_hi;
       if (first || last) {
-        const int k = first ? 0 : 1;
+        // the share's last piece to the warp's slot in shared memory, a
+        // different first piece to its slot in the workspace
+        const int k = last ? 1 : 0;
+        float* dst = last ? red2 + warp * H * D : a.wslot + ((long long)cta * CW + warp) * H * D;
         if (lane < LPR) {
 #pragma unroll
           for (int h = 0; h < H; ++h)
 #pragma unroll
             for (int i = 0; i < 8; i += 2)
-              *reinterpret_cast<float4*>(red2 + ((warp * 2 + k) * H + h) * D + j * kDimsPerLane + 2 * i) =
+              *reinterpret_cast<float4*>(dst + h * D + j * kDimsPerLane + 2 * i) =
                   make_float4(acc[h][i].x, acc[h][i].y, acc[h][i + 1].x, acc[h][i + 1].y);
         }
         if (lane == 0) s_spiece[warp * 2 + k] = pc;
@@ -1233,7 +1234,8 @@ __global__ void __launch_bounds__(kThreads, 1) fused_decode_kernel(FusedArgs a) 
       for (int o = tid; o < H * D; o += NTHR) {
         float s2 = 0.0f;
         for (int k2 = kr.x; k2 < kr.y; ++k2)
-          if (s_spiece[k2] == e) s2 += red2[k2 * H * D + o];
+          if (s_spiece[k2] == e)
+            s2 += (k2 & 1) ? red2[(k2 >> 1) * H * D + o] : __ldcg(a.wslot + ((long long)cta * CW + (k2 >> 1)) * H * D + o);
         const int h = o / D, dd = o % D;
         if (x.owned) {
           d.out[((long long)b * d.Hq + g * H + h) * D + dd] = s2;

@@ -83,6 +83,7 @@ struct FusedArgs {
   int* arrive2;                  // [units] partial outputs published
   float* pstats;                 // [grid][2][H][2]
   float* ppart;                  // [grid][2][H][D]
+  float* wslot;                  // [grid][kWarps][H][D] sparse mode: a warp's first piece when its share holds more than one
   float* cstats;                 // [chunks][H][2]
   int* ulist;                    // [grid][cpc_max][16]
   float* glogits;                // [grid][cpc_max * chunk][H] (when shared memory is short)
