@@ -462,45 +462,47 @@ __global__ void __launch_bounds__(kThreads, 1) fused_decode_kernel(FusedArgs a) 
   __syncthreads();
 
   // ------------------------------------------------------------ unit list
-  {
-    int part = 0;
-    for (int u = tid; u < units; u += NTHR) {
-      int n0, n1;
-      unit_lens(d, u, n0, n1);
-      part += chunks_of(n0) + chunks_of(n1);
-      if (n0 + n1 == 0 && (u % grid) == cta) {  // empty unit: its outputs are zero
-        const int b = u / d.Hkv, g = u % d.Hkv;
-        for (int e = 0; e < H * D; ++e) d.out[((long long)b * d.Hq + g * H + e / D) * D + e % D] = 0.0f;
+  // Every CTA derives the chunk ranges of all units (prefix sums of their
+  // chunk counts), takes an equal contiguous range [k0, k1) of chunks, and
+  // lists the units it touches.  Up to one unit per thread this is one pass
+  // (lengths read once, one block scan); more units take two.
+  if (cta == 0) {  // length checks, spread over the CTA's threads (a serial loop here delays CTA 0)
+    for (int u = tid; u < (d.len_mode == 0 ? d.B : units); u += NTHR) {
+      bool bad;
+      if (d.len_mode == 0) {
+        bad = d.lens[u] < 0 || d.lens[u] > d.T_cap;
+      } else {
+        const int r0 = d.lens[2 * u], r1 = d.lens[2 * u + 1];
+        bad = r0 < 0 || r1 < 0 || (long long)r0 + r1 > d.T_cap;
       }
-    }
-#pragma unroll
-    for (int off = 16; off >= 1; off >>= 1) part += __shfl_xor_sync(kFull, part, off);
-    if (lane == 0) atomicAdd(&s_total, part);
-    if (cta == 0) {  // length checks, spread over the CTA's threads (a serial loop here delays CTA 0)
-      for (int u = tid; u < (d.len_mode == 0 ? d.B : units); u += NTHR) {
-        bool bad;
-        if (d.len_mode == 0) {
-          bad = d.lens[u] < 0 || d.lens[u] > d.T_cap;
-        } else {
-          const int r0 = d.lens[2 * u], r1 = d.lens[2 * u + 1];
-          bad = r0 < 0 || r1 < 0 || (long long)r0 + r1 > d.T_cap;
-        }
-        if (bad) atomicExch(d.status, kStatusInvalidArg);
-      }
+      if (bad) atomicExch(d.status, kStatusInvalidArg);
     }
   }
-  __syncthreads();
-  const int total = s_total;
-  const int cpc = (total + grid - 1) / grid;
-  const int k0 = min(cta * cpc, total), k1 = min(k0 + cpc, total);
-  const int nck = k1 - k0;
-  const int ntile = nck * TPC;
+  int total = 0, cpc = 0, k0 = 0, k1 = 0;
   int* ulist_g = a.ulist + (long long)cta * a.cpc_max * kRec;
   int* ulist_s = reinterpret_cast<int*>(smem_raw + kUlOff);
-  for (int base = 0; base < units; base += NTHR) {
-    const int u = base + tid;
+  // unit u's record, when its chunks [cb, cb + nc) meet [k0, k1)
+  auto put_unit = [&](int u, int cb, int nc, int n0, int n1, int nc0, int idx) {
+    // the list lives in shared memory when it fits, else in the workspace
+    int* recs[2] = {ulist_g + (long long)idx * kRec, idx < kUlCap ? ulist_s + idx * kRec : nullptr};
+    for (int c = 0; c < 2; ++c) {
+      int* rec = recs[c];
+      if (rec == nullptr) continue;
+      rec[0] = u; rec[1] = cb; rec[2] = nc; rec[3] = n0; rec[4] = n1;
+      rec[5] = (cb >= k0 && cb + nc <= k1) ? 1 : 0;
+      rec[6] = nc0;
+    }
+    atomicMax(&s_nent, idx + 1);
+  };
+  auto zero_empty = [&](int u) {  // an empty unit: its outputs are zero
+    const int b = u / d.Hkv, g = u % d.Hkv;
+    for (int e = 0; e < H * D; ++e) d.out[((long long)b * d.Hq + g * H + e / D) * D + e % D] = 0.0f;
+  };
+  if (units <= NTHR) {
+    const int u = tid;
     int n0 = 0, n1 = 0;
     if (u < units) unit_lens(d, u, n0, n1);
+    if (u < units && n0 + n1 == 0 && (u % grid) == cta) zero_empty(u);
     const int nc0 = chunks_of(n0);
     const int nc = nc0 + chunks_of(n1);
     const int ne = nc > 0 ? 1 : 0;
@@ -512,32 +514,67 @@ __global__ void __launch_bounds__(kThreads, 1) fused_decode_kernel(FusedArgs a) 
     }
     if (lane == 31) { s_wsum[warp] = sc; s_wsum[16 + warp] = sn; }
     __syncthreads();
-    int wc = 0, wn = 0, tc = 0, tn = 0;
+    int wc = 0, wn = 0;
     for (int w = 0; w < CW; ++w) {
       if (w < warp) { wc += s_wsum[w]; wn += s_wsum[16 + w]; }
-      tc += s_wsum[w]; tn += s_wsum[16 + w];
+      total += s_wsum[w];
     }
-    const int cb = s_carry_c + wc + sc - nc;
-    const int ne_idx = s_carry_n + wn + sn - ne;
+    cpc = (total + grid - 1) / grid;
+    k0 = min(cta * cpc, total);
+    k1 = min(k0 + cpc, total);
+    const int cb = wc + sc - nc;
+    const int ne_idx = wn + sn - ne;
     if (ne && cb <= k0 && k0 < cb + nc) s_e0 = ne_idx;
     __syncthreads();
-    if (ne && cb < k1 && cb + nc > k0) {
-      const int idx = ne_idx - s_e0;
-      // the list lives in shared memory when it fits, else in the workspace
-      int* recs[2] = {ulist_g + (long long)idx * kRec, idx < kUlCap ? ulist_s + idx * kRec : nullptr};
-      for (int c = 0; c < 2; ++c) {
-        int* rec = recs[c];
-        if (rec == nullptr) continue;
-        rec[0] = u; rec[1] = cb; rec[2] = nc; rec[3] = n0; rec[4] = n1;
-        rec[5] = (cb >= k0 && cb + nc <= k1) ? 1 : 0;
-        rec[6] = nc0;
-      }
-      atomicMax(&s_nent, idx + 1);
+    if (ne && cb < k1 && cb + nc > k0) put_unit(u, cb, nc, n0, n1, nc0, ne_idx - s_e0);
+  } else {
+    int part = 0;
+    for (int u = tid; u < units; u += NTHR) {
+      int n0, n1;
+      unit_lens(d, u, n0, n1);
+      part += chunks_of(n0) + chunks_of(n1);
+      if (n0 + n1 == 0 && (u % grid) == cta) zero_empty(u);
     }
+#pragma unroll
+    for (int off = 16; off >= 1; off >>= 1) part += __shfl_xor_sync(kFull, part, off);
+    if (lane == 0) atomicAdd(&s_total, part);
     __syncthreads();
-    if (tid == 0) { s_carry_c += tc; s_carry_n += tn; }
-    __syncthreads();
+    total = s_total;
+    cpc = (total + grid - 1) / grid;
+    k0 = min(cta * cpc, total);
+    k1 = min(k0 + cpc, total);
+    for (int base = 0; base < units; base += NTHR) {
+      const int u = base + tid;
+      int n0 = 0, n1 = 0;
+      if (u < units) unit_lens(d, u, n0, n1);
+      const int nc0 = chunks_of(n0);
+      const int nc = nc0 + chunks_of(n1);
+      const int ne = nc > 0 ? 1 : 0;
+      int sc = nc, sn = ne;  // warp inclusive scans
+#pragma unroll
+      for (int off = 1; off < 32; off <<= 1) {
+        const int y = __shfl_up_sync(kFull, sc, off), z = __shfl_up_sync(kFull, sn, off);
+        if (lane >= off) { sc += y; sn += z; }
+      }
+      if (lane == 31) { s_wsum[warp] = sc; s_wsum[16 + warp] = sn; }
+      __syncthreads();
+      int wc = 0, wn = 0, tc = 0, tn = 0;
+      for (int w = 0; w < CW; ++w) {
+        if (w < warp) { wc += s_wsum[w]; wn += s_wsum[16 + w]; }
+        tc += s_wsum[w]; tn += s_wsum[16 + w];
+      }
+      const int cb = s_carry_c + wc + sc - nc;
+      const int ne_idx = s_carry_n + wn + sn - ne;
+      if (ne && cb <= k0 && k0 < cb + nc) s_e0 = ne_idx;
+      __syncthreads();
+      if (ne && cb < k1 && cb + nc > k0) put_unit(u, cb, nc, n0, n1, nc0, ne_idx - s_e0);
+      __syncthreads();
+      if (tid == 0) { s_carry_c += tc; s_carry_n += tn; }
+      __syncthreads();
+    }
   }
+  const int nck = k1 - k0;
+  const int ntile = nck * TPC;
   // tile statistics (max, sum, factor per head): shared memory unless many tiles
   float* tsm;
   float* tsl;

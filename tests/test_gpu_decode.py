@@ -117,6 +117,16 @@ def test_decode_tau_above_every_probability_gives_zero(orc):
     assert np.all(out == 0.0) and counts.tolist() == [2 * 32 * 300, 2 * 8 * 300]
 
 
+def test_decode_more_units_than_threads(orc):
+    """576 (sequence, KV head) units, more than one CTA's threads: the unit
+    list takes its two-pass path; ragged lengths including 0, every
+    sequence against the oracle."""
+    cfg = W.scaled(W.CONFIGS[2], B=72, T_cap=320, seq_lo=0, seq_hi=320, seq="uniform", seed=91)
+    out, _, _ = run_case(orc, cfg, 6, 4, 1e-3)
+    zero = np.nonzero(W.make_inputs(cfg)["seq_lens"].numpy() == 0)[0]
+    assert np.all(out[zero] == 0.0)
+
+
 def test_decode_capacity_invariance(orc):
     """The same tokens in a larger cache (more chunks launched, most of them
     empty) give the same skip set and outputs within tolerance."""
