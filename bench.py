@@ -41,10 +41,10 @@ headline keeps the isolated, flushed figure.
 whole step), the way the ncu commands under profiles/ capture it.
 
 e2e is a decode loop through the public API with host buffers: every step
-copies q and the new token's K/V (plus positions and lengths) host->device,
-appends the token (lkv_append_kv), decodes, and reads out and the skip counts
-back device->host; value = the decode + append algorithmic bytes over the
-loop's device time.
+copies q and the new token's K/V (plus positions and lengths) host->device in
+one copy from a pinned staging buffer, appends the token (lkv_append_kv),
+decodes, and reads out and the skip counts back device->host in one copy;
+value = the decode + append algorithmic bytes over the loop's device time.
 
 Multi-GPU: one process per GPU, every rank decodes its own batch (weak
 scaling, no collective on the data path), value = all ranks' decode bytes /
@@ -380,42 +380,54 @@ class Step:
 def run_e2e(step, inp, device, stream, steps):
     """Decode loop through the public API with host buffers.  The cache holds
     the workload's tokens; the loop starts `steps` tokens short of the full
-    context and, every step, copies q, the new token's K/V, its position and
-    the new lengths host->device, appends the token (lkv_append_kv), decodes
-    over the longer sequences, and copies out and the skip counts back."""
+    context and, every step, copies that step's inputs (q, the new token's
+    K/V, its position and the new lengths, packed in one pinned staging
+    buffer) host->device in one copy, appends the token (lkv_append_kv),
+    decodes over the longer sequences, and copies out and the skip counts
+    (adjacent in one device buffer) back in one copy."""
     cfg = step.cfg
     B, Hq, Hkv, D, T, G = step.shape
     L = step.lkv
     s = stream.cuda_stream
     full = inp["seq_lens"].to(torch.int64)
     start = torch.clamp(full - steps, min=0)
-    h_pos = torch.stack([torch.clamp(start + i, max=T - 1) for i in range(steps)]).to(torch.int32)
-    h_len = torch.stack([torch.minimum(start + i + 1, full) for i in range(steps)]).to(torch.int32)
-    idx = h_pos.to(torch.int64)
-    h_k = torch.stack([inp["k"][torch.arange(B), :, idx[i]] for i in range(steps)]).contiguous().pin_memory()
-    h_v = torch.stack([inp["v"][torch.arange(B), :, idx[i]] for i in range(steps)]).contiguous().pin_memory()
-    h_pos, h_len = h_pos.pin_memory(), h_len.pin_memory()
-    h_q = inp["q"].contiguous().pin_memory()
-    d_pos = torch.empty(B, dtype=torch.int32, device=device)
-    d_len = torch.empty(B, dtype=torch.int32, device=device)
-    d_q = torch.empty_like(step.d["q"])
-    d_k = torch.empty(B, Hkv, D, dtype=torch.bfloat16, device=device)
-    d_v = torch.empty(B, Hkv, D, dtype=torch.bfloat16, device=device)
-    h_out = torch.empty(steps, B, Hq, D, dtype=torch.float32).pin_memory()
-    h_cnt = torch.empty(steps, 2, dtype=torch.int64).pin_memory()
+    pos = torch.stack([torch.clamp(start + i, max=T - 1) for i in range(steps)]).to(torch.int32)
+    lens = torch.stack([torch.minimum(start + i + 1, full) for i in range(steps)]).to(torch.int32)
+    idx = pos.to(torch.int64)
+    # staging layout per step (every part a multiple of 16 bytes): q | k | v | pos | lens
+    nq, nkv = B * Hq * D * 2, B * Hkv * D * 2
+    parts = [nq, nkv, nkv, B * 4, B * 4]
+    offs = [sum(parts[:i]) for i in range(len(parts))]
+    per_step = (sum(parts) + 255) // 256 * 256
+    h_in = torch.empty(steps, per_step, dtype=torch.uint8).pin_memory()
+    for i in range(steps):
+        row = h_in[i]
+        row[offs[0]:offs[0] + nq].copy_(inp["q"].contiguous().view(-1).view(torch.uint8))
+        row[offs[1]:offs[1] + nkv].copy_(inp["k"][torch.arange(B), :, idx[i]].contiguous().view(-1).view(torch.uint8))
+        row[offs[2]:offs[2] + nkv].copy_(inp["v"][torch.arange(B), :, idx[i]].contiguous().view(-1).view(torch.uint8))
+        row[offs[3]:offs[3] + B * 4].copy_(pos[i].view(torch.uint8))
+        row[offs[4]:offs[4] + B * 4].copy_(lens[i].view(torch.uint8))
+    d_in = torch.empty(per_step, dtype=torch.uint8, device=device)
+    d_q = d_in[offs[0]:offs[0] + nq].view(torch.bfloat16).view(B, Hq, D)
+    d_k = d_in[offs[1]:offs[1] + nkv].view(torch.bfloat16).view(B, Hkv, D)
+    d_v = d_in[offs[2]:offs[2] + nkv].view(torch.bfloat16).view(B, Hkv, D)
+    d_pos = d_in[offs[3]:offs[3] + B * 4].view(torch.int32)
+    d_len = d_in[offs[4]:offs[4] + B * 4].view(torch.int32)
+    n_out = B * Hq * D * 4
+    d_res = torch.empty(n_out + 16, dtype=torch.uint8, device=device)   # out (f32) then the two skip counts
+    out = d_res[:n_out].view(torch.float32).view(B, Hq, D)
+    cnt = d_res[n_out:].view(torch.int64)
+    h_res = torch.empty(steps, n_out + 16, dtype=torch.uint8).pin_memory()
     c = step.cache
 
     def one(i):
-        d_q.copy_(h_q, non_blocking=True)
-        d_k.copy_(h_k[i], non_blocking=True)
-        d_v.copy_(h_v[i], non_blocking=True)
-        d_pos.copy_(h_pos[i], non_blocking=True)
-        d_len.copy_(h_len[i], non_blocking=True)
+        d_in.copy_(h_in[i], non_blocking=True)
         L.lkv_append_kv((KB, VB, G), B, Hkv, T, D, d_pos, d_k, d_v, c["k_codes"], c["k_sz"], c["v_codes"],
                         c["v_sz"], s)
-        step.decode(s, seq_lens=d_len, q=d_q)
-        h_out[i].copy_(step.out, non_blocking=True)
-        h_cnt[i].copy_(step.cnt, non_blocking=True)
+        L.lkv_decode_attention((KB, VB, G), B, Hq, Hkv, T, D, d_len, d_q, c["k_codes"], c["k_sz"],
+                               c["v_codes"], c["v_sz"], cfg.softmax_scale, cfg.tau, out, None, cnt, step.ws,
+                               step.ws.numel(), s)
+        h_res[i].copy_(d_res, non_blocking=True)
 
     one(0)                                   # warm-up (rewrites the same row)
     torch.cuda.synchronize(device)
@@ -428,15 +440,15 @@ def run_e2e(step, inp, device, stream, steps):
     sec = t0.elapsed_time(t1) * 1e-3
     by = 0
     for i in range(steps):
-        rows = int(h_len[i].to(torch.int64).sum()) * Hkv
-        by += decode_bytes(rows, rows - int(h_cnt[i, 1]), B, Hq, D, G, KB, VB)
+        rows = int(lens[i].to(torch.int64).sum()) * Hkv
+        skipped = int(h_res[i, n_out:].view(torch.int64)[1])
+        by += decode_bytes(rows, rows - skipped, B, Hq, D, G, KB, VB)
         by += quantize_bytes(B * Hkv, D, G, KB, VB)           # the appended rows
-    h2d = (h_q.numel() + h_k[0].numel() + h_v[0].numel()) * 2 + (h_pos[0].numel() + h_len[0].numel()) * 4
-    d2h = h_out[0].numel() * 4 + h_cnt[0].numel() * 8
-    return {"value": round(by / sec / 1e9, 2), "unit": "GB/s", "h2d_bytes_per_step": int(h2d),
-            "d2h_bytes_per_step": int(d2h), "seconds": sec, "bytes": by, "steps": steps,
+    return {"value": round(by / sec / 1e9, 2), "unit": "GB/s", "h2d_bytes_per_step": int(sum(parts)),
+            "d2h_bytes_per_step": int(n_out + 16), "seconds": sec, "bytes": by, "steps": steps,
             "us_per_step": round(sec / steps * 1e6, 2),
-            "loop": "H2D q + new K/V + pos + lengths, lkv_append_kv, lkv_decode_attention, D2H out + counts"}
+            "loop": "one H2D copy of q + new K/V + pos + lengths, lkv_append_kv, lkv_decode_attention, "
+                    "one D2H copy of out + skip counts"}
 
 
 def bench_stream(step, device, stream, args, peak, nbytes, copies=4, blocks=5):
