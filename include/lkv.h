@@ -259,7 +259,7 @@ LKV_API int lkv_decode_attention_mass(lkv_qspec spec, int B, int Hq, int Hkv, in
  * the decode's scratch layout scales with the SM count: the test is
  * lkv_decode_workspace_bytes(...) <= LKV_STATIC_WORKSPACE_BYTES, called with
  * the target device current.  On a 148-SM B200, B = 16, Hkv = 8,
- * T_cap = 8192, D = 128 with groups of 4 query heads needs about 18 MiB.
+ * T_cap = 8192, D = 128 with groups of 4 query heads needs about 23 MiB.
  */
 #define LKV_STATIC_WORKSPACE_BYTES (32u << 20)
 
