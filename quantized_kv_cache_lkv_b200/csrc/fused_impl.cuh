@@ -862,6 +862,29 @@ __global__ void __launch_bounds__(kThreads, 1) fused_decode_kernel(FusedArgs a) 
   // phase 2 reuses: skip straight to the end (the status word says why).
   const bool aborted = *abort_flag != 0;
   const int n_work = aborted ? 0 : nent;
+  // the dense V pass applies when every row is kept and the V rows fit its buffers
+  const bool dense = d.tau <= 0.0f && VB0 <= 6 && VB1 <= 6;
+  const int lcap = a.cand_cap;
+  const bool sparse_try = !dense && lcap > 0 && n_work > 0 && nent <= kUlCap;
+  // sparse mode layout in the ring: the CTA's kept-row list [lcap] rows and
+  // [lcap][H] weights first; behind it the e-values of a round of tiles
+  // during the scan, then the warps' last-piece partial outputs [CW][H][D]
+  // and the V staging slots during the accumulation (a warp's first piece,
+  // when its share holds more than one, goes to its workspace slot)
+  const int lists_bytes = (lcap * (1 + H) * 4 + 127) / 128 * 128;
+  float* const ebuf = reinterpret_cast<float*>(ring + lists_bytes);
+  const int round_tiles = sparse_try ? (a.ring_bytes - lists_bytes) / (TR * H * 4) : 0;
+  // The first round's e-values (each warp's contiguous run of tiles, one
+  // bulk copy per warp on its first dense-pass barrier, unused in sparse
+  // mode) land while the statistics below are merged.
+  const int e_t1 = sparse_try ? min(ntile, round_tiles) : 0;
+  const int e_lo = (e_t1 * warp) / CW, e_hi = (e_t1 * (warp + 1)) / CW;
+  if (sparse_try && lane == 0 && e_hi > e_lo) {
+    fence_proxy_async_global();  // the e-values were written by plain stores in phase 1
+    const uint32_t eb = (uint32_t)(e_hi - e_lo) * TR * H * 4;
+    mbar_arrive_expect_tx(&dbar[warp * 2], eb);
+    bulk_g2s(ebuf + (size_t)e_lo * TR * H, lg + (long long)e_lo * TR * H, eb, &dbar[warp * 2], policy_evict_first());
+  }
 
   // ------------------------------------------------------------ statistics
   // piece statistics: the CTA's tiles of each unit, merged -- one warp per
@@ -965,26 +988,14 @@ __global__ void __launch_bounds__(kThreads, 1) fused_decode_kernel(FusedArgs a) 
   // are last.
   const int red_off = a.ring_bytes - CW * H * D * 4;
   float* red = reinterpret_cast<float*>(ring + red_off);
-  // the dense V pass applies when every row is kept and the V rows fit its buffers
-  const bool dense = d.tau <= 0.0f && VB0 <= 6 && VB1 <= 6;
-  const int lcap = a.cand_cap;
-  const bool sparse_try = !dense && lcap > 0 && n_work > 0 && nent <= kUlCap;
   unsigned long long cnt_heads = 0, cnt_rows = 0;
   uint8_t* const smask = d.skip_mask;
   float* const mass_out = d.mass;
   constexpr int kSzSlot = 8 * ((D / 32) > 2 ? (D / 32) : 2);
   constexpr int kVRowMax = D * (VB0 > VB1 ? VB0 : VB1) / 8;
   constexpr int kSlotBytes = kVRowMax + kSzSlot;
-  // sparse mode layout in the ring: the CTA's kept-row list [lcap] rows and
-  // [lcap][H] weights first; behind it the e-values of a round of tiles
-  // during the scan, then the warps' last-piece partial outputs [CW][H][D]
-  // and the V staging slots during the accumulation (a warp's first piece,
-  // when its share holds more than one, goes to its workspace slot)
   int* const krow = reinterpret_cast<int*>(ring);             // CTA-local row | unit entry << 20
   float* const kw = reinterpret_cast<float*>(krow + lcap);    // weights p (0 for a skipping head)
-  const int lists_bytes = (lcap * (1 + H) * 4 + 127) / 128 * 128;
-  float* const ebuf = reinterpret_cast<float*>(ring + lists_bytes);
-  const int round_tiles = sparse_try ? (a.ring_bytes - lists_bytes) / (TR * H * 4) : 0;
   float* const red2 = reinterpret_cast<float*>(ring + lists_bytes);      // [CW][H][D]
   const int red2_bytes = CW * H * D * 4;
   uint8_t* const stage0 = ring + lists_bytes + red2_bytes;
@@ -1018,18 +1029,26 @@ __global__ void __launch_bounds__(kThreads, 1) fused_decode_kernel(FusedArgs a) 
           nrow = max(0, min(TR, cr.rows - (t % TPC) * TR)); ent = lo2; seg = cr.seg; pos = cr.row0 + (t % TPC) * TR;
         }
       };
-      // copy: the e-values of this warp's tiles (a tile's rows are one run
-      // of nrow * H floats in the workspace, 16-byte aligned)
+      if (T0 == 0) {
+        // the first round's bulk copy, issued after phase 1 (same tiles)
+        if (t_hi > t_lo && !mbar_wait(&dbar[warp * 2], 0, limit_ns)) {
+          atomicExch(d.status, kStatusTimeout);
+          mbar_wait(&dbar[warp * 2], 0, limit_ns);  // never leave the copy in flight
+        }
+      } else {
+        // copy: the e-values of this warp's tiles (a tile's rows are one run
+        // of nrow * H floats in the workspace, 16-byte aligned)
 #pragma unroll 1
-      for (int t = t_lo; t < t_hi; ++t) {
-        int nrow, ent, seg, pos;
-        tile_info(t, nrow, ent, seg, pos);
-        const int nchk = (nrow * H * 4 + 15) / 16;
-        const uint8_t* src = reinterpret_cast<const uint8_t*>(lg + (long long)t * TR * H);
-        uint8_t* dst = reinterpret_cast<uint8_t*>(ebuf + (t - T0) * TR * H);
-        for (int q = lane; q < nchk; q += 32) cp_async16(dst + q * 16, src + q * 16);
+        for (int t = t_lo; t < t_hi; ++t) {
+          int nrow, ent, seg, pos;
+          tile_info(t, nrow, ent, seg, pos);
+          const int nchk = (nrow * H * 4 + 15) / 16;
+          const uint8_t* src = reinterpret_cast<const uint8_t*>(lg + (long long)t * TR * H);
+          uint8_t* dst = reinterpret_cast<uint8_t*>(ebuf + (t - T0) * TR * H);
+          for (int q = lane; q < nchk; q += 32) cp_async16(dst + q * 16, src + q * 16);
+        }
+        cp_async_wait_all();
       }
-      cp_async_wait_all();
       __syncwarp();
       // one pass: the skip decisions; kept rows (with their weights p, 0 for
       // a head that skips) go to the warp's list, in row order
