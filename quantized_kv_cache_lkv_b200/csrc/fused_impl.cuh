@@ -73,8 +73,7 @@ constexpr unsigned kFull = 0xFFFFFFFFu;
 // per warp for the dense pass), per q slot and head A and Z[4] [1024, 1536),
 // misc ints [1536, 2560), tile statistics [2560, 8704), fp16 q of up to
 // kQSlots units [8704, 12800), unit list [12800, 16896), stage descriptors
-// [16896, 17664), tile descriptors [17664, 18688), piece slot ranges
-// [18688, 19200).
+// [16896, 17664), tile descriptors [17664, 18688), spare [18688, 19200).
 constexpr int kBarOff = 0;
 constexpr int kAzOff = 1024;
 constexpr int kMiscOff = 1536;
@@ -84,11 +83,10 @@ constexpr int kUlOff = 12800;
 constexpr int kUlCap = 64;
 constexpr int kDescOff = 16896;
 constexpr int kTinfoOff = 17664;  // per tile (valid rows | segment << 7 | unit entry << 8, first row)
-constexpr int kPrangeOff = 18688; // sparse mode: per piece the range of partial-output slots
 constexpr int kHeader = 19200;
 static_assert(2 * kMaxStages + 2 * kWarps <= 128, "barriers fit their 1024 bytes");
 static_assert(kDescOff + kMaxStages * 32 <= kTinfoOff, "stage descriptors fit");
-static_assert(kTinfoOff + kTsCap * 8 <= kPrangeOff && kPrangeOff + kUlCap * 8 <= kHeader, "tile and piece tables fit");
+static_assert(kTinfoOff + kTsCap * 8 <= kHeader, "tile table fits");
 static_assert(kHeader % 128 == 0, "the ring starts 128-byte aligned");
 
 // Compile-time geometry of one instantiation.
@@ -443,6 +441,7 @@ __global__ void __launch_bounds__(kThreads, 1) fused_decode_kernel(FusedArgs a) 
   int& s_last = misc[6];
   int& s_ovf = misc[7];
   int& s_issued = misc[8];                            // chunks the producer has issued
+  int& s_valid = misc[9];                             // sparse mode: valid rows the scan saw
   int* s_kept = misc + 10;                            // sparse mode: kept (row, head) pairs, kept rows
   int* s_lastu = misc + 12;                           // sparse mode: shared pieces this CTA combines
   int* s_spiece = misc + 128;                         // sparse mode: piece in each warp's two slots
@@ -456,7 +455,7 @@ __global__ void __launch_bounds__(kThreads, 1) fused_decode_kernel(FusedArgs a) 
     for (int s = 0; s < 2 * kWarps; ++s) mbar_init(&dbar[s], 1);
     fence_mbar_init();
     s_total = 0; s_e0 = 0; s_nent = 0; s_abort = 0; s_carry_c = 0; s_carry_n = 0; s_last = 0; s_ovf = 0;
-    s_issued = 0; s_kept[0] = 0; s_kept[1] = 0;
+    s_issued = 0; s_valid = 0; s_kept[0] = 0; s_kept[1] = 0;
   }
   for (int i = tid; i < kUlCap; i += kThreads) s_pdone[i] = 0;
   __syncthreads();
@@ -967,17 +966,21 @@ __global__ void __launch_bounds__(kThreads, 1) fused_decode_kernel(FusedArgs a) 
     }
   }
   __syncthreads();
-  // per-tile factors exp2(max_tile - max) / sum
-  for (int q = tid; q < (n_work > 0 ? ntile * H : 0); q += NTHR) {
-    const int t2 = q / H, h = q % H;
-    const int g = k0 + t2 / TPC;
-    int lo = 0, hi = nent - 1;  // entry holding chunk g
-    while (lo < hi) { const int mid = (lo + hi + 1) >> 1; if (ulist[mid * kRec + 1] <= g) lo = mid; else hi = mid - 1; }
-    const float* st = reinterpret_cast<const float*>(ulist + lo * kRec + 8);
-    const float M = st[2 * h], il = st[2 * h + 1];
-    const float mt = tsm[t2 * H + h];
-    tsf[t2 * H + h] = (il > 0.0f && mt > -INFINITY) ? exp2f(mt - M) * il : 0.0f;
-  }
+  // per-tile factors exp2(max_tile - max) / sum (the sparse scan computes
+  // its own as it goes; a sparse pass that falls back computes them later)
+  auto tile_factors = [&]() {
+    for (int q = tid; q < (n_work > 0 ? ntile * H : 0); q += NTHR) {
+      const int t2 = q / H, h = q % H;
+      const int g = k0 + t2 / TPC;
+      int lo = 0, hi = nent - 1;  // entry holding chunk g
+      while (lo < hi) { const int mid = (lo + hi + 1) >> 1; if (ulist[mid * kRec + 1] <= g) lo = mid; else hi = mid - 1; }
+      const float* st = reinterpret_cast<const float*>(ulist + lo * kRec + 8);
+      const float M = st[2 * h], il = st[2 * h + 1];
+      const float mt = tsm[t2 * H + h];
+      tsf[t2 * H + h] = (il > 0.0f && mt > -INFINITY) ? exp2f(mt - M) * il : 0.0f;
+    }
+  };
+  if (!sparse_try) tile_factors();
   __syncthreads();
 
   // ------------------------------------------------------------ phase 2
@@ -1000,7 +1003,7 @@ __global__ void __launch_bounds__(kThreads, 1) fused_decode_kernel(FusedArgs a) 
   const int red2_bytes = CW * H * D * 4;
   uint8_t* const stage0 = ring + lists_bytes + red2_bytes;
   const int stage_slots = sparse_try ? max(0, (a.ring_bytes - lists_bytes - red2_bytes) / kSlotBytes) : 0;
-  uint32_t kh_lane = 0, kr_lane = 0;  // kept (row, head) pairs and kept rows seen by this lane
+  uint32_t kh_lane = 0, kr_lane = 0, kv_lane = 0;  // kept (row, head) pairs, kept rows and valid rows seen by this lane
   if (sparse_try) {
     // 1. every row of the CTA, in rounds of round_tiles tiles: the round's
     //    e-values come into shared memory in one go (each warp copies its
@@ -1059,7 +1062,16 @@ __global__ void __launch_bounds__(kThreads, 1) fused_decode_kernel(FusedArgs a) 
         tile_info(t, nrow, ent, seg, pos);
         if (nrow == 0) continue;  // the same for the whole warp
         float f[H];
-        lds_heads<H>(tsf + t * H, f);
+        {
+          // the tile's factors exp2(max_tile - max) / sum, from its piece's global statistics
+          const float* st = reinterpret_cast<const float*>(ulist + ent * kRec + 8);
+#pragma unroll
+          for (int h = 0; h < H; ++h) {
+            const float M = st[2 * h], il = st[2 * h + 1];
+            const float mt = tsm[t * H + h];
+            f[h] = (il > 0.0f && mt > -INFINITY) ? exp2f(mt - M) * il : 0.0f;
+          }
+        }
         const float* et = ebuf + (t - T0) * TR * H;
 #pragma unroll
         for (int hf = 0; hf < 2; ++hf) {
@@ -1083,6 +1095,7 @@ __global__ void __launch_bounds__(kThreads, 1) fused_decode_kernel(FusedArgs a) 
           }
           kh_lane += kh;
           kr_lane += need ? 1u : 0u;
+          kv_lane += valid ? 1u : 0u;
           const unsigned bal = __ballot_sync(kFull, need);
           if (need) {
             const int o = n_w + __popc(bal & ((1u << lane) - 1u));
@@ -1122,6 +1135,10 @@ __global__ void __launch_bounds__(kThreads, 1) fused_decode_kernel(FusedArgs a) 
   }
   __syncthreads();
   const bool sparse = sparse_try && !*static_cast<volatile int*>(&s_ovf);
+  if (sparse_try && !sparse) {  // the list overflowed: the per-piece scan below needs the factors
+    tile_factors();
+    __syncthreads();
+  }
   if (sparse) {
     if (tid == 0) {
       int acc_n = 0;
@@ -1133,8 +1150,9 @@ __global__ void __launch_bounds__(kThreads, 1) fused_decode_kernel(FusedArgs a) 
     for (int off = 16; off >= 1; off >>= 1) {
       kh_lane += __shfl_xor_sync(kFull, kh_lane, off);
       kr_lane += __shfl_xor_sync(kFull, kr_lane, off);
+      kv_lane += __shfl_xor_sync(kFull, kv_lane, off);
     }
-    if (lane == 0) { atomicAdd(&s_kept[0], (int)kh_lane); atomicAdd(&s_kept[1], (int)kr_lane); }
+    if (lane == 0) { atomicAdd(&s_kept[0], (int)kh_lane); atomicAdd(&s_kept[1], (int)kr_lane); atomicAdd(&s_valid, (int)kv_lane); }
     if (tid < CW * 2) s_spiece[tid] = -1;
     // 2. the CTA's kept rows are split evenly over the warps; each warp
     //    brings its rows' V codes and (scale, zero) into its staging slots
@@ -1274,22 +1292,13 @@ __global__ void __launch_bounds__(kThreads, 1) fused_decode_kernel(FusedArgs a) 
     // 3. the output of every piece not yet written: the sum of the slots
     //    that hold it, in warp order (zero when no head kept any row); a
     //    piece's slots lie in one range of the warp-ordered slot list
-    int2* const prange = reinterpret_cast<int2*>(smem_raw + kPrangeOff);
-    for (int e = tid; e < n_work; e += NTHR) {
-      int k_lo = CW * 2, k_hi = 0;
-      for (int k2 = 0; k2 < CW * 2; ++k2)
-        if (s_spiece[k2] == e) { k_lo = min(k_lo, k2); k_hi = k2 + 1; }
-      prange[e] = make_int2(k_lo, k_hi);
-    }
-    __syncthreads();
     for (int e = 0; e < n_work; ++e) {
       if (s_pdone[e]) continue;
-      const int2 kr = prange[e];
       const Unit x = load_unit(ulist + e * kRec);
       const int b = x.u / d.Hkv, g = x.u % d.Hkv;
       for (int o = tid; o < H * D; o += NTHR) {
         float s2 = 0.0f;
-        for (int k2 = kr.x; k2 < kr.y; ++k2)
+        for (int k2 = 0; k2 < CW * 2; ++k2)
           if (s_spiece[k2] == e)
             s2 += (k2 & 1) ? red2[(k2 >> 1) * H * D + o] : __ldcg(a.wslot + ((long long)cta * CW + (k2 >> 1)) * H * D + o);
         const int h = o / D, dd = o % D;
@@ -1339,12 +1348,7 @@ __global__ void __launch_bounds__(kThreads, 1) fused_decode_kernel(FusedArgs a) 
     }
     __syncthreads();
     if (tid == 0) {
-      long long valid = 0;
-      for (int e = 0; e < n_work; ++e) {
-        const Unit x = load_unit(ulist + e * kRec);
-        const int ga = max(x.cb, k0), gb = min(x.cb + x.nc, k1);
-        for (int c = ga; c < gb; ++c) valid += chunk_rows(x, c - x.cb).rows;
-      }
+      const long long valid = s_valid;  // every valid row of the CTA passed the scan once
       cnt_heads = (unsigned long long)(valid * H - s_kept[0]);
       cnt_rows = (unsigned long long)(valid - s_kept[1]);
     }
