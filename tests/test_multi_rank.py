@@ -69,3 +69,24 @@ def test_decode_bytes_per_row():
     per (b, h, d)."""
     assert bench.decode_bytes(10, 4, 2, 32, 128, 64, 6, 4) == 10 * 112 + 4 * 80 + 2 * 32 * 128 * 6
     assert bench.quantize_bytes(3, 128, 64, 6, 4) == 3 * (512 + 96 + 64 + 32)
+
+
+def test_reference_arm_prints_one_json_line():
+    """The reference arm (the CPU oracle) runs without a GPU and prints the
+    contract's line: impl, metric, value, unit, config of the GPU arm, a
+    cpu_baseline describing the run and an e2e block with no host copies."""
+    import json
+    import subprocess
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    p = subprocess.run([sys.executable, os.path.join(root, "bench.py"), "--impl", "reference", "--steps", "1",
+                        "--warmup", "3"], capture_output=True, text=True, timeout=600, cwd=root)
+    assert p.returncode == 0, p.stderr[-2000:]
+    lines = [ln for ln in p.stdout.splitlines() if ln.startswith("{")]
+    assert len(lines) == 1
+    line = json.loads(lines[0])
+    assert line["impl"] == "reference" and line["metric"] == bench.METRIC and line["unit"] == "GB/s"
+    assert line["value"] > 0 and line["higher_is_better"] is True
+    assert line["config"]["workload"] == bench.W.CONFIGS[bench.CFG_MAIN].name
+    assert line["cpu_baseline"]["kind"] == "oracle" and line["cpu_baseline"]["value"] == line["value"]
+    assert line["e2e"] == {"value": line["value"], "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}
