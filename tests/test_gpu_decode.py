@@ -127,6 +127,16 @@ def test_decode_more_units_than_threads(orc):
     assert np.all(out[zero] == 0.0)
 
 
+def test_decode_kept_list_overflow_falls_back(orc):
+    """One CTA per unit (112 units) with 4096 rows each and tau 1e-9: nearly
+    every row is kept, more than the 2048 one CTA can list, so the sparse
+    pass falls back to the per-piece scan; outputs, masks and counts still
+    match the oracle."""
+    cfg = W.scaled(W.CONFIGS[2], B=14, T_cap=4096, seed=93)
+    out, mask, counts = run_case(orc, cfg, 6, 4, 1e-9)
+    assert counts[1] < 14 * 8 * 4096 // 10     # most rows kept by some head
+
+
 def test_decode_capacity_invariance(orc):
     """The same tokens in a larger cache (more chunks launched, most of them
     empty) give the same skip set and outputs within tolerance."""
