@@ -196,3 +196,22 @@ def test_binding_raises_without_library(monkeypatch, tmp_path):
     monkeypatch.setattr(lkv, "LIB_PATH", str(tmp_path / "missing.so"))
     with pytest.raises(RuntimeError):
         lkv.lkv_version()
+
+
+def test_plain_c_client(L, tmp_path):
+    """A C11 program that includes only include/lkv.h compiles with gcc
+    (-Wall -Werror), links liblkv.so and gets the documented results of the
+    calls that need no GPU: the boundary is usable from plain C."""
+    import shutil
+    import subprocess
+    cc = shutil.which("gcc") or shutil.which("cc")
+    if cc is None:
+        pytest.skip("no C compiler")
+    pkg = os.path.dirname(lkv.LIB_PATH)
+    exe = tmp_path / "abi_client"
+    build = subprocess.run([cc, "-std=c11", "-Wall", "-Werror", "-I", os.path.join(ROOT, "include"),
+                            os.path.join(ROOT, "tests", "abi_client.c"), "-L", pkg, "-llkv",
+                            f"-Wl,-rpath,{pkg}", "-o", str(exe)], capture_output=True, text=True)
+    assert build.returncode == 0, build.stderr
+    run = subprocess.run([str(exe)], capture_output=True, text=True, timeout=120)
+    assert run.returncode == 0 and run.stdout.strip() == "ok", run.stdout + run.stderr
